@@ -1,0 +1,512 @@
+#!/usr/bin/env python
+"""Decode throughput of DeepSeek-V4 CSA/HCA attention layers on B200.
+
+One step = one decode step (one new token per sequence) through every layer
+of the workload: new-token append + block compression, indexer + top-k (CSA),
+MQA over selected / all entries + window + sink, split-K combine.  The
+default workload is the V4-Pro CSA + HCA layer pair at 1M context, batch 4
+(every decode step of the hot path); the Flash 128K HCA and CSA layers are
+reported beside it under "also".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 runs as one process per GPU (torchrun); sequences are independent, so
+every rank decodes its own batch (weak scaling, no collective on the data
+path); the time is the max over ranks.  One JSON line is printed by rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+HEADLINE = "pro_pair_1m"
+ALSO = ("hca_flash_128k", "csa_flash_128k")
+METRIC = "CSA/HCA layer decode queries/s at 128K & 1M ctx; % of HBM/FP4-TC roofline"
+L2_BYTES = 126 * 1024 * 1024
+FLUSH_BYTES = 320 * 1024 * 1024
+
+
+# ------------------------------------------------------------------ state from synthetic inputs
+
+def desc_for(ly):
+    import long_context_compressed_kv_b200 as v
+    return v.layer_desc(v.CSA if ly.kind == "csa" else v.HCA, ly.m, ly.H, ly.d, ly.d_rope,
+                        n_win=ly.n_win, rope_theta=ly.rope_theta, H_I=ly.H_I, d_I=ly.d_I,
+                        top_k=ly.top_k, kv_dtype=v.E4M3_BF16ROPE if ly.kv_fp8 else v.F32,
+                        idx_dtype=v.MXFP4 if ly.idx_fp4 else v.F32)
+
+
+def build_decode_layer(w, li, inp, in_dtype=None):
+    """A DecodeLayer holding the coded synthetic history of ``synth.decode_layer_inputs``
+    and the new token's inputs, ready for ``step``."""
+    import torch
+    from long_context_compressed_kv_b200.decode import DecodeLayer
+    ly = w.layers[li]
+    p, ring = inp["p"], inp["ring"]
+    lay = DecodeLayer(desc_for(ly), w.B, kv_rows=inp["n_hist"] + 1, swa_rows=ly.n_win,
+                      in_dtype=in_dtype or torch.float32)
+    lay.load_entries(inp["hist_entries"])
+    lay.load_window(inp["swa_hist"], first_token=p - (ly.n_win - 1))
+    names = ["Ca", "Za", "Cb", "Zb"] if ly.kind == "csa" else ["C", "Z"]
+    tail = np.stack([inp["tail_" + nm][:, : ring - 1] for nm in names], 2)
+    itail = None
+    if ly.kind == "csa":
+        itail = np.stack([inp["itail_" + nm][:, : ring - 1] for nm in names], 2)
+    lay.load_tail(tail, p - ring + 1, itail)
+    lay.x_main.copy_(torch.from_numpy(np.stack([inp["tail_" + nm][:, ring - 1] for nm in names], 1)))
+    lay.bias.copy_(torch.from_numpy(inp["bias"]))
+    lay.Q.copy_(torch.from_numpy(inp["Q"]))
+    lay.sink = torch.from_numpy(inp["sink"]).cuda()
+    lay.pos.fill_(p)
+    if ly.kind == "csa":
+        lay.load_keys(inp["hist_keys"])
+        lay.x_idx.copy_(torch.from_numpy(
+            np.stack([inp["itail_" + nm][:, ring - 1] for nm in names], 1)))
+        lay.ibias.copy_(torch.from_numpy(inp["ibias"]))
+        lay.set_index_query(inp["qI"])
+        lay.w.copy_(torch.from_numpy(inp["w"]))
+    lay.max_vis = (p + 1) // ly.m
+    return lay
+
+
+def algorithmic_bytes(w):
+    """Bytes one decode step must move (per the method), per layer: visible or
+    selected entries x 580 B, indexer keys x 68 B, window tokens x 580 B, Q in
+    bf16, indexer q (MXFP4) + weights, the new token's inputs, the output."""
+    out = {}
+    for ly in w.layers:
+        p = w.L - 1
+        n_vis = (p + 1) // ly.m
+        entry = (ly.d - ly.d_rope) + 2 * ly.d_rope + 4
+        q_b = ly.H * ly.d * 2 + ly.H * ly.d * 2
+        if ly.kind == "csa":
+            key_b = ly.d_I // 2 + ly.d_I // 32
+            idx = n_vis * key_b + ly.H_I * (key_b + 4)
+            mqa = (ly.top_k + ly.n_win) * entry + q_b
+            out["csa"] = dict(index=w.B * idx, mqa=w.B * mqa, entries=w.B * (ly.top_k + ly.n_win),
+                              keys=w.B * n_vis)
+        else:
+            mqa = (n_vis + ly.n_win) * entry + q_b
+            out["hca"] = dict(mqa=w.B * mqa, entries=w.B * (n_vis + ly.n_win))
+    return out
+
+
+def algorithmic_flops(w):
+    out = 0
+    for ly in w.layers:
+        n_vis = (w.L) // ly.m
+        if ly.kind == "csa":
+            out += w.B * (n_vis * 2 * ly.H_I * ly.d_I + (ly.top_k + ly.n_win) * 4 * ly.H * ly.d)
+        else:
+            out += w.B * (n_vis + ly.n_win) * 4 * ly.H * ly.d
+    return out
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ timing helpers
+
+def timed_device(run, flush, steps, stream):
+    """Per-step CUDA-event durations (ms) of ``run`` with an L2 flush between
+    steps (outside the timed intervals), all on ``stream``."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            flush()
+            a.record(stream)
+            run()
+            b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def max_over_ranks(x: float, dist):
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist):
+    import torch
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------------ the GPU arm
+
+class Workload:
+    """The decode layers of one workload on this GPU, captured as one graph."""
+
+    def __init__(self, name):
+        import torch
+        self.w = synth.WORKLOADS[name]
+        self.inputs = [synth.decode_layer_inputs(self.w, li) for li in range(len(self.w.layers))]
+        self.layers = [build_decode_layer(self.w, li, inp) for li, inp in enumerate(self.inputs)]
+        torch.cuda.synchronize()
+        self.graph = None
+
+    def step(self):
+        for lay in self.layers:
+            lay.step(lay.max_vis)
+
+    def capture(self):
+        import torch
+        self.step()                               # first launches outside the capture
+        torch.cuda.synchronize()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.step()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step()
+        torch.cuda.synchronize()
+
+    def replay(self):
+        self.graph.replay()
+
+    def queries_per_step(self):
+        return self.w.B
+
+    def launches_per_step(self):
+        n = 0
+        for ly in self.w.layers:
+            # prep + window-KV compress + entry compress (+ key compress)
+            # (+ index scores + top-k) + MQA + combine
+            n += 1 + 2 + (1 if ly.kind == "csa" else 0) + (2 if ly.kind == "csa" else 0) + 2
+        return n
+
+    # per-step host<->device traffic of the end-to-end measurement
+    def host_io(self):
+        import torch
+        ins, outs = [], []
+        for lay in self.layers:
+            for t in ([lay.x_main, lay.Q, lay.pos] +
+                      ([lay.x_idx, lay.qI, lay.qI_sf, lay.w] if lay.csa else [])):
+                if t is None:
+                    continue
+                h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                h.copy_(t)
+                ins.append((h, t))
+            h = torch.empty(lay.out.shape, dtype=lay.out.dtype, pin_memory=True)
+            outs.append((h, lay.out))
+        return ins, outs
+
+
+def run_gpu(args, dist, rank, world):
+    import torch
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    stream = torch.cuda.current_stream()
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def flush():
+        flush_buf.zero_()
+
+    wl = Workload(args.workload)
+    launches = wl.launches_per_step()
+    wl.capture()
+    for _ in range(args.warmup):
+        flush()
+        wl.replay()
+    barrier(dist)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        barrier(dist)
+        per_step = timed_device(wl.replay, flush, args.steps, stream)
+        barrier(dist)
+    ms = max_over_ranks(float(np.mean(per_step)), dist)
+    if args.profile:
+        return dict(profile=True, ms=ms, launches=launches)
+    q_step = wl.queries_per_step()
+    value = world * q_step / (ms / 1e3)
+
+    # ---- dominant kernel: the indexer score kernel of the CSA layer, timed alone
+    import long_context_compressed_kv_b200 as v
+    csa = [lay for lay in wl.layers if lay.csa]
+    roof = None
+    abytes = algorithmic_bytes(wl.w)
+    peaks = _peaks()
+    if csa:
+        lay = csa[0]
+        scores = torch.empty(lay.B, lay.max_vis, dtype=torch.float32, device="cuda")
+
+        def idx_only():
+            v.index_topk(lay.desc, qI=lay.qI, qI_sf=lay.qI_sf, w=lay.w, q_pos=lay.pos,
+                         keys=lay.keys, keys_sf=lay.keys_sf, key_rows=lay.kv_rows,
+                         max_vis=lay.max_vis, idx_out=None, scores_out=scores, ws=lay.ws)
+        for _ in range(3):
+            flush()
+            idx_only()
+        t_idx = float(np.mean(timed_device(idx_only, flush, max(args.steps, 10), stream)))
+        t_idx = max_over_ranks(t_idx, dist)
+        bytes_idx = abytes["csa"]["index"]
+        achieved = bytes_idx / (t_idx / 1e3) / 1e9
+        roof = {"kernel": "index_scores (CSA indexer, MXFP4 keys)", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "peak_source": peaks["source"], "launch_us": round(t_idx * 1e3, 2),
+                "algorithmic_bytes": int(bytes_idx)}
+    step_bytes = sum(sum(vv for kk, vv in d.items() if kk in ("index", "mqa"))
+                     for d in abytes.values())
+    step_roof = {"bytes": int(step_bytes), "us": round(ms * 1e3, 2),
+                 "achieved_gbs": round(step_bytes / (ms / 1e3) / 1e9, 1),
+                 "frac_hbm": round(step_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+
+    # ---- end to end through the public API with host buffers
+    ins, outs = wl.host_io()
+    h2d = sum(h.numel() * h.element_size() for h, _ in ins)
+    d2h = sum(h.numel() * h.element_size() for h, _ in outs)
+
+    def e2e_step():
+        for h, d in ins:
+            d.copy_(h, non_blocking=True)
+        wl.step()
+        for h, d in outs:
+            h.copy_(d, non_blocking=True)
+    for _ in range(args.warmup):
+        flush()
+        e2e_step()
+    barrier(dist)
+    e2e_ms = max_over_ranks(float(np.mean(timed_device(e2e_step, flush, args.steps, stream))), dist)
+    e2e_val = world * q_step / (e2e_ms / 1e3)
+
+    also = {}
+    if not args.no_also and world == 1:
+        del wl
+        torch.cuda.empty_cache()
+        for name in ALSO:
+            w2 = Workload(name)
+            w2.capture()
+            for _ in range(args.warmup):
+                flush()
+                w2.replay()
+            t2 = float(np.mean(timed_device(w2.replay, flush, args.steps, stream)))
+            b2 = algorithmic_bytes(w2.w)
+            sb = sum(sum(vv for kk, vv in d.items() if kk in ("index", "mqa")) for d in b2.values())
+            also[name] = {"queries_per_s": round(w2.queries_per_step() / (t2 / 1e3), 1),
+                          "us_per_step": round(t2 * 1e3, 2),
+                          "frac_hbm": round(sb / (t2 / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+            del w2
+            torch.cuda.empty_cache()
+    return dict(value=value, ms=ms, roof=roof, step_roof=step_roof, clocks=clk.summary(),
+                e2e=dict(value=e2e_val, h2d=h2d, d2h=d2h, ms=e2e_ms), also=also,
+                launches=launches, q_step=q_step,
+                per_step=per_step)
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ the oracle (CPU) arm
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def oracle_sample(name, seconds_target=12.0, max_seqs=None):
+    """Time the CPU oracle's decode step on a bounded sample of the workload:
+    whole sequences (every layer of the workload) until ~seconds_target of
+    CPU work.  Returns (queries/s, sample description, seconds)."""
+    from oracle import pipeline
+    w = synth.WORKLOADS[name]
+    inputs = [synth.decode_layer_inputs(w, li) for li in range(len(w.layers))]
+    caches = [dict() for _ in w.layers]
+    n = 0
+    t_total = 0.0
+    b = 0
+    while t_total < seconds_target and (max_seqs is None or n < max_seqs):
+        t0 = time.perf_counter()
+        for li, ly in enumerate(w.layers):
+            pipeline.decode_layer(inputs[li], ly, [b % w.B])
+        t_total += time.perf_counter() - t0
+        n += 1
+        b += 1
+    return n / t_total, f"{n} sequence(s) x {len(w.layers)} layer(s) of {name}", t_total
+
+
+def run_reference(args):
+    """The reference arm: the fp64 CPU oracle, as it stands, on host cores."""
+    from oracle import pipeline
+    w = synth.WORKLOADS[args.workload]
+    inputs = [synth.decode_layer_inputs(w, li) for li in range(len(w.layers))]
+    times = []
+    for s in range(args.warmup + args.steps):
+        b = s % w.B
+        t0 = time.perf_counter()
+        for li, ly in enumerate(w.layers):
+            pipeline.decode_layer(inputs[li], ly, [b])
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+    value = 1.0 / float(np.mean(times))
+    cores = _blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4),
+            "unit": "queries/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(float(np.mean(times)) * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "batch": w.B, "context": w.L,
+                       "layers": [ly.kind for ly in w.layers], "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "queries/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"per step: 1 sequence through every layer of {args.workload}"},
+            "e2e": {"value": round(value, 4), "unit": "queries/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="v4attn", choices=["v4attn", "reference"])
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-also", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="graph capture, warm-up and timed steps only (for a kernel launch list)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    res = run_gpu(args, dist, rank, world)
+    if res.get("profile"):
+        if rank == 0:
+            print(json.dumps({"profile": args.workload, "ms_per_step": res["ms"],
+                              "launches_per_step": res["launches"]}), flush=True)
+        return
+    if rank == 0:
+        w = synth.WORKLOADS[args.workload]
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            val, sample, secs = oracle_sample(args.workload)
+            cpu = {"value": round(val, 4), "unit": "queries/s", "cores": _blas_threads(),
+                   "kind": "oracle", "sample": sample, "seconds": round(secs, 1)}
+        line = {
+            "metric": METRIC, "value": round(res["value"], 1), "unit": "queries/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(res["ms"], 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3+bf16 KV, mxfp4 indexer, f32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "batch_per_gpu": w.B, "context": w.L,
+                       "layers": [f"{ly.kind} m={ly.m} H={ly.H} d={ly.d}" +
+                                  (f" top_k={ly.top_k} H_I={ly.H_I}x{ly.d_I}" if ly.kind == "csa"
+                                   else "") for ly in w.layers],
+                       "l2": "flushed between steps (320 MB write)",
+                       "parallelism": f"dp{world} (independent sequences)",
+                       "graph": "one CUDA graph per step"},
+            "e2e": {"value": round(res["e2e"]["value"], 1), "unit": "queries/s",
+                    "h2d_bytes_per_step": int(res["e2e"]["h2d"]),
+                    "d2h_bytes_per_step": int(res["e2e"]["d2h"]),
+                    "ms_per_step": round(res["e2e"]["ms"], 5)},
+            "gpu_launches": res["launches"] * args.steps,
+            "roofline": res["roof"],
+            "step_roofline": res["step_roof"],
+            "cpu_baseline": cpu,
+            "clocks": res["clocks"],
+            "also": res["also"],
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,494 @@
+// C-ABI entry points of the v4attn library: argument validation, workspace
+// layout, kernel selection and the decode-step orchestration.
+//
+// Every entry point validates its arguments on the host and returns before
+// launching anything when they are wrong; device-side checks (positions past a
+// cache, indices out of range) skip the access and set a bit of the status
+// word at the start of the workspace, read by v4attn_device_status().
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_kernels.h"
+
+using namespace v4a;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Workspace: [status header | decode scratch | body].  The body holds either
+// the indexer scores of an index_topk call or the split-K partials of an MQA
+// call; the two never live at the same time (stream order), so they overlap.
+size_t dec_bytes(int32_t n_q) { return align_up((size_t)n_q * 3 * sizeof(int64_t)); }
+size_t body0(int32_t n_q) { return align_up(sizeof(WsHeader)) + dec_bytes(n_q); }
+size_t index_need(int32_t n_q, int64_t max_vis) {
+  return align_up((size_t)n_q * (size_t)std::max<int64_t>(max_vis, 1) * sizeof(float));
+}
+int mqa_splits(const v4attn_layer_desc* d, int64_t keys) {
+  const int sk = mqa_split_keys(d);
+  return (int)std::max<int64_t>(1, (keys + sk - 1) / sk);
+}
+size_t mqa_part_o_bytes(const v4attn_layer_desc* d, int32_t n_q, int n_split) {
+  return align_up((size_t)n_q * n_split * d->H * d->d * sizeof(float));
+}
+size_t mqa_need(const v4attn_layer_desc* d, int32_t n_q, int64_t keys) {
+  const int S = mqa_splits(d, keys);
+  return mqa_part_o_bytes(d, n_q, S) + align_up((size_t)n_q * S * d->H * 2 * sizeof(float));
+}
+size_t total_need(const v4attn_layer_desc* d, int32_t n_q, int64_t max_vis) {
+  size_t body = mqa_need(d, n_q, max_vis + d->n_win);
+  if (d->kind == V4A_CSA) {
+    body = std::max(body, index_need(n_q, max_vis));
+    body = std::max(body, mqa_need(d, n_q, (int64_t)d->top_k + d->n_win));
+  }
+  return body0(n_q) + body;
+}
+
+v4attn_status check_desc(const v4attn_layer_desc* d) {
+  if (!d) return V4A_ERR_INVALID_ARG;
+  if (d->kind != V4A_CSA && d->kind != V4A_HCA) return V4A_ERR_INVALID_ARG;
+  if (d->m < 1 || d->m > 128) return V4A_ERR_INVALID_ARG;
+  if (d->n_win < 0 || d->n_win > 1024) return V4A_ERR_INVALID_ARG;
+  if (d->H < 1 || d->H > 128) return V4A_ERR_UNSUPPORTED;
+  if (d->d < 32 || d->d > 512 || d->d % 32) return V4A_ERR_UNSUPPORTED;
+  if (d->d_rope < 0 || d->d_rope > d->d || d->d_rope % 2) return V4A_ERR_INVALID_ARG;
+  if (!(d->rope_theta > 0.f)) return V4A_ERR_INVALID_ARG;
+  if (!(d->rms_eps >= 0.f)) return V4A_ERR_INVALID_ARG;
+  if (d->kv_dtype != V4A_F32 && d->kv_dtype != V4A_E4M3_BF16ROPE) return V4A_ERR_UNSUPPORTED;
+  if (d->kv_dtype == V4A_E4M3_BF16ROPE && (d->d != 512 || d->d_rope != 64))
+    return V4A_ERR_UNSUPPORTED;
+  if (d->kind == V4A_CSA) {
+    if (d->idx_dtype != V4A_F32 && d->idx_dtype != V4A_MXFP4) return V4A_ERR_UNSUPPORTED;
+    if (d->d_I != 32 && d->d_I != 64 && d->d_I != 128) return V4A_ERR_UNSUPPORTED;
+    if (d->H_I < 1 || d->H_I > 64) return V4A_ERR_UNSUPPORTED;
+    if (d->top_k < 1 || d->top_k > 2048) return V4A_ERR_UNSUPPORTED;
+  }
+  return V4A_OK;
+}
+
+float softmax_scale(const v4attn_layer_desc* d) {
+  return d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)d->d);
+}
+
+v4attn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? V4A_OK : V4A_ERR_CUDA; }
+
+v4attn_status run_compress(const v4attn_layer_desc* d, const v4attn_compress_args* a,
+                           cudaStream_t st) {
+  if (!a) return V4A_ERR_INVALID_ARG;
+  if (a->m < 1 || a->m > 128 || a->c < 32 || a->c > 1024 || a->c % 2 || a->B < 1)
+    return V4A_ERR_INVALID_ARG;
+  if (a->n_entries < 0 || a->B > 65535) return V4A_ERR_INVALID_ARG;
+  if (!a->Ca || (!a->Za && a->m != 1) || !a->seq_len || !a->entry_begin || !a->out)
+    return V4A_ERR_INVALID_ARG;
+  if (a->overlap && (!a->Cb || !a->Zb)) return V4A_ERR_INVALID_ARG;
+  if (a->in_dtype != V4A_F32 && a->in_dtype != V4A_BF16) return V4A_ERR_UNSUPPORTED;
+  if (a->in_rows < 1 || a->in_row_stride < a->c || a->out_rows < 1) return V4A_ERR_INVALID_ARG;
+  if (a->out_dtype == V4A_E4M3_BF16ROPE) {
+    if (a->c != 512 || d->d_rope != 64 || !a->out_scale) return V4A_ERR_UNSUPPORTED;
+  } else if (a->out_dtype == V4A_MXFP4) {
+    if (a->c % 32 || !a->out_scale) return V4A_ERR_UNSUPPORTED;
+  } else if (a->out_dtype != V4A_F32) {
+    return V4A_ERR_UNSUPPORTED;
+  }
+  if (a->apply_rope && d->d_rope > a->c) return V4A_ERR_INVALID_ARG;
+  if (a->n_entries == 0) return V4A_OK;
+  CompressParams P;
+  P.m = a->m;
+  P.overlap = a->overlap ? 1 : 0;
+  P.c = a->c;
+  P.Ca = a->Ca;
+  P.Za = a->Za;
+  P.Cb = a->Cb;
+  P.Zb = a->Zb;
+  P.in_dtype = a->in_dtype;
+  P.in_seq_stride = a->in_seq_stride;
+  P.in_row_stride = a->in_row_stride;
+  P.in_rows = a->in_rows;
+  P.bias = a->bias;
+  P.seq_len = a->seq_len;
+  P.entry_begin = a->entry_begin;
+  P.complete_only = a->complete_only;
+  P.apply_rmsnorm = a->apply_rmsnorm;
+  P.apply_rope = a->apply_rope;
+  P.out_dtype = a->out_dtype;
+  P.out = a->out;
+  P.out_scale = a->out_scale;
+  P.out_rows = a->out_rows;
+  P.d_rope = d->d_rope;   // stored-format split; rotation only when apply_rope
+  P.theta = d->rope_theta;
+  P.eps = d->rms_eps;
+  return cuda_status(launch_compress(P, a->B, a->n_entries, st));
+}
+
+v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args* a, void* ws,
+                             size_t ws_bytes, cudaStream_t st) {
+  if (d->kind != V4A_CSA) return V4A_ERR_INVALID_ARG;
+  if (!a || a->n_q < 1 || a->n_q > 65535 || a->B < 1) return V4A_ERR_INVALID_ARG;
+  if (!a->qI || !a->w || !a->q_pos || !a->keys || (!a->idx_out && !a->scores_out))
+    return V4A_ERR_INVALID_ARG;
+  if (d->idx_dtype == V4A_MXFP4 && (!a->qI_sf || !a->keys_sf)) return V4A_ERR_INVALID_ARG;
+  if (a->key_rows < 1 || a->max_vis < 0 || a->max_vis > a->key_rows) return V4A_ERR_INVALID_ARG;
+  if (!ws) return V4A_ERR_WORKSPACE;
+  if (ws_bytes < body0(a->n_q) + index_need(a->n_q, a->max_vis)) return V4A_ERR_WORKSPACE;
+  uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
+  float* scores = a->scores_out ? a->scores_out : reinterpret_cast<float*>(w8 + body0(a->n_q));
+  const int64_t ld = std::max<int64_t>(a->max_vis, 1);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  if (a->max_vis > 0) {
+    IndexParams P;
+    P.n_q = a->n_q;
+    P.B = a->B;
+    P.m = d->m;
+    P.H_I = d->H_I;
+    P.d_I = d->d_I;
+    P.idx_dtype = d->idx_dtype;
+    P.qI = a->qI;
+    P.qI_sf = a->qI_sf;
+    P.w = a->w;
+    P.q_seq = a->q_seq;
+    P.q_pos = a->q_pos;
+    P.keys = a->keys;
+    P.keys_sf = a->keys_sf;
+    P.key_rows = a->key_rows;
+    P.max_vis = a->max_vis;
+    P.scores = scores;
+    P.scores_ld = ld;
+    P.status = status;
+    cudaError_t e = index_scores_dispatch(P, st);
+    if (e != cudaSuccess) return V4A_ERR_CUDA;
+  }
+  if (!a->idx_out) return V4A_OK;   // scores-only call
+  TopkParams T;
+  T.n_q = a->n_q;
+  T.m = d->m;
+  T.k = d->top_k;
+  T.scores = scores;
+  T.scores_ld = ld;
+  T.max_vis = a->max_vis;
+  T.q_pos = a->q_pos;
+  T.idx_out = a->idx_out;
+  return cuda_status(launch_topk(T, st));
+}
+
+v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void* ws,
+                      size_t ws_bytes, cudaStream_t st, bool sparse) {
+  if (!a || a->n_q < 1 || a->n_q > 65535 || a->B < 1) return V4A_ERR_INVALID_ARG;
+  if (!a->Q || !a->q_pos || !a->kv || !a->out) return V4A_ERR_INVALID_ARG;
+  if (d->n_win > 0 && (!a->swa || a->swa_rows < d->n_win)) return V4A_ERR_INVALID_ARG;
+  if (d->kv_dtype == V4A_E4M3_BF16ROPE && (!a->kv_scale || (d->n_win > 0 && !a->swa_scale)))
+    return V4A_ERR_INVALID_ARG;
+  if (a->q_dtype != V4A_F32 && a->q_dtype != V4A_BF16) return V4A_ERR_UNSUPPORTED;
+  if (a->out_dtype != V4A_F32 && a->out_dtype != V4A_BF16) return V4A_ERR_UNSUPPORTED;
+  if (a->kv_rows < 1) return V4A_ERR_INVALID_ARG;
+  if (sparse && (!a->idx || a->n_sel < 1 || a->n_sel > 4096)) return V4A_ERR_INVALID_ARG;
+  if (!sparse && (a->max_vis < 0 || a->max_vis > a->kv_rows)) return V4A_ERR_INVALID_ARG;
+  if (!aligned16(a->kv) || (a->swa && !aligned16(a->swa)) || !aligned16(a->out))
+    return V4A_ERR_INVALID_ARG;
+  if (!ws) return V4A_ERR_WORKSPACE;
+  const int64_t keys = (sparse ? (int64_t)a->n_sel : a->max_vis) + d->n_win;
+  if (ws_bytes < body0(a->n_q) + mqa_need(d, a->n_q, keys)) return V4A_ERR_WORKSPACE;
+  uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
+  MqaParams P;
+  P.n_q = a->n_q;
+  P.B = a->B;
+  P.H = d->H;
+  P.d = d->d;
+  P.d_rope = d->d_rope;
+  P.n_win = d->n_win;
+  P.m = d->m;
+  P.theta = d->rope_theta;
+  P.scale = softmax_scale(d);
+  P.eps = d->rms_eps;
+  P.Q = a->Q;
+  P.q_dtype = a->q_dtype;
+  P.q_rmsnorm = a->q_rmsnorm;
+  P.q_seq = a->q_seq;
+  P.q_pos = a->q_pos;
+  P.kv_dtype = d->kv_dtype;
+  P.kv = reinterpret_cast<const uint8_t*>(a->kv);
+  P.kv_scale = a->kv_scale;
+  P.kv_rows = a->kv_rows;
+  P.swa = reinterpret_cast<const uint8_t*>(a->swa);
+  P.swa_scale = a->swa_scale;
+  P.swa_rows = a->swa_rows > 0 ? a->swa_rows : 1;
+  P.idx = sparse ? a->idx : nullptr;
+  P.n_sel = sparse ? a->n_sel : 0;
+  P.max_vis = sparse ? a->kv_rows : a->max_vis;
+  P.sink = a->sink;
+  P.split_keys = mqa_split_keys(d);
+  P.n_split = mqa_splits(d, keys);
+  P.part_o = reinterpret_cast<float*>(w8 + body0(a->n_q));
+  P.part_ml = reinterpret_cast<float*>(w8 + body0(a->n_q) + mqa_part_o_bytes(d, a->n_q, P.n_split));
+  P.out = a->out;
+  P.out_dtype = a->out_dtype;
+  P.lse = a->lse;
+  P.status = reinterpret_cast<uint32_t*>(ws);
+  cudaError_t e = mqa_dispatch(P, st);
+  if (e != cudaSuccess) return V4A_ERR_CUDA;
+  return cuda_status(launch_mqa_combine(P, st));
+}
+
+__global__ void decode_prep_kernel(int B, const int64_t* pos, int m, int ring, int n_arr, int d,
+                                   const void* x_main, void* tail, int in_elt, int dI,
+                                   const void* x_idx, void* itail, int64_t* lens, int64_t* eb_tok,
+                                   int64_t* eb_ent) {
+  const int b = blockIdx.x;
+  const int64_t p = pos[b];
+  if (threadIdx.x == 0) {
+    lens[b] = p + 1;
+    eb_tok[b] = p;
+    eb_ent[b] = p / m;
+  }
+  const int64_t slot = p % ring;
+  const int64_t nb = (int64_t)n_arr * d * in_elt;
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(x_main) + b * nb;
+  uint8_t* dst = reinterpret_cast<uint8_t*>(tail) + ((int64_t)b * ring + slot) * nb;
+  for (int64_t e = threadIdx.x; e < nb; e += blockDim.x) dst[e] = src[e];
+  if (x_idx) {
+    const int64_t ni = (int64_t)4 * dI * in_elt;
+    const uint8_t* s2 = reinterpret_cast<const uint8_t*>(x_idx) + b * ni;
+    uint8_t* d2 = reinterpret_cast<uint8_t*>(itail) + ((int64_t)b * ring + slot) * ni;
+    for (int64_t e = threadIdx.x; e < ni; e += blockDim.x) d2[e] = s2[e];
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t v4attn_workspace_size(const v4attn_layer_desc* desc, int32_t n_q, int64_t max_vis) {
+  if (check_desc(desc) != V4A_OK || n_q < 1 || max_vis < 0) return 0;
+  return total_need(desc, n_q, max_vis);
+}
+
+v4attn_status v4attn_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!ws || ws_bytes < sizeof(WsHeader)) return V4A_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, sizeof(WsHeader), stream));
+}
+
+v4attn_status v4attn_compress(const v4attn_layer_desc* desc, const v4attn_compress_args* args,
+                              void* ws, size_t ws_bytes, cudaStream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!desc || desc->d_rope < 0 || desc->d_rope % 2 || !(desc->rope_theta > 0.f))
+    return V4A_ERR_INVALID_ARG;
+  return run_compress(desc, args, stream);
+}
+
+v4attn_status v4attn_index_topk(const v4attn_layer_desc* desc, const v4attn_index_args* args,
+                                void* ws, size_t ws_bytes, cudaStream_t stream) {
+  v4attn_status s = check_desc(desc);
+  if (s != V4A_OK) return s;
+  return run_index_topk(desc, args, ws, ws_bytes, stream);
+}
+
+v4attn_status v4attn_sparse_mqa(const v4attn_layer_desc* desc, const v4attn_mqa_args* args,
+                                void* ws, size_t ws_bytes, cudaStream_t stream) {
+  v4attn_status s = check_desc(desc);
+  if (s != V4A_OK) return s;
+  return run_mqa(desc, args, ws, ws_bytes, stream, true);
+}
+
+v4attn_status v4attn_dense_mqa(const v4attn_layer_desc* desc, const v4attn_mqa_args* args,
+                               void* ws, size_t ws_bytes, cudaStream_t stream) {
+  v4attn_status s = check_desc(desc);
+  if (s != V4A_OK) return s;
+  return run_mqa(desc, args, ws, ws_bytes, stream, false);
+}
+
+v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_args* a, void* ws,
+                            size_t ws_bytes, cudaStream_t stream) {
+  v4attn_status s = check_desc(desc);
+  if (s != V4A_OK) return s;
+  if (!a || a->B < 1 || a->B > 65535 || !a->pos || !a->x_main || !a->tail || !a->kv || !a->swa ||
+      !a->Q || !a->out)
+    return V4A_ERR_INVALID_ARG;
+  const bool csa = desc->kind == V4A_CSA;
+  if (csa && (!a->x_idx || !a->itail || !a->keys || !a->qI || !a->w || !a->idx_out))
+    return V4A_ERR_INVALID_ARG;
+  if (a->in_dtype != V4A_F32 && a->in_dtype != V4A_BF16) return V4A_ERR_UNSUPPORTED;
+  if (a->max_vis < 0 || a->max_vis > a->kv_rows || (csa && a->max_vis > a->key_rows))
+    return V4A_ERR_INVALID_ARG;
+  if (!ws) return V4A_ERR_WORKSPACE;
+  if (ws_bytes < total_need(desc, a->B, a->max_vis)) return V4A_ERR_WORKSPACE;
+  uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
+  int64_t* lens = reinterpret_cast<int64_t*>(w8 + align_up(sizeof(WsHeader)));
+  int64_t* eb_tok = lens + a->B;
+  int64_t* eb_ent = eb_tok + a->B;
+  const int m = desc->m;
+  const int ring = csa ? 2 * m : m;
+  const int n_arr = csa ? 4 : 2;
+  const int d = desc->d;
+  const int elt = a->in_dtype == V4A_F32 ? 4 : 2;
+  decode_prep_kernel<<<a->B, 256, 0, stream>>>(a->B, a->pos, m, ring, n_arr, d, a->x_main,
+                                               a->tail, elt, desc->d_I, csa ? a->x_idx : nullptr,
+                                               a->itail, lens, eb_tok, eb_ent);
+  if (cudaGetLastError() != cudaSuccess) return V4A_ERR_CUDA;
+
+  // 1. window KV of the new token (RMSNorm, RoPE at p, stored format)
+  v4attn_compress_args c{};
+  c.m = 1;
+  c.overlap = 0;
+  c.c = d;
+  c.B = a->B;
+  c.Ca = a->x_main;
+  c.in_dtype = a->in_dtype;
+  c.in_seq_stride = (int64_t)n_arr * d;
+  c.in_row_stride = (int64_t)n_arr * d;
+  c.in_rows = 1;
+  c.seq_len = lens;
+  c.entry_begin = eb_tok;
+  c.n_entries = 1;
+  c.apply_rmsnorm = 1;
+  c.apply_rope = 1;
+  c.out_dtype = desc->kv_dtype;
+  c.out = a->swa;
+  c.out_scale = a->swa_scale;
+  c.out_rows = a->swa_rows;
+  s = run_compress(desc, &c, stream);
+  if (s != V4A_OK) return s;
+  // 2. the completed block's entry (and indexer key) from the tail rings
+  const uint8_t* tail = reinterpret_cast<const uint8_t*>(a->tail);
+  v4attn_compress_args e{};
+  e.m = m;
+  e.overlap = csa ? 1 : 0;
+  e.c = d;
+  e.B = a->B;
+  e.Ca = tail;
+  e.Za = tail + (size_t)d * elt;
+  e.Cb = csa ? tail + (size_t)2 * d * elt : nullptr;
+  e.Zb = csa ? tail + (size_t)3 * d * elt : nullptr;
+  e.in_dtype = a->in_dtype;
+  e.in_seq_stride = (int64_t)ring * n_arr * d;
+  e.in_row_stride = (int64_t)n_arr * d;
+  e.in_rows = ring;
+  e.bias = a->bias;
+  e.seq_len = lens;
+  e.entry_begin = eb_ent;
+  e.n_entries = 1;
+  e.complete_only = 1;
+  e.apply_rmsnorm = 1;
+  e.apply_rope = 1;
+  e.out_dtype = desc->kv_dtype;
+  e.out = a->kv;
+  e.out_scale = a->kv_scale;
+  e.out_rows = a->kv_rows;
+  s = run_compress(desc, &e, stream);
+  if (s != V4A_OK) return s;
+  if (csa) {
+    const uint8_t* it = reinterpret_cast<const uint8_t*>(a->itail);
+    const int dI = desc->d_I;
+    v4attn_compress_args k = e;
+    k.c = dI;
+    k.Ca = it;
+    k.Za = it + (size_t)dI * elt;
+    k.Cb = it + (size_t)2 * dI * elt;
+    k.Zb = it + (size_t)3 * dI * elt;
+    k.in_seq_stride = (int64_t)ring * 4 * dI;
+    k.in_row_stride = (int64_t)4 * dI;
+    k.bias = a->ibias;
+    k.apply_rmsnorm = 0;
+    k.apply_rope = 0;
+    k.out_dtype = desc->idx_dtype;
+    k.out = a->keys;
+    k.out_scale = a->keys_sf;
+    k.out_rows = a->key_rows;
+    s = run_compress(desc, &k, stream);
+    if (s != V4A_OK) return s;
+    // 3. indexer + top-k
+    v4attn_index_args ix{};
+    ix.n_q = a->B;
+    ix.B = a->B;
+    ix.qI = a->qI;
+    ix.qI_sf = a->qI_sf;
+    ix.w = a->w;
+    ix.q_seq = nullptr;
+    ix.q_pos = a->pos;
+    ix.keys = a->keys;
+    ix.keys_sf = a->keys_sf;
+    ix.key_rows = a->key_rows;
+    ix.max_vis = a->max_vis;
+    ix.idx_out = a->idx_out;
+    s = run_index_topk(desc, &ix, ws, ws_bytes, stream);
+    if (s != V4A_OK) return s;
+  }
+  // 4. MQA
+  v4attn_mqa_args q{};
+  q.n_q = a->B;
+  q.B = a->B;
+  q.Q = a->Q;
+  q.q_dtype = a->q_dtype;
+  q.q_rmsnorm = 0;
+  q.q_seq = nullptr;
+  q.q_pos = a->pos;
+  q.kv = a->kv;
+  q.kv_scale = a->kv_scale;
+  q.kv_rows = a->kv_rows;
+  q.swa = a->swa;
+  q.swa_scale = a->swa_scale;
+  q.swa_rows = a->swa_rows;
+  q.idx = csa ? a->idx_out : nullptr;
+  q.n_sel = csa ? desc->top_k : 0;
+  q.max_vis = a->max_vis;
+  q.sink = a->sink;
+  q.out = a->out;
+  q.out_dtype = a->out_dtype;
+  q.lse = a->lse;
+  return run_mqa(desc, &q, ws, ws_bytes, stream, csa);
+}
+
+v4attn_status v4attn_project(const v4attn_project_args* a, cudaStream_t stream) {
+  if (!a || a->M < 0 || a->N < 0 || a->K < 0 || !a->X || !a->W || !a->Y) return V4A_ERR_INVALID_ARG;
+  if ((a->x_dtype != V4A_F32 && a->x_dtype != V4A_BF16) || a->w_dtype != a->x_dtype)
+    return V4A_ERR_UNSUPPORTED;
+  if (a->y_dtype != V4A_F32 && a->y_dtype != V4A_BF16) return V4A_ERR_UNSUPPORTED;
+  if (a->ldx < a->K || a->ldw < a->N || a->ldy < a->N) return V4A_ERR_INVALID_ARG;
+  if (a->M == 0 || a->N == 0) return V4A_OK;
+  if (a->M > 65535LL * 64) return V4A_ERR_UNSUPPORTED;
+  ProjectParams P;
+  P.M = a->M;
+  P.N = a->N;
+  P.K = a->K;
+  P.X = a->X;
+  P.x_dtype = a->x_dtype;
+  P.ldx = a->ldx;
+  P.W = a->W;
+  P.ldw = a->ldw;
+  P.Y = a->Y;
+  P.y_dtype = a->y_dtype;
+  P.ldy = a->ldy;
+  return cuda_status(project_dispatch(P, stream));
+}
+
+v4attn_status v4attn_device_status(const void* ws, cudaStream_t stream, uint32_t* bits) {
+  if (!ws) return V4A_ERR_WORKSPACE;
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, ws, sizeof(uint32_t), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return V4A_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return V4A_ERR_CUDA;
+  if (bits) *bits = word;
+  if (word & ST_TIMEOUT) return V4A_ERR_TIMEOUT;
+  if (word) return V4A_ERR_DEVICE_CHECK;
+  return V4A_OK;
+}
+
+const char* v4attn_status_string(v4attn_status s) {
+  switch (s) {
+    case V4A_OK: return "ok";
+    case V4A_ERR_INVALID_ARG: return "invalid argument";
+    case V4A_ERR_UNSUPPORTED: return "unsupported shape or format";
+    case V4A_ERR_WORKSPACE: return "workspace missing or too small";
+    case V4A_ERR_CUDA: return "CUDA launch error";
+    case V4A_ERR_TIMEOUT: return "a bounded device wait ran out";
+    case V4A_ERR_DEVICE_CHECK: return "a device-side argument check failed";
+  }
+  return "unknown status";
+}
+
+const char* v4attn_build_info(void) { return build_info_string(); }
+
+}  // extern "C"

@@ -1,0 +1,352 @@
+// Lightning-indexer scores on the 5th-generation tensor cores: block-scaled
+// MXFP4 x MXFP4 MMA (tcgen05.mma kind::mxf4, E8M0 scale per 32 elements) with
+// the ReLU / head-weighted reduction fused into the TMEM epilogue.
+//
+// Method: "DeepSeek-V4 深读" (ricardokevins.github.io), section
+// "CSA：4× 压缩之后再 top-k" (64 indexer heads, ReLU scores, input-dependent
+// head weights) and section "FP4 QAT、可恢复 rollout 与百万 Token RL" (MXFP4
+// indexer QK path):  s_i = sum_h w_h * max(0, q_h . k_i).
+//
+// Shape of the contraction per query: D[128 keys][H_I heads] = K_tile . Q^T,
+// K-dim = d_I = 128 (two MMAs of K = 64).  A (keys) streams from HBM through a
+// multi-stage TMA ring (64-byte-swizzled K-major tiles); B (the query's H_I x
+// 128 codes) stays in shared memory for the query's whole key range; the E8M0
+// scales of both go to TMEM with tcgen05.cp (row m at lane m % 32 of every
+// sub-partition, column m / 32, byte = 32-element block).  The accumulator is
+// double-buffered in TMEM so the epilogue of tile i overlaps the MMA of tile
+// i+1.  Roles: warp 0 TMA producer, warp 1 MMA issuer (one lane), warps 2..5
+// epilogue (one thread per key row).  The kernel is HBM-bound: 68 bytes per key
+// against 16384 FP4 FLOP.
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+#include "tc_kernels.h"
+
+namespace v4a {
+
+namespace {
+
+constexpr int KT = 128;                 // keys per tile (MMA M)
+constexpr int KROW = 64;                // bytes per key row (128 E2M1)
+constexpr int STAGES = 12;
+constexpr int KTILE_BYTES = KT * KROW;  // 8 KB
+constexpr int SF_BYTES = 512;           // 128 rows x 4 scale bytes
+constexpr int MAXQ = 1024;              // queries per launch on this path
+constexpr int NTHREADS = 192;
+
+struct Smem {
+  alignas(1024) uint8_t keys[STAGES][KTILE_BYTES];
+  alignas(1024) uint8_t q[2][128 * KROW];
+  alignas(128) uint8_t sfa[STAGES][SF_BYTES];
+  alignas(128) uint8_t sfb[2][SF_BYTES];
+  float w[2][128];
+  uint64_t full[STAGES], empty[STAGES], qfull[2], qempty[2], accfull[2], accempty[2];
+  int tile_prefix[MAXQ + 1];
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct TileIter {
+  int q = -1, lt = 0, seg = -1;
+  int qcur = 0;
+};
+
+}  // namespace
+
+__device__ __forceinline__ void fail(Smem& s, uint32_t* status) {
+  s.abort = 1;
+  flag(status, ST_TIMEOUT);
+}
+
+// Decode tile g into (query, local tile); `it` tracks segments (query changes).
+__device__ __forceinline__ void locate(const Smem& s, int n_q, int g, TileIter& t) {
+  while (t.qcur + 1 <= n_q && s.tile_prefix[t.qcur + 1] <= g) ++t.qcur;
+  if (t.qcur != t.q) {
+    t.q = t.qcur;
+    ++t.seg;
+  }
+  t.lt = g - s.tile_prefix[t.q];
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    index_tc_kernel(IndexParams P, const __grid_constant__ CUtensorMap tm_keys,
+                    const __grid_constant__ CUtensorMap tm_q) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = P.H_I;                       // MMA N (multiple of 16, <= 128)
+  const uint32_t TM_COLS = 256;
+
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    s.tile_prefix[0] = 0;
+    for (int q = 0; q < P.n_q; ++q) {
+      int64_t nv = (P.q_pos[q] + 1) / P.m;
+      const int b = P.q_seq ? P.q_seq[q] : q;
+      if (b < 0 || b >= P.B) {
+        flag(P.status, ST_BAD_SEQ);
+        nv = 0;
+      }
+      if (nv > P.key_rows || nv > P.max_vis) {
+        flag(P.status, ST_BAD_POSITION);
+        nv = min(P.key_rows, P.max_vis);
+      }
+      acc += (int)((nv + KT - 1) / KT);
+      s.tile_prefix[q + 1] = acc;
+    }
+    s.abort = 0;
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.qfull[i], 1);
+      mbar_init(&s.qempty[i], 1 + 4);
+      mbar_init(&s.accfull[i], 1);
+      mbar_init(&s.accempty[i], 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(&s.tmem_base, TM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const int total = s.tile_prefix[P.n_q];
+  const int g0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
+  const int g1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
+  const uint32_t tmem = s.tmem_base;
+  // TMEM columns: acc[a] at a*N; SFA[a] at 2N + 4a; SFB[j] at 2N + 8 + 4j
+  const uint32_t col_sfa = 2 * N, col_sfb = 2 * N + 8;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_keys);
+      prefetch_tmap(&tm_q);
+    }
+    TileIter t;
+    const uint32_t* ksf32 = reinterpret_cast<const uint32_t*>(P.keys_sf);
+    const int64_t total_rows = (int64_t)P.B * P.key_rows;
+    int it = 0;
+    for (int g = g0; g < g1 && !s.abort; ++g, ++it) {
+      const int seg_before = t.seg;
+      locate(s, P.n_q, g, t);
+      const int b = P.q_seq ? P.q_seq[t.q] : t.q;
+      if (t.seg != seg_before) {
+        const int j = t.seg & 1, uq = t.seg >> 1;
+        if (uq >= 1 && !mbar_wait(&s.qempty[j], (uq - 1) & 1)) {
+          fail(s, P.status);
+          break;
+        }
+        if (lane == 0) {
+          mbar_expect_tx(&s.qfull[j], (uint32_t)(N * KROW));
+          tma_load_2d(s.q[j], &tm_q, &s.qfull[j], 0, t.q * P.H_I);
+        }
+        // query scales in the tcgen05 scale-factor order, head weights
+        for (int h = lane; h < 128; h += 32) {
+          uint32_t word = 0;
+          if (h < N) word = reinterpret_cast<const uint32_t*>(P.qI_sf)[(int64_t)t.q * P.H_I + h];
+          *reinterpret_cast<uint32_t*>(&s.sfb[j][16 * (h & 31) + 4 * (h >> 5)]) = word;
+          s.w[j][h] = (h < N) ? P.w[(int64_t)t.q * P.H_I + h] : 0.f;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.qfull[j]);
+      }
+      const int st = it % STAGES, u = it / STAGES;
+      if (u >= 1 && !mbar_wait(&s.empty[st], (u - 1) & 1)) {
+        fail(s, P.status);
+        break;
+      }
+      const int64_t row0 = (int64_t)b * P.key_rows + (int64_t)t.lt * KT;
+      if (lane == 0) {
+        mbar_expect_tx(&s.full[st], KTILE_BYTES);
+        tma_load_2d(s.keys[st], &tm_keys, &s.full[st], 0, (int)row0);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int r = lane * 4 + k;
+        const int64_t gr = row0 + r;
+        const uint32_t word = (gr < total_rows) ? ksf32[gr] : 0u;
+        *reinterpret_cast<uint32_t*>(&s.sfa[st][16 * (r & 31) + 4 * (r >> 5)]) = word;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.full[st]);
+    }
+    // drain: no load may still be landing in shared memory when the CTA exits
+    if (s.abort && lane == 0) {
+      for (int k = 0; k < STAGES && k < it; ++k) {
+        const int i2 = it - 1 - k;
+        mbar_wait(&s.full[i2 % STAGES], (i2 / STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    TileIter t;
+    int it = 0;
+    const uint64_t kdesc_bits = smem_desc_bits(16, 8 * KROW, 4);    // K-major, 64B swizzle
+    const uint64_t sf_bits = smem_desc_bits(16, 128, 0);            // 32 rows x 16 B
+    for (int g = g0; g < g1 && !s.abort; ++g, ++it) {
+      const int seg_before = t.seg;
+      locate(s, P.n_q, g, t);
+      const int j = t.seg & 1;
+      if (t.seg != seg_before) {
+        if (!mbar_wait(&s.qfull[j], (t.seg >> 1) & 1)) {
+          fail(s, P.status);
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) tmem_cp_32x128b_warpx4(tmem + col_sfb + 4 * j, smem_desc(s.sfb[j], sf_bits));
+      }
+      const int st = it % STAGES, a = it & 1, ua = it >> 1;
+      if (!mbar_wait(&s.full[st], (it / STAGES) & 1)) {
+        fail(s, P.status);
+        break;
+      }
+      if (ua >= 1 && !mbar_wait(&s.accempty[a], (ua - 1) & 1)) {
+        fail(s, P.status);
+        break;
+      }
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t sfa = tmem + col_sfa + 4 * a;
+        const uint32_t sfb = tmem + col_sfb + 4 * j;
+        tmem_cp_32x128b_warpx4(sfa, smem_desc(s.sfa[st], sf_bits));
+        const uint64_t da = smem_desc(s.keys[st], kdesc_bits);
+        const uint64_t db = smem_desc(s.q[j], kdesc_bits);
+        const uint32_t d = tmem + a * N;
+        // K = 0..63 (scale bytes 0,1), then K = 64..127 (scale bytes 2,3): +32 B
+        mma_mxf4(d, da, db, idesc_mxf4(KT, N, 0, 0), sfa, sfb, 0);
+        mma_mxf4(d, da + 2, db + 2, idesc_mxf4(KT, N, 2, 2), sfa, sfb, 1);
+        tc_commit(&s.empty[st]);
+        tc_commit(&s.accfull[a]);
+        const bool seg_end = (g + 1 == g1) || (g + 1 >= s.tile_prefix[t.q + 1]);
+        if (seg_end) tc_commit(&s.qempty[j]);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;                  // TMEM lanes 32*quad .. +31
+    const int r = quad * 32 + lane;             // key row within the tile
+    // keys beyond the last tile of each query: -inf
+    {
+      const int et = threadIdx.x - 64;
+      for (int q = blockIdx.x; q < P.n_q; q += gridDim.x) {
+        const int64_t from = (int64_t)(s.tile_prefix[q + 1] - s.tile_prefix[q]) * KT;
+        for (int64_t i = from + et; i < P.max_vis; i += 128)
+          P.scores[(int64_t)q * P.scores_ld + i] = -INFINITY;
+      }
+    }
+    TileIter t;
+    int it = 0;
+    for (int g = g0; g < g1 && !s.abort; ++g, ++it) {
+      const int seg_before = t.seg;
+      locate(s, P.n_q, g, t);
+      const int j = t.seg & 1;
+      if (t.seg != seg_before && !mbar_wait(&s.qfull[j], (t.seg >> 1) & 1)) {
+        fail(s, P.status);
+        break;
+      }
+      const int a = it & 1;
+      if (!mbar_wait(&s.accfull[a], (it >> 1) & 1)) {
+        fail(s, P.status);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + a * N;
+      float score = 0.f;
+      for (int c = 0; c < N; c += 32) {
+        float v[32];
+        tmem_ld32(taddr + c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 32; ++h) score = fmaf(s.w[j][c + h], fmaxf(v[h], 0.f), score);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.accempty[a]);
+      const int64_t nv = min((int64_t)(P.q_pos[t.q] + 1) / P.m, min(P.key_rows, P.max_vis));
+      const int64_t i = (int64_t)t.lt * KT + r;
+      if (i < P.max_vis) P.scores[(int64_t)t.q * P.scores_ld + i] = (i < nv) ? score : -INFINITY;
+      const bool seg_end = (g + 1 == g1) || (g + 1 >= s.tile_prefix[t.q + 1]);
+      if (seg_end) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.qempty[j]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D uint8 tensor map: rows of `row_bytes`, box of `box_rows` rows, 64B swizzle.
+bool make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int row_bytes, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || rows < 1 || rows > (1ll << 31)) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+bool index_tc_supported(const IndexParams& P) {
+  return P.idx_dtype == V4A_MXFP4 && P.d_I == 128 && P.H_I % 32 == 0 && P.H_I >= 32 &&
+         P.H_I <= 128 && P.n_q <= MAXQ && encode_fn() != nullptr &&
+         ((uintptr_t)P.keys & 15) == 0 && ((uintptr_t)P.qI & 15) == 0 &&
+         ((uintptr_t)P.keys_sf & 3) == 0 && ((uintptr_t)P.qI_sf & 3) == 0;
+}
+
+cudaError_t launch_index_tc(const IndexParams& P, cudaStream_t st) {
+  CUtensorMap tk, tq;
+  if (!make_rows_map(&tk, P.keys, (int64_t)P.B * P.key_rows, KROW, KT)) return cudaErrorInvalidValue;
+  if (!make_rows_map(&tq, P.qI, (int64_t)P.n_q * P.H_I, KROW, P.H_I)) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(Smem) + 1024;
+  static unsigned long long configured = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !(configured & (1ull << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured |= 1ull << dev;
+  }
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = sms;   // persistent: one CTA per SM, contiguous tile ranges
+  index_tc_kernel<<<grid, NTHREADS, smem, st>>>(P, tk, tq);
+  return cudaGetLastError();
+}
+
+}  // namespace v4a

@@ -1,0 +1,96 @@
+// Kernel parameter blocks and launchers of the v4attn library (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace v4a {
+
+struct CompressParams {
+  int m, overlap, c;
+  const void *Ca, *Za, *Cb, *Zb;
+  int in_dtype;
+  int64_t in_seq_stride, in_row_stride, in_rows;
+  const float* bias;
+  const int64_t* seq_len;
+  const int64_t* entry_begin;
+  int complete_only, apply_rmsnorm, apply_rope;
+  int out_dtype;
+  void* out;
+  void* out_scale;
+  int64_t out_rows;
+  int d_rope;
+  float theta, eps;
+};
+
+struct IndexParams {
+  int n_q, B, m, H_I, d_I, idx_dtype;
+  const void* qI;
+  const uint8_t* qI_sf;
+  const float* w;
+  const int32_t* q_seq;
+  const int64_t* q_pos;
+  const void* keys;
+  const uint8_t* keys_sf;
+  int64_t key_rows, max_vis;
+  float* scores;        // [n_q][max_vis]
+  int64_t scores_ld;
+  uint32_t* status;
+};
+
+struct TopkParams {
+  int n_q, m, k;
+  const float* scores;
+  int64_t scores_ld, max_vis;
+  const int64_t* q_pos;
+  int32_t* idx_out;
+};
+
+struct MqaParams {
+  int n_q, B, H, d, d_rope, n_win, m;
+  float theta, scale, eps;
+  const void* Q;
+  int q_dtype, q_rmsnorm;
+  const int32_t* q_seq;
+  const int64_t* q_pos;
+  int kv_dtype;
+  const uint8_t* kv;
+  const float* kv_scale;
+  int64_t kv_rows;
+  const uint8_t* swa;
+  const float* swa_scale;
+  int64_t swa_rows;
+  const int32_t* idx;   // sparse: [n_q][n_sel]; dense: nullptr
+  int n_sel;
+  int64_t max_vis;
+  const float* sink;
+  int n_split;          // splits per query
+  int split_keys;       // keys per split
+  float* part_o;        // [n_q][n_split][H][d]
+  float* part_ml;       // [n_q][n_split][H][2]
+  void* out;
+  int out_dtype;
+  float* lse;
+  uint32_t* status;
+};
+
+struct ProjectParams {
+  int64_t M, N, K;
+  const void* X;
+  int x_dtype;
+  int64_t ldx;
+  const void* W;
+  int64_t ldw;
+  void* Y;
+  int y_dtype;
+  int64_t ldy;
+};
+
+cudaError_t launch_compress(const CompressParams& P, int B, int n_entries, cudaStream_t st);
+cudaError_t launch_index_scores(const IndexParams& P, cudaStream_t st);
+cudaError_t launch_topk(const TopkParams& P, cudaStream_t st);
+cudaError_t launch_mqa_simt(const MqaParams& P, cudaStream_t st);
+cudaError_t launch_mqa_combine(const MqaParams& P, cudaStream_t st);
+cudaError_t launch_project(const ProjectParams& P, cudaStream_t st);
+
+}  // namespace v4a

@@ -60,9 +60,10 @@ def decode_layer(inp: dict, ly, seqs, need_scores: bool = False) -> dict:
     out = {k: [] for k in ("entry_new", "entry_new_val", "key_new", "key_new_val", "swa_new",
                            "swa_new_val", "scores", "idx", "out", "lse")}
     for b in seqs:
-        hist_store, hist_val = store_kv(inp["hist_entries"][b], ly)
+        hist = inp["hist_entries"][b]
+        n_hist = hist.shape[0]
         tail = lambda nm: (lambda t, arr=inp["tail_" + nm][b]: np.asarray(arr, np.float64)[t - t0])
-        ents = hist_val
+        new_val = None
         if complete:
             if ly.kind == "csa":
                 e = pool(np.array([i_new]), m, True, p + 1, tail("Ca"), tail("Za"), inp["bias"],
@@ -70,10 +71,20 @@ def decode_layer(inp: dict, ly, seqs, need_scores: bool = False) -> dict:
             else:
                 e = pool(np.array([i_new]), m, False, p + 1, tail("C"), tail("Z"), inp["bias"])
             e = finish_main(e, np.array([i_new]), m, ly.d_rope, ly.rope_theta)
-            st, val = store_kv(e, ly)
+            st, new_val = store_kv(e, ly)
             out["entry_new"].append(st)
-            out["entry_new_val"].append(val[0])
-            ents = np.concatenate([hist_val, val], axis=0)
+            out["entry_new_val"].append(new_val[0])
+
+        def entries(rows):
+            """Stored (dequantised) entries for the given entry indices."""
+            rows = np.asarray(rows, dtype=np.int64)
+            old = rows[rows < n_hist]
+            _, val = store_kv(hist[old], ly)
+            res = np.empty((len(rows), ly.d))
+            res[rows < n_hist] = val
+            if np.any(rows >= n_hist):
+                res[rows >= n_hist] = new_val[0]
+            return res
         # window: synthetic history rows for tokens p-n_win+1 .. p-1, then token p
         ca_p = inp["tail_Ca" if ly.kind == "csa" else "tail_C"][b][ring - 1]
         st, swa_p = store_kv(token_kv(ca_p[None, :], np.array([p]), ly), ly)
@@ -98,9 +109,9 @@ def decode_layer(inp: dict, ly, seqs, need_scores: bool = False) -> dict:
             idx = topk(s, n_vis, ly.top_k)
             out["scores"].append(s)
             out["idx"].append(idx)
-            sel = ents[idx[idx >= 0]]
+            sel = entries(idx[idx >= 0])
         else:
-            sel = ents[:n_vis]
+            sel = entries(np.arange(n_vis))
         q = prepare_query(inp["Q"][b], p, ly.d_rope, ly.rope_theta, ly.kv_fp8)
         keys = np.concatenate([sel, swa_val], axis=0)
         o, lse = attend(q, keys, scale, inp["sink"])

@@ -1,0 +1,90 @@
+"""The C-ABI library loads, exports every entry point include/v4attn.h
+declares, its ctypes mirror matches the C struct layouts (checked against a
+gcc-compiled probe of the header), and host-side argument checks reject bad
+calls before anything is launched (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "v4attn.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(v4attn_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_entry_point():
+    from long_context_compressed_kv_b200 import _abi
+    lib = _abi.load()
+    names = _declared_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _abi.SIGNATURES, n
+    # and nothing in the binding is missing from the header
+    assert set(_abi.SIGNATURES) <= set(names)
+
+
+def test_struct_layouts_match_header(tmp_path):
+    from long_context_compressed_kv_b200 import _abi
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "v4attn.h"', "int main(void){"]
+    for cname, cls in _abi.STRUCTS.items():
+        lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
+        for fname, _ in cls._fields_:
+            lines.append(f'printf("{cname}.{fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines.append("return 0;}")
+    src = tmp_path / "probe.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-I", "/usr/local/cuda/include",
+                    str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    got = dict(line.split() for line in out.strip().splitlines())
+    for cname, cls in _abi.STRUCTS.items():
+        assert int(got[cname]) == ctypes.sizeof(cls), cname
+        for fname, _ in cls._fields_:
+            assert int(got[f"{cname}.{fname}"]) == getattr(cls, fname).offset, (cname, fname)
+
+
+def test_host_side_validation_rejects_bad_calls():
+    from long_context_compressed_kv_b200 import _abi
+    lib = _abi.load()
+    d = _abi.LayerDesc(_abi.HCA, 128, 128, 64, 512, 64, 160000.0, 0.0, 0, 0, 0,
+                       _abi.E4M3_BF16ROPE, _abi.MXFP4, 1e-6)
+    assert lib.v4attn_workspace_size(ctypes.byref(d), 16, 1024) > 0
+    bad = _abi.LayerDesc.from_buffer_copy(d)
+    bad.d = 100                                   # not a multiple of 32
+    assert lib.v4attn_workspace_size(ctypes.byref(bad), 16, 1024) == 0
+    assert lib.v4attn_dense_mqa(ctypes.byref(bad), None, None, 0, None) == _abi.ERR_UNSUPPORTED
+    assert lib.v4attn_dense_mqa(ctypes.byref(d), None, None, 0, None) == _abi.ERR_INVALID_ARG
+    a = _abi.MqaArgs()
+    a.n_q = 1
+    a.B = 1
+    assert lib.v4attn_dense_mqa(ctypes.byref(d), ctypes.byref(a), None, 0, None) == \
+        _abi.ERR_INVALID_ARG                      # null pointers
+    fp8_other = _abi.LayerDesc.from_buffer_copy(d)
+    fp8_other.d = 256
+    assert lib.v4attn_workspace_size(ctypes.byref(fp8_other), 1, 1) == 0
+    c = _abi.CompressArgs()
+    assert lib.v4attn_compress(ctypes.byref(d), ctypes.byref(c), None, 0, None) == \
+        _abi.ERR_INVALID_ARG
+    p = _abi.ProjectArgs()
+    p.M, p.N, p.K = 4, 4, 4
+    assert lib.v4attn_project(ctypes.byref(p), None) == _abi.ERR_INVALID_ARG
+    assert lib.v4attn_status_string(_abi.ERR_WORKSPACE) == b"workspace missing or too small"
+    assert b"sm_100a" in lib.v4attn_build_info()
+
+
+def test_csa_workspace_covers_index_and_sparse_mqa():
+    from long_context_compressed_kv_b200 import _abi
+    lib = _abi.load()
+    d = _abi.LayerDesc(_abi.CSA, 4, 128, 128, 512, 64, 160000.0, 0.0, 64, 128, 1024,
+                       _abi.E4M3_BF16ROPE, _abi.MXFP4, 1e-6)
+    n = lib.v4attn_workspace_size(ctypes.byref(d), 4, 262144)
+    assert n >= 4 * 262144 * 4                    # fp32 scores of every visible key

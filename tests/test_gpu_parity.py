@@ -1,0 +1,415 @@
+"""GPU parity: every stage of the CUDA path, called through the C ABI, against
+the fp64 CPU oracle on the same seeded inputs - small cases that span several
+tiles with ragged tails, the edge cases (first entries, partial windows,
+fewer visible keys than k, no sink), and the five workloads at full size with
+sampled sequences."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import codecs, compress as ocomp, indexer as oidx, mqa as omqa, pipeline
+from tests.gpu_util import (F32_ABS_TOL, R16_TOL, DecodeState, check_topk, code_rows,
+                            compare_decode, desc_for, dev, r16, read_keys, read_kv, v4)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+
+
+# ------------------------------------------------------------------ coding (bit-exact)
+
+def test_coding_is_bit_exact():
+    v = v4()
+    rng = np.random.default_rng(11)
+    vals = rng.standard_normal((3, 300, 512)).astype(np.float32)
+    vals[0, :50] *= 1e-3
+    vals[1, :50] *= 1e3
+    vals[2, 7] = 0.0
+    vals[2, 8, :448] = 0.0
+    d = v.layer_desc(v.HCA, 128, 64, 512, 64)
+    rows, sc = code_rows(d, dev(vals), v.E4M3_BF16ROPE)
+    codes, rbits, s = codecs.quantize_kv(vals.astype(np.float64), 64)
+    g = rows.cpu().numpy()
+    assert np.array_equal(g[..., :448], codes)
+    assert np.array_equal(g[..., 448:].copy().view(np.uint16), rbits)
+    assert np.array_equal(sc.cpu().numpy(), s)
+    # MXFP4 (128 channels), including an all-zero block and saturating blocks
+    kv = rng.standard_normal((2, 700, 128)).astype(np.float32)
+    kv[0, 3, :32] = 0.0
+    kv[1, 5] *= 1e-30
+    rows, sf = code_rows(d, dev(kv), v.MXFP4)
+    c2, sf2 = codecs.quantize_mxfp4(kv.astype(np.float64))
+    assert np.array_equal(rows.cpu().numpy(), codecs.pack_e2m1(c2))
+    assert np.array_equal(sf.cpu().numpy(), sf2)
+    rows, _ = code_rows(d, dev(kv), v.F32)
+    assert np.array_equal(rows.cpu().numpy().view(np.float32), kv)
+
+
+# ------------------------------------------------------------------ compression
+
+@pytest.mark.parametrize("kind,m,L,fmt,c,ring", [
+    ("csa", 4, 4 * 37 + 3, "e4m3", 512, None),
+    ("csa", 4, 4 * 200, "mxfp4", 128, None),
+    ("csa", 4, 4 * 61 + 1, "f32", 128, None),
+    ("hca", 128, 128 * 5 + 77, "e4m3", 512, None),
+    ("hca", 128, 128 * 3, "f32", 64, None),
+    ("csa", 4, 4 * 50, "e4m3", 512, 8),      # tail ring input
+    ("hca", 128, 128 * 4, "e4m3", 512, 128),
+])
+@pytest.mark.parametrize("in_bf16", [False, True])
+def test_compress_parity(kind, m, L, fmt, c, ring, in_bf16):
+    v = v4()
+    rng = np.random.default_rng(L + c)
+    B = 2
+    overlap = kind == "csa"
+    arrs = {nm: rng.standard_normal((B, L, c)).astype(np.float32) for nm in ("Ca", "Za", "Cb", "Zb")}
+    if in_bf16:
+        arrs = {k: synth.bf16_values(a) for k, a in arrs.items()}
+    bias = (rng.standard_normal((2 * m if overlap else m, c)) * 0.1).astype(np.float32)
+    n_ent = ocomp.n_entries(L, m)
+    if ring is None:
+        e0, n_e, rows_in = 0, n_ent, L
+        dev_arrs = {k: dev(a, torch.bfloat16 if in_bf16 else torch.float32) for k, a in arrs.items()}
+    else:
+        # only the last complete block, read from a ring of `ring` rows
+        e0, n_e, rows_in = L // m - 1, 1, ring
+        rr = {}
+        for k, a in arrs.items():
+            r = np.zeros((B, ring, c), dtype=np.float32)
+            for t in range(L - ring, L):
+                r[:, t % ring] = a[:, t]
+            rr[k] = dev(r, torch.bfloat16 if in_bf16 else torch.float32)
+        dev_arrs = rr
+    fmt_id = {"e4m3": v.E4M3_BF16ROPE, "mxfp4": v.MXFP4, "f32": v.F32}[fmt]
+    norm_rope = fmt != "mxfp4"
+    d_rope = 64 if c == 512 else (32 if c >= 64 else 0)
+    desc = v.layer_desc(v.CSA if overlap else v.HCA, m, 16, 512, d_rope)
+    out_rows = n_ent + 3
+    rb = v.row_bytes(fmt_id, c, d_rope)
+    out = torch.zeros(B, out_rows, rb, dtype=torch.uint8, device="cuda")
+    sc = (torch.zeros(B, out_rows, dtype=torch.float32, device="cuda") if fmt == "e4m3" else
+          torch.zeros(B, out_rows, c // 32, dtype=torch.uint8, device="cuda") if fmt == "mxfp4"
+          else None)
+    lens = torch.full((B,), L, dtype=torch.int64, device="cuda")
+    eb = torch.full((B,), e0, dtype=torch.int64, device="cuda")
+    v.compress(desc, m=m, overlap=overlap, c=c, Ca=dev_arrs["Ca"], Za=dev_arrs["Za"],
+               Cb=dev_arrs["Cb"] if overlap else None, Zb=dev_arrs["Zb"] if overlap else None,
+               in_rows=rows_in, in_seq_stride=rows_in * c, in_row_stride=c, bias=dev(bias),
+               seq_len=lens, entry_begin=eb, n_entries=n_e, out_dtype=fmt_id, out=out,
+               out_scale=sc, out_rows=out_rows, apply_rmsnorm=norm_rope, apply_rope=norm_rope)
+    torch.cuda.synchronize()
+    ii = np.arange(e0, e0 + n_e)
+    g = out.cpu().numpy()
+    for b in range(B):
+        a64 = {k: a[b].astype(np.float64) for k, a in arrs.items()}
+        e = ocomp.pool(ii, m, overlap, L, a64["Ca"], a64["Za"], bias, a64["Cb"], a64["Zb"])
+        if norm_rope:
+            e = ocomp.finish_main(e, ii, m, d_rope, 160000.0)
+        if fmt == "e4m3":
+            ref = codecs.dequantize_kv(*codecs.quantize_kv(e, 64))
+            got = read_kv(g[b, ii], sc[b, ii].cpu().numpy(), fmt_id)
+            assert r16(got, ref) <= R16_TOL
+            # identical codes except rare fp32-vs-fp64 rounding-boundary decisions
+            assert np.mean(got == ref) > 0.995
+        elif fmt == "mxfp4":
+            c2, sf2 = codecs.quantize_mxfp4(e)
+            ref = codecs.dequantize_mxfp4(c2, sf2)
+            got = read_keys(g[b, ii], sc[b, ii].cpu().numpy(), fmt_id)
+            assert r16(got, ref) <= R16_TOL
+            assert np.mean(got == ref) > 0.995
+        else:
+            got = g[b, ii].view(np.float32).astype(np.float64)
+            assert np.max(np.abs(got - e)) <= F32_ABS_TOL
+    # rows outside the computed range are untouched
+    assert not g[:, n_ent:].any()
+
+
+# ------------------------------------------------------------------ indexer + top-k
+
+@pytest.mark.parametrize("fp4,d_I,H_I", [(True, 128, 64), (False, 32, 4), (True, 64, 16)])
+def test_index_topk_parity(fp4, d_I, H_I):
+    v = v4()
+    rng = np.random.default_rng(d_I + H_I)
+    B, N, k = 3, 3000, 64
+    keys = rng.standard_normal((B, N, d_I)).astype(np.float32)
+    positions = np.array([4 * N - 1, 4 * 700 + 2, 4 * 10 + 1, 2, 4 * N - 5, 4 * 2999 + 3])
+    q_seq = np.array([0, 1, 2, 0, 2, 1], dtype=np.int32)
+    nq = len(positions)
+    qI = rng.standard_normal((nq, H_I, d_I)).astype(np.float32)
+    w = rng.uniform(0, 1, (nq, H_I)).astype(np.float32)
+    ly = synth.Layer("csa", 4, 16, 512, 64, 128, H_I, d_I, k, idx_fp4=fp4)
+    desc = desc_for(ly)
+    kfmt = v.MXFP4 if fp4 else v.F32
+    krows, ksf = code_rows(desc, dev(keys), kfmt)
+    qrows, qsf = code_rows(desc, dev(qI.reshape(1, nq * H_I, d_I)), kfmt)
+    qrows = qrows.reshape(nq, H_I, -1)
+    qsf = None if qsf is None else qsf.reshape(nq, H_I, -1)
+    idx = torch.full((nq, k), -9, dtype=torch.int32, device="cuda")
+    scores = torch.zeros(nq, N, dtype=torch.float32, device="cuda")
+    ws = v.workspace(desc, nq, N)
+    v.index_topk(desc, qI=qrows, qI_sf=qsf, w=dev(w), q_pos=dev(positions, torch.int64),
+                 q_seq=dev(q_seq, torch.int32), B=B, keys=krows, keys_sf=ksf, key_rows=N,
+                 max_vis=N, idx_out=idx, scores_out=scores, ws=ws)
+    torch.cuda.synchronize()
+    assert v.device_status(ws) == 0
+    if fp4:
+        kd = codecs.dequantize_mxfp4(*codecs.quantize_mxfp4(keys.astype(np.float64)))
+        qd = codecs.dequantize_mxfp4(*codecs.quantize_mxfp4(qI.astype(np.float64)))
+    else:
+        kd, qd = keys.astype(np.float64), qI.astype(np.float64)
+    g_idx, g_s = idx.cpu().numpy(), scores.cpu().numpy()
+    for q in range(nq):
+        nv = int(ocomp.n_visible(positions[q], 4))
+        s = oidx.scores(qd[q], w[q], kd[q_seq[q], :nv])
+        scale = max(1.0, float(np.max(np.abs(s)))) if nv else 1.0
+        assert np.max(np.abs(g_s[q, :nv] - s), initial=0.0) <= 1e-5 * scale
+        assert np.all(np.isneginf(g_s[q, nv:]))
+        check_topk(g_idx[q], s, nv, k)
+
+
+def test_topk_ties_go_to_lower_index():
+    """Many exactly equal scores: the selection must be the lowest indices."""
+    v = v4()
+    B, N, k = 1, 5000, 100
+    keys = np.zeros((B, N, 32), dtype=np.float32)
+    keys[0, :, 0] = 1.0                      # every key scores w * q0
+    keys[0, 4000:4010, 0] = 2.0              # ten larger ones
+    ly = synth.Layer("csa", 4, 16, 512, 64, 128, 1, 32, k, idx_fp4=False)
+    desc = desc_for(ly)
+    krows, _ = code_rows(desc, dev(keys), v.F32)
+    qI = np.zeros((1, 1, 32), dtype=np.float32)
+    qI[0, 0, 0] = 1.0
+    idx = torch.zeros(1, k, dtype=torch.int32, device="cuda")
+    ws = v.workspace(desc, 1, N)
+    v.index_topk(desc, qI=dev(qI), w=dev(np.ones((1, 1), np.float32)),
+                 q_pos=dev(np.array([4 * N - 1]), torch.int64), keys=krows, key_rows=N, max_vis=N,
+                 idx_out=idx, ws=ws, B=1)
+    got = idx.cpu().numpy()[0]
+    assert list(got) == list(range(90)) + list(range(4000, 4010))
+
+
+# ------------------------------------------------------------------ MQA
+
+@pytest.mark.parametrize("sparse", [True, False])
+@pytest.mark.parametrize("fp8,H,d,d_rope", [(True, 64, 512, 64), (True, 128, 512, 64),
+                                            (False, 16, 128, 32)])
+def test_mqa_parity(sparse, fp8, H, d, d_rope):
+    v = v4()
+    rng = np.random.default_rng(H + d + sparse)
+    m, B, N, n_win, k = (4 if sparse else 128), 3, 700, 128, 96
+    ly = synth.Layer("csa" if sparse else "hca", m, H, d, d_rope, n_win, 4, 32, k, kv_fp8=fp8,
+                     idx_fp4=False)
+    desc = desc_for(ly)
+    fmt = v.E4M3_BF16ROPE if fp8 else v.F32
+    ents = rng.standard_normal((B, N, d)).astype(np.float32)
+    T = m * N + 50
+    swa_rows = 256
+    swa_vals = rng.standard_normal((B, swa_rows, d)).astype(np.float32)
+    kv, kv_sc = code_rows(desc, dev(ents), fmt, d_rope=d_rope)
+    swa, swa_sc = code_rows(desc, dev(swa_vals), fmt, d_rope=d_rope)
+    positions = np.array([m * N - 1, m * 300 + 1, 5, m * 10, m * N - 2, 200])
+    q_seq = np.array([0, 1, 2, 2, 1, 0], dtype=np.int32)
+    nq = len(positions)
+    Q = synth.bf16_values(rng.standard_normal((nq, H, d)).astype(np.float32))
+    sink = rng.standard_normal(H).astype(np.float32)
+    idx = np.full((nq, k), -1, dtype=np.int32)
+    for q in range(nq):
+        nv = int(ocomp.n_visible(positions[q], m))
+        sel = np.sort(rng.choice(nv, size=min(k, nv), replace=False)) if nv else np.zeros(0, int)
+        idx[q, : len(sel)] = sel
+    out = torch.zeros(nq, H, d, dtype=torch.float32 if not fp8 else torch.bfloat16, device="cuda")
+    lse = torch.zeros(nq, H, dtype=torch.float32, device="cuda")
+    ws = v.workspace(desc, nq, N)
+    kw = dict(Q=dev(Q, torch.bfloat16), q_pos=dev(positions, torch.int64),
+              q_seq=dev(q_seq, torch.int32), B=B, kv=kv, kv_scale=kv_sc, kv_rows=N, swa=swa,
+              swa_scale=swa_sc, swa_rows=swa_rows, out=out, ws=ws, sink=dev(sink), lse=lse)
+    if sparse:
+        v.sparse_mqa(desc, idx=dev(idx, torch.int32), **kw)
+    else:
+        v.dense_mqa(desc, max_vis=N, **kw)
+    torch.cuda.synchronize()
+    assert v.device_status(ws) == 0
+    g_out, g_lse = out.float().cpu().numpy(), lse.cpu().numpy()
+    if fp8:
+        e_val = codecs.dequantize_kv(*codecs.quantize_kv(ents.astype(np.float64), 64))
+        s_val = codecs.dequantize_kv(*codecs.quantize_kv(swa_vals.astype(np.float64), 64))
+    else:
+        e_val, s_val = ents.astype(np.float64), swa_vals.astype(np.float64)
+    for q in range(nq):
+        p, b = int(positions[q]), int(q_seq[q])
+        nv = int(ocomp.n_visible(p, m))
+        rows = idx[q][idx[q] >= 0] if sparse else np.arange(nv)
+        toks = omqa.window_tokens(p, n_win)
+        keys = np.concatenate([e_val[b, rows], s_val[b, toks % swa_rows]], 0)
+        qq = omqa.prepare_query(Q[q], p, d_rope, 160000.0, fp8)
+        o, l = omqa.attend(qq, keys, 1 / np.sqrt(d), sink)
+        o = omqa.finish_output(o, p, d_rope, 160000.0)
+        if fp8:
+            assert r16(g_out[q], o) <= R16_TOL, q
+        else:
+            assert np.max(np.abs(g_out[q] - o)) <= F32_ABS_TOL, q
+        assert np.max(np.abs(g_lse[q] - l)) <= 1e-3, q
+
+
+def test_mqa_no_sink_and_empty_selection():
+    v = v4()
+    rng = np.random.default_rng(5)
+    ly = synth.Layer("csa", 4, 64, 512, 64, 128, 4, 32, 32)
+    desc = desc_for(ly)
+    ents = rng.standard_normal((1, 50, 512)).astype(np.float32)
+    kv, kv_sc = code_rows(desc, dev(ents), v.E4M3_BF16ROPE)
+    swa, swa_sc = code_rows(desc, dev(ents[:, :128 if 50 > 128 else 50]), v.E4M3_BF16ROPE,
+                            rows=128)
+    Q = synth.bf16_values(rng.standard_normal((1, 64, 512)).astype(np.float32))
+    idx = torch.full((1, 32), -1, dtype=torch.int32, device="cuda")     # nothing selected
+    out = torch.zeros(1, 64, 512, dtype=torch.bfloat16, device="cuda")
+    ws = v.workspace(desc, 1, 50)
+    v.sparse_mqa(desc, Q=dev(Q, torch.bfloat16), q_pos=dev(np.array([40]), torch.int64), kv=kv,
+                 kv_scale=kv_sc, kv_rows=50, swa=swa, swa_scale=swa_sc, swa_rows=128, idx=idx,
+                 out=out, ws=ws, B=1)
+    torch.cuda.synchronize()
+    ev = codecs.dequantize_kv(*codecs.quantize_kv(ents[0].astype(np.float64), 64))
+    qq = omqa.prepare_query(Q[0], 40, 64, 160000.0, True)
+    o, _ = omqa.attend(qq, ev[:41], 1 / np.sqrt(512), None)          # window = tokens 0..40
+    o = omqa.finish_output(o, 40, 64, 160000.0)
+    assert r16(out.float().cpu().numpy()[0], o) <= R16_TOL
+
+
+# ------------------------------------------------------------------ decode steps
+
+def _small(kind, L, B):
+    base = synth.WORKLOADS["csa_flash_128k" if kind == "csa" else "hca_flash_128k"]
+    return synth.scaled(base, B=B, L=L, top_k=64, name=f"small_{kind}")
+
+
+@pytest.mark.parametrize("kind,L", [("csa", 4 * 3000), ("hca", 128 * 40), ("csa", 4 * 1000 + 2),
+                                    ("hca", 128 * 9 + 50)])
+def test_decode_step_small(kind, L):
+    w = _small(kind, L, 3)
+    inp = synth.decode_layer_inputs(w, 0)
+    st = DecodeState(w, 0, inp)
+    st.step()
+    ref = pipeline.decode_layer(inp, w.layers[0], [0, 1, 2])
+    compare_decode(st, ref, [0, 1, 2])
+
+
+def test_decode_is_deterministic_and_batch_invariant():
+    w = _small("csa", 4 * 2000, 3)
+    inp = synth.decode_layer_inputs(w, 0)
+    st = DecodeState(w, 0, inp)
+    st.step()
+    out1, idx1 = st.out.clone(), st.idx.clone()
+    st.step()                       # same step again: the appends rewrite the same rows
+    assert torch.equal(out1, st.out) and torch.equal(idx1, st.idx)
+    # changing another sequence's query leaves sequence 1 bit-identical
+    st.Q[0].neg_()
+    st.qI[2] = st.qI[0]
+    st.step()
+    assert torch.equal(out1[1], st.out[1]) and torch.equal(idx1[1], st.idx[1])
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def test_tiny_csa_fp32_full():
+    """The fp32 CSA layer (L = 8192, 32 queries): projections, pooling of all
+    entries and keys, window KV, indexer + top-k, sparse MQA, all in fp32."""
+    v = v4()
+    w = synth.WORKLOADS["tiny_csa_fp32"]
+    ly = w.layers[0]
+    inp = synth.tiny_inputs(w)
+    ref = pipeline.tiny_layer(inp, w)
+    desc = desc_for(ly)
+    L, c, cI = w.L, ly.d, ly.d_I
+    x = dev(inp["x"])
+    Wcat = dev(np.concatenate([inp["W_kv"], inp["W_z"], inp["W_kvI"], inp["W_zI"]], 1))
+    CZ = torch.empty(L, Wcat.shape[1], dtype=torch.float32, device="cuda")
+    v.project(x, Wcat, CZ)
+    ld = CZ.shape[1]
+    n_ent = L // 4
+    one = lambda val: torch.full((1,), val, dtype=torch.int64, device="cuda")
+    ents = torch.zeros(1, n_ent, 4 * c, dtype=torch.uint8, device="cuda")
+    v.compress(desc, m=4, overlap=True, c=c, Ca=CZ[:, :c], Za=CZ[:, c:2 * c], Cb=CZ[:, :c],
+               Zb=CZ[:, c:2 * c], in_rows=L, in_seq_stride=L * ld, in_row_stride=ld,
+               bias=dev(inp["bias"]), seq_len=one(L), entry_begin=one(0), n_entries=n_ent,
+               out_dtype=v.F32, out=ents, out_rows=n_ent)
+    keys = torch.zeros(1, n_ent, 4 * cI, dtype=torch.uint8, device="cuda")
+    v.compress(desc, m=4, overlap=True, c=cI, Ca=CZ[:, 2 * c:2 * c + cI],
+               Za=CZ[:, 2 * c + cI:2 * c + 2 * cI], Cb=CZ[:, 2 * c:2 * c + cI],
+               Zb=CZ[:, 2 * c + cI:2 * c + 2 * cI], in_rows=L, in_seq_stride=L * ld,
+               in_row_stride=ld, bias=dev(inp["ibias"]), seq_len=one(L), entry_begin=one(0),
+               n_entries=n_ent, out_dtype=v.F32, out=keys, out_rows=n_ent, apply_rmsnorm=False,
+               apply_rope=False)
+    swa = torch.zeros(1, L, 4 * c, dtype=torch.uint8, device="cuda")
+    v.compress(desc, m=1, overlap=False, c=c, Ca=CZ[:, :c], Za=None, in_rows=L,
+               in_seq_stride=L * ld, in_row_stride=ld, seq_len=one(L), entry_begin=one(0),
+               n_entries=L, out_dtype=v.F32, out=swa, out_rows=L)
+    pos = inp["positions"]
+    nq = len(pos)
+    xq = x[torch.from_numpy(pos).cuda()]
+    Wq = dev(np.concatenate([inp["W_dq"], inp["W_w"], inp["W_q"]], 1))
+    QQ = torch.empty(nq, Wq.shape[1], dtype=torch.float32, device="cuda")
+    v.project(xq, Wq, QQ)
+    r = w.low_rank
+    qI = torch.empty(nq, ly.H_I * cI, dtype=torch.float32, device="cuda")
+    v.project(QQ[:, :r], dev(inp["W_uq"]), qI)
+    wh = QQ[:, r:r + ly.H_I].contiguous()
+    Q = QQ[:, r + ly.H_I:].contiguous().reshape(nq, ly.H, c)
+    q_pos = dev(pos, torch.int64)
+    q_seq = torch.zeros(nq, dtype=torch.int32, device="cuda")
+    idx = torch.zeros(nq, ly.top_k, dtype=torch.int32, device="cuda")
+    scores = torch.zeros(nq, n_ent, dtype=torch.float32, device="cuda")
+    ws = v.workspace(desc, nq, n_ent)
+    v.index_topk(desc, qI=qI.reshape(nq, ly.H_I, cI), w=wh, q_pos=q_pos, q_seq=q_seq, B=1,
+                 keys=keys, key_rows=n_ent, max_vis=n_ent, idx_out=idx, scores_out=scores, ws=ws)
+    out = torch.zeros(nq, ly.H, c, dtype=torch.float32, device="cuda")
+    lse = torch.zeros(nq, ly.H, dtype=torch.float32, device="cuda")
+    v.sparse_mqa(desc, Q=Q, q_pos=q_pos, q_seq=q_seq, B=1, kv=ents, kv_rows=n_ent, swa=swa,
+                 swa_rows=L, idx=idx, out=out, ws=ws, sink=dev(inp["sink"]), lse=lse,
+                 q_rmsnorm=True)
+    torch.cuda.synchronize()
+    assert v.device_status(ws) == 0
+    assert np.max(np.abs(ents.cpu().numpy()[0].view(np.float32) - ref["entries"])) <= F32_ABS_TOL
+    assert np.max(np.abs(keys.cpu().numpy()[0].view(np.float32) - ref["keys"])) <= F32_ABS_TOL
+    assert np.max(np.abs(swa.cpu().numpy()[0].view(np.float32) - ref["swa"])) <= F32_ABS_TOL
+    g_idx, g_s, g_o, g_l = (idx.cpu().numpy(), scores.cpu().numpy(), out.cpu().numpy(),
+                            lse.cpu().numpy())
+    for q in range(nq):
+        nv = len(ref["scores"][q])
+        s = ref["scores"][q]
+        assert np.max(np.abs(g_s[q, :nv] - s)) <= 1e-4 * max(1.0, np.max(np.abs(s)))
+        check_topk(g_idx[q], s, nv, ly.top_k)
+        sel_same = np.array_equal(g_idx[q], ref["idx"][q])
+        if sel_same:
+            assert np.max(np.abs(g_o[q] - ref["out"][q])) <= F32_ABS_TOL, q
+        assert np.max(np.abs(g_l[q] - ref["lse"][q])) <= 1e-3
+
+
+def _full_decode(name, seqs):
+    w = synth.WORKLOADS[name]
+    for li in range(len(w.layers)):
+        inp = synth.decode_layer_inputs(w, li)
+        st = DecodeState(w, li, inp)
+        st.step()
+        ref = pipeline.decode_layer(inp, w.layers[li], seqs)
+        rep = compare_decode(st, ref, seqs)
+        print(name, li, rep)
+        del st
+        torch.cuda.empty_cache()
+
+
+def test_full_hca_flash_128k():
+    _full_decode("hca_flash_128k", [0, 15])
+
+
+def test_full_csa_flash_128k():
+    _full_decode("csa_flash_128k", [0, 31])
+
+
+def test_full_pro_pair_1m():
+    _full_decode("pro_pair_1m", [0, 3])
