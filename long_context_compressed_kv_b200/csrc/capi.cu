@@ -64,7 +64,7 @@ v4attn_status check_desc(const v4attn_layer_desc* d) {
   if (d->kind == V4A_CSA) {
     if (d->idx_dtype != V4A_F32 && d->idx_dtype != V4A_MXFP4) return V4A_ERR_UNSUPPORTED;
     if (d->d_I != 32 && d->d_I != 64 && d->d_I != 128) return V4A_ERR_UNSUPPORTED;
-    if (d->H_I < 1 || d->H_I > 64) return V4A_ERR_UNSUPPORTED;
+    if (d->H_I < 1 || d->H_I > 128) return V4A_ERR_UNSUPPORTED;
     if (d->top_k < 1 || d->top_k > 2048) return V4A_ERR_UNSUPPORTED;
   }
   return V4A_OK;

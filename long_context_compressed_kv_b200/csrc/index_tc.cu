@@ -32,7 +32,9 @@ constexpr int STAGES = 12;
 constexpr int KTILE_BYTES = KT * KROW;  // 8 KB
 constexpr int SF_BYTES = 512;           // 128 rows x 4 scale bytes
 constexpr int MAXQ = 1024;              // queries per launch on this path
-constexpr int NTHREADS = 192;
+constexpr int EPI_GROUPS = 2;           // epilogue warp groups, alternating tiles
+constexpr int NTHREADS = 64 + EPI_GROUPS * 128;
+constexpr int MAX_ACC = 4;              // accumulator stages in TMEM
 
 struct Smem {
   alignas(1024) uint8_t keys[STAGES][KTILE_BYTES];
@@ -40,7 +42,8 @@ struct Smem {
   alignas(128) uint8_t sfa[STAGES][SF_BYTES];
   alignas(128) uint8_t sfb[2][SF_BYTES];
   float w[2][128];
-  uint64_t full[STAGES], empty[STAGES], qfull[2], qempty[2], accfull[2], accempty[2];
+  uint64_t full[STAGES], empty[STAGES], qfull[2], qempty[2], accfull[MAX_ACC],
+      accempty[MAX_ACC], done;
   int tile_prefix[MAXQ + 1];
   uint32_t tmem_base;
   int abort;
@@ -68,6 +71,7 @@ __device__ __forceinline__ void locate(const Smem& s, int n_q, int g, TileIter& 
   t.lt = g - s.tile_prefix[t.q];
 }
 
+template <int N>   // indexer heads = MMA N
 __global__ void __launch_bounds__(NTHREADS, 1)
     index_tc_kernel(IndexParams P, const __grid_constant__ CUtensorMap tm_keys,
                     const __grid_constant__ CUtensorMap tm_q) {
@@ -75,8 +79,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   Smem& s = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int N = P.H_I;                       // MMA N (multiple of 16, <= 128)
-  const uint32_t TM_COLS = 256;
+  constexpr int NACC = (4 * N + 24 <= 512) ? 4 : 2;        // accumulator stages
+  constexpr uint32_t TM_COLS = (NACC * N + 24 <= 256) ? 256 : 512;
+  constexpr bool W_IN_REGS = N <= 64;
 
   if (threadIdx.x == 0) {
     int acc = 0;
@@ -97,15 +102,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     s.abort = 0;
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&s.full[i], 1);
+      mbar_init(&s.full[i], 32);   // one cp.async arrive per producer lane (+ TMA bytes)
       mbar_init(&s.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.qfull[i], 1);
-      mbar_init(&s.qempty[i], 1 + 4);
+      mbar_init(&s.qempty[i], 1 + 4 * EPI_GROUPS);
+    }
+    for (int i = 0; i < MAX_ACC; ++i) {
       mbar_init(&s.accfull[i], 1);
       mbar_init(&s.accempty[i], 4);
     }
+    mbar_init(&s.done, 1);
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(&s.tmem_base, TM_COLS);
@@ -117,8 +125,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int g0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
   const int g1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
   const uint32_t tmem = s.tmem_base;
-  // TMEM columns: acc[a] at a*N; SFA[a] at 2N + 4a; SFB[j] at 2N + 8 + 4j
-  const uint32_t col_sfa = 2 * N, col_sfb = 2 * N + 8;
+  // TMEM columns: acc[a] at a*N; SFA[a] at NACC*N + 4a; SFB[j] after them
+  const uint32_t col_sfa = NACC * N, col_sfb = NACC * N + 4 * NACC;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -165,16 +173,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_expect_tx(&s.full[st], KTILE_BYTES);
         tma_load_2d(s.keys[st], &tm_keys, &s.full[st], 0, (int)row0);
       }
+      // key scales straight into the tcgen05 scale-factor order, asynchronously
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int r = lane * 4 + k;
         const int64_t gr = row0 + r;
-        const uint32_t word = (gr < total_rows) ? ksf32[gr] : 0u;
-        *reinterpret_cast<uint32_t*>(&s.sfa[st][16 * (r & 31) + 4 * (r >> 5)]) = word;
+        const bool ok = gr < total_rows;
+        cp_async4(&s.sfa[st][16 * (r & 31) + 4 * (r >> 5)], ksf32 + (ok ? gr : 0), ok);
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.full[st]);
+      cp_async_arrive_noinc(&s.full[st]);
     }
     // drain: no load may still be landing in shared memory when the CTA exits
     if (s.abort && lane == 0) {
@@ -201,7 +208,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         if (lane == 0) tmem_cp_32x128b_warpx4(tmem + col_sfb + 4 * j, smem_desc(s.sfb[j], sf_bits));
       }
-      const int st = it % STAGES, a = it & 1, ua = it >> 1;
+      const int st = it % STAGES, a = it % NACC, ua = it / NACC;
       if (!mbar_wait(&s.full[st], (it / STAGES) & 1)) {
         fail(s, P.status);
         break;
@@ -211,6 +218,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       tc_fence_after();
+      fence_proxy_async_smem();   // scales were written by cp.async (generic proxy)
       if (lane == 0) {
         const uint32_t sfa = tmem + col_sfa + 4 * a;
         const uint32_t sfb = tmem + col_sfb + 4 * j;
@@ -228,51 +236,81 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       __syncwarp();
     }
+    // every MMA / copy this warp issued has completed before TMEM is released
+    if (lane == 0) {
+      tc_commit(&s.done);
+      if (!mbar_wait(&s.done, 0)) flag(P.status, ST_TIMEOUT);
+    }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;                  // TMEM lanes 32*quad .. +31
+    // group g handles the tiles with it % 2 == g; within a group, warp w reads
+    // TMEM lanes 32*(w%4) .. +31 (one key row per thread)
+    const int grp = (warp - 2) >> 2;
+    const int quad = warp & 3;
     const int r = quad * 32 + lane;             // key row within the tile
-    // keys beyond the last tile of each query: -inf
     {
+      // keys beyond the last tile of each query: -inf
       const int et = threadIdx.x - 64;
       for (int q = blockIdx.x; q < P.n_q; q += gridDim.x) {
         const int64_t from = (int64_t)(s.tile_prefix[q + 1] - s.tile_prefix[q]) * KT;
-        for (int64_t i = from + et; i < P.max_vis; i += 128)
+        for (int64_t i = from + et; i < P.max_vis; i += EPI_GROUPS * 128)
           P.scores[(int64_t)q * P.scores_ld + i] = -INFINITY;
       }
     }
     TileIter t;
     int it = 0;
+    float wreg[W_IN_REGS ? N : 1];
+    int64_t nv = 0;
     for (int g = g0; g < g1 && !s.abort; ++g, ++it) {
       const int seg_before = t.seg;
       locate(s, P.n_q, g, t);
       const int j = t.seg & 1;
-      if (t.seg != seg_before && !mbar_wait(&s.qfull[j], (t.seg >> 1) & 1)) {
-        fail(s, P.status);
-        break;
-      }
-      const int a = it & 1;
-      if (!mbar_wait(&s.accfull[a], (it >> 1) & 1)) {
-        fail(s, P.status);
-        break;
-      }
-      tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + a * N;
-      float score = 0.f;
-      for (int c = 0; c < N; c += 32) {
-        float v[32];
-        tmem_ld32(taddr + c, v);
-        tmem_ld_wait();
+      if (t.seg != seg_before) {
+        if (!mbar_wait(&s.qfull[j], (t.seg >> 1) & 1)) {
+          fail(s, P.status);
+          break;
+        }
+        if constexpr (W_IN_REGS) {
 #pragma unroll
-        for (int h = 0; h < 32; ++h) score = fmaf(s.w[j][c + h], fmaxf(v[h], 0.f), score);
+          for (int h = 0; h < N; ++h) wreg[h] = s.w[j][h];
+        }
+        nv = min((int64_t)(P.q_pos[t.q] + 1) / P.m, min(P.key_rows, P.max_vis));
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.accempty[a]);
-      const int64_t nv = min((int64_t)(P.q_pos[t.q] + 1) / P.m, min(P.key_rows, P.max_vis));
-      const int64_t i = (int64_t)t.lt * KT + r;
-      if (i < P.max_vis) P.scores[(int64_t)t.q * P.scores_ld + i] = (i < nv) ? score : -INFINITY;
       const bool seg_end = (g + 1 == g1) || (g + 1 >= s.tile_prefix[t.q + 1]);
+      if ((it & 1) == grp) {
+        const int a = it % NACC;
+        if (!mbar_wait(&s.accfull[a], (it / NACC) & 1)) {
+          fail(s, P.status);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + a * N;
+        float s0 = 0.f, s1 = 0.f;
+        constexpr int CH = N <= 64 ? N : 64;      // columns per TMEM round trip
+#pragma unroll
+        for (int c0 = 0; c0 < N; c0 += CH) {
+          uint32_t v[CH];
+#pragma unroll
+          for (int c = 0; c < CH; c += 32) tmem_ld32_nowait(taddr + c0 + c, v + c);
+          tmem_ld_wait();
+          if (c0 + CH == N) {                     // accumulator fully read: release it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.accempty[a]);
+          }
+#pragma unroll
+          for (int h = 0; h < CH; h += 2) {
+            const float w0 = W_IN_REGS ? wreg[(c0 + h) % (W_IN_REGS ? N : 1)] : s.w[j][c0 + h];
+            const float w1 = W_IN_REGS ? wreg[(c0 + h + 1) % (W_IN_REGS ? N : 1)] : s.w[j][c0 + h + 1];
+            s0 = fmaf(w0, fmaxf(__uint_as_float(v[h]), 0.f), s0);
+            s1 = fmaf(w1, fmaxf(__uint_as_float(v[h + 1]), 0.f), s1);
+          }
+        }
+        const float score = s0 + s1;
+        const int64_t i = (int64_t)t.lt * KT + r;
+        if (i < P.max_vis) P.scores[(int64_t)t.q * P.scores_ld + i] = (i < nv) ? score : -INFINITY;
+      }
       if (seg_end) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.qempty[j]);
@@ -322,8 +360,8 @@ bool make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int row_byt
 }
 
 bool index_tc_supported(const IndexParams& P) {
-  return P.idx_dtype == V4A_MXFP4 && P.d_I == 128 && P.H_I % 32 == 0 && P.H_I >= 32 &&
-         P.H_I <= 128 && P.n_q <= MAXQ && encode_fn() != nullptr &&
+  return P.idx_dtype == V4A_MXFP4 && P.d_I == 128 &&
+         (P.H_I == 32 || P.H_I == 64 || P.H_I == 128) && P.n_q <= MAXQ && encode_fn() != nullptr &&
          ((uintptr_t)P.keys & 15) == 0 && ((uintptr_t)P.qI & 15) == 0 &&
          ((uintptr_t)P.keys_sf & 3) == 0 && ((uintptr_t)P.qI_sf & 3) == 0;
 }
@@ -337,15 +375,24 @@ cudaError_t launch_index_tc(const IndexParams& P, cudaStream_t st) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !(configured & (1ull << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaSuccess;
+    e = cudaFuncSetAttribute(index_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(index_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(index_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured |= 1ull << dev;
   }
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = sms;   // persistent: one CTA per SM, contiguous tile ranges
-  index_tc_kernel<<<grid, NTHREADS, smem, st>>>(P, tk, tq);
+  switch (P.H_I) {
+    case 32: index_tc_kernel<32><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
+    case 64: index_tc_kernel<64><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
+    case 128: index_tc_kernel<128><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
+    default: return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

@@ -86,6 +86,17 @@ __global__ void __launch_bounds__(128) index_scores_simt(IndexParams P) {
 cudaError_t launch_index_scores(const IndexParams& P, cudaStream_t st) {
   dim3 grid((unsigned)((P.max_vis + 127) / 128), P.n_q);
   const size_t smem = (size_t)(P.H_I * P.d_I + P.H_I) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaSuccess;
+    switch (P.d_I) {
+      case 64: e = cudaFuncSetAttribute(index_scores_simt<64>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); break;
+      case 128: e = cudaFuncSetAttribute(index_scores_simt<128>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); break;
+      default: break;
+    }
+    if (e != cudaSuccess) return e;
+  }
   switch (P.d_I) {
     case 32: index_scores_simt<32><<<grid, 128, smem, st>>>(P); break;
     case 64: index_scores_simt<64><<<grid, 128, smem, st>>>(P); break;

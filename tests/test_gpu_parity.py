@@ -132,7 +132,8 @@ def test_compress_parity(kind, m, L, fmt, c, ring, in_bf16):
 
 # ------------------------------------------------------------------ indexer + top-k
 
-@pytest.mark.parametrize("fp4,d_I,H_I", [(True, 128, 64), (False, 32, 4), (True, 64, 16)])
+@pytest.mark.parametrize("fp4,d_I,H_I", [(True, 128, 64), (False, 32, 4), (True, 64, 16),
+                                          (True, 128, 128), (True, 128, 32)])
 def test_index_topk_parity(fp4, d_I, H_I):
     v = v4()
     rng = np.random.default_rng(d_I + H_I)
