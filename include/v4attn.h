@@ -250,6 +250,34 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
                             void* ws, size_t ws_bytes, cudaStream_t stream);
 v4attn_status v4attn_project(const v4attn_project_args* args, cudaStream_t stream);
 
+/* ---------------------------------------------------------------- no-allocation variant
+ * The paper has no counterpart to this call; it is a convenience of this
+ * library.  It is v4attn_index_topk without a caller-supplied workspace, for
+ * callers that cannot call cudaMalloc: code that runs inside a host framework
+ * which owns the device allocator and exposes none of it, or a serving loop
+ * that is not allowed to allocate device memory once it has started.
+ *   - The scratch it needs (a status word and the fp32 scores) is one array
+ *     compiled into the library, so every GPU that loads libv4attn holds it
+ *     (about 8.4 MB) until the process exits.
+ *   - Limit: n_q * max(max_vis, 1) <= V4A_NOALLOC_MAX_SCORES and n_q <= 1365;
+ *     a larger call returns V4A_ERR_UNSUPPORTED before launching anything.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - Every call shares the one array, which keeps the last call's contents:
+ *     the call clears the status word and rewrites every score it reads, but
+ *     two calls whose work overlaps on the GPU (unordered streams, or several
+ *     host threads) race on the array; the caller must order them.
+ *   - Device-side check bits land in the array's status word, which the API
+ *     does not expose; out-of-range positions are skipped as in
+ *     v4attn_index_topk.
+ * Arguments and results are those of v4attn_index_topk (scores_out may be
+ * given; idx_out may be NULL only when scores_out is given). */
+#define V4A_NOALLOC_MAX_SCORES 2097152
+v4attn_status v4attn_index_topk_noalloc(const v4attn_layer_desc* desc,
+                                        const v4attn_index_args* args, cudaStream_t stream);
+
 /* Synchronise `stream`, read the status word the kernels left in `ws` and
  * map it: 0 -> V4A_OK, a bounds / argument check -> V4A_ERR_DEVICE_CHECK,
  * a bounded wait that ran out -> V4A_ERR_TIMEOUT.  *bits (if not NULL)

@@ -21,7 +21,8 @@ from ._abi import (BF16, CSA, E4M3_BF16ROPE, F32, HCA, MXFP4, CompressArgs, Deco
 _lib = _abi.load()
 
 __all__ = ["F32", "BF16", "E4M3_BF16ROPE", "MXFP4", "CSA", "HCA", "V4AttnError", "layer_desc",
-           "workspace", "workspace_size", "compress", "index_topk", "sparse_mqa", "dense_mqa",
+           "workspace", "workspace_size", "compress", "index_topk", "index_topk_noalloc",
+           "sparse_mqa", "dense_mqa",
            "decode", "project", "device_status", "build_info", "row_bytes"]
 
 
@@ -112,6 +113,19 @@ def index_topk(desc: LayerDesc, *, qI, w, q_pos, keys, key_rows: int, max_vis: i
                   _p(scores_out))
     _check("v4attn_index_topk", _lib.v4attn_index_topk(ctypes.byref(desc), ctypes.byref(a),
                                                        _p(ws), ws.numel(), _stream(stream)))
+
+
+def index_topk_noalloc(desc: LayerDesc, *, qI, w, q_pos, keys, key_rows: int, max_vis: int,
+                       idx_out, qI_sf=None, keys_sf=None, q_seq=None, B: Optional[int] = None,
+                       scores_out=None, stream=None):
+    """index_topk with the library's built-in scratch instead of a workspace,
+    for callers that cannot allocate device memory (see include/v4attn.h)."""
+    n_q = int(q_pos.numel())
+    a = IndexArgs(n_q, B if B is not None else n_q, _p(qI), _p(qI_sf), _p(w), _p(q_seq),
+                  _p(q_pos), _p(keys), _p(keys_sf), key_rows, max_vis, _p(idx_out),
+                  _p(scores_out))
+    _check("v4attn_index_topk_noalloc",
+           _lib.v4attn_index_topk_noalloc(ctypes.byref(desc), ctypes.byref(a), _stream(stream)))
 
 
 def _mqa(fn, desc, Q, q_pos, kv, kv_rows, swa, swa_rows, out, ws, kv_scale, swa_scale, q_seq, B,

@@ -11,6 +11,7 @@ LIB_PATH = os.path.join(HERE, "libv4attn.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_CHECK = range(7)
 # dtypes
 F32, BF16, E4M3_BF16ROPE, MXFP4 = range(4)
+NOALLOC_MAX_SCORES = 2097152   # V4A_NOALLOC_MAX_SCORES
 # layer kinds
 CSA, HCA = 0, 1
 
@@ -85,6 +86,8 @@ SIGNATURES = {
     "v4attn_decode": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.POINTER(DecodeArgs),
                                      c_ptr, c_sz, c_ptr]),
     "v4attn_project": (ctypes.c_int, [ctypes.POINTER(ProjectArgs), c_ptr]),
+    "v4attn_index_topk_noalloc": (ctypes.c_int, [ctypes.POINTER(LayerDesc),
+                                                 ctypes.POINTER(IndexArgs), c_ptr]),
     "v4attn_device_status": (ctypes.c_int, [c_ptr, c_ptr, ctypes.POINTER(ctypes.c_uint32)]),
     "v4attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "v4attn_build_info": (ctypes.c_char_p, []),
@@ -101,7 +104,7 @@ def load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise RuntimeError(
             f"{LIB_PATH} is missing: build it with "
-            "`python -m long_context_compressed_kv_b200.csrc.build` (there is no CPU fallback)")
+            "`python long_context_compressed_kv_b200/csrc/build.py` (there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)

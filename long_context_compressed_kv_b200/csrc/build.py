@@ -1,6 +1,6 @@
 """Build libv4attn.so (sm_100a) in-tree with nvcc.
 
-    python -m long_context_compressed_kv_b200.csrc.build [--force]
+    python long_context_compressed_kv_b200/csrc/build.py [--force]
 
 Compiles every .cu file of this directory for sm_100a and links them into
 ``long_context_compressed_kv_b200/libv4attn.so``.  Objects go to ``_build/``

@@ -492,3 +492,39 @@ const char* v4attn_status_string(v4attn_status s) {
 const char* v4attn_build_info(void) { return build_info_string(); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation variant
+// Scratch of v4attn_index_topk_noalloc, for callers that cannot allocate
+// device memory: status header, decode region and the fp32 scores of up to
+// V4A_NOALLOC_MAX_SCORES (query, key) pairs.  It is a file-scope device array,
+// so every GPU that loads this library holds it (about 8.4 MB) until the
+// process exits.  In host code the symbol is only a host-side stand-in, never
+// a device address: the device address comes from cudaGetSymbolAddress, looked
+// up once per device with that device current, on the first call there.
+namespace {
+constexpr size_t kNoallocBytes = 256 + 32768 + (size_t)V4A_NOALLOC_MAX_SCORES * sizeof(float);
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocBytes];
+void* g_noalloc_ptr[64] = {nullptr};
+}  // namespace
+
+extern "C" v4attn_status v4attn_index_topk_noalloc(const v4attn_layer_desc* desc,
+                                                   const v4attn_index_args* args,
+                                                   cudaStream_t stream) {
+  v4attn_status s = check_desc(desc);
+  if (s != V4A_OK) return s;
+  if (!args || args->n_q < 1 || args->max_vis < 0) return V4A_ERR_INVALID_ARG;
+  if ((int64_t)args->n_q * std::max<int64_t>(args->max_vis, 1) > V4A_NOALLOC_MAX_SCORES ||
+      body0(args->n_q) + index_need(args->n_q, args->max_vis) > kNoallocBytes)
+    return V4A_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return V4A_ERR_CUDA;
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return V4A_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  void* ws = g_noalloc_ptr[dev];
+  // the status word must start at zero; the scores are fully rewritten by the call
+  if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), stream) != cudaSuccess) return V4A_ERR_CUDA;
+  return run_index_topk(desc, args, ws, kNoallocBytes, stream);
+}
