@@ -28,22 +28,19 @@ size_t body0(int32_t n_q) { return align_up(sizeof(WsHeader)) + dec_bytes(n_q); 
 size_t index_need(int32_t n_q, int64_t max_vis) {
   return align_up((size_t)n_q * (size_t)std::max<int64_t>(max_vis, 1) * sizeof(float));
 }
-int mqa_splits(const v4attn_layer_desc* d, int64_t keys) {
-  const int sk = mqa_split_keys(d);
-  return (int)std::max<int64_t>(1, (keys + sk - 1) / sk);
-}
 size_t mqa_part_o_bytes(const v4attn_layer_desc* d, int32_t n_q, int n_split) {
   return align_up((size_t)n_q * n_split * d->H * d->d * sizeof(float));
 }
-size_t mqa_need(const v4attn_layer_desc* d, int32_t n_q, int64_t keys) {
-  const int S = mqa_splits(d, keys);
+// partials for at most n_main_max entries per query (selected or visible)
+size_t mqa_need(const v4attn_layer_desc* d, int32_t n_q, int64_t n_main_max) {
+  const int S = mqa_num_splits(d, n_main_max);
   return mqa_part_o_bytes(d, n_q, S) + align_up((size_t)n_q * S * d->H * 2 * sizeof(float));
 }
 size_t total_need(const v4attn_layer_desc* d, int32_t n_q, int64_t max_vis) {
-  size_t body = mqa_need(d, n_q, max_vis + d->n_win);
+  size_t body = mqa_need(d, n_q, max_vis);
   if (d->kind == V4A_CSA) {
     body = std::max(body, index_need(n_q, max_vis));
-    body = std::max(body, mqa_need(d, n_q, (int64_t)d->top_k + d->n_win));
+    body = std::max(body, mqa_need(d, n_q, (int64_t)d->top_k));
   }
   return body0(n_q) + body;
 }
@@ -171,7 +168,7 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
   T.max_vis = a->max_vis;
   T.q_pos = a->q_pos;
   T.idx_out = a->idx_out;
-  return cuda_status(launch_topk(T, st));
+  return cuda_status(topk_dispatch(T, st));
 }
 
 v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void* ws,
@@ -189,8 +186,8 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
   if (!aligned16(a->kv) || (a->swa && !aligned16(a->swa)) || !aligned16(a->out))
     return V4A_ERR_INVALID_ARG;
   if (!ws) return V4A_ERR_WORKSPACE;
-  const int64_t keys = (sparse ? (int64_t)a->n_sel : a->max_vis) + d->n_win;
-  if (ws_bytes < body0(a->n_q) + mqa_need(d, a->n_q, keys)) return V4A_ERR_WORKSPACE;
+  const int64_t n_main_max = sparse ? (int64_t)a->n_sel : a->max_vis;
+  if (ws_bytes < body0(a->n_q) + mqa_need(d, a->n_q, n_main_max)) return V4A_ERR_WORKSPACE;
   uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
   MqaParams P;
   P.n_q = a->n_q;
@@ -220,7 +217,7 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
   P.max_vis = sparse ? a->kv_rows : a->max_vis;
   P.sink = a->sink;
   P.split_keys = mqa_split_keys(d);
-  P.n_split = mqa_splits(d, keys);
+  P.n_split = mqa_num_splits(d, n_main_max);
   P.part_o = reinterpret_cast<float*>(w8 + body0(a->n_q));
   P.part_ml = reinterpret_cast<float*>(w8 + body0(a->n_q) + mqa_part_o_bytes(d, a->n_q, P.n_split));
   P.out = a->out;

@@ -5,8 +5,16 @@
 namespace v4a {
 
 int mqa_split_keys(const v4attn_layer_desc* d) {
-  (void)d;
+  if (d->kv_dtype == V4A_E4M3_BF16ROPE && d->d == 512)      // tensor-core kernel
+    return d->kind == V4A_CSA ? 128 : 256;
   return kSimtSplitKeys;
+}
+
+int mqa_num_splits(const v4attn_layer_desc* d, int64_t n_main_max) {
+  const int64_t pad = 64;
+  const int64_t keys = (n_main_max + pad - 1) / pad * pad + (d->n_win + pad - 1) / pad * pad;
+  const int sk = mqa_split_keys(d);
+  return (int)std::max<int64_t>(1, (keys + sk - 1) / sk);
 }
 
 cudaError_t index_scores_dispatch(const IndexParams& P, cudaStream_t st) {
@@ -14,14 +22,21 @@ cudaError_t index_scores_dispatch(const IndexParams& P, cudaStream_t st) {
   return launch_index_scores(P, st);
 }
 
-cudaError_t mqa_dispatch(const MqaParams& P, cudaStream_t st) { return launch_mqa_simt(P, st); }
+cudaError_t topk_dispatch(const TopkParams& P, cudaStream_t st) {
+  if (topk_cluster_supported(P)) return launch_topk_cluster(P, st);
+  return launch_topk(P, st);
+}
+
+cudaError_t mqa_dispatch(const MqaParams& P, cudaStream_t st) {
+  return launch_mqa_simt(P, st);
+}
 
 cudaError_t project_dispatch(const ProjectParams& P, cudaStream_t st) {
   return launch_project(P, st);
 }
 
 const char* build_info_string() {
-  return "v4attn sm_100a: compress(simt) index(tcgen05 mxf4 | simt) topk(radix) mqa(simt) project(simt)";
+  return "v4attn sm_100a: compress(simt) index(tcgen05 mxf4 | simt) topk(cluster radix | radix) mqa(simt) project(simt)";
 }
 
 }  // namespace v4a

@@ -39,9 +39,11 @@ constexpr int MAX_ACC = 4;              // accumulator stages in TMEM
 struct Smem {
   alignas(1024) uint8_t keys[STAGES][KTILE_BYTES];
   alignas(1024) uint8_t q[2][128 * KROW];
-  alignas(128) uint8_t sfa[STAGES][SF_BYTES];
+  alignas(128) uint8_t sfa[STAGES][SF_BYTES];      // scale-factor order (tcgen05.cp source)
+  alignas(128) uint32_t sfa_raw[STAGES][KT];        // key scales as loaded (row-major)
   alignas(128) uint8_t sfb[2][SF_BYTES];
-  float w[2][128];
+  alignas(128) uint32_t sfb_raw[2][128];
+  alignas(16) float w[2][128];
   uint64_t full[STAGES], empty[STAGES], qfull[2], qempty[2], accfull[MAX_ACC],
       accempty[MAX_ACC], done;
   int tile_prefix[MAXQ + 1];
@@ -83,26 +85,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   constexpr uint32_t TM_COLS = (NACC * N + 24 <= 256) ? 256 : 512;
   constexpr bool W_IN_REGS = N <= 64;
 
+  // tiles per query, loaded in parallel, then a serial prefix over shared memory
+  for (int q = threadIdx.x; q < P.n_q; q += NTHREADS) {
+    int64_t nv = (P.q_pos[q] + 1) / P.m;
+    const int b = P.q_seq ? P.q_seq[q] : q;
+    if (b < 0 || b >= P.B) {
+      flag(P.status, ST_BAD_SEQ);
+      nv = 0;
+    }
+    if (nv > P.key_rows || nv > P.max_vis) {
+      flag(P.status, ST_BAD_POSITION);
+      nv = min(P.key_rows, P.max_vis);
+    }
+    s.tile_prefix[q + 1] = (int)((nv + KT - 1) / KT);
+  }
+  __syncthreads();
   if (threadIdx.x == 0) {
     int acc = 0;
     s.tile_prefix[0] = 0;
     for (int q = 0; q < P.n_q; ++q) {
-      int64_t nv = (P.q_pos[q] + 1) / P.m;
-      const int b = P.q_seq ? P.q_seq[q] : q;
-      if (b < 0 || b >= P.B) {
-        flag(P.status, ST_BAD_SEQ);
-        nv = 0;
-      }
-      if (nv > P.key_rows || nv > P.max_vis) {
-        flag(P.status, ST_BAD_POSITION);
-        nv = min(P.key_rows, P.max_vis);
-      }
-      acc += (int)((nv + KT - 1) / KT);
+      acc += s.tile_prefix[q + 1];
       s.tile_prefix[q + 1] = acc;
     }
     s.abort = 0;
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&s.full[i], 32);   // one cp.async arrive per producer lane (+ TMA bytes)
+      mbar_init(&s.full[i], 1);    // the producer lane's arrive + TMA / bulk bytes
       mbar_init(&s.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -149,19 +156,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           break;
         }
         if (lane == 0) {
-          mbar_expect_tx(&s.qfull[j], (uint32_t)(N * KROW));
+          // query codes (TMA), query scales and head weights (bulk copies)
+          mbar_arrive_expect_tx(&s.qfull[j], (uint32_t)(N * KROW + 2 * N * 4));
           tma_load_2d(s.q[j], &tm_q, &s.qfull[j], 0, t.q * P.H_I);
+          bulk_load(s.sfb_raw[j], reinterpret_cast<const uint32_t*>(P.qI_sf) + (int64_t)t.q * P.H_I,
+                    N * 4, &s.qfull[j]);
+          bulk_load(s.w[j], P.w + (int64_t)t.q * P.H_I, N * 4, &s.qfull[j]);
         }
-        // query scales in the tcgen05 scale-factor order, head weights
-        for (int h = lane; h < 128; h += 32) {
-          uint32_t word = 0;
-          if (h < N) word = reinterpret_cast<const uint32_t*>(P.qI_sf)[(int64_t)t.q * P.H_I + h];
-          *reinterpret_cast<uint32_t*>(&s.sfb[j][16 * (h & 31) + 4 * (h >> 5)]) = word;
-          s.w[j][h] = (h < N) ? P.w[(int64_t)t.q * P.H_I + h] : 0.f;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.qfull[j]);
       }
       const int st = it % STAGES, u = it / STAGES;
       if (u >= 1 && !mbar_wait(&s.empty[st], (u - 1) & 1)) {
@@ -170,18 +171,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       const int64_t row0 = (int64_t)b * P.key_rows + (int64_t)t.lt * KT;
       if (lane == 0) {
-        mbar_expect_tx(&s.full[st], KTILE_BYTES);
+        // key codes (TMA tile) + their scales (bulk copy of the in-range rows,
+        // 4 at a time; a ragged end of the key array goes by 4-byte cp.async)
+        const int64_t rows_left = total_rows - row0;
+        const int nrow = (int)(rows_left < KT ? rows_left : KT);
+        const int nbulk = nrow & ~3;
+        mbar_expect_tx(&s.full[st], KTILE_BYTES + nbulk * 4);
         tma_load_2d(s.keys[st], &tm_keys, &s.full[st], 0, (int)row0);
+        if (nbulk) bulk_load(s.sfa_raw[st], ksf32 + row0, nbulk * 4, &s.full[st]);
+        for (int r = nbulk; r < nrow; ++r) cp_async4(&s.sfa_raw[st][r], ksf32 + row0 + r, true);
+        cp_async_arrive_noinc(&s.full[st]);
       }
-      // key scales straight into the tcgen05 scale-factor order, asynchronously
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int r = lane * 4 + k;
-        const int64_t gr = row0 + r;
-        const bool ok = gr < total_rows;
-        cp_async4(&s.sfa[st][16 * (r & 31) + 4 * (r >> 5)], ksf32 + (ok ? gr : 0), ok);
-      }
-      cp_async_arrive_noinc(&s.full[st]);
     }
     // drain: no load may still be landing in shared memory when the CTA exits
     if (s.abort && lane == 0) {
@@ -205,6 +205,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           fail(s, P.status);
           break;
         }
+        // query scales into the tcgen05 scale-factor order (rows >= N zero)
+        for (int h = lane; h < 128; h += 32)
+          *reinterpret_cast<uint32_t*>(&s.sfb[j][16 * (h & 31) + 4 * (h >> 5)]) =
+              (h < N) ? s.sfb_raw[j][h] : 0u;
+        fence_proxy_async_smem();
+        __syncwarp();
         tc_fence_after();
         if (lane == 0) tmem_cp_32x128b_warpx4(tmem + col_sfb + 4 * j, smem_desc(s.sfb[j], sf_bits));
       }
@@ -217,8 +223,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fail(s, P.status);
         break;
       }
+      // key scales into the tcgen05 scale-factor order (row r -> lane r%32, column r/32)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int r = k * 32 + lane;
+        *reinterpret_cast<uint32_t*>(&s.sfa[st][16 * lane + 4 * k]) = s.sfa_raw[st][r];
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
       tc_fence_after();
-      fence_proxy_async_smem();   // scales were written by cp.async (generic proxy)
       if (lane == 0) {
         const uint32_t sfa = tmem + col_sfa + 4 * a;
         const uint32_t sfb = tmem + col_sfb + 4 * j;
@@ -359,11 +372,34 @@ bool make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int row_byt
          CUDA_SUCCESS;
 }
 
+// 2-D uint8 tensor map over rows of `row_bytes`: box of `box_bytes` x `box_rows`
+// starting at any 16-byte-aligned column, with a 32/64/128-byte swizzle.
+bool make_rows_map_sw(CUtensorMap* map, const void* base, int64_t rows, int row_bytes,
+                      int box_bytes, int box_rows, int swizzle_bytes) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || rows < 1 || rows > (1ll << 31) || (row_bytes & 15)) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool index_tc_supported(const IndexParams& P) {
+  // the scale and weight rows are moved by 1-D bulk copies: 16-byte aligned
+  // sources, i.e. 16-byte aligned bases and a key row count divisible by 4
   return P.idx_dtype == V4A_MXFP4 && P.d_I == 128 &&
-         (P.H_I == 32 || P.H_I == 64 || P.H_I == 128) && P.n_q <= MAXQ && encode_fn() != nullptr &&
+         (P.H_I == 32 || P.H_I == 64 || P.H_I == 128) && P.n_q <= MAXQ &&
+         encode_fn() != nullptr && P.key_rows % 4 == 0 &&
          ((uintptr_t)P.keys & 15) == 0 && ((uintptr_t)P.qI & 15) == 0 &&
-         ((uintptr_t)P.keys_sf & 3) == 0 && ((uintptr_t)P.qI_sf & 3) == 0;
+         ((uintptr_t)P.keys_sf & 15) == 0 && ((uintptr_t)P.qI_sf & 15) == 0 &&
+         ((uintptr_t)P.w & 15) == 0;
 }
 
 cudaError_t launch_index_tc(const IndexParams& P, cudaStream_t st) {

@@ -1,0 +1,616 @@
+// Shared-KV MQA on the 5th-generation tensor cores (tcgen05), decode form:
+// one query's H heads against a chunk of selected (CSA) or visible (HCA)
+// compressed entries and its window tokens, split-K partials out.
+//
+// Method: "DeepSeek-V4 深读" (ricardokevins.github.io), model-spec table (64 /
+// 128 query heads of dim 512 over one shared KV head) and section
+// "其他稳定性细节" (448 FP8 + 64 BF16 RoPE dims, sink, inverse RoPE on the
+// output, which the combine applies); "拆解 DeepSeekv4", section "细节".
+//
+// Layout of the work.  A CTA owns (query, key chunk of split_keys keys, half
+// of the 512 output dims).  Output dims are split because fp32 O for 128
+// heads x 512 dims is all of TMEM (512 columns x 128 lanes): each CTA keeps
+// O[128 x 256] in TMEM columns 256..511 and S for two 64-key tiles in
+// columns 0..255, and recomputes S = Q K^T (the two halves of a chunk run on
+// neighbouring CTAs, so the second read of the chunk's rows comes from L2).
+//
+// Per 64-key tile:
+//   S_nope = Q_nope(E4M3) . K_nope(E4M3)^T   14 x tcgen05.mma kind::f8f6f4, K=32
+//   S_rope = Q_rope(BF16) . K_rope(BF16)^T    4 x tcgen05.mma kind::f16,   K=16
+//   s_j    = scale * (q_scale * k_scale_j * S_nope + S_rope)
+//   P'_j   = 2^8 exp2(s_j log2e + log2 k_scale_j - M_u)     (E4M3 hi + lo parts)
+//   P_j    = exp2(s_j log2e - M_s)                          (BF16, RoPE dims)
+//   O_nope += P'_hi V_nope + P'_lo V_nope                    kind::f8f6f4, V MN-major
+//   O_rope += P V_rope                                       kind::f16,    V MN-major
+// The entry scale k_scale_j of the FP8 dims is folded into P', which keeps its
+// own running maximum M_u so that P' never exceeds E4M3's range; O is
+// rescaled in TMEM only when a running maximum grows.  The same shared-memory
+// tile serves as the K-major B operand of Q K^T and the MN-major B operand of
+// P V.  Rows arrive by TMA: tile mode for contiguous HCA entries, tile::gather4
+// (4 rows per instruction, box one row high) for selected entries and window
+// tokens.  Roles: warp 0 loads, warp 1 issues MMAs (one lane), warps 2..5 do
+// the query preparation, the softmax and the epilogue (one head row each).
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+#include "tc_kernels.h"
+
+namespace v4a {
+
+namespace {
+
+constexpr int NK = 64;          // keys per tile
+constexpr int KST = 3;          // tile stages in flight
+constexpr int NTHR = 192;
+constexpr int ROWB = 576;       // stored row: 448 E4M3 + 64 bf16
+constexpr int SKMAX = 512;      // keys per split, at most
+constexpr int TILE_BYTES = NK * (4 * 128 + 64);
+
+struct Smem {
+  alignas(1024) uint8_t qn[3][128 * 128];     // Q nope bytes 0..383, K-major SW128
+  alignas(1024) uint8_t qn3[128 * 64];        // Q nope bytes 384..447, K-major SW64
+  alignas(1024) uint8_t qr[128 * 128];        // Q rope (bf16), K-major SW128
+  alignas(1024) uint8_t kv[KST][4][NK * 128]; // nope blocks 0..2 and the rope block, SW128
+  alignas(1024) uint8_t kv3[KST][NK * 64];    // nope bytes 384..447, SW64
+  alignas(1024) uint8_t p_hi[128 * 64];       // P' high part, E4M3, K-major SW64
+  alignas(1024) uint8_t p_lo[128 * 64];       // P' low part
+  alignas(1024) uint8_t p_bf[128 * 128];      // P for the RoPE dims, bf16, K-major SW128
+  float kscale[KST][NK];
+  int idx[SKMAX];
+  float cs[32], sn[32];
+  uint64_t full[KST], empty[KST], sfull[2], sfree[2], pfull, pempty, qready, ofinal, done;
+  uint32_t tmem_base;
+};
+
+struct Maps {
+  CUtensorMap kv128, kv64;      // tile mode, boxes {128 B | 64 B} x NK rows
+  CUtensorMap kvg128, kvg64;    // gather4 over entry rows, boxes one row high
+  CUtensorMap swg128, swg64;    // gather4 over window rows
+};
+
+__device__ __forceinline__ void gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                        int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// byte offset of (row, byte c) in a K-major tile of 128-byte rows, 128B swizzle
+__device__ __forceinline__ int sw128(int row, int c) {
+  return (row >> 3) * 1024 + (row & 7) * 128 + ((((c >> 4) ^ (row & 7)) & 7) << 4) + (c & 15);
+}
+// ... of 64-byte rows, 64B swizzle
+__device__ __forceinline__ int sw64(int row, int c) {
+  return (row >> 3) * 512 + (row & 7) * 64 + ((((c >> 4) ^ ((row & 7) >> 1)) & 3) << 4) + (c & 15);
+}
+
+struct Geo {
+  int b;
+  int64_t p, n_vis;
+  int n_main, n_swa, nmp, total, s0, T;
+};
+
+__device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
+  Geo g;
+  g.b = P.q_seq ? P.q_seq[q] : q;
+  g.p = P.q_pos[q];
+  g.n_vis = (g.p + 1) / P.m;
+  if (g.b < 0 || g.b >= P.B) {
+    if (threadIdx.x == 0) flag(P.status, ST_BAD_SEQ);
+    g.b = 0;
+    g.n_vis = 0;
+    g.p = -1;
+  }
+  if (g.n_vis > P.kv_rows) {
+    if (threadIdx.x == 0) flag(P.status, ST_BAD_POSITION);
+    g.n_vis = P.kv_rows;
+  }
+  int64_t nm = P.idx ? (int64_t)P.n_sel : g.n_vis;
+  if (!P.idx && nm > P.max_vis) {
+    if (threadIdx.x == 0) flag(P.status, ST_BAD_POSITION);
+    nm = P.max_vis;
+  }
+  g.n_main = (int)nm;
+  g.n_swa = (int)min((int64_t)P.n_win, g.p + 1);
+  if (g.n_swa < 0) g.n_swa = 0;
+  g.nmp = (g.n_main + NK - 1) / NK * NK;
+  g.total = g.nmp + (g.n_swa + NK - 1) / NK * NK;
+  g.s0 = split * P.split_keys;
+  const int len = min(P.split_keys, g.total - g.s0);
+  g.T = len > 0 ? len / NK : 0;
+  return g;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(NTHR, 1)
+    mqa_tc_kernel(MqaParams P, const __grid_constant__ Maps maps) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int dh = blockIdx.x & 1;
+  const int rest = blockIdx.x >> 1;
+  const int split = rest % P.n_split, q = rest / P.n_split;
+  const Geo g = geometry(P, q, split);
+  const int64_t pbase = ((int64_t)q * P.n_split + split) * P.H;
+
+  if (g.T == 0) {                     // nothing in this chunk: an empty partial
+    if (dh == 0)
+      for (int h = threadIdx.x; h < P.H; h += NTHR) {
+        P.part_ml[(pbase + h) * 2] = -INFINITY;
+        P.part_ml[(pbase + h) * 2 + 1] = 0.f;
+      }
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < KST; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.sfull[i], 1);
+      mbar_init(&s.sfree[i], 4);
+    }
+    mbar_init(&s.pfull, 4);
+    mbar_init(&s.pempty, 1);
+    mbar_init(&s.qready, 1);
+    mbar_init(&s.ofinal, 1);
+    mbar_init(&s.done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && P.idx) {
+    // this chunk's selected entries (-1 marks an empty slot)
+    for (int i = lane; i < P.split_keys; i += 32) {
+      const int j = g.s0 + i;
+      s.idx[i] = (j < g.n_main) ? P.idx[(int64_t)q * P.n_sel + j] : -1;
+    }
+  }
+  if (warp == 1) tmem_alloc(&s.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ loads
+    const int64_t kv_base = (int64_t)g.b * P.kv_rows, sw_base = (int64_t)g.b * P.swa_rows;
+    for (int t = 0; t < g.T; ++t) {
+      const int st = t % KST, u = t / KST;
+      if (u >= 1 && !mbar_wait(&s.empty[st], (u - 1) & 1)) {
+        flag(P.status, ST_TIMEOUT);
+        break;
+      }
+      const int vk = g.s0 + t * NK;
+      const bool main_tile = vk < g.nmp;
+      const bool contiguous = main_tile && !P.idx && vk + NK <= g.n_main;
+      if (lane == 0) mbar_expect_tx(&s.full[st], TILE_BYTES);
+      __syncwarp();
+      if (contiguous) {
+        if (lane == 0) {
+          const int y = (int)(kv_base + vk);
+          tma_load_2d(s.kv[st][0], &maps.kv128, &s.full[st], 0, y);
+          tma_load_2d(s.kv[st][1], &maps.kv128, &s.full[st], 128, y);
+          tma_load_2d(s.kv[st][2], &maps.kv128, &s.full[st], 256, y);
+          tma_load_2d(s.kv3[st], &maps.kv64, &s.full[st], 384, y);
+          tma_load_2d(s.kv[st][3], &maps.kv128, &s.full[st], 448, y);
+        }
+      } else if (lane < NK / 4) {
+        int rows[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int r = lane * 4 + k;
+          if (main_tile) {
+            const int jj = vk + r;
+            int e = -1;
+            if (jj < g.n_main) e = P.idx ? s.idx[jj - g.s0] : jj;
+            if (e >= g.n_vis) {
+              flag(P.status, ST_BAD_INDEX);
+              e = -1;
+            }
+            rows[k] = (int)(kv_base + (e >= 0 ? e : 0));
+          } else {
+            const int w = vk - g.nmp + r;
+            const int64_t tok = g.p - g.n_swa + 1 + (w < g.n_swa ? w : 0);
+            rows[k] = (int)(sw_base + (tok >= 0 ? tok % P.swa_rows : 0));
+          }
+        }
+        const CUtensorMap* m128 = main_tile ? &maps.kvg128 : &maps.swg128;
+        const CUtensorMap* m64 = main_tile ? &maps.kvg64 : &maps.swg64;
+        const int o128 = lane * 4 * 128, o64 = lane * 4 * 64;
+        gather4(s.kv[st][0] + o128, m128, &s.full[st], 0, rows[0], rows[1], rows[2], rows[3]);
+        gather4(s.kv[st][1] + o128, m128, &s.full[st], 128, rows[0], rows[1], rows[2], rows[3]);
+        gather4(s.kv[st][2] + o128, m128, &s.full[st], 256, rows[0], rows[1], rows[2], rows[3]);
+        gather4(s.kv3[st] + o64, m64, &s.full[st], 384, rows[0], rows[1], rows[2], rows[3]);
+        gather4(s.kv[st][3] + o128, m128, &s.full[st], 448, rows[0], rows[1], rows[2], rows[3]);
+      }
+      if (lane == 0) {
+        // entry scales, one 4-byte copy per row (window rows from their own array)
+        for (int r = 0; r < NK; ++r) {
+          const float* src;
+          bool ok = true;
+          if (main_tile) {
+            const int jj = vk + r;
+            int e = -1;
+            if (jj < g.n_main) e = P.idx ? s.idx[jj - g.s0] : jj;
+            ok = e >= 0 && e < g.n_vis;
+            src = P.kv_scale + kv_base + (ok ? e : 0);
+          } else {
+            const int w = vk - g.nmp + r;
+            ok = w < g.n_swa;
+            const int64_t tok = g.p - g.n_swa + 1 + (ok ? w : 0);
+            src = P.swa_scale + sw_base + (tok >= 0 ? tok % P.swa_rows : 0);
+          }
+          cp_async4(&s.kscale[st][r], src, ok);
+        }
+        cp_async_arrive_noinc(&s.full[st]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    const uint64_t kq128 = smem_desc_bits(16, 1024, 2);   // K-major, 128B swizzle
+    const uint64_t kq64 = smem_desc_bits(16, 512, 4);     // K-major, 64B swizzle
+    const uint64_t mn128 = smem_desc_bits(NK * 128, 1024, 2);  // MN-major, 128B swizzle
+    const uint64_t mn64 = smem_desc_bits(16, 512, 4);      // MN-major, 64B swizzle
+    const uint32_t id_qk8 = idesc_f(0, 0, 128, NK, false, false);
+    const uint32_t id_qk16 = idesc_f(1, 1, 128, NK, false, false);
+    const uint32_t id_pv256 = idesc_f(0, 0, 128, 256, false, true);
+    const uint32_t id_pv128 = idesc_f(0, 0, 128, 128, false, true);
+    const uint32_t id_pv64 = idesc_f(0, 0, 128, 64, false, true);
+    const uint32_t id_pvr = idesc_f(1, 1, 128, 64, false, true);
+    const uint32_t O = tmem + 256;
+    bool ok = mbar_wait(&s.qready, 0);
+    auto pv = [&](int tt) -> bool {
+      const int st = tt % KST;
+      if (!mbar_wait(&s.pfull, tt & 1)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint64_t ahi = smem_desc(s.p_hi, kq64), alo = smem_desc(s.p_lo, kq64);
+        if (dh == 0) {
+          const uint64_t bv = smem_desc(s.kv[st][0], mn128);
+          for (int ks = 0; ks < 2; ++ks) {
+            const uint64_t bk = bv + (uint64_t)(ks * 32 * 128 >> 4);
+            mma_f8f6f4(O, ahi + 2 * ks, bk, id_pv256, (tt | ks) != 0);
+            mma_f8f6f4(O, alo + 2 * ks, bk, id_pv256, 1);
+          }
+        } else {
+          const uint64_t b2 = smem_desc(s.kv[st][2], mn128);
+          const uint64_t b3 = smem_desc(s.kv3[st], mn64);
+          const uint64_t br = smem_desc(s.kv[st][3], mn128);
+          const uint64_t apb = smem_desc(s.p_bf, kq128);
+          for (int ks = 0; ks < 2; ++ks) {
+            const uint64_t bk2 = b2 + (uint64_t)(ks * 32 * 128 >> 4);
+            const uint64_t bk3 = b3 + (uint64_t)(ks * 32 * 64 >> 4);
+            mma_f8f6f4(O, ahi + 2 * ks, bk2, id_pv128, (tt | ks) != 0);
+            mma_f8f6f4(O, alo + 2 * ks, bk2, id_pv128, 1);
+            mma_f8f6f4(O + 128, ahi + 2 * ks, bk3, id_pv64, (tt | ks) != 0);
+            mma_f8f6f4(O + 128, alo + 2 * ks, bk3, id_pv64, 1);
+          }
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f16(O + 192, apb + 2 * ks, br + (uint64_t)(ks * 16 * 128 >> 4), id_pvr,
+                    (tt | ks) != 0);
+        }
+        tc_commit(&s.pempty);
+        tc_commit(&s.empty[st]);
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int t = 0; t < g.T && ok; ++t) {
+      const int st = t % KST, a = t & 1, ua = t >> 1;
+      if (!mbar_wait(&s.full[st], (t / KST) & 1)) { ok = false; break; }
+      if (ua >= 1 && !mbar_wait(&s.sfree[a], (ua - 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t Sn = tmem + a * 128, Sr = Sn + 64;
+        for (int kb = 0; kb < 3; ++kb) {
+          const uint64_t aq = smem_desc(s.qn[kb], kq128), bk = smem_desc(s.kv[st][kb], kq128);
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f8f6f4(Sn, aq + 2 * ks, bk + 2 * ks, id_qk8, (kb | ks) != 0);
+        }
+        {
+          const uint64_t aq = smem_desc(s.qn3, kq64), bk = smem_desc(s.kv3[st], kq64);
+          for (int ks = 0; ks < 2; ++ks) mma_f8f6f4(Sn, aq + 2 * ks, bk + 2 * ks, id_qk8, 1);
+        }
+        {
+          const uint64_t aq = smem_desc(s.qr, kq128), bk = smem_desc(s.kv[st][3], kq128);
+          for (int ks = 0; ks < 4; ++ks) mma_f16(Sr, aq + 2 * ks, bk + 2 * ks, id_qk16, ks != 0);
+        }
+        tc_commit(&s.sfull[a]);
+      }
+      __syncwarp();
+      if (t >= 1 && !pv(t - 1)) { ok = false; break; }
+    }
+    if (ok) ok = pv(g.T - 1);
+    if (!ok) flag(P.status, ST_TIMEOUT);
+    if (lane == 0) {
+      tc_commit(&s.ofinal);
+      tc_commit(&s.done);
+      if (!mbar_wait(&s.done, 0)) flag(P.status, ST_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ query prep, softmax, epilogue
+    const int ts = threadIdx.x - 64;          // 0..127
+    const int quad = warp & 3;
+    const int h = quad * 32 + lane;           // head row == TMEM lane
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    if (ts < 32 && g.p >= 0) {
+      float c, sn;
+      rope_cs(g.p, ts, P.d_rope, P.theta, c, sn);
+      s.cs[ts] = c;
+      s.sn[ts] = sn;
+    }
+    softmax_bar();
+    float qsc = 1.f;
+    {
+      // Q row h: RoPE at p on dims 448..511, E4M3 coding of dims 0..447 with a
+      // power-of-two scale, written in the swizzled MMA layouts
+      uint32_t wq[256];                       // 512 bf16 as pairs
+      if (h < P.H) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            reinterpret_cast<const __nv_bfloat16*>(P.Q) + ((int64_t)q * P.H + h) * 512);
+#pragma unroll 4
+        for (int i = 0; i < 64; ++i) {
+          const uint4 v = src[i];
+          wq[4 * i] = v.x; wq[4 * i + 1] = v.y; wq[4 * i + 2] = v.z; wq[4 * i + 3] = v.w;
+        }
+      } else {
+#pragma unroll 4
+        for (int i = 0; i < 256; ++i) wq[i] = 0u;
+      }
+      float amax = 0.f;
+#pragma unroll 8
+      for (int i = 0; i < 224; ++i) {
+        const float x0 = bf16_bits_to_f32((uint16_t)(wq[i] & 0xFFFF));
+        const float x1 = bf16_bits_to_f32((uint16_t)(wq[i] >> 16));
+        amax = fmaxf(amax, fmaxf(fabsf(x0), fabsf(x1)));
+      }
+      const int se = e4m3_scale_exp(amax);
+      qsc = exp2i(se);
+      // non-RoPE dims: 16 bytes at a time
+      for (int c16 = 0; c16 < 28; ++c16) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t w0 = wq[c16 * 8 + 2 * k], w1 = wq[c16 * 8 + 2 * k + 1];
+          const uint32_t b0 = f32_to_e4m3(scale_pow2(bf16_bits_to_f32((uint16_t)(w0 & 0xFFFF)), se));
+          const uint32_t b1 = f32_to_e4m3(scale_pow2(bf16_bits_to_f32((uint16_t)(w0 >> 16)), se));
+          const uint32_t b2 = f32_to_e4m3(scale_pow2(bf16_bits_to_f32((uint16_t)(w1 & 0xFFFF)), se));
+          const uint32_t b3 = f32_to_e4m3(scale_pow2(bf16_bits_to_f32((uint16_t)(w1 >> 16)), se));
+          pk[k] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        }
+        const int c = c16 * 16;
+        uint8_t* dst = (c < 384) ? s.qn[c >> 7] + sw128(h, c & 127) : s.qn3 + sw64(h, c - 384);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      // bytes 64..127 of the SW64 block stay unused; RoPE dims (pairs 224..255)
+      for (int c16 = 0; c16 < 8; ++c16) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int pr = c16 * 4 + k;         // RoPE pair index 0..31
+          const uint32_t wv = wq[224 + pr];
+          const float x0 = bf16_bits_to_f32((uint16_t)(wv & 0xFFFF));
+          const float x1 = bf16_bits_to_f32((uint16_t)(wv >> 16));
+          const float cs = s.cs[pr], sn = s.sn[pr];
+          const float r0 = x0 * cs - x1 * sn, r1 = x0 * sn + x1 * cs;
+          pk[k] = (uint32_t)f32_to_bf16_bits(r0) | ((uint32_t)f32_to_bf16_bits(r1) << 16);
+        }
+        *reinterpret_cast<uint4*>(s.qr + sw128(h, c16 * 16)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+    }
+    fence_proxy_async_smem();
+    softmax_bar();
+    if (ts == 0) mbar_arrive(&s.qready);
+
+    const float sl2 = P.scale * 1.4426950408889634f;     // softmax scale x log2(e)
+    float Ms = -INFINITY, Mu = -INFINITY, l = 0.f;
+    bool wrote = false;                                  // O holds a PV result
+    for (int t = 0; t < g.T; ++t) {
+      const int a = t & 1, st = t % KST;
+      if (!mbar_wait(&s.sfull[a], (t >> 1) & 1) || !mbar_wait(&s.full[st], (t / KST) & 1)) {
+        flag(P.status, ST_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      uint32_t sn_[NK], sr_[NK];
+      const uint32_t ta = tmem + lane_off + a * 128;
+      tmem_ld32_nowait(ta, sn_);
+      tmem_ld32_nowait(ta + 32, sn_ + 32);
+      tmem_ld32_nowait(ta + 64, sr_);
+      tmem_ld32_nowait(ta + 96, sr_ + 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.sfree[a]);
+      const int vk = g.s0 + t * NK;
+      const bool main_tile = vk < g.nmp;
+      float s2[NK], u2[NK];
+      float ms = -INFINITY, mu = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < NK; ++j) {
+        bool valid;
+        if (main_tile) {
+          const int jj = vk + j;
+          valid = jj < g.n_main;
+          if (valid && P.idx) {
+            const int e = s.idx[jj - g.s0];
+            valid = e >= 0 && e < g.n_vis;
+          }
+        } else {
+          valid = (vk - g.nmp + j) < g.n_swa;
+        }
+        const float ksc = s.kscale[st][j];
+        const float v = (qsc * ksc * __uint_as_float(sn_[j]) + __uint_as_float(sr_[j])) * sl2;
+        const int ke = (int)((__float_as_uint(ksc) >> 23) & 0xFF) - 127;
+        s2[j] = valid ? v : -INFINITY;
+        u2[j] = valid ? v + (float)ke : -INFINITY;
+        ms = fmaxf(ms, s2[j]);
+        mu = fmaxf(mu, u2[j]);
+      }
+      const float Ms_new = fmaxf(Ms, ms), Mu_new = fmaxf(Mu, mu);
+      const float as = (Ms_new == -INFINITY) ? 1.f : exp2f(Ms - Ms_new);
+      const float au = (Mu_new == -INFINITY) ? 1.f : exp2f(Mu - Mu_new);
+      float lsum = 0.f;
+      uint32_t phi[NK / 4], plo[NK / 4], pbf[NK / 2];
+#pragma unroll
+      for (int j = 0; j < NK; j += 4) {
+        uint32_t hw = 0, lw = 0;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float pj = (s2[j + k] == -INFINITY) ? 0.f : exp2f(s2[j + k] - Ms_new);
+          const float pp = (u2[j + k] == -INFINITY) ? 0.f : exp2f(u2[j + k] - Mu_new + 8.f);
+          lsum += pj;
+          const uint32_t hi = f32_to_e4m3(pp);
+          const uint32_t lo = f32_to_e4m3(pp - e4m3_to_f32((uint8_t)hi));
+          hw |= hi << (8 * k);
+          lw |= lo << (8 * k);
+          if (k & 1) {
+            const float p0 = (s2[j + k - 1] == -INFINITY) ? 0.f : exp2f(s2[j + k - 1] - Ms_new);
+            pbf[(j + k) >> 1] = (uint32_t)f32_to_bf16_bits(p0) | ((uint32_t)f32_to_bf16_bits(pj) << 16);
+          }
+        }
+        phi[j >> 2] = hw;
+        plo[j >> 2] = lw;
+      }
+      l = l * as + lsum;
+      // PV of the previous tile must be done before O or P change
+      if (t >= 1 && !mbar_wait(&s.pempty, (t - 1) & 1)) {
+        flag(P.status, ST_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      if (wrote && (au < 1.f || (dh == 1 && as < 1.f))) {
+        const uint32_t ob = tmem + lane_off + 256;
+        for (int c = 0; c < 256; c += 32) {
+          const float f = (dh == 1 && c >= 192) ? as : au;
+          if (f == 1.f) continue;
+          uint32_t r[32];
+          tmem_ld32_nowait(ob + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * f);
+          tmem_st32(ob + c, r);
+        }
+        tmem_st_wait();
+      }
+      Ms = Ms_new;
+      Mu = Mu_new;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(s.p_hi + sw64(h, 16 * c)) =
+            make_uint4(phi[4 * c], phi[4 * c + 1], phi[4 * c + 2], phi[4 * c + 3]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(s.p_lo + sw64(h, 16 * c)) =
+            make_uint4(plo[4 * c], plo[4 * c + 1], plo[4 * c + 2], plo[4 * c + 3]);
+      if (dh == 1) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(s.p_bf + sw128(h, 16 * c)) =
+              make_uint4(pbf[4 * c], pbf[4 * c + 1], pbf[4 * c + 2], pbf[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.pfull);
+      wrote = true;
+    }
+    // ------------------------------------------------------------ epilogue
+    const bool fin = mbar_wait(&s.ofinal, 0);
+    tc_fence_after();
+    if (!fin) flag(P.status, ST_TIMEOUT);
+    // O_nope is in units of 2^8 exp2(. - Mu); express it in units of exp2(. - Ms)
+    const float fn = (Ms == -INFINITY) ? 0.f : exp2f(Mu - 8.f - Ms);
+    const uint32_t ob = tmem + lane_off + 256;
+    float* dst = P.part_o + (pbase + h) * 512 + dh * 256;
+    for (int c = 0; c < 256; c += 32) {
+      uint32_t r[32];
+      tmem_ld32_nowait(ob + c, r);
+      tmem_ld_wait();
+      const float f = (dh == 1 && c >= 192) ? (Ms == -INFINITY ? 0.f : 1.f) : fn;
+      if (h < P.H && fin) {
+#pragma unroll
+        for (int k = 0; k < 32; k += 4)
+          *reinterpret_cast<float4*>(dst + c + k) =
+              make_float4(__uint_as_float(r[k]) * f, __uint_as_float(r[k + 1]) * f,
+                          __uint_as_float(r[k + 2]) * f, __uint_as_float(r[k + 3]) * f);
+      }
+    }
+    if (dh == 0 && h < P.H) {
+      P.part_ml[(pbase + h) * 2] = (Ms == -INFINITY) ? -INFINITY : Ms * 0.6931471805599453f;
+      P.part_ml[(pbase + h) * 2 + 1] = l;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+bool make_rows_map_sw(CUtensorMap* map, const void* base, int64_t rows, int row_bytes,
+                      int box_bytes, int box_rows, int swizzle_bytes);
+
+bool mqa_tc_supported(const MqaParams& P) {
+  return P.kv_dtype == V4A_E4M3_BF16ROPE && P.d == 512 && P.d_rope == 64 && P.H <= 128 &&
+         P.q_dtype == V4A_BF16 && !P.q_rmsnorm && P.split_keys % NK == 0 &&
+         P.split_keys <= SKMAX && P.n_win <= 1024 && ((uintptr_t)P.kv & 15) == 0 &&
+         (P.n_win == 0 || ((uintptr_t)P.swa & 15) == 0) && ((uintptr_t)P.Q & 15) == 0 &&
+         (int64_t)P.B * P.kv_rows < (1ll << 31) && (int64_t)P.B * P.swa_rows < (1ll << 31);
+}
+
+cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
+  Maps m;
+  const int64_t kv_rows = (int64_t)P.B * P.kv_rows;
+  const int64_t sw_rows = (int64_t)P.B * P.swa_rows;
+  const void* swa = P.swa ? (const void*)P.swa : (const void*)P.kv;
+  const int64_t swr = P.swa ? sw_rows : kv_rows;
+  if (!make_rows_map_sw(&m.kv128, P.kv, kv_rows, ROWB, 128, NK, 128) ||
+      !make_rows_map_sw(&m.kv64, P.kv, kv_rows, ROWB, 64, NK, 64) ||
+      !make_rows_map_sw(&m.kvg128, P.kv, kv_rows, ROWB, 128, 1, 128) ||
+      !make_rows_map_sw(&m.kvg64, P.kv, kv_rows, ROWB, 64, 1, 64) ||
+      !make_rows_map_sw(&m.swg128, swa, swr, ROWB, 128, 1, 128) ||
+      !make_rows_map_sw(&m.swg64, swa, swr, ROWB, 64, 1, 64))
+    return cudaErrorInvalidValue;
+  const size_t smem = sizeof(Smem) + 1024;
+  static unsigned long long configured = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !(configured & (1ull << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured |= 1ull << dev;
+  }
+  const int64_t grid = (int64_t)P.n_q * P.n_split * 2;
+  if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  mqa_tc_kernel<<<(unsigned)grid, NTHR, smem, st>>>(P, m);
+  return cudaGetLastError();
+}
+
+}  // namespace v4a

@@ -66,6 +66,8 @@ class DecodeLayer:
         self.m, self.d, self.d_rope = desc.m, desc.d, desc.d_rope
         self.ring = 2 * desc.m if self.csa else desc.m
         self.n_arr = 4 if self.csa else 2
+        # capacity rounded up to whole 128-row tiles (aligned rows for the TMA paths)
+        kv_rows = (kv_rows + 127) // 128 * 128
         self.kv_rows = kv_rows
         self.swa_rows = swa_rows or max(desc.n_win, 1)
         self.in_dtype = in_dtype

@@ -195,6 +195,37 @@ def test_topk_ties_go_to_lower_index():
     assert list(got) == list(range(90)) + list(range(4000, 4010))
 
 
+@pytest.mark.parametrize("n_vis,k,mode", [(300000, 1024, "ties"), (300000, 777, "random"),
+                                          (262144, 1024, "random"), (70000, 512, "ties"),
+                                          (9, 64, "random"), (4096, 2048, "random")])
+def test_topk_selection_exact(n_vis, k, mode):
+    """The selection alone, fed exact scores through index_topk's F32 path:
+    ties spanning the cluster's slices, more keys than the CTAs keep in shared
+    memory, k equal to the number of keys, fewer keys than k."""
+    v = v4()
+    rng = np.random.default_rng(n_vis + k)
+    d_I = 32
+    keys = np.zeros((1, n_vis, d_I), dtype=np.float32)
+    if mode == "ties":
+        keys[0, :, 0] = rng.integers(0, 3, n_vis).astype(np.float32)    # massive ties
+    else:
+        keys[0, :, 0] = rng.standard_normal(n_vis).astype(np.float32) ** 2
+    ly = synth.Layer("csa", 4, 16, 512, 64, 128, 1, d_I, min(k, 2048), idx_fp4=False)
+    desc = desc_for(ly)
+    krows, _ = code_rows(desc, dev(keys), v.F32)
+    qI = np.zeros((1, 1, d_I), dtype=np.float32)
+    qI[0, 0, 0] = 1.0
+    idx = torch.full((1, k), -3, dtype=torch.int32, device="cuda")
+    ws = v.workspace(desc, 1, n_vis)
+    v.index_topk(desc, qI=dev(qI), w=dev(np.ones((1, 1), np.float32)),
+                 q_pos=dev(np.array([4 * n_vis - 1]), torch.int64), keys=krows, key_rows=n_vis,
+                 max_vis=n_vis, idx_out=idx, ws=ws, B=1)
+    torch.cuda.synchronize()
+    s = keys[0, :, 0].astype(np.float64)
+    want = oidx.topk(s, n_vis, k)
+    assert np.array_equal(idx.cpu().numpy()[0], want)
+
+
 # ------------------------------------------------------------------ MQA
 
 @pytest.mark.parametrize("sparse", [True, False])
