@@ -28,6 +28,7 @@ cudaError_t topk_dispatch(const TopkParams& P, cudaStream_t st) {
 }
 
 cudaError_t mqa_dispatch(const MqaParams& P, cudaStream_t st) {
+  if (mqa_tc_supported(P)) return launch_mqa_tc(P, st);
   return launch_mqa_simt(P, st);
 }
 
@@ -36,7 +37,7 @@ cudaError_t project_dispatch(const ProjectParams& P, cudaStream_t st) {
 }
 
 const char* build_info_string() {
-  return "v4attn sm_100a: compress(simt) index(tcgen05 mxf4 | simt) topk(cluster radix | radix) mqa(simt) project(simt)";
+  return "v4attn sm_100a: compress(simt) index(tcgen05 mxf4 | simt) topk(cluster radix | radix) mqa(tcgen05 fp8/bf16 | simt) project(simt)";
 }
 
 }  // namespace v4a

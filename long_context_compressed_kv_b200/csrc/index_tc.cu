@@ -145,13 +145,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t* ksf32 = reinterpret_cast<const uint32_t*>(P.keys_sf);
     const int64_t total_rows = (int64_t)P.B * P.key_rows;
     int it = 0;
-    for (int g = g0; g < g1 && !s.abort; ++g, ++it) {
+    for (int g = g0; g < g1 && !__any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s.abort)); ++g, ++it) {
       const int seg_before = t.seg;
       locate(s, P.n_q, g, t);
       const int b = P.q_seq ? P.q_seq[t.q] : t.q;
       if (t.seg != seg_before) {
         const int j = t.seg & 1, uq = t.seg >> 1;
-        if (uq >= 1 && !mbar_wait(&s.qempty[j], (uq - 1) & 1)) {
+        if (uq >= 1 && !mbar_wait_warp(&s.qempty[j], (uq - 1) & 1, P.status)) {
           fail(s, P.status);
           break;
         }
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       const int st = it % STAGES, u = it / STAGES;
-      if (u >= 1 && !mbar_wait(&s.empty[st], (u - 1) & 1)) {
+      if (u >= 1 && !mbar_wait_warp(&s.empty[st], (u - 1) & 1, P.status)) {
         fail(s, P.status);
         break;
       }
@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (s.abort && lane == 0) {
       for (int k = 0; k < STAGES && k < it; ++k) {
         const int i2 = it - 1 - k;
-        mbar_wait(&s.full[i2 % STAGES], (i2 / STAGES) & 1);
+        mbar_wait(&s.full[i2 % STAGES], (i2 / STAGES) & 1);   // time bound only
       }
     }
   } else if (warp == 1) {
@@ -196,12 +196,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int it = 0;
     const uint64_t kdesc_bits = smem_desc_bits(16, 8 * KROW, 4);    // K-major, 64B swizzle
     const uint64_t sf_bits = smem_desc_bits(16, 128, 0);            // 32 rows x 16 B
-    for (int g = g0; g < g1 && !s.abort; ++g, ++it) {
+    for (int g = g0; g < g1 && !__any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s.abort)); ++g, ++it) {
       const int seg_before = t.seg;
       locate(s, P.n_q, g, t);
       const int j = t.seg & 1;
       if (t.seg != seg_before) {
-        if (!mbar_wait(&s.qfull[j], (t.seg >> 1) & 1)) {
+        if (!mbar_wait_warp(&s.qfull[j], (t.seg >> 1) & 1, P.status)) {
           fail(s, P.status);
           break;
         }
@@ -215,11 +215,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) tmem_cp_32x128b_warpx4(tmem + col_sfb + 4 * j, smem_desc(s.sfb[j], sf_bits));
       }
       const int st = it % STAGES, a = it % NACC, ua = it / NACC;
-      if (!mbar_wait(&s.full[st], (it / STAGES) & 1)) {
+      if (!mbar_wait_warp(&s.full[st], (it / STAGES) & 1, P.status)) {
         fail(s, P.status);
         break;
       }
-      if (ua >= 1 && !mbar_wait(&s.accempty[a], (ua - 1) & 1)) {
+      if (ua >= 1 && !mbar_wait_warp(&s.accempty[a], (ua - 1) & 1, P.status)) {
         fail(s, P.status);
         break;
       }
@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // every MMA / copy this warp issued has completed before TMEM is released
     if (lane == 0) {
       tc_commit(&s.done);
-      if (!mbar_wait(&s.done, 0)) flag(P.status, ST_TIMEOUT);
+      if (!mbar_wait(&s.done, 0)) flag(P.status, ST_TIMEOUT);   // time bound only
     }
     __syncwarp();
   } else {
@@ -275,12 +275,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int it = 0;
     float wreg[W_IN_REGS ? N : 1];
     int64_t nv = 0;
-    for (int g = g0; g < g1 && !s.abort; ++g, ++it) {
+    for (int g = g0; g < g1 && !__any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s.abort)); ++g, ++it) {
       const int seg_before = t.seg;
       locate(s, P.n_q, g, t);
       const int j = t.seg & 1;
       if (t.seg != seg_before) {
-        if (!mbar_wait(&s.qfull[j], (t.seg >> 1) & 1)) {
+        if (!mbar_wait_warp(&s.qfull[j], (t.seg >> 1) & 1, P.status)) {
           fail(s, P.status);
           break;
         }
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const bool seg_end = (g + 1 == g1) || (g + 1 >= s.tile_prefix[t.q + 1]);
       if ((it & 1) == grp) {
         const int a = it % NACC;
-        if (!mbar_wait(&s.accfull[a], (it / NACC) & 1)) {
+        if (!mbar_wait_warp(&s.accfull[a], (it / NACC) & 1, P.status)) {
           fail(s, P.status);
           break;
         }

@@ -26,9 +26,10 @@
 // own running maximum M_u so that P' never exceeds E4M3's range; O is
 // rescaled in TMEM only when a running maximum grows.  The same shared-memory
 // tile serves as the K-major B operand of Q K^T and the MN-major B operand of
-// P V.  Rows arrive by TMA: tile mode for contiguous HCA entries, tile::gather4
-// (4 rows per instruction, box one row high) for selected entries and window
-// tokens.  Roles: warp 0 loads, warp 1 issues MMAs (one lane), warps 2..5 do
+// P V.  Rows arrive by tile-mode TMA for contiguous HCA entries and by 16-byte
+// cp.async for selected entries and window tokens: a swizzled TMA destination
+// must sit on the swizzle's repeat (1024 bytes for 128-byte rows), which a
+// 4-row gather into the middle of an 8-row swizzle atom does not.  Roles: warp 0 loads, warp 1 issues MMAs (one lane), warps 2..5 do
 // the query preparation, the softmax and the epilogue (one head row each).
 #include "common.cuh"
 #include "kernels.h"
@@ -64,19 +65,8 @@ struct Smem {
 
 struct Maps {
   CUtensorMap kv128, kv64;      // tile mode, boxes {128 B | 64 B} x NK rows
-  CUtensorMap kvg128, kvg64;    // gather4 over entry rows, boxes one row high
-  CUtensorMap swg128, swg64;    // gather4 over window rows
 };
 
-__device__ __forceinline__ void gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
-                                        int r0, int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1),
-      "r"(r2), "r"(r3)
-      : "memory");
-}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
@@ -194,20 +184,48 @@ __global__ void __launch_bounds__(NTHR, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ loads
+    // Contiguous entry tiles go by tile-mode TMA (complete_tx bytes on full[st]).
+    // Selected entries and window tokens go by 16-byte cp.async straight into
+    // the swizzled positions (lanes walk the 36 chunks of each 576-byte row in
+    // order, so a warp's copies are coalesced); so do the 64 entry scales.
+    // Tile t is published once tile t+1 has been issued: wait for all but the
+    // newest cp.async group, fence the generic-proxy writes against the async
+    // proxy that the MMAs read through, then lane 0 arrives on full[st].
     const int64_t kv_base = (int64_t)g.b * P.kv_rows, sw_base = (int64_t)g.b * P.swa_rows;
-    for (int t = 0; t < g.T; ++t) {
+    const uint8_t* kvb = reinterpret_cast<const uint8_t*>(P.kv);
+    const uint8_t* swb = reinterpret_cast<const uint8_t*>(P.swa ? P.swa : P.kv);
+    // global row of key r of tile vk, or -1 when the slot is empty
+    auto row_of = [&](int vk, int r, bool main_tile) -> int64_t {
+      if (main_tile) {
+        const int jj = vk + r;
+        if (jj >= g.n_main) return -1;
+        const int e = P.idx ? s.idx[jj - g.s0] : jj;
+        if (e < 0) return -1;
+        if (e >= g.n_vis) {
+          flag(P.status, ST_BAD_INDEX);
+          return -1;
+        }
+        return kv_base + e;
+      }
+      const int w = vk - g.nmp + r;
+      if (w >= g.n_swa) return -1;
+      const int64_t tok = g.p - g.n_swa + 1 + w;
+      return sw_base + tok % P.swa_rows;
+    };
+    bool issued_ok = true;
+    int t = 0;
+    for (; t < g.T; ++t) {
       const int st = t % KST, u = t / KST;
-      if (u >= 1 && !mbar_wait(&s.empty[st], (u - 1) & 1)) {
-        flag(P.status, ST_TIMEOUT);
+      if (u >= 1 && !mbar_wait_warp(&s.empty[st], (u - 1) & 1, P.status, 0)) {
+        issued_ok = false;
         break;
       }
       const int vk = g.s0 + t * NK;
       const bool main_tile = vk < g.nmp;
       const bool contiguous = main_tile && !P.idx && vk + NK <= g.n_main;
-      if (lane == 0) mbar_expect_tx(&s.full[st], TILE_BYTES);
-      __syncwarp();
       if (contiguous) {
         if (lane == 0) {
+          mbar_expect_tx(&s.full[st], TILE_BYTES);
           const int y = (int)(kv_base + vk);
           tma_load_2d(s.kv[st][0], &maps.kv128, &s.full[st], 0, y);
           tma_load_2d(s.kv[st][1], &maps.kv128, &s.full[st], 128, y);
@@ -215,57 +233,36 @@ __global__ void __launch_bounds__(NTHR, 1)
           tma_load_2d(s.kv3[st], &maps.kv64, &s.full[st], 384, y);
           tma_load_2d(s.kv[st][3], &maps.kv128, &s.full[st], 448, y);
         }
-      } else if (lane < NK / 4) {
-        int rows[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int r = lane * 4 + k;
-          if (main_tile) {
-            const int jj = vk + r;
-            int e = -1;
-            if (jj < g.n_main) e = P.idx ? s.idx[jj - g.s0] : jj;
-            if (e >= g.n_vis) {
-              flag(P.status, ST_BAD_INDEX);
-              e = -1;
-            }
-            rows[k] = (int)(kv_base + (e >= 0 ? e : 0));
-          } else {
-            const int w = vk - g.nmp + r;
-            const int64_t tok = g.p - g.n_swa + 1 + (w < g.n_swa ? w : 0);
-            rows[k] = (int)(sw_base + (tok >= 0 ? tok % P.swa_rows : 0));
-          }
+      } else {
+        for (int i = lane; i < NK * 36; i += 32) {
+          const int r = i / 36, ch = i - r * 36;
+          const int64_t row = row_of(vk, r, main_tile);
+          const uint8_t* src = (main_tile ? kvb : swb) + (row >= 0 ? row : 0) * ROWB + ch * 16;
+          uint8_t* dst;
+          if (ch < 24) dst = s.kv[st][ch >> 3] + sw128(r, (ch & 7) * 16);
+          else if (ch < 28) dst = s.kv3[st] + sw64(r, (ch - 24) * 16);
+          else dst = s.kv[st][3] + sw128(r, (ch - 28) * 16);
+          cp_async16(dst, src, row >= 0);
         }
-        const CUtensorMap* m128 = main_tile ? &maps.kvg128 : &maps.swg128;
-        const CUtensorMap* m64 = main_tile ? &maps.kvg64 : &maps.swg64;
-        const int o128 = lane * 4 * 128, o64 = lane * 4 * 64;
-        gather4(s.kv[st][0] + o128, m128, &s.full[st], 0, rows[0], rows[1], rows[2], rows[3]);
-        gather4(s.kv[st][1] + o128, m128, &s.full[st], 128, rows[0], rows[1], rows[2], rows[3]);
-        gather4(s.kv[st][2] + o128, m128, &s.full[st], 256, rows[0], rows[1], rows[2], rows[3]);
-        gather4(s.kv3[st] + o64, m64, &s.full[st], 384, rows[0], rows[1], rows[2], rows[3]);
-        gather4(s.kv[st][3] + o128, m128, &s.full[st], 448, rows[0], rows[1], rows[2], rows[3]);
       }
-      if (lane == 0) {
-        // entry scales, one 4-byte copy per row (window rows from their own array)
-        for (int r = 0; r < NK; ++r) {
-          const float* src;
-          bool ok = true;
-          if (main_tile) {
-            const int jj = vk + r;
-            int e = -1;
-            if (jj < g.n_main) e = P.idx ? s.idx[jj - g.s0] : jj;
-            ok = e >= 0 && e < g.n_vis;
-            src = P.kv_scale + kv_base + (ok ? e : 0);
-          } else {
-            const int w = vk - g.nmp + r;
-            ok = w < g.n_swa;
-            const int64_t tok = g.p - g.n_swa + 1 + (ok ? w : 0);
-            src = P.swa_scale + sw_base + (tok >= 0 ? tok % P.swa_rows : 0);
-          }
-          cp_async4(&s.kscale[st][r], src, ok);
-        }
-        cp_async_arrive_noinc(&s.full[st]);
+      for (int r = lane; r < NK; r += 32) {
+        const int64_t row = row_of(vk, r, main_tile);
+        const float* src = (main_tile ? P.kv_scale : P.swa_scale) + (row >= 0 ? row : 0);
+        cp_async4(&s.kscale[st][r], src, row >= 0);
+      }
+      cp_async_commit();
+      if (t >= 1) {
+        cp_async_wait<1>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.full[(t - 1) % KST]);
       }
     }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (issued_ok && lane == 0 && t >= 1) mbar_arrive(&s.full[(t - 1) % KST]);
+    if (!issued_ok) flag(P.status, ST_TIMEOUT);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     const uint64_t kq128 = smem_desc_bits(16, 1024, 2);   // K-major, 128B swizzle
@@ -279,10 +276,10 @@ __global__ void __launch_bounds__(NTHR, 1)
     const uint32_t id_pv64 = idesc_f(0, 0, 128, 64, false, true);
     const uint32_t id_pvr = idesc_f(1, 1, 128, 64, false, true);
     const uint32_t O = tmem + 256;
-    bool ok = mbar_wait(&s.qready, 0);
+    bool ok = mbar_wait_warp(&s.qready, 0, P.status, 1);
     auto pv = [&](int tt) -> bool {
       const int st = tt % KST;
-      if (!mbar_wait(&s.pfull, tt & 1)) return false;
+      if (!mbar_wait_warp(&s.pfull, tt & 1, P.status, 2)) return false;
       tc_fence_after();
       if (lane == 0) {
         const uint64_t ahi = smem_desc(s.p_hi, kq64), alo = smem_desc(s.p_lo, kq64);
@@ -318,8 +315,8 @@ __global__ void __launch_bounds__(NTHR, 1)
     };
     for (int t = 0; t < g.T && ok; ++t) {
       const int st = t % KST, a = t & 1, ua = t >> 1;
-      if (!mbar_wait(&s.full[st], (t / KST) & 1)) { ok = false; break; }
-      if (ua >= 1 && !mbar_wait(&s.sfree[a], (ua - 1) & 1)) { ok = false; break; }
+      if (!mbar_wait_warp(&s.full[st], (t / KST) & 1, P.status, 3)) { ok = false; break; }
+      if (ua >= 1 && !mbar_wait_warp(&s.sfree[a], (ua - 1) & 1, P.status, 4)) { ok = false; break; }
       tc_fence_after();
       if (lane == 0) {
         const uint32_t Sn = tmem + a * 128, Sr = Sn + 64;
@@ -346,7 +343,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     if (lane == 0) {
       tc_commit(&s.ofinal);
       tc_commit(&s.done);
-      if (!mbar_wait(&s.done, 0)) flag(P.status, ST_TIMEOUT);
+      if (!mbar_wait(&s.done, 0)) flag(P.status, ST_TIMEOUT | (1u << (16 + 5)));   // time bound only
     }
     __syncwarp();
   } else {
@@ -429,7 +426,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     bool wrote = false;                                  // O holds a PV result
     for (int t = 0; t < g.T; ++t) {
       const int a = t & 1, st = t % KST;
-      if (!mbar_wait(&s.sfull[a], (t >> 1) & 1) || !mbar_wait(&s.full[st], (t / KST) & 1)) {
+      if (!mbar_wait_warp(&s.sfull[a], (t >> 1) & 1, P.status, 6) || !mbar_wait_warp(&s.full[st], (t / KST) & 1, P.status, 7)) {
         flag(P.status, ST_TIMEOUT);
         break;
       }
@@ -496,16 +493,22 @@ __global__ void __launch_bounds__(NTHR, 1)
       }
       l = l * as + lsum;
       // PV of the previous tile must be done before O or P change
-      if (t >= 1 && !mbar_wait(&s.pempty, (t - 1) & 1)) {
+      if (t >= 1 && !mbar_wait_warp(&s.pempty, (t - 1) & 1, P.status, 8)) {
         flag(P.status, ST_TIMEOUT);
         break;
       }
       tc_fence_after();
-      if (wrote && (au < 1.f || (dh == 1 && as < 1.f))) {
+      // Rescale O when a running maximum grew.  tcgen05.ld / st are warp-wide
+      // (.sync.aligned): the decision is taken per warp and every lane takes
+      // part, scaling its own row by its own factor (1 where nothing changed).
+      const bool grow_u = __any_sync(0xffffffffu, wrote && au < 1.f);
+      const bool grow_s = __any_sync(0xffffffffu, wrote && dh == 1 && as < 1.f);
+      if (grow_u || grow_s) {
         const uint32_t ob = tmem + lane_off + 256;
         for (int c = 0; c < 256; c += 32) {
-          const float f = (dh == 1 && c >= 192) ? as : au;
-          if (f == 1.f) continue;
+          const bool rope_cols = dh == 1 && c >= 192;
+          if (rope_cols ? !grow_s : !grow_u) continue;     // uniform across the warp
+          const float f = rope_cols ? as : au;
           uint32_t r[32];
           tmem_ld32_nowait(ob + c, r);
           tmem_ld_wait();
@@ -538,7 +541,7 @@ __global__ void __launch_bounds__(NTHR, 1)
       wrote = true;
     }
     // ------------------------------------------------------------ epilogue
-    const bool fin = mbar_wait(&s.ofinal, 0);
+    const bool fin = mbar_wait_warp(&s.ofinal, 0, P.status, 9);
     tc_fence_after();
     if (!fin) flag(P.status, ST_TIMEOUT);
     // O_nope is in units of 2^8 exp2(. - Mu); express it in units of exp2(. - Ms)
@@ -587,15 +590,8 @@ bool mqa_tc_supported(const MqaParams& P) {
 cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   Maps m;
   const int64_t kv_rows = (int64_t)P.B * P.kv_rows;
-  const int64_t sw_rows = (int64_t)P.B * P.swa_rows;
-  const void* swa = P.swa ? (const void*)P.swa : (const void*)P.kv;
-  const int64_t swr = P.swa ? sw_rows : kv_rows;
   if (!make_rows_map_sw(&m.kv128, P.kv, kv_rows, ROWB, 128, NK, 128) ||
-      !make_rows_map_sw(&m.kv64, P.kv, kv_rows, ROWB, 64, NK, 64) ||
-      !make_rows_map_sw(&m.kvg128, P.kv, kv_rows, ROWB, 128, 1, 128) ||
-      !make_rows_map_sw(&m.kvg64, P.kv, kv_rows, ROWB, 64, 1, 64) ||
-      !make_rows_map_sw(&m.swg128, swa, swr, ROWB, 128, 1, 128) ||
-      !make_rows_map_sw(&m.swg64, swa, swr, ROWB, 64, 1, 64))
+      !make_rows_map_sw(&m.kv64, P.kv, kv_rows, ROWB, 64, NK, 64))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
   static unsigned long long configured = 0;

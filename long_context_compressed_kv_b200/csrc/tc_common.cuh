@@ -19,9 +19,13 @@
 
 namespace v4a {
 
-// Spin limit of every mbarrier wait (~ seconds at worst); on expiry the wait
-// reports failure and the kernel records ST_TIMEOUT and winds down.
-constexpr uint32_t kWaitLimit = 1u << 26;
+// Wall-clock limit of every mbarrier wait.  A failed try_wait may suspend the
+// thread for a while, so the bound is in time (%globaltimer), not iterations.
+// On expiry the wait reports failure; the kernel records ST_TIMEOUT in the
+// status word, and every other wait of the grid gives up as soon as it sees
+// that bit, so a stuck kernel ends within about one limit.
+constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s
+constexpr uint32_t kStatusTimeout = 1u << 8;            // == ST_TIMEOUT
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -61,11 +65,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase with the given parity; false on expiry.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait that, on expiry, also records its call site (bit 16 + site of
+// the status word) so a report says which wait gave up.
+__device__ __forceinline__ bool mbar_wait_at(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                             int site);
+
+// Bounded wait for the phase with the given parity; false on expiry or when
+// `status` (the grid's status word, may be null) already records a timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          const uint32_t* status = nullptr) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (status && (*reinterpret_cast<const volatile uint32_t*>(status) & kStatusTimeout))
+      return false;
+    if (global_ns() - t0 > kWaitNs) return false;
+  }
+}
+__device__ __forceinline__ bool mbar_wait_at(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                             int site) {
+  if (mbar_wait(bar, parity, status)) return true;
+  if (status) atomicOr(status, kStatusTimeout | (1u << (16 + (site & 15))));
   return false;
+}
+
+// The same wait taken by all 32 lanes of a warp, with one answer for all of
+// them: a warp never splits at a timeout, so the warp-wide (.sync.aligned)
+// tcgen05 loads and stores that follow always see every lane.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                               int site = -1) {
+  const bool ok = site >= 0 ? mbar_wait_at(bar, parity, status, site)
+                            : mbar_wait(bar, parity, status);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // 4-byte asynchronous global->shared copy (zero-filled when !valid) and the
@@ -74,6 +112,20 @@ __device__ __forceinline__ void cp_async4(void* dst, const void* src, bool valid
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src),
                "r"(valid ? 4 : 0)
                : "memory");
+}
+// 16-byte copy that bypasses L1 (zero-filled when !valid); both addresses 16-byte aligned.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
