@@ -114,8 +114,9 @@ typedef struct {
   const void* Cb;             /* device, branch-b values (overlap only) */
   const void* Zb;             /* device, branch-b logits (overlap only) */
   int32_t in_dtype;           /* V4A_F32 or V4A_BF16 */
-  int64_t in_seq_stride;      /* elements between sequences */
-  int64_t in_row_stride;      /* elements between token rows (>= c) */
+  int64_t in_seq_stride;      /* elements between sequences (even) */
+  int64_t in_row_stride;      /* elements between token rows (>= c, even); Ca/Za/Cb/Zb aligned
+                                 to 2 elements, bias to 8 bytes, else V4A_ERR_INVALID_ARG */
   int64_t in_rows;            /* rows per sequence in the input arrays */
   const float* bias;          /* device [2m or m][c] position bias; NULL = 0 */
   const int64_t* seq_len;     /* device [B] tokens present (window tokens >= it are left out) */

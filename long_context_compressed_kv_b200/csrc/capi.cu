@@ -32,9 +32,15 @@ size_t mqa_part_o_bytes(const v4attn_layer_desc* d, int32_t n_q, int n_split) {
   return align_up((size_t)n_q * n_split * d->H * d->d * sizeof(float));
 }
 // partials for at most n_main_max entries per query (selected or visible)
+size_t mqa_part_ml_bytes(const v4attn_layer_desc* d, int32_t n_q, int n_split) {
+  return align_up((size_t)n_q * n_split * d->H * 2 * sizeof(float));
+}
+size_t mqa_qbuf_bytes(const v4attn_layer_desc* d, int32_t n_q) {
+  return d->kv_dtype == V4A_E4M3_BF16ROPE ? align_up((size_t)n_q * kMqaQImageStride) : 0;
+}
 size_t mqa_need(const v4attn_layer_desc* d, int32_t n_q, int64_t n_main_max) {
   const int S = mqa_num_splits(d, n_main_max);
-  return mqa_part_o_bytes(d, n_q, S) + align_up((size_t)n_q * S * d->H * 2 * sizeof(float));
+  return mqa_part_o_bytes(d, n_q, S) + mqa_part_ml_bytes(d, n_q, S) + mqa_qbuf_bytes(d, n_q);
 }
 size_t total_need(const v4attn_layer_desc* d, int32_t n_q, int64_t max_vis) {
   size_t body = mqa_need(d, n_q, max_vis);
@@ -84,6 +90,14 @@ v4attn_status run_compress(const v4attn_layer_desc* d, const v4attn_compress_arg
   if (a->overlap && (!a->Cb || !a->Zb)) return V4A_ERR_INVALID_ARG;
   if (a->in_dtype != V4A_F32 && a->in_dtype != V4A_BF16) return V4A_ERR_UNSUPPORTED;
   if (a->in_rows < 1 || a->in_row_stride < a->c || a->out_rows < 1) return V4A_ERR_INVALID_ARG;
+  {
+    // channel pairs are read as one 2-element load: even strides, bases aligned to 2 elements
+    const uintptr_t al = a->in_dtype == V4A_F32 ? 8 : 4;
+    if ((a->in_row_stride | a->in_seq_stride) & 1) return V4A_ERR_INVALID_ARG;
+    for (const void* p : {a->Ca, a->Za, a->Cb, a->Zb})
+      if (p && (reinterpret_cast<uintptr_t>(p) % al)) return V4A_ERR_INVALID_ARG;
+    if (a->bias && (reinterpret_cast<uintptr_t>(a->bias) % 8)) return V4A_ERR_INVALID_ARG;
+  }
   if (a->out_dtype == V4A_E4M3_BF16ROPE) {
     if (a->c != 512 || d->d_rope != 64 || !a->out_scale) return V4A_ERR_UNSUPPORTED;
   } else if (a->out_dtype == V4A_MXFP4) {
@@ -220,6 +234,10 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
   P.n_split = mqa_num_splits(d, n_main_max);
   P.part_o = reinterpret_cast<float*>(w8 + body0(a->n_q));
   P.part_ml = reinterpret_cast<float*>(w8 + body0(a->n_q) + mqa_part_o_bytes(d, a->n_q, P.n_split));
+  P.qbuf = mqa_qbuf_bytes(d, a->n_q)
+               ? w8 + body0(a->n_q) + mqa_part_o_bytes(d, a->n_q, P.n_split) +
+                     mqa_part_ml_bytes(d, a->n_q, P.n_split)
+               : nullptr;
   P.out = a->out;
   P.out_dtype = a->out_dtype;
   P.lse = a->lse;

@@ -8,17 +8,51 @@
 // non-RoPE dims + BF16 RoPE dims); "AI深一度 第15期|DeepSeek V4", section
 // "一、CSA与HCA" (softmax gate with a learnable position bias).
 //
-// One CTA computes one entry of one sequence; thread k owns the channel pair
-// (2k, 2k+1), which is also a RoPE pair.  The softmax over the window is an
-// online (running-max) softmax per channel, so the window is read once; rows
-// are read coalesced (consecutive threads, consecutive channels).  This step
-// moves 2-4 x c values per token and is HBM / latency bound.
+// One CTA computes one entry of one sequence.  Thread k of a row slice owns
+// the channel pair (2k, 2k+1), which is also a RoPE pair; the window's rows
+// are split over up to 4 row slices of the CTA.  Each slice runs an online
+// (running-max) softmax per channel over its rows, 8 rows per batch with the
+// batch's loads issued before its arithmetic, and the slices' (max, sum,
+// weighted sum) triples are merged through shared memory.  Rows are read
+// coalesced (consecutive threads, consecutive channels).  The step moves
+// 2-4 x c values per window token and is HBM / latency bound.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace v4a {
 
-__device__ void compress_entry(const CompressParams& P, int b, int64_t i, float* red) {
+namespace {
+constexpr int kRowBatch = 8;
+
+__device__ __forceinline__ float2 load_pair(const void* p, int dtype, int64_t i) {
+  if (dtype == V4A_F32) return *reinterpret_cast<const float2*>(reinterpret_cast<const float*>(p) + i);
+  const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(
+      reinterpret_cast<const __nv_bfloat16*>(p) + i);
+  return make_float2(__bfloat162float(v.x), __bfloat162float(v.y));
+}
+
+// fold a batch of (value, logit) pairs into the running (max, sum, acc) of one channel
+__device__ __forceinline__ void fold(float& mx, float& sm, float& acc, const float* z,
+                                     const float* v) {
+  float m = mx;
+#pragma unroll
+  for (int u = 0; u < kRowBatch; ++u) m = fmaxf(m, z[u]);
+  if (m == -INFINITY) return;
+  const float al = __expf(mx - m);        // 0 when mx is still -inf
+  acc *= al;
+  sm *= al;
+#pragma unroll
+  for (int u = 0; u < kRowBatch; ++u) {
+    const float e = __expf(z[u] - m);     // 0 for the -inf fillers
+    acc += e * v[u];
+    sm += e;
+  }
+  mx = m;
+}
+}  // namespace
+
+__device__ void compress_entry(const CompressParams& P, int b, int64_t i, float* red, float* mrg,
+                               int PT, int RS) {
   const int64_t L = P.seq_len[b];
   const int m = P.m;
   const int c = P.c;
@@ -26,55 +60,77 @@ __device__ void compress_entry(const CompressParams& P, int b, int64_t i, float*
   if (i < 0 || (int64_t)m * i >= L) return;
   if (P.complete_only && (int64_t)m * (i + 1) > L) return;
 
-  const int k = threadIdx.x;
+  const int k = threadIdx.x % PT, slice = threadIdx.x / PT;
   const int c0 = 2 * k;
   const bool active = c0 < c;
+  const bool owner = active && slice == 0;
   const int R = P.overlap ? 2 * m : m;
+  const int per = (R + RS - 1) / RS;
+  const int r_lo = min(R, slice * per), r_hi = min(R, r_lo + per);
   const int64_t jbase = P.overlap ? (int64_t)m * (i - 1) : (int64_t)m * i;
   const int64_t seq_off = (int64_t)b * P.in_seq_stride;
 
   float mx0 = -INFINITY, mx1 = -INFINITY, s0 = 0.f, s1 = 0.f, a0 = 0.f, a1 = 0.f;
   if (active) {
-    for (int r = 0; r < R; ++r) {
-      const int64_t j = jbase + r;
-      if (j < 0 || j >= L) continue;
-      const bool br_a = !P.overlap || r >= m;
-      const void* Cp = br_a ? P.Ca : P.Cb;
-      const void* Zp = br_a ? P.Za : P.Zb;
-      const int64_t off = seq_off + (j % P.in_rows) * P.in_row_stride + c0;
-      const float v0 = load_in(Cp, P.in_dtype, off);
-      const float v1 = load_in(Cp, P.in_dtype, off + 1);
-      float z0 = Zp ? load_in(Zp, P.in_dtype, off) : 0.f;
-      float z1 = Zp ? load_in(Zp, P.in_dtype, off + 1) : 0.f;
-      if (P.bias) {
-        z0 += P.bias[(int64_t)r * c + c0];
-        z1 += P.bias[(int64_t)r * c + c0 + 1];
+    for (int r0 = r_lo; r0 < r_hi; r0 += kRowBatch) {
+      float v0[kRowBatch], v1[kRowBatch], z0[kRowBatch], z1[kRowBatch];
+#pragma unroll
+      for (int u = 0; u < kRowBatch; ++u) {
+        const int r = r0 + u;
+        const int64_t j = jbase + r;
+        v0[u] = v1[u] = 0.f;
+        z0[u] = z1[u] = -INFINITY;
+        if (r < r_hi && j >= 0 && j < L) {
+          const bool br_a = !P.overlap || r >= m;
+          const void* Cp = br_a ? P.Ca : P.Cb;
+          const void* Zp = br_a ? P.Za : P.Zb;
+          const int64_t off = seq_off + (j % P.in_rows) * P.in_row_stride + c0;
+          const float2 v = load_pair(Cp, P.in_dtype, off);
+          float2 z = Zp ? load_pair(Zp, P.in_dtype, off) : make_float2(0.f, 0.f);
+          if (P.bias) {
+            const float2 bb = *reinterpret_cast<const float2*>(P.bias + (int64_t)r * c + c0);
+            z.x += bb.x;
+            z.y += bb.y;
+          }
+          v0[u] = v.x;
+          v1[u] = v.y;
+          z0[u] = z.x;
+          z1[u] = z.y;
+        }
       }
-      // running-max softmax accumulation (channel 0 of the pair)
-      if (z0 > mx0) {
-        const float al = __expf(mx0 - z0);
-        a0 = a0 * al + v0;
-        s0 = s0 * al + 1.f;
-        mx0 = z0;
-      } else {
-        const float e = __expf(z0 - mx0);
-        a0 += e * v0;
-        s0 += e;
+      fold(mx0, s0, a0, z0, v0);
+      fold(mx1, s1, a1, z1, v1);
+    }
+  }
+  if (RS > 1) {
+    // merge the row slices into slice 0
+    float* my = mrg + (size_t)threadIdx.x * 6;
+    my[0] = mx0; my[1] = s0; my[2] = a0; my[3] = mx1; my[4] = s1; my[5] = a1;
+    __syncthreads();
+    if (slice == 0 && active) {
+      float M0 = -INFINITY, M1 = -INFINITY;
+      for (int q = 0; q < RS; ++q) {
+        M0 = fmaxf(M0, mrg[(size_t)(q * PT + k) * 6]);
+        M1 = fmaxf(M1, mrg[(size_t)(q * PT + k) * 6 + 3]);
       }
-      if (z1 > mx1) {
-        const float al = __expf(mx1 - z1);
-        a1 = a1 * al + v1;
-        s1 = s1 * al + 1.f;
-        mx1 = z1;
-      } else {
-        const float e = __expf(z1 - mx1);
-        a1 += e * v1;
-        s1 += e;
+      s0 = a0 = s1 = a1 = 0.f;
+      for (int q = 0; q < RS; ++q) {
+        const float* o = mrg + (size_t)(q * PT + k) * 6;
+        if (o[0] != -INFINITY) {
+          const float f = __expf(o[0] - M0);
+          s0 += f * o[1];
+          a0 += f * o[2];
+        }
+        if (o[3] != -INFINITY) {
+          const float f = __expf(o[3] - M1);
+          s1 += f * o[4];
+          a1 += f * o[5];
+        }
       }
     }
   }
-  float e0 = active ? a0 / s0 : 0.f;
-  float e1 = active ? a1 / s1 : 0.f;
+  float e0 = owner ? a0 / s0 : 0.f;
+  float e1 = owner ? a1 / s1 : 0.f;
 
   if (P.apply_rmsnorm) {
     const float ss = block_sum(e0 * e0 + e1 * e1, red);
@@ -82,7 +138,7 @@ __device__ void compress_entry(const CompressParams& P, int b, int64_t i, float*
     e0 *= inv;
     e1 *= inv;
   }
-  if (P.apply_rope && active && c0 >= c - P.d_rope) {
+  if (P.apply_rope && owner && c0 >= c - P.d_rope) {
     float cs, sn;
     rope_cs((int64_t)m * i, (c0 - (c - P.d_rope)) / 2, P.d_rope, P.theta, cs, sn);
     const float r0 = e0 * cs - e1 * sn;
@@ -95,13 +151,13 @@ __device__ void compress_entry(const CompressParams& P, int b, int64_t i, float*
   const int64_t rb = row_bytes(P.out_dtype, c, P.d_rope);
   uint8_t* out = reinterpret_cast<uint8_t*>(P.out) + ((int64_t)b * P.out_rows + row) * rb;
   if (P.out_dtype == V4A_F32) {
-    if (active) reinterpret_cast<float2*>(out)[k] = make_float2(e0, e1);
+    if (owner) reinterpret_cast<float2*>(out)[k] = make_float2(e0, e1);
   } else if (P.out_dtype == V4A_E4M3_BF16ROPE) {
     const int dn = c - P.d_rope;
-    const float am = (active && c0 < dn) ? fmaxf(fabsf(e0), fabsf(e1)) : 0.f;
+    const float am = (owner && c0 < dn) ? fmaxf(fabsf(e0), fabsf(e1)) : 0.f;
     const float amax = block_max(am, red);
     const int se = e4m3_scale_exp(amax);
-    if (active) {
+    if (owner) {
       if (c0 < dn) {
         const uint16_t pr = (uint16_t)f32_to_e4m3(scale_pow2(e0, se)) |
                             ((uint16_t)f32_to_e4m3(scale_pow2(e1, se)) << 8);
@@ -114,11 +170,11 @@ __device__ void compress_entry(const CompressParams& P, int b, int64_t i, float*
     if (threadIdx.x == 0)
       reinterpret_cast<float*>(P.out_scale)[(int64_t)b * P.out_rows + row] = exp2i(se);
   } else {  // V4A_MXFP4: 16 threads (32 channels) per scale block
-    float am = active ? fmaxf(fabsf(e0), fabsf(e1)) : 0.f;
+    float am = owner ? fmaxf(fabsf(e0), fabsf(e1)) : 0.f;
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
     const int X = mx_scale_exp(am);
-    if (active) {
+    if (owner) {
       const uint8_t lo = f32_to_e2m1(scale_pow2(e0, X));
       const uint8_t hi = f32_to_e2m1(scale_pow2(e1, X));
       out[k] = (uint8_t)(lo | (hi << 4));
@@ -130,21 +186,27 @@ __device__ void compress_entry(const CompressParams& P, int b, int64_t i, float*
 }
 
 // Grid-stride over the entries of sequence blockIdx.y.
-__global__ void compress_kernel(CompressParams P, int n_entries) {
+__global__ void __launch_bounds__(1024) compress_kernel(CompressParams P, int n_entries, int PT, int RS) {
   __shared__ float red[32];
+  extern __shared__ float mrg[];
   const int b = blockIdx.y;
   const int64_t e0 = P.entry_begin[b];
   for (int e = blockIdx.x; e < n_entries; e += gridDim.x) {
-    compress_entry(P, b, e0 + e, red);
+    compress_entry(P, b, e0 + e, red, mrg, PT, RS);
     __syncthreads();
   }
 }
 
 cudaError_t launch_compress(const CompressParams& P, int B, int n_entries, cudaStream_t st) {
-  int threads = ((P.c / 2 + 31) / 32) * 32;
-  if (threads < 32) threads = 32;
+  int PT = ((P.c / 2 + 31) / 32) * 32;     // threads per row slice
+  if (PT < 32) PT = 32;
+  const int R = P.overlap ? 2 * P.m : P.m;
+  int RS = R / (2 * kRowBatch);            // row slices: at least 2 batches each
+  RS = RS < 1 ? 1 : (RS > 4 ? 4 : RS);
+  while (RS > 1 && PT * RS > 1024) --RS;
+  const size_t smem = RS > 1 ? (size_t)PT * RS * 6 * sizeof(float) : 0;
   dim3 grid(n_entries < 8192 ? n_entries : 8192, B);
-  compress_kernel<<<grid, threads, 0, st>>>(P, n_entries);
+  compress_kernel<<<grid, PT * RS, smem, st>>>(P, n_entries, PT, RS);
   return cudaGetLastError();
 }
 

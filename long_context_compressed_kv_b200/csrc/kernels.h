@@ -46,6 +46,10 @@ struct TopkParams {
   int32_t* idx_out;
 };
 
+// Bytes per query of the tensor-core MQA's coded query image (73728 bytes of
+// swizzled E4M3 / bf16 tiles + 512 bytes of per-head scales, 1024-aligned).
+constexpr int64_t kMqaQImageStride = 74752;
+
 struct MqaParams {
   int n_q, B, H, d, d_rope, n_win, m;
   float theta, scale, eps;
@@ -68,6 +72,7 @@ struct MqaParams {
   int split_keys;       // keys per split
   float* part_o;        // [n_q][n_split][H][d]
   float* part_ml;       // [n_q][n_split][H][2]
+  uint8_t* qbuf;        // tensor-core path: [n_q] coded query images (kMqaQImageStride bytes)
   void* out;
   int out_dtype;
   float* lse;

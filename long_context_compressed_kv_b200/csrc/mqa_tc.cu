@@ -7,30 +7,41 @@
 // "其他稳定性细节" (448 FP8 + 64 BF16 RoPE dims, sink, inverse RoPE on the
 // output, which the combine applies); "拆解 DeepSeekv4", section "细节".
 //
-// Layout of the work.  A CTA owns (query, key chunk of split_keys keys, half
-// of the 512 output dims).  Output dims are split because fp32 O for 128
-// heads x 512 dims is all of TMEM (512 columns x 128 lanes): each CTA keeps
-// O[128 x 256] in TMEM columns 256..511 and S for two 64-key tiles in
-// columns 0..255, and recomputes S = Q K^T (the two halves of a chunk run on
-// neighbouring CTAs, so the second read of the chunk's rows comes from L2).
+// Layout of the work.  A small pre-kernel codes each query once (RoPE at its
+// position on dims 448..511, E4M3 with a power-of-two scale on dims 0..447)
+// straight into the swizzled shared-memory image the MMAs read; every CTA of
+// the query copies that image in with bulk copies.  A CTA owns (query, key
+// chunk of split_keys keys, half of the 512 output dims).  Output dims are
+// split because fp32 O for 128 heads x 512 dims is all of TMEM (512 columns x
+// 128 lanes): each CTA keeps O[128 x 256] in TMEM columns 256..511 and S for
+// two 64-key tiles in columns 0..255, and recomputes S = Q K^T (the two
+// halves of a chunk run on neighbouring CTAs, so the second read of the
+// chunk's rows comes from L2).
 //
 // Per 64-key tile:
 //   S_nope = Q_nope(E4M3) . K_nope(E4M3)^T   14 x tcgen05.mma kind::f8f6f4, K=32
 //   S_rope = Q_rope(BF16) . K_rope(BF16)^T    4 x tcgen05.mma kind::f16,   K=16
-//   s_j    = scale * (q_scale * k_scale_j * S_nope + S_rope)
-//   P'_j   = 2^8 exp2(s_j log2e + log2 k_scale_j - M_u)     (E4M3 hi + lo parts)
-//   P_j    = exp2(s_j log2e - M_s)                          (BF16, RoPE dims)
-//   O_nope += P'_hi V_nope + P'_lo V_nope                    kind::f8f6f4, V MN-major
-//   O_rope += P V_rope                                       kind::f16,    V MN-major
+//   s_j    = scale * (q_scale * k_scale_j * S_nope + S_rope)       (log2 units)
+//   P_j    = exp2(s_j - M_s)                                        (BF16, RoPE dims)
+//   P'_j   = P_j * k_scale_j * 2^(M_s - M_u + 8) = 2^(s_j + log2 k_scale_j - M_u + 8)
+//   O_nope += P'_hi V_nope + P'_lo V_nope     (E4M3 hi + lo parts), kind::f8f6f4, V MN-major
+//   O_rope += P V_rope                                              kind::f16, V MN-major
 // The entry scale k_scale_j of the FP8 dims is folded into P', which keeps its
-// own running maximum M_u so that P' never exceeds E4M3's range; O is
-// rescaled in TMEM only when a running maximum grows.  The same shared-memory
-// tile serves as the K-major B operand of Q K^T and the MN-major B operand of
-// P V.  Rows arrive by tile-mode TMA for contiguous HCA entries and by 16-byte
-// cp.async for selected entries and window tokens: a swizzled TMA destination
-// must sit on the swizzle's repeat (1024 bytes for 128-byte rows), which a
-// 4-row gather into the middle of an 8-row swizzle atom does not.  Roles: warp 0 loads, warp 1 issues MMAs (one lane), warps 2..5 do
-// the query preparation, the softmax and the epilogue (one head row each).
+// own running maximum M_u so that P' never exceeds 2^8 (inside E4M3's range);
+// one exp2 per key serves both.  O is rescaled in TMEM only when a running
+// maximum grows.  The same shared-memory tile serves as the K-major B operand
+// of Q K^T and the MN-major B operand of P V.
+//
+// Rows arrive by tile-mode TMA for contiguous HCA entries and by 16-byte
+// cp.async for selected entries and window tokens (a swizzled TMA destination
+// must sit on the swizzle's 1024-byte repeat, which a 4-row gather into the
+// middle of an 8-row atom does not).  Roles: warp 0 loads, warp 1 issues the
+// MMAs (one lane), warps 2..9 run the softmax and the epilogue: two warps per
+// TMEM lane quarter, one per 32-key half of each tile, exchanging row maxima
+// through shared memory.  Every cross-warp hand-off is an mbarrier with a
+// bounded, warp-uniform wait, so a stalled kernel ends with a status bit.
+#include <cstddef>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -42,26 +53,39 @@ namespace {
 
 constexpr int NK = 64;          // keys per tile
 constexpr int KST = 3;          // tile stages in flight
-constexpr int NTHR = 192;
+constexpr int NSM = 8;          // softmax / epilogue warps
+constexpr int NTHR = 64 + 32 * NSM;
 constexpr int ROWB = 576;       // stored row: 448 E4M3 + 64 bf16
 constexpr int SKMAX = 512;      // keys per split, at most
 constexpr int TILE_BYTES = NK * (4 * 128 + 64);
+// query image: Q nope bytes 0..383 as three K-major SW128 blocks, bytes
+// 384..447 as one K-major SW64 block, the RoPE dims (bf16) as one K-major SW128
+// block, then the per-head E4M3 scale
+constexpr int Q_NOPE3 = 3 * 16384, Q_ROPE = Q_NOPE3 + 8192, QTILE = Q_ROPE + 16384;
+constexpr int QIMG = QTILE + 128 * 4;
+constexpr int QCHUNK = QIMG / 4;
+static_assert(QCHUNK % 16 == 0, "bulk copies move multiples of 16 bytes");
 
 struct Smem {
-  alignas(1024) uint8_t qn[3][128 * 128];     // Q nope bytes 0..383, K-major SW128
-  alignas(1024) uint8_t qn3[128 * 64];        // Q nope bytes 384..447, K-major SW64
-  alignas(1024) uint8_t qr[128 * 128];        // Q rope (bf16), K-major SW128
+  alignas(1024) uint8_t q[QTILE];
+  float qsc[128];                             // contiguous with q: one image
   alignas(1024) uint8_t kv[KST][4][NK * 128]; // nope blocks 0..2 and the rope block, SW128
   alignas(1024) uint8_t kv3[KST][NK * 64];    // nope bytes 384..447, SW64
   alignas(1024) uint8_t p_hi[128 * 64];       // P' high part, E4M3, K-major SW64
   alignas(1024) uint8_t p_lo[128 * 64];       // P' low part
   alignas(1024) uint8_t p_bf[128 * 128];      // P for the RoPE dims, bf16, K-major SW128
   float kscale[KST][NK];
+  uint32_t vmask[KST][2];                     // valid keys of a tile, 32 per word
   int idx[SKMAX];
-  float cs[32], sn[32];
-  uint64_t full[KST], empty[KST], sfull[2], sfree[2], pfull, pempty, qready, ofinal, done;
+  float xmax[2][2][2][128];                   // [tile parity][key half][M_s, M_u][row]
+  float xl[128];                              // the second half's row sums, for the epilogue
+  uint64_t full[KST], empty[KST], sfull[2], sfree[2], xbar[2];
+  uint64_t pfull, pempty, qready, ofinal, done, lbar;
   uint32_t tmem_base;
 };
+
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory per CTA");
+static_assert(offsetof(Smem, qsc) == QTILE, "the query image is one contiguous copy");
 
 struct Maps {
   CUtensorMap kv128, kv64;      // tile mode, boxes {128 B | 64 B} x NK rows
@@ -82,7 +106,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // byte offset of (row, byte c) in a K-major tile of 128-byte rows, 128B swizzle
 __device__ __forceinline__ int sw128(int row, int c) {
@@ -92,6 +115,17 @@ __device__ __forceinline__ int sw128(int row, int c) {
 __device__ __forceinline__ int sw64(int row, int c) {
   return (row >> 3) * 512 + (row & 7) * 64 + ((((c >> 4) ^ ((row & 7) >> 1)) & 3) << 4) + (c & 15);
 }
+
+// two floats -> two E4M3 codes (saturating, round to nearest even), low byte = a
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t c) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)c, __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 struct Geo {
   int b;
@@ -132,6 +166,70 @@ __device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
 
 }  // namespace
 
+// One CTA per query, one thread per head row: the query image of the main kernel.
+__global__ void __launch_bounds__(128) mqa_tc_qprep_kernel(MqaParams P) {
+  __shared__ float cs[32], sn[32];
+  const int q = blockIdx.x, h = threadIdx.x;
+  const int64_t p = P.q_pos[q];
+  if (h < 32) {
+    float c = 1.f, sv = 0.f;
+    if (p >= 0) rope_cs(p, h, 64, P.theta, c, sv);
+    cs[h] = c;
+    sn[h] = sv;
+  }
+  __syncthreads();
+  uint8_t* img = P.qbuf + (int64_t)q * kMqaQImageStride;
+  const bool live = h < P.H;
+  const uint4* src = reinterpret_cast<const uint4*>(
+      reinterpret_cast<const __nv_bfloat16*>(P.Q) + ((int64_t)q * P.H + (live ? h : 0)) * 512);
+  float amax = 0.f;
+  if (live)
+    for (int i = 0; i < 56; ++i) {
+      const uint4 v = src[i];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[k])), fabsf(bf16hi(w[k]))));
+    }
+  const int se = e4m3_scale_exp(amax);
+  // dims 0..447: 16 E4M3 codes per 16-byte chunk
+  for (int c16 = 0; c16 < 28; ++c16) {
+    uint32_t pk[4] = {0u, 0u, 0u, 0u};
+    if (live) {
+      const uint4 a = src[2 * c16], b = src[2 * c16 + 1];
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t lo = e4m3x2(scale_pow2(bf16lo(w[2 * k]), se), scale_pow2(bf16hi(w[2 * k]), se));
+        const uint32_t hi =
+            e4m3x2(scale_pow2(bf16lo(w[2 * k + 1]), se), scale_pow2(bf16hi(w[2 * k + 1]), se));
+        pk[k] = lo | (hi << 16);
+      }
+    }
+    const int c = c16 * 16;
+    uint8_t* dst = (c < 384) ? img + (c >> 7) * 16384 + sw128(h, c & 127)
+                             : img + Q_NOPE3 + sw64(h, c - 384);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+  // dims 448..511: RoPE at the query position, kept in bf16
+  for (int c16 = 0; c16 < 8; ++c16) {
+    uint32_t pk[4] = {0u, 0u, 0u, 0u};
+    if (live) {
+      const uint4 v = src[56 + c16];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int pr = c16 * 4 + k;
+        const float x0 = bf16lo(w[k]), x1 = bf16hi(w[k]);
+        const float r0 = x0 * cs[pr] - x1 * sn[pr], r1 = x0 * sn[pr] + x1 * cs[pr];
+        pk[k] = (uint32_t)f32_to_bf16_bits(r0) | ((uint32_t)f32_to_bf16_bits(r1) << 16);
+      }
+    }
+    *reinterpret_cast<uint4*>(img + Q_ROPE + sw128(h, c16 * 16)) =
+        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+  reinterpret_cast<float*>(img + QTILE)[h] = exp2i(se);
+}
+
 __global__ void __launch_bounds__(NTHR, 1)
     mqa_tc_kernel(MqaParams P, const __grid_constant__ Maps maps) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -160,13 +258,15 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.sfull[i], 1);
-      mbar_init(&s.sfree[i], 4);
+      mbar_init(&s.sfree[i], NSM);
+      mbar_init(&s.xbar[i], NSM);
     }
-    mbar_init(&s.pfull, 4);
+    mbar_init(&s.pfull, NSM);
     mbar_init(&s.pempty, 1);
     mbar_init(&s.qready, 1);
     mbar_init(&s.ofinal, 1);
     mbar_init(&s.done, 1);
+    mbar_init(&s.lbar, NSM / 2);
     fence_mbar_init();
   }
   if (warp == 0 && P.idx) {
@@ -184,16 +284,23 @@ __global__ void __launch_bounds__(NTHR, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ loads
-    // Contiguous entry tiles go by tile-mode TMA (complete_tx bytes on full[st]).
-    // Selected entries and window tokens go by 16-byte cp.async straight into
-    // the swizzled positions (lanes walk the 36 chunks of each 576-byte row in
-    // order, so a warp's copies are coalesced); so do the 64 entry scales.
-    // Tile t is published once tile t+1 has been issued: wait for all but the
-    // newest cp.async group, fence the generic-proxy writes against the async
-    // proxy that the MMAs read through, then lane 0 arrives on full[st].
+    // The query image by four bulk copies on qready.  Contiguous entry tiles
+    // go by tile-mode TMA (complete_tx bytes on full[st]).  Selected entries
+    // and window tokens go by 16-byte cp.async straight into the swizzled
+    // positions (lanes walk the 36 chunks of each 576-byte row in order, so a
+    // warp's copies are coalesced); so do the 64 entry scales.  Tile t is
+    // published once tile t+1 has been issued: wait for all but the newest
+    // cp.async group, fence the generic-proxy writes against the async proxy
+    // that the MMAs read through, then lane 0 arrives on full[st].
+    if (lane == 0) {
+      const uint8_t* qimg = P.qbuf + (int64_t)q * kMqaQImageStride;
+      mbar_arrive_expect_tx(&s.qready, QIMG);
+      for (int k = 0; k < 4; ++k)
+        bulk_load(s.q + k * QCHUNK, qimg + k * QCHUNK, QCHUNK, &s.qready);
+    }
     const int64_t kv_base = (int64_t)g.b * P.kv_rows, sw_base = (int64_t)g.b * P.swa_rows;
-    const uint8_t* kvb = reinterpret_cast<const uint8_t*>(P.kv);
-    const uint8_t* swb = reinterpret_cast<const uint8_t*>(P.swa ? P.swa : P.kv);
+    const uint8_t* kvb = P.kv;
+    const uint8_t* swb = P.swa ? P.swa : P.kv;
     // global row of key r of tile vk, or -1 when the slot is empty
     auto row_of = [&](int vk, int r, bool main_tile) -> int64_t {
       if (main_tile) {
@@ -245,10 +352,20 @@ __global__ void __launch_bounds__(NTHR, 1)
           cp_async16(dst, src, row >= 0);
         }
       }
-      for (int r = lane; r < NK; r += 32) {
+      bool ok2[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int r = lane + 32 * k;
         const int64_t row = row_of(vk, r, main_tile);
         const float* src = (main_tile ? P.kv_scale : P.swa_scale) + (row >= 0 ? row : 0);
         cp_async4(&s.kscale[st][r], src, row >= 0);
+        ok2[k] = row >= 0;
+      }
+      const uint32_t m0 = __ballot_sync(0xffffffffu, ok2[0]);
+      const uint32_t m1 = __ballot_sync(0xffffffffu, ok2[1]);
+      if (lane == 0) {
+        s.vmask[st][0] = m0;
+        s.vmask[st][1] = m1;
       }
       cp_async_commit();
       if (t >= 1) {
@@ -321,16 +438,16 @@ __global__ void __launch_bounds__(NTHR, 1)
       if (lane == 0) {
         const uint32_t Sn = tmem + a * 128, Sr = Sn + 64;
         for (int kb = 0; kb < 3; ++kb) {
-          const uint64_t aq = smem_desc(s.qn[kb], kq128), bk = smem_desc(s.kv[st][kb], kq128);
+          const uint64_t aq = smem_desc(s.q + kb * 16384, kq128), bk = smem_desc(s.kv[st][kb], kq128);
           for (int ks = 0; ks < 4; ++ks)
             mma_f8f6f4(Sn, aq + 2 * ks, bk + 2 * ks, id_qk8, (kb | ks) != 0);
         }
         {
-          const uint64_t aq = smem_desc(s.qn3, kq64), bk = smem_desc(s.kv3[st], kq64);
+          const uint64_t aq = smem_desc(s.q + Q_NOPE3, kq64), bk = smem_desc(s.kv3[st], kq64);
           for (int ks = 0; ks < 2; ++ks) mma_f8f6f4(Sn, aq + 2 * ks, bk + 2 * ks, id_qk8, 1);
         }
         {
-          const uint64_t aq = smem_desc(s.qr, kq128), bk = smem_desc(s.kv[st][3], kq128);
+          const uint64_t aq = smem_desc(s.q + Q_ROPE, kq128), bk = smem_desc(s.kv[st][3], kq128);
           for (int ks = 0; ks < 4; ++ks) mma_f16(Sr, aq + 2 * ks, bk + 2 * ks, id_qk16, ks != 0);
         }
         tc_commit(&s.sfull[a]);
@@ -347,165 +464,97 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ query prep, softmax, epilogue
-    const int ts = threadIdx.x - 64;          // 0..127
+    // ------------------------------------------------------------ softmax, epilogue
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;         // keys half*32 .. +31 of each tile
     const int h = quad * 32 + lane;           // head row == TMEM lane
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    if (ts < 32 && g.p >= 0) {
-      float c, sn;
-      rope_cs(g.p, ts, P.d_rope, P.theta, c, sn);
-      s.cs[ts] = c;
-      s.sn[ts] = sn;
-    }
-    softmax_bar();
-    float qsc = 1.f;
-    {
-      // Q row h: RoPE at p on dims 448..511, E4M3 coding of dims 0..447 with a
-      // power-of-two scale, written in the swizzled MMA layouts
-      uint32_t wq[256];                       // 512 bf16 as pairs
-      if (h < P.H) {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            reinterpret_cast<const __nv_bfloat16*>(P.Q) + ((int64_t)q * P.H + h) * 512);
-#pragma unroll 4
-        for (int i = 0; i < 64; ++i) {
-          const uint4 v = src[i];
-          wq[4 * i] = v.x; wq[4 * i + 1] = v.y; wq[4 * i + 2] = v.z; wq[4 * i + 3] = v.w;
-        }
-      } else {
-#pragma unroll 4
-        for (int i = 0; i < 256; ++i) wq[i] = 0u;
-      }
-      float amax = 0.f;
-#pragma unroll 8
-      for (int i = 0; i < 224; ++i) {
-        const float x0 = bf16_bits_to_f32((uint16_t)(wq[i] & 0xFFFF));
-        const float x1 = bf16_bits_to_f32((uint16_t)(wq[i] >> 16));
-        amax = fmaxf(amax, fmaxf(fabsf(x0), fabsf(x1)));
-      }
-      const int se = e4m3_scale_exp(amax);
-      qsc = exp2i(se);
-      // non-RoPE dims: 16 bytes at a time
-      for (int c16 = 0; c16 < 28; ++c16) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t w0 = wq[c16 * 8 + 2 * k], w1 = wq[c16 * 8 + 2 * k + 1];
-          const uint32_t b0 = f32_to_e4m3(scale_pow2(bf16_bits_to_f32((uint16_t)(w0 & 0xFFFF)), se));
-          const uint32_t b1 = f32_to_e4m3(scale_pow2(bf16_bits_to_f32((uint16_t)(w0 >> 16)), se));
-          const uint32_t b2 = f32_to_e4m3(scale_pow2(bf16_bits_to_f32((uint16_t)(w1 & 0xFFFF)), se));
-          const uint32_t b3 = f32_to_e4m3(scale_pow2(bf16_bits_to_f32((uint16_t)(w1 >> 16)), se));
-          pk[k] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-        }
-        const int c = c16 * 16;
-        uint8_t* dst = (c < 384) ? s.qn[c >> 7] + sw128(h, c & 127) : s.qn3 + sw64(h, c - 384);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
-      // bytes 64..127 of the SW64 block stay unused; RoPE dims (pairs 224..255)
-      for (int c16 = 0; c16 < 8; ++c16) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int pr = c16 * 4 + k;         // RoPE pair index 0..31
-          const uint32_t wv = wq[224 + pr];
-          const float x0 = bf16_bits_to_f32((uint16_t)(wv & 0xFFFF));
-          const float x1 = bf16_bits_to_f32((uint16_t)(wv >> 16));
-          const float cs = s.cs[pr], sn = s.sn[pr];
-          const float r0 = x0 * cs - x1 * sn, r1 = x0 * sn + x1 * cs;
-          pk[k] = (uint32_t)f32_to_bf16_bits(r0) | ((uint32_t)f32_to_bf16_bits(r1) << 16);
-        }
-        *reinterpret_cast<uint4*>(s.qr + sw128(h, c16 * 16)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
-    }
-    fence_proxy_async_smem();
-    softmax_bar();
-    if (ts == 0) mbar_arrive(&s.qready);
-
     const float sl2 = P.scale * 1.4426950408889634f;     // softmax scale x log2(e)
     float Ms = -INFINITY, Mu = -INFINITY, l = 0.f;
     bool wrote = false;                                  // O holds a PV result
-    for (int t = 0; t < g.T; ++t) {
-      const int a = t & 1, st = t % KST;
-      if (!mbar_wait_warp(&s.sfull[a], (t >> 1) & 1, P.status, 6) || !mbar_wait_warp(&s.full[st], (t / KST) & 1, P.status, 7)) {
-        flag(P.status, ST_TIMEOUT);
+    bool live = mbar_wait_warp(&s.qready, 0, P.status, 1);
+    const float qs = s.qsc[h];
+    for (int t = 0; t < g.T && live; ++t) {
+      const int a = t & 1, st = t % KST, xb = t & 1;
+      if (!mbar_wait_warp(&s.sfull[a], (t >> 1) & 1, P.status, 6) ||
+          !mbar_wait_warp(&s.full[st], (t / KST) & 1, P.status, 7)) {
+        live = false;
         break;
       }
       tc_fence_after();
-      uint32_t sn_[NK], sr_[NK];
-      const uint32_t ta = tmem + lane_off + a * 128;
+      uint32_t sn_[32], sr_[32];
+      const uint32_t ta = tmem + lane_off + a * 128 + half * 32;
       tmem_ld32_nowait(ta, sn_);
-      tmem_ld32_nowait(ta + 32, sn_ + 32);
       tmem_ld32_nowait(ta + 64, sr_);
-      tmem_ld32_nowait(ta + 96, sr_ + 32);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.sfree[a]);
-      const int vk = g.s0 + t * NK;
-      const bool main_tile = vk < g.nmp;
-      float s2[NK], u2[NK];
+      const uint32_t vm = s.vmask[st][half];
+      const float* ksc = &s.kscale[st][half * 32];
+      float s2[32];
       float ms = -INFINITY, mu = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < NK; ++j) {
-        bool valid;
-        if (main_tile) {
-          const int jj = vk + j;
-          valid = jj < g.n_main;
-          if (valid && P.idx) {
-            const int e = s.idx[jj - g.s0];
-            valid = e >= 0 && e < g.n_vis;
-          }
-        } else {
-          valid = (vk - g.nmp + j) < g.n_swa;
-        }
-        const float ksc = s.kscale[st][j];
-        const float v = (qsc * ksc * __uint_as_float(sn_[j]) + __uint_as_float(sr_[j])) * sl2;
-        const int ke = (int)((__float_as_uint(ksc) >> 23) & 0xFF) - 127;
-        s2[j] = valid ? v : -INFINITY;
-        u2[j] = valid ? v + (float)ke : -INFINITY;
+      for (int j = 0; j < 32; ++j) {
+        const float kj = ksc[j];
+        const float v = (qs * kj * __uint_as_float(sn_[j]) + __uint_as_float(sr_[j])) * sl2;
+        const int ke = (int)((__float_as_uint(kj) >> 23) & 0xFF) - 127;
+        s2[j] = ((vm >> j) & 1u) ? v : -INFINITY;
         ms = fmaxf(ms, s2[j]);
-        mu = fmaxf(mu, u2[j]);
+        mu = fmaxf(mu, s2[j] + (float)ke);
       }
+      // row maxima over the whole tile: exchange with the other key half
+      s.xmax[xb][half][0][h] = ms;
+      s.xmax[xb][half][1][h] = mu;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.xbar[xb]);
+      if (!mbar_wait_warp(&s.xbar[xb], (t >> 1) & 1, P.status, 10)) {
+        live = false;
+        break;
+      }
+      ms = fmaxf(ms, s.xmax[xb][half ^ 1][0][h]);
+      mu = fmaxf(mu, s.xmax[xb][half ^ 1][1][h]);
       const float Ms_new = fmaxf(Ms, ms), Mu_new = fmaxf(Mu, mu);
       const float as = (Ms_new == -INFINITY) ? 1.f : exp2f(Ms - Ms_new);
       const float au = (Mu_new == -INFINITY) ? 1.f : exp2f(Mu - Mu_new);
+      const float crow = (Mu_new == -INFINITY) ? 0.f : exp2f(Ms_new - Mu_new + 8.f);
       float lsum = 0.f;
-      uint32_t phi[NK / 4], plo[NK / 4], pbf[NK / 2];
+      uint32_t phi[8], plo[8], pbf[16];
 #pragma unroll
-      for (int j = 0; j < NK; j += 4) {
-        uint32_t hw = 0, lw = 0;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float pj = (s2[j + k] == -INFINITY) ? 0.f : exp2f(s2[j + k] - Ms_new);
-          const float pp = (u2[j + k] == -INFINITY) ? 0.f : exp2f(u2[j + k] - Mu_new + 8.f);
-          lsum += pj;
-          const uint32_t hi = f32_to_e4m3(pp);
-          const uint32_t lo = f32_to_e4m3(pp - e4m3_to_f32((uint8_t)hi));
-          hw |= hi << (8 * k);
-          lw |= lo << (8 * k);
-          if (k & 1) {
-            const float p0 = (s2[j + k - 1] == -INFINITY) ? 0.f : exp2f(s2[j + k - 1] - Ms_new);
-            pbf[(j + k) >> 1] = (uint32_t)f32_to_bf16_bits(p0) | ((uint32_t)f32_to_bf16_bits(pj) << 16);
-          }
+      for (int j = 0; j < 32; j += 2) {
+        const float p0 = (s2[j] == -INFINITY) ? 0.f : exp2f(s2[j] - Ms_new);
+        const float p1 = (s2[j + 1] == -INFINITY) ? 0.f : exp2f(s2[j + 1] - Ms_new);
+        lsum += p0 + p1;
+        const float u0 = p0 * ksc[j] * crow, u1 = p1 * ksc[j + 1] * crow;
+        const uint32_t hi = e4m3x2(u0, u1);
+        const float2 hf = e4m3x2_to_f32(hi);
+        const uint32_t lo = e4m3x2(u0 - hf.x, u1 - hf.y);
+        const int sh = (j & 3) * 8;
+        if ((j & 3) == 0) {
+          phi[j >> 2] = hi;
+          plo[j >> 2] = lo;
+        } else {
+          phi[j >> 2] |= hi << sh;
+          plo[j >> 2] |= lo << sh;
         }
-        phi[j >> 2] = hw;
-        plo[j >> 2] = lw;
+        pbf[j >> 1] = (uint32_t)f32_to_bf16_bits(p0) | ((uint32_t)f32_to_bf16_bits(p1) << 16);
       }
       l = l * as + lsum;
       // PV of the previous tile must be done before O or P change
       if (t >= 1 && !mbar_wait_warp(&s.pempty, (t - 1) & 1, P.status, 8)) {
-        flag(P.status, ST_TIMEOUT);
+        live = false;
         break;
       }
       tc_fence_after();
-      // Rescale O when a running maximum grew.  tcgen05.ld / st are warp-wide
-      // (.sync.aligned): the decision is taken per warp and every lane takes
-      // part, scaling its own row by its own factor (1 where nothing changed).
+      // Rescale this warp's half of O (columns half*128 .. +127) when a running
+      // maximum grew.  tcgen05.ld / st are warp-wide (.sync.aligned): the
+      // decision is taken per warp, every lane takes part with its own factor.
       const bool grow_u = __any_sync(0xffffffffu, wrote && au < 1.f);
       const bool grow_s = __any_sync(0xffffffffu, wrote && dh == 1 && as < 1.f);
       if (grow_u || grow_s) {
         const uint32_t ob = tmem + lane_off + 256;
-        for (int c = 0; c < 256; c += 32) {
+        for (int cc = 0; cc < 128; cc += 32) {
+          const int c = half * 128 + cc;
           const bool rope_cols = dh == 1 && c >= 192;
           if (rope_cols ? !grow_s : !grow_u) continue;     // uniform across the warp
           const float f = rope_cols ? as : au;
@@ -521,17 +570,16 @@ __global__ void __launch_bounds__(NTHR, 1)
       Ms = Ms_new;
       Mu = Mu_new;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        *reinterpret_cast<uint4*>(s.p_hi + sw64(h, 16 * c)) =
+      for (int c = 0; c < 2; ++c) {
+        *reinterpret_cast<uint4*>(s.p_hi + sw64(h, half * 32 + 16 * c)) =
             make_uint4(phi[4 * c], phi[4 * c + 1], phi[4 * c + 2], phi[4 * c + 3]);
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        *reinterpret_cast<uint4*>(s.p_lo + sw64(h, 16 * c)) =
+        *reinterpret_cast<uint4*>(s.p_lo + sw64(h, half * 32 + 16 * c)) =
             make_uint4(plo[4 * c], plo[4 * c + 1], plo[4 * c + 2], plo[4 * c + 3]);
+      }
       if (dh == 1) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(s.p_bf + sw128(h, 16 * c)) =
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(s.p_bf + sw128(h, half * 64 + 16 * c)) =
               make_uint4(pbf[4 * c], pbf[4 * c + 1], pbf[4 * c + 2], pbf[4 * c + 3]);
       }
       fence_proxy_async_smem();
@@ -540,15 +588,26 @@ __global__ void __launch_bounds__(NTHR, 1)
       if (lane == 0) mbar_arrive(&s.pfull);
       wrote = true;
     }
+    if (!live) flag(P.status, ST_TIMEOUT);
     // ------------------------------------------------------------ epilogue
-    const bool fin = mbar_wait_warp(&s.ofinal, 0, P.status, 9);
+    bool fin = mbar_wait_warp(&s.ofinal, 0, P.status, 9);
     tc_fence_after();
-    if (!fin) flag(P.status, ST_TIMEOUT);
+    // row sum of both key halves
+    if (half == 1) {
+      s.xl[h] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.lbar);
+    } else {
+      fin = mbar_wait_warp(&s.lbar, 0, P.status, 11) && fin;
+      l += s.xl[h];
+    }
+    fin = fin && live;
     // O_nope is in units of 2^8 exp2(. - Mu); express it in units of exp2(. - Ms)
     const float fn = (Ms == -INFINITY) ? 0.f : exp2f(Mu - 8.f - Ms);
     const uint32_t ob = tmem + lane_off + 256;
     float* dst = P.part_o + (pbase + h) * 512 + dh * 256;
-    for (int c = 0; c < 256; c += 32) {
+    for (int cc = 0; cc < 128; cc += 32) {
+      const int c = half * 128 + cc;
       uint32_t r[32];
       tmem_ld32_nowait(ob + c, r);
       tmem_ld_wait();
@@ -561,7 +620,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                           __uint_as_float(r[k + 2]) * f, __uint_as_float(r[k + 3]) * f);
       }
     }
-    if (dh == 0 && h < P.H) {
+    if (dh == 0 && half == 0 && h < P.H) {
       P.part_ml[(pbase + h) * 2] = (Ms == -INFINITY) ? -INFINITY : Ms * 0.6931471805599453f;
       P.part_ml[(pbase + h) * 2 + 1] = l;
     }
@@ -582,6 +641,7 @@ bool make_rows_map_sw(CUtensorMap* map, const void* base, int64_t rows, int row_
 bool mqa_tc_supported(const MqaParams& P) {
   return P.kv_dtype == V4A_E4M3_BF16ROPE && P.d == 512 && P.d_rope == 64 && P.H <= 128 &&
          P.q_dtype == V4A_BF16 && !P.q_rmsnorm && P.split_keys % NK == 0 &&
+         P.qbuf != nullptr && ((uintptr_t)P.qbuf & 15) == 0 &&
          P.split_keys <= SKMAX && P.n_win <= 1024 && ((uintptr_t)P.kv & 15) == 0 &&
          (P.n_win == 0 || ((uintptr_t)P.swa & 15) == 0) && ((uintptr_t)P.Q & 15) == 0 &&
          (int64_t)P.B * P.kv_rows < (1ll << 31) && (int64_t)P.B * P.swa_rows < (1ll << 31);
@@ -605,6 +665,7 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   }
   const int64_t grid = (int64_t)P.n_q * P.n_split * 2;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  mqa_tc_qprep_kernel<<<P.n_q, 128, 0, st>>>(P);
   mqa_tc_kernel<<<(unsigned)grid, NTHR, smem, st>>>(P, m);
   return cudaGetLastError();
 }
