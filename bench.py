@@ -116,6 +116,28 @@ def algorithmic_flops(w):
 
 # ------------------------------------------------------------------ clocks
 
+def graph_kernel_nodes(graph):
+    """Number of kernel nodes in a captured torch CUDA graph (None if the
+    runtime bindings are unavailable)."""
+    try:
+        from cuda.bindings import runtime as rt
+        g = rt.cudaGraph_t(init_value=graph.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(g, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(g, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kern = 0
+        for nd in nodes[:n]:
+            err, ty = rt.cudaGraphNodeGetType(nd)
+            if err == rt.cudaError_t.cudaSuccess and ty == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                kern += 1
+        return kern
+    except Exception:
+        return None
+
+
 class ClockSampler:
     """SM clock and clock-event reasons sampled through NVML every few
     milliseconds from a host thread; only samples taken between ``start()``
@@ -275,10 +297,11 @@ class Workload:
             self.step()
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
-        self.graph = torch.cuda.CUDAGraph()
+        self.graph = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(self.graph):
             self.step()
         torch.cuda.synchronize()
+        self.kernel_nodes = graph_kernel_nodes(self.graph)
 
     def replay(self):
         self.graph.replay()
@@ -287,11 +310,16 @@ class Workload:
         return self.w.B
 
     def launches_per_step(self):
+        """Kernel launches of one step: the kernel nodes of the captured graph
+        (every one of them is a library kernel; the step makes no other call)."""
+        if getattr(self, "kernel_nodes", None):
+            return self.kernel_nodes
         n = 0
         for ly in self.w.layers:
             # prep + window-KV compress + entry compress (+ key compress)
-            # (+ index scores + top-k) + MQA + combine
-            n += 1 + 2 + (1 if ly.kind == "csa" else 0) + (2 if ly.kind == "csa" else 0) + 2
+            # (+ index scores + top-k) (+ query coding) + MQA + combine
+            tc_mqa = ly.kv_fp8 and ly.d == 512
+            n += 1 + 2 + (3 if ly.kind == "csa" else 0) + (1 if tc_mqa else 0) + 2
         return n
 
     # per-step host<->device traffic of the end-to-end measurement

@@ -247,6 +247,19 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
   return cuda_status(launch_mqa_combine(P, st));
 }
 
+// Block-wide copy of n bytes between non-overlapping buffers, 16 bytes per
+// thread and step when both ends and n allow it.
+__device__ __forceinline__ void copy_bytes(uint8_t* __restrict__ dst,
+                                           const uint8_t* __restrict__ src, int64_t n) {
+  if (((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src) | (uintptr_t)n) & 15) == 0) {
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+    uint4* d = reinterpret_cast<uint4*>(dst);
+    for (int64_t e = threadIdx.x; e < n / 16; e += blockDim.x) d[e] = s[e];
+  } else {
+    for (int64_t e = threadIdx.x; e < n; e += blockDim.x) dst[e] = src[e];
+  }
+}
+
 __global__ void decode_prep_kernel(int B, const int64_t* pos, int m, int ring, int n_arr, int d,
                                    const void* x_main, void* tail, int in_elt, int dI,
                                    const void* x_idx, void* itail, int64_t* lens, int64_t* eb_tok,
@@ -262,12 +275,12 @@ __global__ void decode_prep_kernel(int B, const int64_t* pos, int m, int ring, i
   const int64_t nb = (int64_t)n_arr * d * in_elt;
   const uint8_t* src = reinterpret_cast<const uint8_t*>(x_main) + b * nb;
   uint8_t* dst = reinterpret_cast<uint8_t*>(tail) + ((int64_t)b * ring + slot) * nb;
-  for (int64_t e = threadIdx.x; e < nb; e += blockDim.x) dst[e] = src[e];
+  copy_bytes(dst, src, nb);
   if (x_idx) {
     const int64_t ni = (int64_t)4 * dI * in_elt;
     const uint8_t* s2 = reinterpret_cast<const uint8_t*>(x_idx) + b * ni;
     uint8_t* d2 = reinterpret_cast<uint8_t*>(itail) + ((int64_t)b * ring + slot) * ni;
-    for (int64_t e = threadIdx.x; e < ni; e += blockDim.x) d2[e] = s2[e];
+    copy_bytes(d2, s2, ni);
   }
 }
 

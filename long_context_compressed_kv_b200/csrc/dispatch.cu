@@ -6,7 +6,7 @@ namespace v4a {
 
 int mqa_split_keys(const v4attn_layer_desc* d) {
   if (d->kv_dtype == V4A_E4M3_BF16ROPE && d->d == 512)      // tensor-core kernel
-    return d->kind == V4A_CSA ? 128 : 256;
+    return d->kind == V4A_CSA ? 128 : 512;
   return kSimtSplitKeys;
 }
 

@@ -32,10 +32,9 @@
 // maximum grows.  The same shared-memory tile serves as the K-major B operand
 // of Q K^T and the MN-major B operand of P V.
 //
-// Rows arrive by tile-mode TMA for contiguous HCA entries and by 16-byte
-// cp.async for selected entries and window tokens (a swizzled TMA destination
-// must sit on the swizzle's 1024-byte repeat, which a 4-row gather into the
-// middle of an 8-row atom does not).  Roles: warp 0 loads, warp 1 issues the
+// Rows arrive by TMA: tile mode for contiguous HCA entries, tile::gather4 (4
+// rows per instruction) for selected entries and window tokens; the entry
+// scales by 4-byte cp.async.  Roles: warp 0 loads, warp 1 issues the
 // MMAs (one lane), warps 2..9 run the softmax and the epilogue: two warps per
 // TMEM lane quarter, one per 32-key half of each tile, exchanging row maxima
 // through shared memory.  Every cross-warp hand-off is an mbarrier with a
@@ -89,7 +88,23 @@ static_assert(offsetof(Smem, qsc) == QTILE, "the query image is one contiguous c
 
 struct Maps {
   CUtensorMap kv128, kv64;      // tile mode, boxes {128 B | 64 B} x NK rows
+  CUtensorMap kvg128, kvg64;    // tile::gather4 over entry rows, boxes one row high
+  CUtensorMap swg128, swg64;    // tile::gather4 over window rows
 };
+
+// Four rows (r0..r3, 4 x the box width) into consecutive rows of a swizzled
+// tile.  The swizzle follows the absolute shared-memory address, so a group
+// may start in the middle of an 8-row swizzle atom (rows 4..7 at +512 bytes
+// for 128-byte rows, checked on B200).
+__device__ __forceinline__ void gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                        int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3)
+      : "memory");
+}
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
   asm volatile(
@@ -166,68 +181,76 @@ __device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
 
 }  // namespace
 
-// One CTA per query, one thread per head row: the query image of the main kernel.
-__global__ void __launch_bounds__(128) mqa_tc_qprep_kernel(MqaParams P) {
+// One CTA per query, four threads per head row (7 of the 28 E4M3 chunks and 2
+// of the 8 RoPE chunks each): the query image of the main kernel.  Each
+// thread issues all of its loads before the RoPE angles (double precision,
+// positions up to 2^20 and beyond) are computed.
+__global__ void __launch_bounds__(512) mqa_tc_qprep_kernel(MqaParams P) {
   __shared__ float cs[32], sn[32];
-  const int q = blockIdx.x, h = threadIdx.x;
+  const int q = blockIdx.x;
+  const int h = threadIdx.x >> 2, part = threadIdx.x & 3;
   const int64_t p = P.q_pos[q];
-  if (h < 32) {
-    float c = 1.f, sv = 0.f;
-    if (p >= 0) rope_cs(p, h, 64, P.theta, c, sv);
-    cs[h] = c;
-    sn[h] = sv;
-  }
-  __syncthreads();
   uint8_t* img = P.qbuf + (int64_t)q * kMqaQImageStride;
   const bool live = h < P.H;
   const uint4* src = reinterpret_cast<const uint4*>(
       reinterpret_cast<const __nv_bfloat16*>(P.Q) + ((int64_t)q * P.H + (live ? h : 0)) * 512);
+  uint4 nope[14], rope[2];
+#pragma unroll
+  for (int i = 0; i < 14; ++i) nope[i] = live ? src[part * 14 + i] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) rope[i] = live ? src[56 + part * 2 + i] : make_uint4(0u, 0u, 0u, 0u);
+  if (threadIdx.x < 32) {
+    float c = 1.f, sv = 0.f;
+    if (p >= 0) rope_cs(p, threadIdx.x, 64, P.theta, c, sv);
+    cs[threadIdx.x] = c;
+    sn[threadIdx.x] = sv;
+  }
   float amax = 0.f;
-  if (live)
-    for (int i = 0; i < 56; ++i) {
-      const uint4 v = src[i];
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[k])), fabsf(bf16hi(w[k]))));
-    }
+  for (int i = 0; i < 14; ++i) {
+    const uint32_t w[4] = {nope[i].x, nope[i].y, nope[i].z, nope[i].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[k])), fabsf(bf16hi(w[k]))));
+  }
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
   const int se = e4m3_scale_exp(amax);
-  // dims 0..447: 16 E4M3 codes per 16-byte chunk
-  for (int c16 = 0; c16 < 28; ++c16) {
-    uint32_t pk[4] = {0u, 0u, 0u, 0u};
-    if (live) {
-      const uint4 a = src[2 * c16], b = src[2 * c16 + 1];
-      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  // dims 0..447: 16 E4M3 codes per 16-byte chunk (chunks part*7 .. part*7+6)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t lo = e4m3x2(scale_pow2(bf16lo(w[2 * k]), se), scale_pow2(bf16hi(w[2 * k]), se));
-        const uint32_t hi =
-            e4m3x2(scale_pow2(bf16lo(w[2 * k + 1]), se), scale_pow2(bf16hi(w[2 * k + 1]), se));
-        pk[k] = lo | (hi << 16);
-      }
+  for (int j = 0; j < 7; ++j) {
+    const uint4 a = nope[2 * j], b = nope[2 * j + 1];
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t pk[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t lo = e4m3x2(scale_pow2(bf16lo(w[2 * k]), se), scale_pow2(bf16hi(w[2 * k]), se));
+      const uint32_t hi =
+          e4m3x2(scale_pow2(bf16lo(w[2 * k + 1]), se), scale_pow2(bf16hi(w[2 * k + 1]), se));
+      pk[k] = lo | (hi << 16);
     }
-    const int c = c16 * 16;
+    const int c = (part * 7 + j) * 16;
     uint8_t* dst = (c < 384) ? img + (c >> 7) * 16384 + sw128(h, c & 127)
                              : img + Q_NOPE3 + sw64(h, c - 384);
     *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
+  __syncthreads();                          // RoPE angles
   // dims 448..511: RoPE at the query position, kept in bf16
-  for (int c16 = 0; c16 < 8; ++c16) {
-    uint32_t pk[4] = {0u, 0u, 0u, 0u};
-    if (live) {
-      const uint4 v = src[56 + c16];
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int pr = c16 * 4 + k;
-        const float x0 = bf16lo(w[k]), x1 = bf16hi(w[k]);
-        const float r0 = x0 * cs[pr] - x1 * sn[pr], r1 = x0 * sn[pr] + x1 * cs[pr];
-        pk[k] = (uint32_t)f32_to_bf16_bits(r0) | ((uint32_t)f32_to_bf16_bits(r1) << 16);
-      }
+  for (int j = 0; j < 2; ++j) {
+    const int c16 = part * 2 + j;
+    const uint32_t w[4] = {rope[j].x, rope[j].y, rope[j].z, rope[j].w};
+    uint32_t pk[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int pr = c16 * 4 + k;
+      const float x0 = bf16lo(w[k]), x1 = bf16hi(w[k]);
+      const float r0 = x0 * cs[pr] - x1 * sn[pr], r1 = x0 * sn[pr] + x1 * cs[pr];
+      pk[k] = (uint32_t)f32_to_bf16_bits(r0) | ((uint32_t)f32_to_bf16_bits(r1) << 16);
     }
     *reinterpret_cast<uint4*>(img + Q_ROPE + sw128(h, c16 * 16)) =
         make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
-  reinterpret_cast<float*>(img + QTILE)[h] = exp2i(se);
+  if (part == 0) reinterpret_cast<float*>(img + QTILE)[h] = exp2i(se);
 }
 
 __global__ void __launch_bounds__(NTHR, 1)
@@ -284,14 +307,11 @@ __global__ void __launch_bounds__(NTHR, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ loads
-    // The query image by four bulk copies on qready.  Contiguous entry tiles
-    // go by tile-mode TMA (complete_tx bytes on full[st]).  Selected entries
-    // and window tokens go by 16-byte cp.async straight into the swizzled
-    // positions (lanes walk the 36 chunks of each 576-byte row in order, so a
-    // warp's copies are coalesced); so do the 64 entry scales.  Tile t is
-    // published once tile t+1 has been issued: wait for all but the newest
-    // cp.async group, fence the generic-proxy writes against the async proxy
-    // that the MMAs read through, then lane 0 arrives on full[st].
+    // The query image by four bulk copies on qready.  Entry / window rows by
+    // TMA (complete_tx bytes on full[st]); the 64 entry scales by cp.async
+    // (zero-filled for empty slots) with the valid-key mask beside them.  Tile
+    // t is published once tile t+1 has been issued: wait for all but the
+    // newest cp.async group, then lane 0 arrives on full[st].
     if (lane == 0) {
       const uint8_t* qimg = P.qbuf + (int64_t)q * kMqaQImageStride;
       mbar_arrive_expect_tx(&s.qready, QIMG);
@@ -299,8 +319,6 @@ __global__ void __launch_bounds__(NTHR, 1)
         bulk_load(s.q + k * QCHUNK, qimg + k * QCHUNK, QCHUNK, &s.qready);
     }
     const int64_t kv_base = (int64_t)g.b * P.kv_rows, sw_base = (int64_t)g.b * P.swa_rows;
-    const uint8_t* kvb = P.kv;
-    const uint8_t* swb = P.swa ? P.swa : P.kv;
     // global row of key r of tile vk, or -1 when the slot is empty
     auto row_of = [&](int vk, int r, bool main_tile) -> int64_t {
       if (main_tile) {
@@ -341,15 +359,25 @@ __global__ void __launch_bounds__(NTHR, 1)
           tma_load_2d(s.kv[st][3], &maps.kv128, &s.full[st], 448, y);
         }
       } else {
-        for (int i = lane; i < NK * 36; i += 32) {
-          const int r = i / 36, ch = i - r * 36;
-          const int64_t row = row_of(vk, r, main_tile);
-          const uint8_t* src = (main_tile ? kvb : swb) + (row >= 0 ? row : 0) * ROWB + ch * 16;
-          uint8_t* dst;
-          if (ch < 24) dst = s.kv[st][ch >> 3] + sw128(r, (ch & 7) * 16);
-          else if (ch < 28) dst = s.kv3[st] + sw64(r, (ch - 24) * 16);
-          else dst = s.kv[st][3] + sw128(r, (ch - 28) * 16);
-          cp_async16(dst, src, row >= 0);
+        // 4 rows per tile::gather4 (box one row high); an empty slot repeats
+        // the chunk's first row (its scale is zero-filled and it is masked)
+        if (lane == 0) mbar_expect_tx(&s.full[st], TILE_BYTES);
+        __syncwarp();
+        if (lane < NK / 4) {
+          int rows[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int64_t row = row_of(vk, lane * 4 + k, main_tile);
+            rows[k] = (int)(row >= 0 ? row : (main_tile ? kv_base : sw_base));
+          }
+          const CUtensorMap* m128 = main_tile ? &maps.kvg128 : &maps.swg128;
+          const CUtensorMap* m64 = main_tile ? &maps.kvg64 : &maps.swg64;
+          const int o128 = lane * 4 * 128, o64 = lane * 4 * 64;
+          gather4(s.kv[st][0] + o128, m128, &s.full[st], 0, rows[0], rows[1], rows[2], rows[3]);
+          gather4(s.kv[st][1] + o128, m128, &s.full[st], 128, rows[0], rows[1], rows[2], rows[3]);
+          gather4(s.kv[st][2] + o128, m128, &s.full[st], 256, rows[0], rows[1], rows[2], rows[3]);
+          gather4(s.kv3[st] + o64, m64, &s.full[st], 384, rows[0], rows[1], rows[2], rows[3]);
+          gather4(s.kv[st][3] + o128, m128, &s.full[st], 448, rows[0], rows[1], rows[2], rows[3]);
         }
       }
       bool ok2[2];
@@ -604,20 +632,26 @@ __global__ void __launch_bounds__(NTHR, 1)
     fin = fin && live;
     // O_nope is in units of 2^8 exp2(. - Mu); express it in units of exp2(. - Ms)
     const float fn = (Ms == -INFINITY) ? 0.f : exp2f(Mu - 8.f - Ms);
+    // O rows leave through a per-warp 32 x 32 staging block in shared memory
+    // (the key stages are free once ofinal has fired), so that every global
+    // store writes one 128-byte row segment.
     const uint32_t ob = tmem + lane_off + 256;
-    float* dst = P.part_o + (pbase + h) * 512 + dh * 256;
+    float* stg = reinterpret_cast<float*>(&s.kv[0][0][0]) + (warp - 2) * (32 * 33);
+    const int64_t row0 = pbase + quad * 32;
     for (int cc = 0; cc < 128; cc += 32) {
       const int c = half * 128 + cc;
       uint32_t r[32];
       tmem_ld32_nowait(ob + c, r);
       tmem_ld_wait();
       const float f = (dh == 1 && c >= 192) ? (Ms == -INFINITY ? 0.f : 1.f) : fn;
-      if (h < P.H && fin) {
+      if (fin) {
 #pragma unroll
-        for (int k = 0; k < 32; k += 4)
-          *reinterpret_cast<float4*>(dst + c + k) =
-              make_float4(__uint_as_float(r[k]) * f, __uint_as_float(r[k + 1]) * f,
-                          __uint_as_float(r[k + 2]) * f, __uint_as_float(r[k + 3]) * f);
+        for (int k = 0; k < 32; ++k) stg[lane * 33 + k] = __uint_as_float(r[k]) * f;
+        __syncwarp();
+        for (int rr = 0; rr < 32; ++rr)
+          if (quad * 32 + rr < P.H)
+            P.part_o[(row0 + rr) * 512 + dh * 256 + c + lane] = stg[rr * 33 + lane];
+        __syncwarp();
       }
     }
     if (dh == 0 && half == 0 && h < P.H) {
@@ -650,8 +684,15 @@ bool mqa_tc_supported(const MqaParams& P) {
 cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   Maps m;
   const int64_t kv_rows = (int64_t)P.B * P.kv_rows;
+  const int64_t sw_rows = (int64_t)P.B * P.swa_rows;
+  const void* swa = P.swa ? (const void*)P.swa : (const void*)P.kv;
+  const int64_t swr = P.swa ? sw_rows : kv_rows;
   if (!make_rows_map_sw(&m.kv128, P.kv, kv_rows, ROWB, 128, NK, 128) ||
-      !make_rows_map_sw(&m.kv64, P.kv, kv_rows, ROWB, 64, NK, 64))
+      !make_rows_map_sw(&m.kv64, P.kv, kv_rows, ROWB, 64, NK, 64) ||
+      !make_rows_map_sw(&m.kvg128, P.kv, kv_rows, ROWB, 128, 1, 128) ||
+      !make_rows_map_sw(&m.kvg64, P.kv, kv_rows, ROWB, 64, 1, 64) ||
+      !make_rows_map_sw(&m.swg128, swa, swr, ROWB, 128, 1, 128) ||
+      !make_rows_map_sw(&m.swg64, swa, swr, ROWB, 64, 1, 64))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
   static unsigned long long configured = 0;
@@ -665,7 +706,7 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   }
   const int64_t grid = (int64_t)P.n_q * P.n_split * 2;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  mqa_tc_qprep_kernel<<<P.n_q, 128, 0, st>>>(P);
+  mqa_tc_qprep_kernel<<<P.n_q, 512, 0, st>>>(P);
   mqa_tc_kernel<<<(unsigned)grid, NTHR, smem, st>>>(P, m);
   return cudaGetLastError();
 }
