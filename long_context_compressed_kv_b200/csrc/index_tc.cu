@@ -145,11 +145,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t* ksf32 = reinterpret_cast<const uint32_t*>(P.keys_sf);
     const int64_t total_rows = (int64_t)P.B * P.key_rows;
     int it = 0;
+    int b = 0;                                  // sequence of the current query
     for (int g = g0; g < g1 && !__any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s.abort)); ++g, ++it) {
       const int seg_before = t.seg;
       locate(s, P.n_q, g, t);
-      const int b = P.q_seq ? P.q_seq[t.q] : t.q;
       if (t.seg != seg_before) {
+        // read once per query: a global load per tile would sit on the issue path
+        b = P.q_seq ? P.q_seq[t.q] : t.q;
         const int j = t.seg & 1, uq = t.seg >> 1;
         if (uq >= 1 && !mbar_wait_warp(&s.qempty[j], (uq - 1) & 1, P.status)) {
           fail(s, P.status);
