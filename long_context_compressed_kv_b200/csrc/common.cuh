@@ -85,14 +85,26 @@ __device__ __forceinline__ float scale_pow2(float x, int e) {
 }
 
 // ---------------------------------------------------------------- RoPE
-// Angle (cos, sin) of pair k at position pos, computed in double so that
-// positions up to 2^20 and beyond keep full accuracy.
+// Angle (cos, sin) of pair k at position pos, a = pos * theta^(-2k/d_rope),
+// computed in double so that positions up to 2^20 and beyond keep full
+// accuracy.  The frequency is exp2(-(2k/d_rope) * log2(theta)); the angle
+// (up to ~2^31 rad) is first brought into [-pi, pi] by Cody-Waite reduction
+// with 2*pi split into two doubles (W. J. Cody and W. Waite, "Software Manual
+// for the Elementary Functions", 1980), so that sincos always sees a small
+// argument.  n < 2^31 and the product n * 2pi_hi is exact in the fma, so the
+// reduced angle is accurate to about 2^-52 absolute.
 __device__ __forceinline__ void rope_cs(int64_t pos, int k, int d_rope, float theta, float& c,
                                         float& s) {
-  double inv = pow((double)theta, -(2.0 * k) / (double)d_rope);
-  double a = (double)pos * inv;
+  constexpr double kTwoPiHi = 6.283185307179586232;       // 2*pi rounded to double
+  constexpr double kTwoPiLo = 2.4492935982947064e-16;     // 2*pi - kTwoPiHi
+  constexpr double kInvTwoPi = 0.15915494309189533577;
+  const double w = exp2(-(2.0 * k / (double)d_rope) * log2((double)theta));
+  const double a = (double)pos * w;
+  const double n = rint(a * kInvTwoPi);
+  double r = fma(-n, kTwoPiHi, a);
+  r = fma(-n, kTwoPiLo, r);
   double sd, cd;
-  sincos(a, &sd, &cd);
+  sincos(r, &sd, &cd);
   c = (float)cd;
   s = (float)sd;
 }

@@ -23,21 +23,22 @@
 //   S_rope = Q_rope(BF16) . K_rope(BF16)^T    4 x tcgen05.mma kind::f16,   K=16
 //   s_j    = scale * (q_scale * k_scale_j * S_nope + S_rope)       (log2 units)
 //   P_j    = exp2(s_j - M_s)                                        (BF16, RoPE dims)
-//   P'_j   = P_j * k_scale_j * 2^(M_s - M_u + 8) = 2^(s_j + log2 k_scale_j - M_u + 8)
-//   O_nope += P'_hi V_nope + P'_lo V_nope     (E4M3 hi + lo parts), kind::f8f6f4, V MN-major
+//   P'_j   = P_j * k_scale_j * 2^(8 - tau - K)                      (E4M3 hi + lo parts)
+//   O_nope += P'_hi V_nope + P'_lo V_nope                           kind::f8f6f4, V MN-major
 //   O_rope += P V_rope                                              kind::f16, V MN-major
-// The entry scale k_scale_j of the FP8 dims is folded into P', which keeps its
-// own running maximum M_u so that P' never exceeds 2^8 (inside E4M3's range);
-// one exp2 per key serves both.  O is rescaled in TMEM only when a running
-// maximum grows.  The same shared-memory tile serves as the K-major B operand
+// The entry scale k_scale_j (a power of two) of the FP8 dims is folded into
+// P'; K is the CTA's running maximum of log2 k_scale, the same for every head
+// row.  M_s is the row's running score maximum, moved only when a tile beats
+// it by more than tau = 4, so P <= 2^tau and P' <= 2^8 (inside E4M3's range);
+// O is rescaled in TMEM only when M_s or K moves.  The same shared-memory tile serves as the K-major B operand
 // of Q K^T and the MN-major B operand of P V.
 //
 // Rows arrive by TMA: tile mode for contiguous HCA entries, tile::gather4 (4
 // rows per instruction) for selected entries and window tokens; the entry
 // scales by 4-byte cp.async.  Roles: warp 0 loads, warp 1 issues the
-// MMAs (one lane), warps 2..9 run the softmax and the epilogue: two warps per
-// TMEM lane quarter, one per 32-key half of each tile, exchanging row maxima
-// through shared memory.  Every cross-warp hand-off is an mbarrier with a
+// MMAs (one lane), warps 2..17 run the softmax and the epilogue: four warps
+// per TMEM lane quarter, one per 16-key group of each tile, exchanging row
+// maxima through shared memory.  Every cross-warp hand-off is an mbarrier with a
 // bounded, warp-uniform wait, so a stalled kernel ends with a status bit.
 #include <cstddef>
 
@@ -52,11 +53,15 @@ namespace {
 
 constexpr int NK = 64;          // keys per tile
 constexpr int KST = 3;          // tile stages in flight
-constexpr int NSM = 8;          // softmax / epilogue warps
+constexpr int KG = 4;           // key groups per tile = softmax warps per TMEM lane quarter
+constexpr int KPG = 64 / KG;    // keys per group
+constexpr int NSM = 4 * KG;     // softmax / epilogue warps
 constexpr int NTHR = 64 + 32 * NSM;
 constexpr int ROWB = 576;       // stored row: 448 E4M3 + 64 bf16
 constexpr int SKMAX = 512;      // keys per split, at most
+constexpr int SKMAX_SEL = 128;  // keys per split of a selected-entry (sparse) call
 constexpr int TILE_BYTES = NK * (4 * 128 + 64);
+constexpr float kTau = 4.f;     // lazy-rescale margin of the running score maximum (log2 units)
 // query image: Q nope bytes 0..383 as three K-major SW128 blocks, bytes
 // 384..447 as one K-major SW64 block, the RoPE dims (bf16) as one K-major SW128
 // block, then the per-head E4M3 scale
@@ -74,10 +79,9 @@ struct Smem {
   alignas(1024) uint8_t p_lo[128 * 64];       // P' low part
   alignas(1024) uint8_t p_bf[128 * 128];      // P for the RoPE dims, bf16, K-major SW128
   float kscale[KST][NK];
-  uint32_t vmask[KST][2];                     // valid keys of a tile, 32 per word
-  int idx[SKMAX];
-  float xmax[2][2][2][128];                   // [tile parity][key half][M_s, M_u][row]
-  float xl[128];                              // the second half's row sums, for the epilogue
+  int idx[SKMAX_SEL];
+  float xmax[2][KG][2][128];                  // [tile parity][key group][M_s, M_u][row]
+  float xl[KG - 1][128];                      // the other groups' row sums, for the epilogue
   uint64_t full[KST], empty[KST], sfull[2], sfree[2], xbar[2];
   uint64_t pfull, pempty, qready, ofinal, done, lbar;
   uint32_t tmem_base;
@@ -139,6 +143,12 @@ __device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t c) {
   const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)c, __NV_E4M3);
   return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
+// 2^x by the SFU (ex2.approx, flush to zero; 2^-inf = 0)
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -181,14 +191,14 @@ __device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
 
 }  // namespace
 
-// One CTA per query, four threads per head row (7 of the 28 E4M3 chunks and 2
-// of the 8 RoPE chunks each): the query image of the main kernel.  Each
-// thread issues all of its loads before the RoPE angles (double precision,
-// positions up to 2^20 and beyond) are computed.
-__global__ void __launch_bounds__(512) mqa_tc_qprep_kernel(MqaParams P) {
+// Eight CTAs per query (16 head rows each, so that a query's 128 KB of bf16 Q
+// is read by eight SMs), four threads per head row (7 of the 28 E4M3 chunks
+// and 2 of the 8 RoPE chunks each): the query image of the main kernel.  Each
+// thread issues all of its loads before the RoPE angles are computed.
+__global__ void __launch_bounds__(64) mqa_tc_qprep_kernel(MqaParams P) {
   __shared__ float cs[32], sn[32];
   const int q = blockIdx.x;
-  const int h = threadIdx.x >> 2, part = threadIdx.x & 3;
+  const int h = blockIdx.y * 16 + (threadIdx.x >> 2), part = threadIdx.x & 3;
   const int64_t p = P.q_pos[q];
   uint8_t* img = P.qbuf + (int64_t)q * kMqaQImageStride;
   const bool live = h < P.H;
@@ -276,7 +286,7 @@ __global__ void __launch_bounds__(NTHR, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < KST; ++i) {
-      mbar_init(&s.full[i], 1);
+      mbar_init(&s.full[i], 32);   // the producer lanes' scale arrivals + TMA bytes
       mbar_init(&s.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -289,7 +299,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     mbar_init(&s.qready, 1);
     mbar_init(&s.ofinal, 1);
     mbar_init(&s.done, 1);
-    mbar_init(&s.lbar, NSM / 2);
+    mbar_init(&s.lbar, NSM - 4);
     fence_mbar_init();
   }
   if (warp == 0 && P.idx) {
@@ -308,10 +318,10 @@ __global__ void __launch_bounds__(NTHR, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ loads
     // The query image by four bulk copies on qready.  Entry / window rows by
-    // TMA (complete_tx bytes on full[st]); the 64 entry scales by cp.async
-    // (zero-filled for empty slots) with the valid-key mask beside them.  Tile
-    // t is published once tile t+1 has been issued: wait for all but the
-    // newest cp.async group, then lane 0 arrives on full[st].
+    // TMA (complete_tx bytes on full[st]); the 64 entry scales by cp.async,
+    // zero-filled for empty slots (a stored scale is a nonzero power of two,
+    // so a zero scale marks an empty slot); every lane arrives on full[st]
+    // through cp.async.mbarrier.arrive.noinc once its scale copies land.
     if (lane == 0) {
       const uint8_t* qimg = P.qbuf + (int64_t)q * kMqaQImageStride;
       mbar_arrive_expect_tx(&s.qready, QIMG);
@@ -338,8 +348,7 @@ __global__ void __launch_bounds__(NTHR, 1)
       return sw_base + tok % P.swa_rows;
     };
     bool issued_ok = true;
-    int t = 0;
-    for (; t < g.T; ++t) {
+    for (int t = 0; t < g.T; ++t) {
       const int st = t % KST, u = t / KST;
       if (u >= 1 && !mbar_wait_warp(&s.empty[st], (u - 1) & 1, P.status, 0)) {
         issued_ok = false;
@@ -348,9 +357,10 @@ __global__ void __launch_bounds__(NTHR, 1)
       const int vk = g.s0 + t * NK;
       const bool main_tile = vk < g.nmp;
       const bool contiguous = main_tile && !P.idx && vk + NK <= g.n_main;
+      if (lane == 0) mbar_expect_tx(&s.full[st], TILE_BYTES);
+      __syncwarp();
       if (contiguous) {
         if (lane == 0) {
-          mbar_expect_tx(&s.full[st], TILE_BYTES);
           const int y = (int)(kv_base + vk);
           tma_load_2d(s.kv[st][0], &maps.kv128, &s.full[st], 0, y);
           tma_load_2d(s.kv[st][1], &maps.kv128, &s.full[st], 128, y);
@@ -358,55 +368,36 @@ __global__ void __launch_bounds__(NTHR, 1)
           tma_load_2d(s.kv3[st], &maps.kv64, &s.full[st], 384, y);
           tma_load_2d(s.kv[st][3], &maps.kv128, &s.full[st], 448, y);
         }
-      } else {
+      } else if (lane < NK / 4) {
         // 4 rows per tile::gather4 (box one row high); an empty slot repeats
-        // the chunk's first row (its scale is zero-filled and it is masked)
-        if (lane == 0) mbar_expect_tx(&s.full[st], TILE_BYTES);
-        __syncwarp();
-        if (lane < NK / 4) {
-          int rows[4];
+        // a valid row (its scale is zero-filled, which marks it empty)
+        int rows[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int64_t row = row_of(vk, lane * 4 + k, main_tile);
-            rows[k] = (int)(row >= 0 ? row : (main_tile ? kv_base : sw_base));
-          }
-          const CUtensorMap* m128 = main_tile ? &maps.kvg128 : &maps.swg128;
-          const CUtensorMap* m64 = main_tile ? &maps.kvg64 : &maps.swg64;
-          const int o128 = lane * 4 * 128, o64 = lane * 4 * 64;
-          gather4(s.kv[st][0] + o128, m128, &s.full[st], 0, rows[0], rows[1], rows[2], rows[3]);
-          gather4(s.kv[st][1] + o128, m128, &s.full[st], 128, rows[0], rows[1], rows[2], rows[3]);
-          gather4(s.kv[st][2] + o128, m128, &s.full[st], 256, rows[0], rows[1], rows[2], rows[3]);
-          gather4(s.kv3[st] + o64, m64, &s.full[st], 384, rows[0], rows[1], rows[2], rows[3]);
-          gather4(s.kv[st][3] + o128, m128, &s.full[st], 448, rows[0], rows[1], rows[2], rows[3]);
+        for (int k = 0; k < 4; ++k) {
+          const int64_t row = row_of(vk, lane * 4 + k, main_tile);
+          rows[k] = (int)(row >= 0 ? row : (main_tile ? kv_base : sw_base));
         }
+        const CUtensorMap* m128 = main_tile ? &maps.kvg128 : &maps.swg128;
+        const CUtensorMap* m64 = main_tile ? &maps.kvg64 : &maps.swg64;
+        const int o128 = lane * 4 * 128, o64 = lane * 4 * 64;
+        gather4(s.kv[st][0] + o128, m128, &s.full[st], 0, rows[0], rows[1], rows[2], rows[3]);
+        gather4(s.kv[st][1] + o128, m128, &s.full[st], 128, rows[0], rows[1], rows[2], rows[3]);
+        gather4(s.kv[st][2] + o128, m128, &s.full[st], 256, rows[0], rows[1], rows[2], rows[3]);
+        gather4(s.kv3[st] + o64, m64, &s.full[st], 384, rows[0], rows[1], rows[2], rows[3]);
+        gather4(s.kv[st][3] + o128, m128, &s.full[st], 448, rows[0], rows[1], rows[2], rows[3]);
       }
-      bool ok2[2];
+      // entry scales (zero for an empty slot), then this lane's arrival, which
+      // fires once its scale copies have landed
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
         const int r = lane + 32 * k;
         const int64_t row = row_of(vk, r, main_tile);
         const float* src = (main_tile ? P.kv_scale : P.swa_scale) + (row >= 0 ? row : 0);
         cp_async4(&s.kscale[st][r], src, row >= 0);
-        ok2[k] = row >= 0;
       }
-      const uint32_t m0 = __ballot_sync(0xffffffffu, ok2[0]);
-      const uint32_t m1 = __ballot_sync(0xffffffffu, ok2[1]);
-      if (lane == 0) {
-        s.vmask[st][0] = m0;
-        s.vmask[st][1] = m1;
-      }
-      cp_async_commit();
-      if (t >= 1) {
-        cp_async_wait<1>();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.full[(t - 1) % KST]);
-      }
+      cp_async_arrive_noinc(&s.full[st]);
     }
     cp_async_wait<0>();
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (issued_ok && lane == 0 && t >= 1) mbar_arrive(&s.full[(t - 1) % KST]);
     if (!issued_ok) flag(P.status, ST_TIMEOUT);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
@@ -494,11 +485,16 @@ __global__ void __launch_bounds__(NTHR, 1)
   } else {
     // ------------------------------------------------------------ softmax, epilogue
     const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;         // keys half*32 .. +31 of each tile
+    const int grp = (warp - 2) >> 2;          // keys grp*KPG .. +KPG-1 of each tile
     const int h = quad * 32 + lane;           // head row == TMEM lane
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const float sl2 = P.scale * 1.4426950408889634f;     // softmax scale x log2(e)
-    float Ms = -INFINITY, Mu = -INFINITY, l = 0.f;
+    // Ms: the row's running score maximum (log2 units), moved only when a tile
+    // exceeds it by more than kTau, so P <= 2^kTau; K: the CTA's running
+    // maximum entry-scale exponent, so P' = P k_scale 2^(8 - kTau - K) <= 2^8.
+    float Ms = -INFINITY, l = 0.f;
+    int K = -1000;                                       // no key seen yet
+    float cu = 0.f;                                      // 2^(8 - kTau - K), exponent clamped
     bool wrote = false;                                  // O holds a PV result
     bool live = mbar_wait_warp(&s.qready, 0, P.status, 1);
     const float qs = s.qsc[h];
@@ -510,62 +506,68 @@ __global__ void __launch_bounds__(NTHR, 1)
         break;
       }
       tc_fence_after();
-      uint32_t sn_[32], sr_[32];
-      const uint32_t ta = tmem + lane_off + a * 128 + half * 32;
-      tmem_ld32_nowait(ta, sn_);
-      tmem_ld32_nowait(ta + 64, sr_);
+      uint32_t sn_[KPG], sr_[KPG];
+      const uint32_t ta = tmem + lane_off + a * 128 + grp * KPG;
+      tmem_ld16_nowait(ta, sn_);
+      tmem_ld16_nowait(ta + 64, sr_);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.sfree[a]);
-      const uint32_t vm = s.vmask[st][half];
-      const float* ksc = &s.kscale[st][half * 32];
-      float s2[32];
-      float ms = -INFINITY, mu = -INFINITY;
+      const float* ksc = &s.kscale[st][grp * KPG];
+      float s2[KPG];
+      float ms = -INFINITY;
+      uint32_t kbits = 0;                                // largest scale bits of the group's keys
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
+      for (int j = 0; j < KPG; ++j) {
         const float kj = ksc[j];
         const float v = (qs * kj * __uint_as_float(sn_[j]) + __uint_as_float(sr_[j])) * sl2;
-        const int ke = (int)((__float_as_uint(kj) >> 23) & 0xFF) - 127;
-        s2[j] = ((vm >> j) & 1u) ? v : -INFINITY;
+        s2[j] = (kj != 0.f) ? v : -INFINITY;
         ms = fmaxf(ms, s2[j]);
-        mu = fmaxf(mu, s2[j] + (float)ke);
+        kbits = max(kbits, __float_as_uint(kj));
       }
-      // row maxima over the whole tile: exchange with the other key half
-      s.xmax[xb][half][0][h] = ms;
-      s.xmax[xb][half][1][h] = mu;
+      // tile maxima (row score, scale exponent): exchange with the other key groups
+      s.xmax[xb][grp][0][h] = ms;
+      s.xmax[xb][grp][1][h] = __uint_as_float(kbits);
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.xbar[xb]);
       if (!mbar_wait_warp(&s.xbar[xb], (t >> 1) & 1, P.status, 10)) {
         live = false;
         break;
       }
-      ms = fmaxf(ms, s.xmax[xb][half ^ 1][0][h]);
-      mu = fmaxf(mu, s.xmax[xb][half ^ 1][1][h]);
-      const float Ms_new = fmaxf(Ms, ms), Mu_new = fmaxf(Mu, mu);
-      const float as = (Ms_new == -INFINITY) ? 1.f : exp2f(Ms - Ms_new);
-      const float au = (Mu_new == -INFINITY) ? 1.f : exp2f(Mu - Mu_new);
-      const float crow = (Mu_new == -INFINITY) ? 0.f : exp2f(Ms_new - Mu_new + 8.f);
-      float lsum = 0.f;
-      uint32_t phi[8], plo[8], pbf[16];
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float p0 = (s2[j] == -INFINITY) ? 0.f : exp2f(s2[j] - Ms_new);
-        const float p1 = (s2[j + 1] == -INFINITY) ? 0.f : exp2f(s2[j + 1] - Ms_new);
+      for (int o = 0; o < KG; ++o) {
+        ms = fmaxf(ms, s.xmax[xb][o][0][h]);
+        kbits = max(kbits, __float_as_uint(s.xmax[xb][o][1][h]));
+      }
+      const int kt = (int)((kbits >> 23) & 0xFF) - 127;      // exponent of the tile's largest scale
+      const bool upd = ms > Ms + kTau;
+      const float Ms_new = upd ? ms : Ms;
+      const int K_new = (kbits != 0 && kt > K) ? kt : K;
+      const float as = (upd && Ms != -INFINITY) ? ex2f(Ms - Ms_new) : 1.f;
+      const float cu_new =
+          (K_new == -1000) ? 0.f : exp2i(min(126, max(-126, 8 - (int)kTau - K_new)));
+      const float ak = (cu > 0.f && cu_new != cu) ? cu_new / cu : 1.f;   // exact: powers of two
+      const float ms_ref = (Ms_new == -INFINITY) ? 0.f : Ms_new;
+      float lsum = 0.f;
+      uint32_t phi[KPG / 4], plo[KPG / 4], pbf[KPG / 2];
+#pragma unroll
+      for (int j = 0; j < KPG; j += 2) {
+        const float p0 = ex2f(s2[j] - ms_ref), p1 = ex2f(s2[j + 1] - ms_ref);   // 0 for -inf
         lsum += p0 + p1;
-        const float u0 = p0 * ksc[j] * crow, u1 = p1 * ksc[j + 1] * crow;
+        const float u0 = p0 * ksc[j] * cu_new, u1 = p1 * ksc[j + 1] * cu_new;   // P' = P k_scale cu
         const uint32_t hi = e4m3x2(u0, u1);
         const float2 hf = e4m3x2_to_f32(hi);
         const uint32_t lo = e4m3x2(u0 - hf.x, u1 - hf.y);
-        const int sh = (j & 3) * 8;
         if ((j & 3) == 0) {
           phi[j >> 2] = hi;
           plo[j >> 2] = lo;
         } else {
-          phi[j >> 2] |= hi << sh;
-          plo[j >> 2] |= lo << sh;
+          phi[j >> 2] |= hi << 16;
+          plo[j >> 2] |= lo << 16;
         }
-        pbf[j >> 1] = (uint32_t)f32_to_bf16_bits(p0) | ((uint32_t)f32_to_bf16_bits(p1) << 16);
+        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+        pbf[j >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
       }
       l = l * as + lsum;
       // PV of the previous tile must be done before O or P change
@@ -574,18 +576,20 @@ __global__ void __launch_bounds__(NTHR, 1)
         break;
       }
       tc_fence_after();
-      // Rescale this warp's half of O (columns half*128 .. +127) when a running
-      // maximum grew.  tcgen05.ld / st are warp-wide (.sync.aligned): the
-      // decision is taken per warp, every lane takes part with its own factor.
-      const bool grow_u = __any_sync(0xffffffffu, wrote && au < 1.f);
-      const bool grow_s = __any_sync(0xffffffffu, wrote && dh == 1 && as < 1.f);
-      if (grow_u || grow_s) {
+      // Rescale this warp's share of O (columns grp*64 .. +63): the FP8 part
+      // by as*ak, the RoPE part by as.  tcgen05.ld / st are warp-wide
+      // (.sync.aligned): the decision is taken per warp, every lane takes part
+      // with its own factor.
+      const float an = as * ak;
+      const bool grow_n = __any_sync(0xffffffffu, wrote && an < 1.f);
+      const bool grow_r = __any_sync(0xffffffffu, wrote && dh == 1 && as < 1.f);
+      if (grow_n || grow_r) {
         const uint32_t ob = tmem + lane_off + 256;
-        for (int cc = 0; cc < 128; cc += 32) {
-          const int c = half * 128 + cc;
+        for (int cc = 0; cc < 256 / KG; cc += 32) {
+          const int c = grp * (256 / KG) + cc;
           const bool rope_cols = dh == 1 && c >= 192;
-          if (rope_cols ? !grow_s : !grow_u) continue;     // uniform across the warp
-          const float f = rope_cols ? as : au;
+          if (rope_cols ? !grow_r : !grow_n) continue;     // uniform across the warp
+          const float f = rope_cols ? as : an;
           uint32_t r[32];
           tmem_ld32_nowait(ob + c, r);
           tmem_ld_wait();
@@ -596,18 +600,14 @@ __global__ void __launch_bounds__(NTHR, 1)
         tmem_st_wait();
       }
       Ms = Ms_new;
-      Mu = Mu_new;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        *reinterpret_cast<uint4*>(s.p_hi + sw64(h, half * 32 + 16 * c)) =
-            make_uint4(phi[4 * c], phi[4 * c + 1], phi[4 * c + 2], phi[4 * c + 3]);
-        *reinterpret_cast<uint4*>(s.p_lo + sw64(h, half * 32 + 16 * c)) =
-            make_uint4(plo[4 * c], plo[4 * c + 1], plo[4 * c + 2], plo[4 * c + 3]);
-      }
+      K = K_new;
+      cu = cu_new;
+      *reinterpret_cast<uint4*>(s.p_hi + sw64(h, grp * KPG)) = make_uint4(phi[0], phi[1], phi[2], phi[3]);
+      *reinterpret_cast<uint4*>(s.p_lo + sw64(h, grp * KPG)) = make_uint4(plo[0], plo[1], plo[2], plo[3]);
       if (dh == 1) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(s.p_bf + sw128(h, half * 64 + 16 * c)) =
+        for (int c = 0; c < 2; ++c)
+          *reinterpret_cast<uint4*>(s.p_bf + sw128(h, grp * 2 * KPG + 16 * c)) =
               make_uint4(pbf[4 * c], pbf[4 * c + 1], pbf[4 * c + 2], pbf[4 * c + 3]);
       }
       fence_proxy_async_smem();
@@ -620,26 +620,27 @@ __global__ void __launch_bounds__(NTHR, 1)
     // ------------------------------------------------------------ epilogue
     bool fin = mbar_wait_warp(&s.ofinal, 0, P.status, 9);
     tc_fence_after();
-    // row sum of both key halves
-    if (half == 1) {
-      s.xl[h] = l;
+    // row sums of all key groups
+    if (grp > 0) {
+      s.xl[grp - 1][h] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.lbar);
     } else {
       fin = mbar_wait_warp(&s.lbar, 0, P.status, 11) && fin;
-      l += s.xl[h];
+#pragma unroll
+      for (int o = 0; o < KG - 1; ++o) l += s.xl[o][h];
     }
     fin = fin && live;
-    // O_nope is in units of 2^8 exp2(. - Mu); express it in units of exp2(. - Ms)
-    const float fn = (Ms == -INFINITY) ? 0.f : exp2f(Mu - 8.f - Ms);
+    // O_nope is in units of cu exp2(. - Ms); express it in units of exp2(. - Ms)
+    const float fn = (Ms == -INFINITY || cu == 0.f) ? 0.f : 1.f / cu;
     // O rows leave through a per-warp 32 x 32 staging block in shared memory
     // (the key stages are free once ofinal has fired), so that every global
     // store writes one 128-byte row segment.
     const uint32_t ob = tmem + lane_off + 256;
     float* stg = reinterpret_cast<float*>(&s.kv[0][0][0]) + (warp - 2) * (32 * 33);
     const int64_t row0 = pbase + quad * 32;
-    for (int cc = 0; cc < 128; cc += 32) {
-      const int c = half * 128 + cc;
+    for (int cc = 0; cc < 256 / KG; cc += 32) {
+      const int c = grp * (256 / KG) + cc;
       uint32_t r[32];
       tmem_ld32_nowait(ob + c, r);
       tmem_ld_wait();
@@ -654,7 +655,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         __syncwarp();
       }
     }
-    if (dh == 0 && half == 0 && h < P.H) {
+    if (dh == 0 && grp == 0 && h < P.H) {
       P.part_ml[(pbase + h) * 2] = (Ms == -INFINITY) ? -INFINITY : Ms * 0.6931471805599453f;
       P.part_ml[(pbase + h) * 2 + 1] = l;
     }
@@ -676,7 +677,7 @@ bool mqa_tc_supported(const MqaParams& P) {
   return P.kv_dtype == V4A_E4M3_BF16ROPE && P.d == 512 && P.d_rope == 64 && P.H <= 128 &&
          P.q_dtype == V4A_BF16 && !P.q_rmsnorm && P.split_keys % NK == 0 &&
          P.qbuf != nullptr && ((uintptr_t)P.qbuf & 15) == 0 &&
-         P.split_keys <= SKMAX && P.n_win <= 1024 && ((uintptr_t)P.kv & 15) == 0 &&
+         P.split_keys <= SKMAX && (!P.idx || P.split_keys <= SKMAX_SEL) && P.n_win <= 1024 && ((uintptr_t)P.kv & 15) == 0 &&
          (P.n_win == 0 || ((uintptr_t)P.swa & 15) == 0) && ((uintptr_t)P.Q & 15) == 0 &&
          (int64_t)P.B * P.kv_rows < (1ll << 31) && (int64_t)P.B * P.swa_rows < (1ll << 31);
 }
@@ -706,7 +707,7 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   }
   const int64_t grid = (int64_t)P.n_q * P.n_split * 2;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  mqa_tc_qprep_kernel<<<P.n_q, 512, 0, st>>>(P);
+  mqa_tc_qprep_kernel<<<dim3((unsigned)P.n_q, 8), 64, 0, st>>>(P);
   mqa_tc_kernel<<<(unsigned)grid, NTHR, smem, st>>>(P, m);
   return cudaGetLastError();
 }
