@@ -138,6 +138,21 @@ def graph_kernel_nodes(graph):
         return None
 
 
+def _index_traffic():
+    """DRAM bytes (read + write) per indexer launch from the committed ncu
+    capture, or None when the kernel's sources have changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "index_tc_pro_pair_1m_counters.json")
+    try:
+        rec = json.load(open(path))
+        h = hashlib.sha256()
+        for f in rec["sources"]:
+            h.update(open(os.path.join(ROOT, f), "rb").read())
+        return int(rec["dram_bytes_per_launch"]) if h.hexdigest() == rec["source_sha256"] else None
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 class ClockSampler:
     """SM clock and clock-event reasons sampled through NVML every few
     milliseconds from a host thread; only samples taken between ``start()``
@@ -392,7 +407,7 @@ def run_gpu(args, dist, rank, world):
         achieved = bytes_idx / (t_idx / 1e3) / 1e9
         roof = {"kernel": "index_scores (CSA indexer, MXFP4 keys)", "bound": "hbm",
                 "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": _index_traffic(),
                 "peak_source": peaks["source"], "launch_us": round(t_idx * 1e3, 2),
                 "algorithmic_bytes": int(bytes_idx)}
     step_bytes = sum(sum(vv for kk, vv in d.items() if kk in ("index", "mqa"))
