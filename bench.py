@@ -269,11 +269,17 @@ def capture_graph(fn):
     return g
 
 
+def _dist_device(dist):
+    import torch
+    return "cuda" if torch.cuda.is_available() and dist.get_backend() == "nccl" else "cpu"
+
+
 def max_over_ranks(x: float, dist):
+    """The largest of the ranks' values (every rank gets it)."""
     if dist is None:
         return x
     import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_dist_device(dist))
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -282,7 +288,29 @@ def barrier(dist):
     import torch
     if dist is not None:
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def rank_workload(name: str, rank: int):
+    """Rank r's share of a weak-scaling run: the workload's recipe at its own
+    batch size, drawn under a rank-specific seed, so that every rank holds
+    different sequences (global sequences r*B .. r*B+B-1); rank 0's draws are
+    those of a one-GPU run."""
+    import dataclasses
+    w = synth.WORKLOADS[name]
+    return w if rank == 0 else dataclasses.replace(w, seed=w.seed + 7919 * rank)
+
+
+def shard(rank: int, world: int, B: int):
+    """Global sequence ids of rank ``rank`` (weak scaling: B per rank)."""
+    assert 0 <= rank < world
+    return range(rank * B, (rank + 1) * B)
+
+
+def job_value(ms_max: float, B: int, world: int) -> float:
+    """Whole-job queries/s: every rank's B sequences in the slowest rank's time."""
+    return world * B / (ms_max / 1e3)
 
 
 # ------------------------------------------------------------------ the GPU arm
@@ -290,9 +318,9 @@ def barrier(dist):
 class Workload:
     """The decode layers of one workload on this GPU, captured as one graph."""
 
-    def __init__(self, name):
+    def __init__(self, name, rank: int = 0):
         import torch
-        self.w = synth.WORKLOADS[name]
+        self.w = rank_workload(name, rank)
         self.inputs = [synth.decode_layer_inputs(self.w, li) for li in range(len(self.w.layers))]
         self.layers = [build_decode_layer(self.w, li, inp) for li, inp in enumerate(self.inputs)]
         torch.cuda.synchronize()
@@ -363,7 +391,7 @@ def run_gpu(args, dist, rank, world):
     def flush():
         flush_buf.zero_()
 
-    wl = Workload(args.workload)
+    wl = Workload(args.workload, rank)
     launches = wl.launches_per_step()
     wl.capture()
     for _ in range(args.warmup):
@@ -380,7 +408,7 @@ def run_gpu(args, dist, rank, world):
     if args.profile:
         return dict(profile=True, ms=ms, launches=launches)
     q_step = wl.queries_per_step()
-    value = world * q_step / (ms / 1e3)
+    value = job_value(ms, q_step, world)
 
     # ---- dominant kernel: the indexer score kernel of the CSA layer, timed alone
     import long_context_compressed_kv_b200 as v
@@ -439,7 +467,7 @@ def run_gpu(args, dist, rank, world):
         del wl
         torch.cuda.empty_cache()
         for name in ALSO:
-            w2 = Workload(name)
+            w2 = Workload(name, rank)
             w2.capture()
             for _ in range(args.warmup):
                 flush()
