@@ -138,7 +138,7 @@ typedef struct {
  * then the top_k largest s_i (exact ties to the lower index), written in
  * ascending index order, -1 padded when n_vis < top_k.  */
 typedef struct {
-  int32_t n_q;                /* queries */
+  int32_t n_q;                /* queries, 1 .. 2^20 */
   int32_t B;                  /* sequences */
   const void* qI;             /* device MXFP4: uint8 [n_q][H_I][d_I/2]; F32: float [n_q][H_I][d_I] */
   const uint8_t* qI_sf;       /* device MXFP4: E8M0 [n_q][H_I][d_I/32]; else NULL */
@@ -165,7 +165,7 @@ typedef struct {
  *   o_h   = sum_j exp(s_hj) k_j / (exp(sink_h) + sum_j exp(s_hj))   (V = K)
  *   out   = o_h with its RoPE dims rotated by -p;  lse_h = log of the denominator.  */
 typedef struct {
-  int32_t n_q;
+  int32_t n_q;                /* queries, 1 .. 2^20 */
   int32_t B;
   const void* Q;              /* device [n_q][H][d] */
   int32_t q_dtype;            /* V4A_F32 or V4A_BF16 */
@@ -233,7 +233,11 @@ typedef struct {
 } v4attn_project_args;
 
 /* Bytes of workspace the calls below need for this layer, n_q queries and at
- * most max_vis visible entries per query (>= 256; includes the status word). */
+ * most max_vis visible entries per query (>= 256; includes the status word).
+ * index_topk and the MQA calls process their queries in chunks of 1024 (up to
+ * 2^20 queries per call), so the body of the workspace holds the scores or
+ * split-K partials of one chunk; the size grows with n_q only by 24 bytes per
+ * query beyond that. */
 size_t v4attn_workspace_size(const v4attn_layer_desc* desc, int32_t n_q, int64_t max_vis);
 
 /* Zero the workspace's status word (stream-ordered). */

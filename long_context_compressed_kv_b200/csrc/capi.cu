@@ -25,8 +25,14 @@ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 // call; the two never live at the same time (stream order), so they overlap.
 size_t dec_bytes(int32_t n_q) { return align_up((size_t)n_q * 3 * sizeof(int64_t)); }
 size_t body0(int32_t n_q) { return align_up(sizeof(WsHeader)) + dec_bytes(n_q); }
+// index_topk and the MQA calls walk their queries in chunks of kQChunk; the
+// scores / split-K partials of one chunk live in the workspace body, reused
+// by the next chunk in stream order.
+constexpr int32_t kQChunk = 1024;
+constexpr int32_t kMaxQueries = 1 << 20;   // queries per index_topk / MQA call
+inline int32_t q_chunk(int32_t n_q) { return std::min(n_q, kQChunk); }
 size_t index_need(int32_t n_q, int64_t max_vis) {
-  return align_up((size_t)n_q * (size_t)std::max<int64_t>(max_vis, 1) * sizeof(float));
+  return align_up((size_t)q_chunk(n_q) * (size_t)std::max<int64_t>(max_vis, 1) * sizeof(float));
 }
 size_t mqa_part_o_bytes(const v4attn_layer_desc* d, int32_t n_q, int n_split) {
   return align_up((size_t)n_q * n_split * d->H * d->d * sizeof(float));
@@ -40,7 +46,8 @@ size_t mqa_qbuf_bytes(const v4attn_layer_desc* d, int32_t n_q) {
 }
 size_t mqa_need(const v4attn_layer_desc* d, int32_t n_q, int64_t n_main_max) {
   const int S = mqa_num_splits(d, n_main_max);
-  return mqa_part_o_bytes(d, n_q, S) + mqa_part_ml_bytes(d, n_q, S) + mqa_qbuf_bytes(d, n_q);
+  const int32_t c = q_chunk(n_q);
+  return mqa_part_o_bytes(d, c, S) + mqa_part_ml_bytes(d, c, S) + mqa_qbuf_bytes(d, c);
 }
 size_t total_need(const v4attn_layer_desc* d, int32_t n_q, int64_t max_vis) {
   size_t body = mqa_need(d, n_q, max_vis);
@@ -138,7 +145,7 @@ v4attn_status run_compress(const v4attn_layer_desc* d, const v4attn_compress_arg
 v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args* a, void* ws,
                              size_t ws_bytes, cudaStream_t st) {
   if (d->kind != V4A_CSA) return V4A_ERR_INVALID_ARG;
-  if (!a || a->n_q < 1 || a->n_q > 65535 || a->B < 1) return V4A_ERR_INVALID_ARG;
+  if (!a || a->n_q < 1 || a->n_q > kMaxQueries || a->B < 1) return V4A_ERR_INVALID_ARG;
   if (!a->qI || !a->w || !a->q_pos || !a->keys || (!a->idx_out && !a->scores_out))
     return V4A_ERR_INVALID_ARG;
   if (d->idx_dtype == V4A_MXFP4 && (!a->qI_sf || !a->keys_sf)) return V4A_ERR_INVALID_ARG;
@@ -146,48 +153,55 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
   if (!ws) return V4A_ERR_WORKSPACE;
   if (ws_bytes < body0(a->n_q) + index_need(a->n_q, a->max_vis)) return V4A_ERR_WORKSPACE;
   uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
-  float* scores = a->scores_out ? a->scores_out : reinterpret_cast<float*>(w8 + body0(a->n_q));
   const int64_t ld = std::max<int64_t>(a->max_vis, 1);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
-  if (a->max_vis > 0) {
-    IndexParams P;
-    P.n_q = a->n_q;
-    P.B = a->B;
-    P.m = d->m;
-    P.H_I = d->H_I;
-    P.d_I = d->d_I;
-    P.idx_dtype = d->idx_dtype;
-    P.qI = a->qI;
-    P.qI_sf = a->qI_sf;
-    P.w = a->w;
-    P.q_seq = a->q_seq;
-    P.q_pos = a->q_pos;
-    P.keys = a->keys;
-    P.keys_sf = a->keys_sf;
-    P.key_rows = a->key_rows;
-    P.max_vis = a->max_vis;
-    P.scores = scores;
-    P.scores_ld = ld;
-    P.status = status;
-    cudaError_t e = index_scores_dispatch(P, st);
-    if (e != cudaSuccess) return V4A_ERR_CUDA;
+  const bool fp4 = d->idx_dtype == V4A_MXFP4;
+  const size_t qrow = fp4 ? (size_t)d->d_I / 2 : (size_t)d->d_I * sizeof(float);
+  for (int32_t q0 = 0; q0 < a->n_q; q0 += kQChunk) {
+    const int32_t cn = std::min(kQChunk, a->n_q - q0);
+    float* scores = a->scores_out ? a->scores_out + (int64_t)q0 * ld
+                                  : reinterpret_cast<float*>(w8 + body0(a->n_q));
+    if (a->max_vis > 0) {
+      IndexParams P;
+      P.n_q = cn;
+      P.B = a->B;
+      P.m = d->m;
+      P.H_I = d->H_I;
+      P.d_I = d->d_I;
+      P.idx_dtype = d->idx_dtype;
+      P.qI = reinterpret_cast<const uint8_t*>(a->qI) + (size_t)q0 * d->H_I * qrow;
+      P.qI_sf = fp4 ? a->qI_sf + (size_t)q0 * d->H_I * (d->d_I / 32) : nullptr;
+      P.w = a->w + (size_t)q0 * d->H_I;
+      P.q_seq = a->q_seq ? a->q_seq + q0 : nullptr;
+      P.q_base = q0;
+      P.q_pos = a->q_pos + q0;
+      P.keys = a->keys;
+      P.keys_sf = a->keys_sf;
+      P.key_rows = a->key_rows;
+      P.max_vis = a->max_vis;
+      P.scores = scores;
+      P.scores_ld = ld;
+      P.status = status;
+      if (index_scores_dispatch(P, st) != cudaSuccess) return V4A_ERR_CUDA;
+    }
+    if (!a->idx_out) continue;   // scores-only call
+    TopkParams T;
+    T.n_q = cn;
+    T.m = d->m;
+    T.k = d->top_k;
+    T.scores = scores;
+    T.scores_ld = ld;
+    T.max_vis = a->max_vis;
+    T.q_pos = a->q_pos + q0;
+    T.idx_out = a->idx_out + (int64_t)q0 * d->top_k;
+    if (topk_dispatch(T, st) != cudaSuccess) return V4A_ERR_CUDA;
   }
-  if (!a->idx_out) return V4A_OK;   // scores-only call
-  TopkParams T;
-  T.n_q = a->n_q;
-  T.m = d->m;
-  T.k = d->top_k;
-  T.scores = scores;
-  T.scores_ld = ld;
-  T.max_vis = a->max_vis;
-  T.q_pos = a->q_pos;
-  T.idx_out = a->idx_out;
-  return cuda_status(topk_dispatch(T, st));
+  return V4A_OK;
 }
 
 v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void* ws,
                       size_t ws_bytes, cudaStream_t st, bool sparse) {
-  if (!a || a->n_q < 1 || a->n_q > 65535 || a->B < 1) return V4A_ERR_INVALID_ARG;
+  if (!a || a->n_q < 1 || a->n_q > kMaxQueries || a->B < 1) return V4A_ERR_INVALID_ARG;
   if (!a->Q || !a->q_pos || !a->kv || !a->out) return V4A_ERR_INVALID_ARG;
   if (d->n_win > 0 && (!a->swa || a->swa_rows < d->n_win)) return V4A_ERR_INVALID_ARG;
   if (d->kv_dtype == V4A_E4M3_BF16ROPE && (!a->kv_scale || (d->n_win > 0 && !a->swa_scale)))
@@ -203,48 +217,54 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
   const int64_t n_main_max = sparse ? (int64_t)a->n_sel : a->max_vis;
   if (ws_bytes < body0(a->n_q) + mqa_need(d, a->n_q, n_main_max)) return V4A_ERR_WORKSPACE;
   uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
-  MqaParams P;
-  P.n_q = a->n_q;
-  P.B = a->B;
-  P.H = d->H;
-  P.d = d->d;
-  P.d_rope = d->d_rope;
-  P.n_win = d->n_win;
-  P.m = d->m;
-  P.theta = d->rope_theta;
-  P.scale = softmax_scale(d);
-  P.eps = d->rms_eps;
-  P.Q = a->Q;
-  P.q_dtype = a->q_dtype;
-  P.q_rmsnorm = a->q_rmsnorm;
-  P.q_seq = a->q_seq;
-  P.q_pos = a->q_pos;
-  P.kv_dtype = d->kv_dtype;
-  P.kv = reinterpret_cast<const uint8_t*>(a->kv);
-  P.kv_scale = a->kv_scale;
-  P.kv_rows = a->kv_rows;
-  P.swa = reinterpret_cast<const uint8_t*>(a->swa);
-  P.swa_scale = a->swa_scale;
-  P.swa_rows = a->swa_rows > 0 ? a->swa_rows : 1;
-  P.idx = sparse ? a->idx : nullptr;
-  P.n_sel = sparse ? a->n_sel : 0;
-  P.max_vis = sparse ? a->kv_rows : a->max_vis;
-  P.sink = a->sink;
-  P.split_keys = mqa_split_keys(d);
-  P.n_split = mqa_num_splits(d, n_main_max);
-  P.part_o = reinterpret_cast<float*>(w8 + body0(a->n_q));
-  P.part_ml = reinterpret_cast<float*>(w8 + body0(a->n_q) + mqa_part_o_bytes(d, a->n_q, P.n_split));
-  P.qbuf = mqa_qbuf_bytes(d, a->n_q)
-               ? w8 + body0(a->n_q) + mqa_part_o_bytes(d, a->n_q, P.n_split) +
-                     mqa_part_ml_bytes(d, a->n_q, P.n_split)
-               : nullptr;
-  P.out = a->out;
-  P.out_dtype = a->out_dtype;
-  P.lse = a->lse;
-  P.status = reinterpret_cast<uint32_t*>(ws);
-  cudaError_t e = mqa_dispatch(P, st);
-  if (e != cudaSuccess) return V4A_ERR_CUDA;
-  return cuda_status(launch_mqa_combine(P, st));
+  const int32_t c = q_chunk(a->n_q);
+  const size_t qb = (size_t)d->H * d->d * (a->q_dtype == V4A_BF16 ? 2 : 4);
+  const size_t ob = (size_t)d->H * d->d * (a->out_dtype == V4A_BF16 ? 2 : 4);
+  for (int32_t q0 = 0; q0 < a->n_q; q0 += kQChunk) {
+    MqaParams P;
+    P.n_q = std::min(kQChunk, a->n_q - q0);
+    P.B = a->B;
+    P.H = d->H;
+    P.d = d->d;
+    P.d_rope = d->d_rope;
+    P.n_win = d->n_win;
+    P.m = d->m;
+    P.theta = d->rope_theta;
+    P.scale = softmax_scale(d);
+    P.eps = d->rms_eps;
+    P.Q = reinterpret_cast<const uint8_t*>(a->Q) + (size_t)q0 * qb;
+    P.q_dtype = a->q_dtype;
+    P.q_rmsnorm = a->q_rmsnorm;
+    P.q_seq = a->q_seq ? a->q_seq + q0 : nullptr;
+    P.q_base = q0;
+    P.q_pos = a->q_pos + q0;
+    P.kv_dtype = d->kv_dtype;
+    P.kv = reinterpret_cast<const uint8_t*>(a->kv);
+    P.kv_scale = a->kv_scale;
+    P.kv_rows = a->kv_rows;
+    P.swa = reinterpret_cast<const uint8_t*>(a->swa);
+    P.swa_scale = a->swa_scale;
+    P.swa_rows = a->swa_rows > 0 ? a->swa_rows : 1;
+    P.idx = sparse ? a->idx + (int64_t)q0 * a->n_sel : nullptr;
+    P.n_sel = sparse ? a->n_sel : 0;
+    P.max_vis = sparse ? a->kv_rows : a->max_vis;
+    P.sink = a->sink;
+    P.split_keys = mqa_split_keys(d);
+    P.n_split = mqa_num_splits(d, n_main_max);
+    P.part_o = reinterpret_cast<float*>(w8 + body0(a->n_q));
+    P.part_ml =
+        reinterpret_cast<float*>(w8 + body0(a->n_q) + mqa_part_o_bytes(d, c, P.n_split));
+    P.qbuf = mqa_qbuf_bytes(d, c) ? w8 + body0(a->n_q) + mqa_part_o_bytes(d, c, P.n_split) +
+                                        mqa_part_ml_bytes(d, c, P.n_split)
+                                  : nullptr;
+    P.out = reinterpret_cast<uint8_t*>(a->out) + (size_t)q0 * ob;
+    P.out_dtype = a->out_dtype;
+    P.lse = a->lse ? a->lse + (int64_t)q0 * d->H : nullptr;
+    P.status = reinterpret_cast<uint32_t*>(ws);
+    if (mqa_dispatch(P, st) != cudaSuccess) return V4A_ERR_CUDA;
+    if (launch_mqa_combine(P, st) != cudaSuccess) return V4A_ERR_CUDA;
+  }
+  return V4A_OK;
 }
 
 // Block-wide copy of n bytes between non-overlapping buffers, 16 bytes per

@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // tiles per query, loaded in parallel, then a serial prefix over shared memory
   for (int q = threadIdx.x; q < P.n_q; q += NTHREADS) {
     int64_t nv = (P.q_pos[q] + 1) / P.m;
-    const int b = P.q_seq ? P.q_seq[q] : q;
+    const int b = P.q_seq ? P.q_seq[q] : P.q_base + q;
     if (b < 0 || b >= P.B) {
       flag(P.status, ST_BAD_SEQ);
       nv = 0;
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       locate(s, P.n_q, g, t);
       if (t.seg != seg_before) {
         // read once per query: a global load per tile would sit on the issue path
-        b = P.q_seq ? P.q_seq[t.q] : t.q;
+        b = P.q_seq ? P.q_seq[t.q] : P.q_base + t.q;
         const int j = t.seg & 1, uq = t.seg >> 1;
         if (uq >= 1 && !mbar_wait_warp(&s.qempty[j], (uq - 1) & 1, P.status)) {
           fail(s, P.status);

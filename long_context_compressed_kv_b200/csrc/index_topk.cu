@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(128) index_scores_simt(IndexParams P) {
   float* qs = sm;
   float* ws = sm + P.H_I * DI;
   const int q = blockIdx.y;
-  int b = P.q_seq ? P.q_seq[q] : q;
+  int b = P.q_seq ? P.q_seq[q] : P.q_base + q;
   const int64_t p = P.q_pos[q];
   int64_t nv = (p + 1) / P.m;
   if (b < 0 || b >= P.B) {

@@ -29,6 +29,7 @@ struct IndexParams {
   const uint8_t* qI_sf;
   const float* w;
   const int32_t* q_seq;
+  int q_base = 0;       // without q_seq, query q belongs to sequence q_base + q
   const int64_t* q_pos;
   const void* keys;
   const uint8_t* keys_sf;
@@ -56,6 +57,7 @@ struct MqaParams {
   const void* Q;
   int q_dtype, q_rmsnorm;
   const int32_t* q_seq;
+  int q_base = 0;       // without q_seq, query q belongs to sequence q_base + q
   const int64_t* q_pos;
   int kv_dtype;
   const uint8_t* kv;

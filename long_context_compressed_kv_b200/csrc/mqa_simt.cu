@@ -129,7 +129,7 @@ __device__ __forceinline__ int resolve_key(const MqaParams& P, int q, int b, int
 
 __device__ __forceinline__ void query_geometry(const MqaParams& P, int q, int& b, int64_t& p,
                                                int64_t& n_vis, int64_t& n_main, int& n_swa) {
-  b = P.q_seq ? P.q_seq[q] : q;
+  b = P.q_seq ? P.q_seq[q] : P.q_base + q;
   p = P.q_pos[q];
   n_vis = (p + 1) / P.m;
   if (b < 0 || b >= P.B) {

@@ -160,7 +160,7 @@ struct Geo {
 
 __device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
   Geo g;
-  g.b = P.q_seq ? P.q_seq[q] : q;
+  g.b = P.q_seq ? P.q_seq[q] : P.q_base + q;
   g.p = P.q_pos[q];
   g.n_vis = (g.p + 1) / P.m;
   if (g.b < 0 || g.b >= P.B) {

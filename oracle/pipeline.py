@@ -160,3 +160,122 @@ def tiny_layer(inp: dict, w, query_rows=None) -> dict:
         res["w"].append(wh)
         res["Q"].append(Q)
     return res
+
+
+PREFILL_COLS = ("Ca", "Cb", "Za", "Zb", "ICa", "ICb", "IZa", "IZb", "C", "Z")
+
+
+def prefill_columns(csa, hca) -> dict:
+    """Column range of each projected array in the prefill pair's projection
+    output: the CSA main arrays (Ca, Cb, Za, Zb; d columns each), the CSA
+    indexer arrays (ICa, ICb, IZa, IZb; d_I each), the HCA arrays (C, Z; d each)."""
+    widths = [csa.d] * 4 + [csa.d_I] * 4 + [hca.d] * 2
+    out, c0 = {}, 0
+    for nm, wd in zip(PREFILL_COLS, widths):
+        out[nm] = (c0, c0 + wd)
+        c0 += wd
+    return out
+
+
+def prefill_pair(w, x, W, qin_csa: dict, qin_hca: dict, query_rows) -> dict:
+    """Chunked prefill of a CSA + HCA layer pair ([deep-read] "CSA：4× 压缩之后再
+    top-k", "HCA：128× 压缩后保留 dense 全局视野"): the raw tokens x [L, d_model]
+    are projected by W into the compressor inputs of both layers; every
+    complete entry / indexer key is pooled from them and every token's window
+    KV is its own RMSNorm'd, RoPE'd C^a (R4); then each query at position
+    prefix + row (rows ``query_rows``) runs the indexer + top-k + sparse MQA
+    (CSA) and the dense MQA over all visible entries (HCA).  ``qin_csa`` /
+    ``qin_hca`` hold the per-query inputs of those rows, in that order.
+
+    Only the projections a query needs are formed: the indexer arrays and the
+    HCA arrays of every token, the CSA main arrays of the selected entries'
+    windows and of the window tokens.  Returns per-query lists plus, for every
+    CSA key, CSA entry and HCA entry that was formed, its stored (dequantised)
+    value and its value before coding."""
+    csa, hca = w.layers
+    x = np.asarray(x, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    cols = prefill_columns(csa, hca)
+    L = w.L
+    proj_cache = {}
+
+    def proj(nm, rows=None):
+        """Projection of array ``nm`` for token rows (all tokens when None)."""
+        c0, c1 = cols[nm]
+        if rows is None:
+            if nm not in proj_cache:
+                proj_cache[nm] = x @ W[:, c0:c1]
+            return proj_cache[nm]
+        return x[np.asarray(rows)] @ W[:, c0:c1]
+
+    def lookup(arr_rows, arr):
+        """(token -> row) view of a projection restricted to some tokens."""
+        pos = {int(t): i for i, t in enumerate(arr_rows)}
+        return lambda t: arr[np.vectorize(pos.__getitem__)(t)]
+
+    scale_c, scale_h = 1.0 / np.sqrt(csa.d), 1.0 / np.sqrt(hca.d)
+    # CSA indexer keys of every complete entry
+    n_csa = L // csa.m
+    ii = np.arange(n_csa)
+    keys = pool(ii, csa.m, True, L, proj("ICa"), proj("IZa"), qin_csa["ibias"],
+                proj("ICb"), proj("IZb"))
+    _, key_val = store_key(keys, csa)
+    # HCA entries of every complete block
+    n_hca = L // hca.m
+    jj = np.arange(n_hca)
+    hca_ent = finish_main(pool(jj, hca.m, False, L, proj("C"), proj("Z"), qin_hca["bias"]),
+                          jj, hca.m, hca.d_rope, hca.rope_theta)
+    _, hca_val = store_kv(hca_ent, hca)
+    out = {"hca_raw": hca_ent, "csa_raw": {}, "detail": []}
+    out.update({k: [] for k in ("positions", "scores", "idx", "csa_out", "csa_lse", "hca_out",
+                           "hca_lse", "csa_entries")})
+    out["key_val"] = key_val
+    out["key_raw"] = keys
+    out["hca_val"] = hca_val
+    csa_cache = {}
+    for r, row in enumerate(query_rows):
+        p = w.prefix + int(row)
+        out["positions"].append(p)
+        # ---- CSA: indexer, top-k, sparse MQA
+        nv = int(n_visible(p, csa.m))
+        _, qv = store_key(np.asarray(qin_csa["qI"][r], dtype=np.float64), csa)
+        s = index_scores(qv, qin_csa["w"][r], key_val[:nv])
+        idx = topk(s, nv, csa.top_k)
+        sel = idx[idx >= 0]
+        need = [i for i in sel.tolist() if i not in csa_cache]
+        if need:
+            need = np.asarray(need)
+            toks = np.unique(np.concatenate([np.arange(csa.m * (i - 1), csa.m * (i + 1))
+                                             for i in need]))
+            toks = toks[(toks >= 0) & (toks < L)]
+            arrs = {nm: lookup(toks, proj(nm, toks)) for nm in ("Ca", "Za", "Cb", "Zb")}
+            e = finish_main(pool(need, csa.m, True, L, arrs["Ca"], arrs["Za"], qin_csa["bias"],
+                                 arrs["Cb"], arrs["Zb"]), need, csa.m, csa.d_rope, csa.rope_theta)
+            _, ev = store_kv(e, csa)
+            for i, v, raw in zip(need.tolist(), ev, e):
+                csa_cache[i] = v
+                out["csa_raw"][i] = raw
+        wt = window_tokens(p, csa.n_win)
+        _, swa_c = store_kv(token_kv(proj("Ca", wt), wt, csa), csa)
+        keys_c = np.concatenate([np.stack([csa_cache[i] for i in sel.tolist()])
+                                 if len(sel) else np.zeros((0, csa.d)), swa_c], axis=0)
+        q = prepare_query(qin_csa["Q"][r], p, csa.d_rope, csa.rope_theta, csa.kv_fp8)
+        o, lse, a_c, _ = attend(q, keys_c, scale_c, qin_csa["sink"], return_weights=True)
+        det = dict(csa_sel=sel, csa_win=wt, csa_keys=keys_c, csa_q=q, csa_a=a_c, csa_o=o)
+        out["scores"].append(s)
+        out["idx"].append(idx)
+        out["csa_out"].append(finish_output(o, p, csa.d_rope, csa.rope_theta))
+        out["csa_lse"].append(lse)
+        # ---- HCA: dense MQA over the visible entries + window
+        nvh = int(n_visible(p, hca.m))
+        wt = window_tokens(p, hca.n_win)
+        _, swa_h = store_kv(token_kv(proj("C", wt), wt, hca), hca)
+        keys_h = np.concatenate([hca_val[:nvh], swa_h], axis=0)
+        qh = prepare_query(qin_hca["Q"][r], p, hca.d_rope, hca.rope_theta, hca.kv_fp8)
+        o, lse, a_h, _ = attend(qh, keys_h, scale_h, qin_hca["sink"], return_weights=True)
+        det.update(hca_n=nvh, hca_win=wt, hca_keys=keys_h, hca_q=qh, hca_a=a_h, hca_o=o)
+        out["detail"].append(det)
+        out["hca_out"].append(finish_output(o, p, hca.d_rope, hca.rope_theta))
+        out["hca_lse"].append(lse)
+    out["csa_entries"] = csa_cache
+    return out

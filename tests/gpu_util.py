@@ -111,6 +111,58 @@ def check_topk(gpu_idx, oracle_scores, n_vis, k, extra_tol=None):
     return len(diff) // 2
 
 
+def check_coded_row(got, ref, ref_raw, d_rope=64, what=""):
+    """One stored E4M3 + bf16 row against the oracle's coded row.  Codes may
+    differ only where the two sides took a rounding decision differently: the
+    oracle's value before coding lies within 1e-4 relative of the midpoint of
+    the two decoded values (fp32 pooling against fp64 pooling), and such
+    flips are rare; a changed power-of-two scale is allowed only when the
+    oracle's amax / 448 lies within 1e-4 (log2) of a power of two."""
+    got, ref, raw = (np.asarray(a, dtype=np.float64) for a in (got, ref, ref_raw))
+    if r16(got, ref) <= R16_TOL:
+        return
+    dn = len(raw) - d_rope
+    t = np.max(np.abs(raw[:dn])) / codecs.E4M3_MAX
+    if t > 0 and abs(np.log2(t) - np.round(np.log2(t))) < 1e-4:
+        assert r16(got, ref) <= 8 * R16_TOL, (what, "scale boundary", r16(got, ref))
+        return
+    d = got != ref
+    mid = 0.5 * (got + ref)
+    near = np.abs(raw - mid) <= 1e-4 * np.maximum(np.abs(raw), 1e-6)
+    assert np.all(near[d]), (what, "code differs away from a rounding midpoint",
+                             np.flatnonzero(d & ~near)[:8])
+    assert d.mean() < 0.01, (what, "too many flipped codes", int(d.sum()))
+
+
+def coding_bound(keys_ref, keys_gpu, a, q, o, scale, d_rope=64):
+    """First-order bound on how much the MQA output of one query moves when
+    its key rows change from the oracle's codes (keys_ref [n, d]) to the
+    codes the GPU stored (keys_gpu), both valid roundings of nearly equal
+    values: |do_h| <= sum_j a_hj |dk_j| + sum_j a_hj |k_j - o_h| scale |q_h . dk_j|
+    (V = K), with a [H, n] the oracle's attention weights and o [H, d] its
+    output before the inverse RoPE.  The RoPE dims are rotated afterwards, so
+    a pair gets the larger bound of its two dims times sqrt(2).  [H, d]."""
+    dk = np.asarray(keys_gpu, np.float64) - np.asarray(keys_ref, np.float64)
+    rows = np.flatnonzero(np.any(dk != 0, axis=1))
+    b = np.zeros_like(np.asarray(o, np.float64))
+    if len(rows) == 0:
+        return b
+    dk, kr, ar = dk[rows], np.asarray(keys_ref, np.float64)[rows], np.asarray(a)[:, rows]
+    ds = scale * np.abs(np.asarray(q, np.float64) @ dk.T)                 # [H, m]
+    b = ar @ np.abs(dk) + np.einsum("hm,hmd->hd", ar * ds, np.abs(kr[None] - o[:, None, :]))
+    dn = b.shape[1] - d_rope
+    pair = np.maximum(b[:, dn::2], b[:, dn + 1::2]) * np.sqrt(2.0)
+    b[:, dn::2] = pair
+    b[:, dn + 1::2] = pair
+    return b
+
+
+def r16_excess(got, ref, bound):
+    """max(|got - ref| - bound, 0) over the RMS of ref."""
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    return float(np.max(np.maximum(np.abs(got - ref) - bound, 0.0)) / np.sqrt(np.mean(ref * ref)))
+
+
 class DecodeState:
     """The decode layer exactly as bench.py builds and times it (coded synthetic
     history, window ring, tail rings, queries), plus what the checks need."""
