@@ -267,42 +267,6 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
   return V4A_OK;
 }
 
-// Block-wide copy of n bytes between non-overlapping buffers, 16 bytes per
-// thread and step when both ends and n allow it.
-__device__ __forceinline__ void copy_bytes(uint8_t* __restrict__ dst,
-                                           const uint8_t* __restrict__ src, int64_t n) {
-  if (((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src) | (uintptr_t)n) & 15) == 0) {
-    const uint4* s = reinterpret_cast<const uint4*>(src);
-    uint4* d = reinterpret_cast<uint4*>(dst);
-    for (int64_t e = threadIdx.x; e < n / 16; e += blockDim.x) d[e] = s[e];
-  } else {
-    for (int64_t e = threadIdx.x; e < n; e += blockDim.x) dst[e] = src[e];
-  }
-}
-
-__global__ void decode_prep_kernel(int B, const int64_t* pos, int m, int ring, int n_arr, int d,
-                                   const void* x_main, void* tail, int in_elt, int dI,
-                                   const void* x_idx, void* itail, int64_t* lens, int64_t* eb_tok,
-                                   int64_t* eb_ent) {
-  const int b = blockIdx.x;
-  const int64_t p = pos[b];
-  if (threadIdx.x == 0) {
-    lens[b] = p + 1;
-    eb_tok[b] = p;
-    eb_ent[b] = p / m;
-  }
-  const int64_t slot = p % ring;
-  const int64_t nb = (int64_t)n_arr * d * in_elt;
-  const uint8_t* src = reinterpret_cast<const uint8_t*>(x_main) + b * nb;
-  uint8_t* dst = reinterpret_cast<uint8_t*>(tail) + ((int64_t)b * ring + slot) * nb;
-  copy_bytes(dst, src, nb);
-  if (x_idx) {
-    const int64_t ni = (int64_t)4 * dI * in_elt;
-    const uint8_t* s2 = reinterpret_cast<const uint8_t*>(x_idx) + b * ni;
-    uint8_t* d2 = reinterpret_cast<uint8_t*>(itail) + ((int64_t)b * ring + slot) * ni;
-    copy_bytes(d2, s2, ni);
-  }
-}
 
 }  // namespace
 
@@ -363,90 +327,53 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
     return V4A_ERR_INVALID_ARG;
   if (!ws) return V4A_ERR_WORKSPACE;
   if (ws_bytes < total_need(desc, a->B, a->max_vis)) return V4A_ERR_WORKSPACE;
-  uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
-  int64_t* lens = reinterpret_cast<int64_t*>(w8 + align_up(sizeof(WsHeader)));
-  int64_t* eb_tok = lens + a->B;
-  int64_t* eb_ent = eb_tok + a->B;
   const int m = desc->m;
   const int ring = csa ? 2 * m : m;
   const int n_arr = csa ? 4 : 2;
   const int d = desc->d;
   const int elt = a->in_dtype == V4A_F32 ? 4 : 2;
-  decode_prep_kernel<<<a->B, 256, 0, stream>>>(a->B, a->pos, m, ring, n_arr, d, a->x_main,
-                                               a->tail, elt, desc->d_I, csa ? a->x_idx : nullptr,
-                                               a->itail, lens, eb_tok, eb_ent);
-  if (cudaGetLastError() != cudaSuccess) return V4A_ERR_CUDA;
-
-  // 1. window KV of the new token (RMSNorm, RoPE at p, stored format)
-  v4attn_compress_args c{};
-  c.m = 1;
-  c.overlap = 0;
-  c.c = d;
-  c.B = a->B;
-  c.Ca = a->x_main;
-  c.in_dtype = a->in_dtype;
-  c.in_seq_stride = (int64_t)n_arr * d;
-  c.in_row_stride = (int64_t)n_arr * d;
-  c.in_rows = 1;
-  c.seq_len = lens;
-  c.entry_begin = eb_tok;
-  c.n_entries = 1;
-  c.apply_rmsnorm = 1;
-  c.apply_rope = 1;
-  c.out_dtype = desc->kv_dtype;
-  c.out = a->swa;
-  c.out_scale = a->swa_scale;
-  c.out_rows = a->swa_rows;
-  s = run_compress(desc, &c, stream);
-  if (s != V4A_OK) return s;
-  // 2. the completed block's entry (and indexer key) from the tail rings
-  const uint8_t* tail = reinterpret_cast<const uint8_t*>(a->tail);
-  v4attn_compress_args e{};
-  e.m = m;
-  e.overlap = csa ? 1 : 0;
-  e.c = d;
-  e.B = a->B;
-  e.Ca = tail;
-  e.Za = tail + (size_t)d * elt;
-  e.Cb = csa ? tail + (size_t)2 * d * elt : nullptr;
-  e.Zb = csa ? tail + (size_t)3 * d * elt : nullptr;
-  e.in_dtype = a->in_dtype;
-  e.in_seq_stride = (int64_t)ring * n_arr * d;
-  e.in_row_stride = (int64_t)n_arr * d;
-  e.in_rows = ring;
-  e.bias = a->bias;
-  e.seq_len = lens;
-  e.entry_begin = eb_ent;
-  e.n_entries = 1;
-  e.complete_only = 1;
-  e.apply_rmsnorm = 1;
-  e.apply_rope = 1;
-  e.out_dtype = desc->kv_dtype;
-  e.out = a->kv;
-  e.out_scale = a->kv_scale;
-  e.out_rows = a->kv_rows;
-  s = run_compress(desc, &e, stream);
-  if (s != V4A_OK) return s;
+  {
+    // channel pairs are read as one 2-element load
+    const uintptr_t al = 2 * (uintptr_t)elt;
+    for (const void* p : {a->x_main, (const void*)a->tail, a->x_idx, (const void*)a->itail})
+      if (p && (reinterpret_cast<uintptr_t>(p) % al)) return V4A_ERR_INVALID_ARG;
+    for (const void* p : {(const void*)a->bias, (const void*)a->ibias})
+      if (p && (reinterpret_cast<uintptr_t>(p) % 8)) return V4A_ERR_INVALID_ARG;
+  }
+  // 1.-2. tail rings, the new token's window KV (RMSNorm, RoPE at p), the
+  // entry (and indexer key) its block completes: one launch
+  AppendParams A;
+  A.B = a->B;
+  A.csa = csa ? 1 : 0;
+  A.pos = a->pos;
+  A.in_dtype = a->in_dtype;
+  A.x_main = a->x_main;
+  A.tail = a->tail;
+  A.m = m;
+  A.ring = ring;
+  A.n_arr = n_arr;
+  A.d = d;
+  A.bias = a->bias;
+  A.x_idx = csa ? a->x_idx : nullptr;
+  A.itail = csa ? a->itail : nullptr;
+  A.dI = desc->d_I;
+  A.ibias = a->ibias;
+  A.kv_dtype = desc->kv_dtype;
+  A.idx_dtype = desc->idx_dtype;
+  A.d_rope = desc->d_rope;
+  A.theta = desc->rope_theta;
+  A.eps = desc->rms_eps;
+  A.swa = a->swa;
+  A.swa_scale = a->swa_scale;
+  A.swa_rows = a->swa_rows;
+  A.kv = a->kv;
+  A.kv_scale = a->kv_scale;
+  A.kv_rows = a->kv_rows;
+  A.keys = csa ? a->keys : nullptr;
+  A.keys_sf = csa ? a->keys_sf : nullptr;
+  A.key_rows = csa ? a->key_rows : 0;
+  if (launch_decode_append(A, stream) != cudaSuccess) return V4A_ERR_CUDA;
   if (csa) {
-    const uint8_t* it = reinterpret_cast<const uint8_t*>(a->itail);
-    const int dI = desc->d_I;
-    v4attn_compress_args k = e;
-    k.c = dI;
-    k.Ca = it;
-    k.Za = it + (size_t)dI * elt;
-    k.Cb = it + (size_t)2 * dI * elt;
-    k.Zb = it + (size_t)3 * dI * elt;
-    k.in_seq_stride = (int64_t)ring * 4 * dI;
-    k.in_row_stride = (int64_t)4 * dI;
-    k.bias = a->ibias;
-    k.apply_rmsnorm = 0;
-    k.apply_rope = 0;
-    k.out_dtype = desc->idx_dtype;
-    k.out = a->keys;
-    k.out_scale = a->keys_sf;
-    k.out_rows = a->key_rows;
-    s = run_compress(desc, &k, stream);
-    if (s != V4A_OK) return s;
     // 3. indexer + top-k
     v4attn_index_args ix{};
     ix.n_q = a->B;

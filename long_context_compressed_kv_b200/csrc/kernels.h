@@ -21,6 +21,36 @@ struct CompressParams {
   int64_t out_rows;
   int d_rope;
   float theta, eps;
+  // decode: the token at position new_pos[b] is read from the *_new arrays
+  // (row b at new_seq_stride) instead of the input ring; seq_len / entry_begin
+  // may instead be derived from new_pos (L = p + 1; entry p for m = 1, p / m
+  // otherwise) when the pointers are null
+  const int64_t* new_pos = nullptr;
+  const void *Ca_new = nullptr, *Za_new = nullptr, *Cb_new = nullptr, *Zb_new = nullptr;
+  int64_t new_seq_stride = 0;
+};
+
+// One decode step's appends (see decode_append_kernel).
+struct AppendParams {
+  int B, csa;
+  const int64_t* pos;
+  int in_dtype;                               // of x_main / tail / x_idx / itail
+  const void* x_main;                         // [B][n_arr][d]
+  void* tail;                                 // [B][ring][n_arr][d]
+  int m, ring, n_arr, d;
+  const float* bias;
+  const void* x_idx;                          // CSA: [B][4][dI]
+  void* itail;                                // CSA: [B][ring][4][dI]
+  int dI;
+  const float* ibias;
+  int kv_dtype, idx_dtype, d_rope;
+  float theta, eps;
+  void *swa, *swa_scale;
+  int64_t swa_rows;
+  void *kv, *kv_scale;
+  int64_t kv_rows;
+  void *keys, *keys_sf;
+  int64_t key_rows;
 };
 
 struct IndexParams {
@@ -94,6 +124,7 @@ struct ProjectParams {
 };
 
 cudaError_t launch_compress(const CompressParams& P, int B, int n_entries, cudaStream_t st);
+cudaError_t launch_decode_append(const AppendParams& A, cudaStream_t st);
 cudaError_t launch_index_scores(const IndexParams& P, cudaStream_t st);
 cudaError_t launch_topk(const TopkParams& P, cudaStream_t st);
 cudaError_t launch_mqa_simt(const MqaParams& P, cudaStream_t st);
