@@ -288,30 +288,59 @@ cudaError_t launch_mqa_simt(const MqaParams& P, cudaStream_t st) {
 
 // ---------------------------------------------------------------- combine
 // One CTA per (head, query); thread k owns the output pair (2k, 2k+1).
+// One CTA per (head, query): merge the split partials with their running
+// maxima, add the sink to the denominator, rotate the RoPE dims back by -p,
+// cast.  The splits' (m, l) pairs are read into shared memory in parallel and
+// the partial rows with 8 independent loads in flight per thread.
 __global__ void mqa_combine_kernel(MqaParams P) {
+  extern __shared__ float wgt[];                       // [n_split]
+  __shared__ float red[32];
   const int h = blockIdx.x, q = blockIdx.y;
   const int k = threadIdx.x;
   const int64_t p = P.q_pos[q];
   const int64_t pbase = (int64_t)q * P.n_split * P.H;
-  float M = -INFINITY;
-  for (int s = 0; s < P.n_split; ++s) M = fmaxf(M, P.part_ml[((pbase + (int64_t)s * P.H) + h) * 2]);
+  const int S = P.n_split;
+  // splits' maxima -> M
+  float mloc = -INFINITY;
+  for (int s = k; s < S; s += blockDim.x) {
+    const float ms = P.part_ml[((pbase + (int64_t)s * P.H) + h) * 2];
+    wgt[s] = ms;
+    mloc = fmaxf(mloc, ms);
+  }
   const float z = P.sink ? P.sink[h] : -INFINITY;
+  float M = block_max(mloc, red);
   M = fmaxf(M, z);
-  float o0 = 0.f, o1 = 0.f, den = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < P.n_split; ++s) {
-      const int64_t r = (pbase + (int64_t)s * P.H) + h;
-      const float ms = P.part_ml[r * 2];
-      if (ms == -INFINITY) continue;
-      const float wgt = __expf(ms - M);
-      den += P.part_ml[r * 2 + 1] * wgt;
-      if (2 * k < P.d) {
-        const float2 v = reinterpret_cast<const float2*>(P.part_o + r * P.d)[k];
-        o0 = fmaf(v.x, wgt, o0);
-        o1 = fmaf(v.y, wgt, o1);
+  // weights exp(m_s - M) and the denominator
+  float dloc = 0.f;
+  for (int s = k; s < S; s += blockDim.x) {
+    const float ms = wgt[s];
+    const float w = (ms == -INFINITY || M == -INFINITY) ? 0.f : __expf(ms - M);
+    wgt[s] = w;
+    dloc += w * P.part_ml[((pbase + (int64_t)s * P.H) + h) * 2 + 1];
+  }
+  float den = block_sum(dloc, red);
+  if (P.sink && M != -INFINITY) den += __expf(z - M);
+  float o0 = 0.f, o1 = 0.f;
+  if (2 * k < P.d && M != -INFINITY) {
+    const float2* base = reinterpret_cast<const float2*>(P.part_o + (pbase + h) * P.d) + k;
+    const int64_t step = (int64_t)P.H * P.d / 2;           // float2 between splits
+    int s = 0;
+    for (; s + 8 <= S; s += 8) {
+      float2 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = wgt[s + u] != 0.f ? base[(s + u) * step] : make_float2(0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        o0 = fmaf(v[u].x, wgt[s + u], o0);
+        o1 = fmaf(v[u].y, wgt[s + u], o1);
       }
     }
-    if (P.sink) den += __expf(z - M);
+    for (; s < S; ++s)
+      if (wgt[s] != 0.f) {
+        const float2 v = base[s * step];
+        o0 = fmaf(v.x, wgt[s], o0);
+        o1 = fmaf(v.y, wgt[s], o1);
+      }
   }
   const float inv = den > 0.f ? 1.0f / den : 0.f;
   o0 *= inv;
@@ -340,7 +369,14 @@ __global__ void mqa_combine_kernel(MqaParams P) {
 cudaError_t launch_mqa_combine(const MqaParams& P, cudaStream_t st) {
   int threads = ((P.d / 2 + 31) / 32) * 32;
   dim3 grid(P.H, P.n_q);
-  mqa_combine_kernel<<<grid, threads, 0, st>>>(P);
+  const size_t smem = (size_t)P.n_split * sizeof(float);
+  if (smem > 200 * 1024) return cudaErrorInvalidValue;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(mqa_combine_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  mqa_combine_kernel<<<grid, threads, smem, st>>>(P);
   return cudaGetLastError();
 }
 
