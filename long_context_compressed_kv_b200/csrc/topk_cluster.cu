@@ -5,7 +5,8 @@
 // query; Flash k = 512, Pro k = 1024).  Ties go to the lower index and the
 // selection is written in ascending index order, -1 padded.
 //
-// The 8 CTAs of a cluster split the query's visible scores into slices and
+// The 16 (or, where a 16-CTA cluster cannot be resident, 8) CTAs of a
+// cluster split the query's visible scores into slices and
 // keep their slice in shared memory (as order-preserving uint32 keys).  A
 // cluster-wide min / max first finds the key bits that every visible score
 // shares; an exact radix select then resolves the remaining bits 8 at a time.
@@ -32,7 +33,7 @@
 namespace v4a {
 
 namespace {
-constexpr int CL = 8;             // CTAs per cluster = slices per query
+constexpr int CL_MAX = 16;        // CTAs per cluster = slices per query (8 or 16, set at launch)
 constexpr int TPB = 512;          // threads per CTA
 constexpr int CACHE = 32768;      // keys a CTA keeps in shared memory (+1/64 padding)
 constexpr int PAD_CACHE = CACHE + CACHE / 64;
@@ -86,8 +87,7 @@ __device__ __forceinline__ uint32_t high_mask(int bits) {   // the top `bits` bi
 }
 }  // namespace
 
-__global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(TPB, 1)
-    topk_cluster_kernel(TopkParams P) {
+__global__ void __launch_bounds__(TPB, 1) topk_cluster_kernel(TopkParams P) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(16) uint32_t dyn[];
@@ -103,6 +103,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(TPB, 1)
   __shared__ uint32_t mm[2];                    // this CTA's (min, max) key, read by the cluster
   __shared__ int cnt[2];                        // this CTA's (#gt, #eq), read by the cluster
   const uint32_t rank = cluster_rank();
+  const int CL = (int)cluster.num_blocks();
   const int q = blockIdx.x / CL;
   const int lane = threadIdx.x & 31;
   int64_t nv64 = (P.q_pos[q] + 1) / P.m;
@@ -174,7 +175,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(TPB, 1)
   if (threadIdx.x < 32) {
     // lanes 0..CL-1 read one CTA's (min, max) each
     uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
-    if (threadIdx.x < CL) {
+    if ((int)threadIdx.x < CL) {
       const uint32_t* rm = cluster.map_shared_rank(mm, (unsigned)threadIdx.x);
       gmin = rm[0];
       gmax = rm[1];
@@ -357,17 +358,49 @@ bool topk_cluster_supported(const TopkParams& P) { return P.n_q <= (1 << 20); }
 
 cudaError_t launch_topk_cluster(const TopkParams& P, cudaStream_t st) {
   const size_t smem = SMEM_WORDS * sizeof(uint32_t);
-  static unsigned long long configured = 0;
+  static int cluster_size[64] = {0};                 // per device: 16 if it can be resident, else 8
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !(configured & (1ull << dev))) {
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  if (!cluster_size[dev]) {
     cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    configured |= 1ull << dev;
+    int cs = 8;
+    if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                             1) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(CL_MAX, 1, 1);
+      cfg.blockDim = dim3(TPB, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = CL_MAX;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel, &cfg) == cudaSuccess && n >= 1)
+        cs = CL_MAX;
+    }
+    cudaGetLastError();                              // a refused query leaves the portable size
+    cluster_size[dev] = cs;
   }
-  topk_cluster_kernel<<<P.n_q * CL, TPB, smem, st>>>(P);
-  return cudaGetLastError();
+  const int CL = cluster_size[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(P.n_q * CL), 1, 1);
+  cfg.blockDim = dim3(TPB, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, P);
 }
 
 }  // namespace v4a
