@@ -387,9 +387,14 @@ def run_gpu(args, dist, rank, world):
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     stream = torch.cuda.current_stream()
     flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_sink = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     def flush():
+        # write a buffer larger than L2, then read it back: the step starts with
+        # nothing of its own in L2 and with no dirty line whose write-back it
+        # would otherwise pay for
         flush_buf.zero_()
+        flush_sink.copy_(flush_buf.view(torch.int32).amax().view(1))
 
     wl = Workload(args.workload, rank)
     launches = wl.launches_per_step()
@@ -611,7 +616,7 @@ def main():
                        "layers": [f"{ly.kind} m={ly.m} H={ly.H} d={ly.d}" +
                                   (f" top_k={ly.top_k} H_I={ly.H_I}x{ly.d_I}" if ly.kind == "csa"
                                    else "") for ly in w.layers],
-                       "l2": "flushed between steps (320 MB write)",
+                       "l2": "flushed between steps (320 MB write, then read back: cold and clean)",
                        "parallelism": f"dp{world} (independent sequences)",
                        "graph": "one CUDA graph per step"},
             "e2e": {"value": round(res["e2e"]["value"], 1), "unit": "queries/s",

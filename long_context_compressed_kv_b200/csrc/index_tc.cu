@@ -12,11 +12,15 @@
 // multi-stage TMA ring (64-byte-swizzled K-major tiles); B (the query's H_I x
 // 128 codes) stays in shared memory for the query's whole key range; the E8M0
 // scales of both go to TMEM with tcgen05.cp (row m at lane m % 32 of every
-// sub-partition, column m / 32, byte = 32-element block).  The accumulator is
-// double-buffered in TMEM so the epilogue of tile i overlaps the MMA of tile
-// i+1.  Roles: warp 0 TMA producer, warp 1 MMA issuer (one lane), warps 2..5
-// epilogue (one thread per key row).  The kernel is HBM-bound: 68 bytes per key
-// against 16384 FP4 FLOP.
+// sub-partition, column m / 32, byte = 32-element block).  A ring stage holds up
+// to four consecutive 128-key tiles of one query (32 KB): on this part a
+// streaming read over one stage per barrier round trip reaches HBM speed only
+// from about 32 KB per stage on, while the work is still split between CTAs
+// tile by tile.  The accumulator has several TMEM stages so the epilogue of
+// tile i overlaps the MMAs of the tiles after it.  Roles: warp 0 TMA producer,
+// warp 1 MMA issuer (one lane), warps 2..5 and 6..9 two epilogue groups on
+// alternate tiles (one thread per key row).  The kernel is HBM-bound: 68 bytes
+// per key against 16384 FP4 FLOP.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -28,19 +32,27 @@ namespace {
 
 constexpr int KT = 128;                 // keys per tile (MMA M)
 constexpr int KROW = 64;                // bytes per key row (128 E2M1)
-constexpr int STAGES = 12;
+constexpr int TPS = 4;                  // tiles per ring stage (32 KB of key codes)
+constexpr int STAGES = 5;
 constexpr int KTILE_BYTES = KT * KROW;  // 8 KB
 constexpr int SF_BYTES = 512;           // 128 rows x 4 scale bytes
 constexpr int MAXQ = 1024;              // queries per launch on this path
 constexpr int EPI_GROUPS = 2;           // epilogue warp groups, alternating tiles
 constexpr int NTHREADS = 64 + EPI_GROUPS * 128;
-constexpr int MAX_ACC = 4;              // accumulator stages in TMEM
+constexpr int MAX_ACC = 8;              // accumulator stages in TMEM
+constexpr uint32_t TM_COLS = 512;
+
+// accumulator stages that fit in 512 TMEM columns next to their key scales (4
+// columns each) and the two query-scale slots (4 columns each)
+__host__ __device__ constexpr int n_acc(int N) {
+  return (512 - 8) / (N + 4) < MAX_ACC ? (512 - 8) / (N + 4) : MAX_ACC;
+}
 
 struct Smem {
-  alignas(1024) uint8_t keys[STAGES][KTILE_BYTES];
+  alignas(1024) uint8_t keys[STAGES][TPS][KTILE_BYTES];
   alignas(1024) uint8_t q[2][128 * KROW];
-  alignas(128) uint8_t sfa[STAGES][SF_BYTES];      // scale-factor order (tcgen05.cp source)
-  alignas(128) uint32_t sfa_raw[STAGES][KT];        // key scales as loaded (row-major)
+  alignas(128) uint8_t sfa[MAX_ACC][SF_BYTES];      // scale-factor order, per accumulator
+  alignas(128) uint32_t sfa_raw[STAGES][TPS * KT];  // key scales as loaded (row-major)
   alignas(128) uint8_t sfb[2][SF_BYTES];
   alignas(128) uint32_t sfb_raw[2][128];
   alignas(16) float w[2][128];
@@ -73,6 +85,14 @@ __device__ __forceinline__ void locate(const Smem& s, int n_q, int g, TileIter& 
   t.lt = g - s.tile_prefix[t.q];
 }
 
+// Tiles in the stage that starts at tile g: up to TPS, all of one query, all
+// inside this CTA's range.  Every role walks the stages with this same rule.
+__device__ __forceinline__ int stage_tiles(const Smem& s, const TileIter& t, int g, int g1) {
+  const int to_seg = s.tile_prefix[t.q + 1] - g, to_end = g1 - g;
+  const int n = to_seg < to_end ? to_seg : to_end;
+  return n < TPS ? n : TPS;
+}
+
 template <int N>   // indexer heads = MMA N
 __global__ void __launch_bounds__(NTHREADS, 1)
     index_tc_kernel(IndexParams P, const __grid_constant__ CUtensorMap tm_keys,
@@ -81,8 +101,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   Smem& s = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NACC = (4 * N + 24 <= 512) ? 4 : 2;        // accumulator stages
-  constexpr uint32_t TM_COLS = (NACC * N + 24 <= 256) ? 256 : 512;
+  constexpr int NACC = n_acc(N);
+  static_assert(NACC >= 2 && NACC * (N + 4) + 8 <= (int)TM_COLS, "TMEM budget");
   constexpr bool W_IN_REGS = N <= 64;
 
   // tiles per query, loaded in parallel, then a serial prefix over shared memory
@@ -134,6 +154,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = s.tmem_base;
   // TMEM columns: acc[a] at a*N; SFA[a] at NACC*N + 4a; SFB[j] after them
   const uint32_t col_sfa = NACC * N, col_sfb = NACC * N + 4 * NACC;
+  auto aborted = [&]() {
+    return __any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s.abort)) != 0;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -144,13 +167,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     TileIter t;
     const uint32_t* ksf32 = reinterpret_cast<const uint32_t*>(P.keys_sf);
     const int64_t total_rows = (int64_t)P.B * P.key_rows;
-    int it = 0;
+    int stg = 0;
     int b = 0;                                  // sequence of the current query
-    for (int g = g0; g < g1 && !__any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s.abort)); ++g, ++it) {
+    for (int g = g0; g < g1 && !aborted(); ++stg) {
       const int seg_before = t.seg;
       locate(s, P.n_q, g, t);
+      const int n = stage_tiles(s, t, g, g1);
       if (t.seg != seg_before) {
-        // read once per query: a global load per tile would sit on the issue path
+        // read once per query: a global load per stage would sit on the issue path
         b = P.q_seq ? P.q_seq[t.q] : P.q_base + t.q;
         const int j = t.seg & 1, uq = t.seg >> 1;
         if (uq >= 1 && !mbar_wait_warp(&s.qempty[j], (uq - 1) & 1, P.status)) {
@@ -166,41 +190,46 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           bulk_load(s.w[j], P.w + (int64_t)t.q * P.H_I, N * 4, &s.qfull[j]);
         }
       }
-      const int st = it % STAGES, u = it / STAGES;
+      const int st = stg % STAGES, u = stg / STAGES;
       if (u >= 1 && !mbar_wait_warp(&s.empty[st], (u - 1) & 1, P.status)) {
         fail(s, P.status);
         break;
       }
       const int64_t row0 = (int64_t)b * P.key_rows + (int64_t)t.lt * KT;
       if (lane == 0) {
-        // key codes (TMA tile) + their scales (bulk copy of the in-range rows,
-        // 4 at a time; a ragged end of the key array goes by 4-byte cp.async)
+        // key codes (one TMA tile per 128 keys) + their scales (bulk copy of
+        // the in-range rows, 4 at a time; a ragged end of the key array goes by
+        // 4-byte cp.async)
         const int64_t rows_left = total_rows - row0;
-        const int nrow = (int)(rows_left < KT ? rows_left : KT);
+        const int nrow = (int)(rows_left < n * KT ? rows_left : n * KT);
         const int nbulk = nrow & ~3;
-        mbar_expect_tx(&s.full[st], KTILE_BYTES + nbulk * 4);
-        tma_load_2d(s.keys[st], &tm_keys, &s.full[st], 0, (int)row0);
+        mbar_expect_tx(&s.full[st], (uint32_t)(n * KTILE_BYTES + nbulk * 4));
+        for (int k = 0; k < n; ++k)
+          tma_load_2d(s.keys[st][k], &tm_keys, &s.full[st], 0, (int)(row0 + k * KT));
         if (nbulk) bulk_load(s.sfa_raw[st], ksf32 + row0, nbulk * 4, &s.full[st]);
         for (int r = nbulk; r < nrow; ++r) cp_async4(&s.sfa_raw[st][r], ksf32 + row0 + r, true);
         cp_async_arrive_noinc(&s.full[st]);
       }
+      g += n;
     }
     // drain: no load may still be landing in shared memory when the CTA exits
     if (s.abort && lane == 0) {
-      for (int k = 0; k < STAGES && k < it; ++k) {
-        const int i2 = it - 1 - k;
+      for (int k = 0; k < STAGES && k < stg; ++k) {
+        const int i2 = stg - 1 - k;
         mbar_wait(&s.full[i2 % STAGES], (i2 / STAGES) & 1);   // time bound only
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     TileIter t;
-    int it = 0;
+    int stg = 0;
+    bool ok = true;
     const uint64_t kdesc_bits = smem_desc_bits(16, 8 * KROW, 4);    // K-major, 64B swizzle
     const uint64_t sf_bits = smem_desc_bits(16, 128, 0);            // 32 rows x 16 B
-    for (int g = g0; g < g1 && !__any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s.abort)); ++g, ++it) {
+    for (int g = g0; ok && g < g1 && !aborted(); ++stg) {
       const int seg_before = t.seg;
       locate(s, P.n_q, g, t);
+      const int n = stage_tiles(s, t, g, g1);
       const int j = t.seg & 1;
       if (t.seg != seg_before) {
         if (!mbar_wait_warp(&s.qfull[j], (t.seg >> 1) & 1, P.status)) {
@@ -216,40 +245,47 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         if (lane == 0) tmem_cp_32x128b_warpx4(tmem + col_sfb + 4 * j, smem_desc(s.sfb[j], sf_bits));
       }
-      const int st = it % STAGES, a = it % NACC, ua = it / NACC;
-      if (!mbar_wait_warp(&s.full[st], (it / STAGES) & 1, P.status)) {
+      const int st = stg % STAGES;
+      if (!mbar_wait_warp(&s.full[st], (stg / STAGES) & 1, P.status)) {
         fail(s, P.status);
         break;
       }
-      if (ua >= 1 && !mbar_wait_warp(&s.accempty[a], (ua - 1) & 1, P.status)) {
-        fail(s, P.status);
-        break;
-      }
-      // key scales into the tcgen05 scale-factor order (row r -> lane r%32, column r/32)
+      for (int k = 0; k < n; ++k) {
+        const int it = g - g0 + k, a = it % NACC, ua = it / NACC;
+        if (ua >= 1 && !mbar_wait_warp(&s.accempty[a], (ua - 1) & 1, P.status)) {
+          fail(s, P.status);
+          ok = false;
+          break;
+        }
+        // key scales into the tcgen05 scale-factor order (row r -> lane r%32, column r/32)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int r = k * 32 + lane;
-        *reinterpret_cast<uint32_t*>(&s.sfa[st][16 * lane + 4 * k]) = s.sfa_raw[st][r];
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint32_t*>(&s.sfa[a][16 * lane + 4 * c]) = s.sfa_raw[st][k * KT + c * 32 + lane];
+        fence_proxy_async_smem();
+        __syncwarp();
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t sfa = tmem + col_sfa + 4 * a;
+          const uint32_t sfb = tmem + col_sfb + 4 * j;
+          tmem_cp_32x128b_warpx4(sfa, smem_desc(s.sfa[a], sf_bits));
+          const uint64_t da = smem_desc(s.keys[st][k], kdesc_bits);
+          const uint64_t db = smem_desc(s.q[j], kdesc_bits);
+          const uint32_t d = tmem + a * N;
+          // K = 0..63 (scale bytes 0,1), then K = 64..127 (scale bytes 2,3): +32 B
+          mma_mxf4(d, da, db, idesc_mxf4(KT, N, 0, 0), sfa, sfb, 0);
+          mma_mxf4(d, da + 2, db + 2, idesc_mxf4(KT, N, 2, 2), sfa, sfb, 1);
+          tc_commit(&s.accfull[a]);
+        }
+        __syncwarp();
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      tc_fence_after();
+      if (!ok) break;
       if (lane == 0) {
-        const uint32_t sfa = tmem + col_sfa + 4 * a;
-        const uint32_t sfb = tmem + col_sfb + 4 * j;
-        tmem_cp_32x128b_warpx4(sfa, smem_desc(s.sfa[st], sf_bits));
-        const uint64_t da = smem_desc(s.keys[st], kdesc_bits);
-        const uint64_t db = smem_desc(s.q[j], kdesc_bits);
-        const uint32_t d = tmem + a * N;
-        // K = 0..63 (scale bytes 0,1), then K = 64..127 (scale bytes 2,3): +32 B
-        mma_mxf4(d, da, db, idesc_mxf4(KT, N, 0, 0), sfa, sfb, 0);
-        mma_mxf4(d, da + 2, db + 2, idesc_mxf4(KT, N, 2, 2), sfa, sfb, 1);
         tc_commit(&s.empty[st]);
-        tc_commit(&s.accfull[a]);
-        const bool seg_end = (g + 1 == g1) || (g + 1 >= s.tile_prefix[t.q + 1]);
+        const bool seg_end = (g + n == g1) || (g + n >= s.tile_prefix[t.q + 1]);
         if (seg_end) tc_commit(&s.qempty[j]);
       }
       __syncwarp();
+      g += n;
     }
     // every MMA / copy this warp issued has completed before TMEM is released
     if (lane == 0) {
@@ -274,12 +310,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
     TileIter t;
-    int it = 0;
+    bool ok = true;
     float wreg[W_IN_REGS ? N : 1];
     int64_t nv = 0;
-    for (int g = g0; g < g1 && !__any_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&s.abort)); ++g, ++it) {
+    for (int g = g0; ok && g < g1 && !aborted();) {
       const int seg_before = t.seg;
       locate(s, P.n_q, g, t);
+      const int n = stage_tiles(s, t, g, g1);
       const int j = t.seg & 1;
       if (t.seg != seg_before) {
         if (!mbar_wait_warp(&s.qfull[j], (t.seg >> 1) & 1, P.status)) {
@@ -292,11 +329,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         nv = min((int64_t)(P.q_pos[t.q] + 1) / P.m, min(P.key_rows, P.max_vis));
       }
-      const bool seg_end = (g + 1 == g1) || (g + 1 >= s.tile_prefix[t.q + 1]);
-      if ((it & 1) == grp) {
+      for (int k = 0; k < n; ++k) {
+        const int it = g - g0 + k;
+        if ((it & 1) != grp) continue;
         const int a = it % NACC;
         if (!mbar_wait_warp(&s.accfull[a], (it / NACC) & 1, P.status)) {
           fail(s, P.status);
+          ok = false;
           break;
         }
         tc_fence_after();
@@ -323,13 +362,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
         const float score = s0 + s1;
-        const int64_t i = (int64_t)t.lt * KT + r;
+        const int64_t i = (int64_t)(t.lt + k) * KT + r;
         if (i < P.max_vis) P.scores[(int64_t)t.q * P.scores_ld + i] = (i < nv) ? score : -INFINITY;
       }
+      if (!ok) break;
+      const bool seg_end = (g + n == g1) || (g + n >= s.tile_prefix[t.q + 1]);
       if (seg_end) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.qempty[j]);
       }
+      g += n;
     }
   }
   tc_fence_before();
