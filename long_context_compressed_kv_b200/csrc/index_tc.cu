@@ -12,7 +12,14 @@
 // multi-stage TMA ring (64-byte-swizzled K-major tiles); B (the query's H_I x
 // 128 codes) stays in shared memory for the query's whole key range; the E8M0
 // scales of both go to TMEM with tcgen05.cp (row m at lane m % 32 of every
-// sub-partition, column m / 32, byte = 32-element block).  A ring stage holds up
+// sub-partition, column m / 32, byte = 32-element block).  The key tile is
+// loaded through a 3-D view of the key array (64 B x rows/4 x 4, strides 256 B
+// and 64 B) so that MMA row 32c + l holds key 4l + c: in that order the key
+// scales, stored row-major (4 bytes a key), are already the scale-factor
+// layout, and go from the bulk-copied stage straight to TMEM without a pass
+// through registers (a generic-proxy rewrite would need a proxy fence per
+// stage, which waits behind the stage loads still in flight).  The epilogue
+// maps TMEM lane 32c + l back to key 4l + c.  A ring stage holds up
 // to four consecutive 128-key tiles of one query (32 KB): on this part a
 // streaming read over one stage per barrier round trip reaches HBM speed only
 // from about 32 KB per stage on, while the work is still split between CTAs
@@ -51,7 +58,6 @@ __host__ __device__ constexpr int n_acc(int N) {
 struct Smem {
   alignas(1024) uint8_t keys[STAGES][TPS][KTILE_BYTES];
   alignas(1024) uint8_t q[2][128 * KROW];
-  alignas(128) uint8_t sfa[MAX_ACC][SF_BYTES];      // scale-factor order, per accumulator
   alignas(128) uint32_t sfa_raw[STAGES][TPS * KT];  // key scales as loaded (row-major)
   alignas(128) uint8_t sfb[2][SF_BYTES];
   alignas(128) uint32_t sfb_raw[2][128];
@@ -204,8 +210,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int nrow = (int)(rows_left < n * KT ? rows_left : n * KT);
         const int nbulk = nrow & ~3;
         mbar_expect_tx(&s.full[st], (uint32_t)(n * KTILE_BYTES + nbulk * 4));
-        for (int k = 0; k < n; ++k)
-          tma_load_2d(s.keys[st][k], &tm_keys, &s.full[st], 0, (int)(row0 + k * KT));
+        for (int k = 0; k < n; ++k)   // rows row0 + 4l + c land at tile row 32c + l
+          tma_load_3d(s.keys[st][k], &tm_keys, &s.full[st], 0, (int)((row0 + k * KT) >> 2), 0);
         if (nbulk) bulk_load(s.sfa_raw[st], ksf32 + row0, nbulk * 4, &s.full[st]);
         for (int r = nbulk; r < nrow; ++r) cp_async4(&s.sfa_raw[st][r], ksf32 + row0 + r, true);
         cp_async_arrive_noinc(&s.full[st]);
@@ -250,6 +256,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fail(s, P.status);
         break;
       }
+      // every accumulator of the stage free first; then all scale copies, then
+      // the MMAs tile by tile, each tile committed to its own barrier (a copy
+      // issued behind an MMA waits for it, and back-to-back commits to one
+      // barrier serialise)
       for (int k = 0; k < n; ++k) {
         const int it = g - g0 + k, a = it % NACC, ua = it / NACC;
         if (ua >= 1 && !mbar_wait_warp(&s.accempty[a], (ua - 1) & 1, P.status)) {
@@ -257,28 +267,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = false;
           break;
         }
-        // key scales into the tcgen05 scale-factor order (row r -> lane r%32, column r/32)
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint32_t*>(&s.sfa[a][16 * lane + 4 * c]) = s.sfa_raw[st][k * KT + c * 32 + lane];
-        fence_proxy_async_smem();
-        __syncwarp();
-        tc_fence_after();
-        if (lane == 0) {
+      }
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t sfb = tmem + col_sfb + 4 * j;
+        const uint64_t db = smem_desc(s.q[j], kdesc_bits);
+        for (int k = 0; k < n; ++k) {
+          const int a = (g - g0 + k) % NACC;
+          tmem_cp_32x128b_warpx4(tmem + col_sfa + 4 * a, smem_desc(&s.sfa_raw[st][k * KT], sf_bits));
+        }
+        for (int k = 0; k < n; ++k) {
+          const int a = (g - g0 + k) % NACC;
           const uint32_t sfa = tmem + col_sfa + 4 * a;
-          const uint32_t sfb = tmem + col_sfb + 4 * j;
-          tmem_cp_32x128b_warpx4(sfa, smem_desc(s.sfa[a], sf_bits));
           const uint64_t da = smem_desc(s.keys[st][k], kdesc_bits);
-          const uint64_t db = smem_desc(s.q[j], kdesc_bits);
           const uint32_t d = tmem + a * N;
           // K = 0..63 (scale bytes 0,1), then K = 64..127 (scale bytes 2,3): +32 B
           mma_mxf4(d, da, db, idesc_mxf4(KT, N, 0, 0), sfa, sfb, 0);
           mma_mxf4(d, da + 2, db + 2, idesc_mxf4(KT, N, 2, 2), sfa, sfb, 1);
           tc_commit(&s.accfull[a]);
         }
-        __syncwarp();
       }
-      if (!ok) break;
+      __syncwarp();
       if (lane == 0) {
         tc_commit(&s.empty[st]);
         const bool seg_end = (g + n == g1) || (g + n >= s.tile_prefix[t.q + 1]);
@@ -296,10 +306,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     // group g handles the tiles with it % 2 == g; within a group, warp w reads
-    // TMEM lanes 32*(w%4) .. +31 (one key row per thread)
+    // TMEM lanes 32*(w%4) .. +31 (one key per thread)
     const int grp = (warp - 2) >> 2;
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;             // key row within the tile
+    const int r = 4 * lane + quad;              // key of TMEM lane 32 * quad + lane
     {
       // keys beyond the last tile of each query: -inf
       const int et = threadIdx.x - 64;
@@ -435,6 +445,22 @@ bool make_rows_map_sw(CUtensorMap* map, const void* base, int64_t rows, int row_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D uint8 view of the MXFP4 key codes (64-byte rows, row count divisible by
+// 4): dims {64 B, rows / 4, 4} with strides {256 B, 64 B}.  A box {64, 32, 4}
+// at (0, row0 / 4, 0) lands rows row0 + 4l + c at shared-memory row 32c + l,
+// 64-byte swizzled; rows past the end of the array read as zero.
+static bool make_keys_map(CUtensorMap* map, const void* base, int64_t rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || rows < 4 || (rows & 3) || rows > (1ll << 31)) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)KROW, (cuuint64_t)(rows / 4), 4};
+  cuuint64_t strides[2] = {(cuuint64_t)(4 * KROW), (cuuint64_t)KROW};
+  cuuint32_t box[3] = {(cuuint32_t)KROW, 32, 4};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool index_tc_supported(const IndexParams& P) {
   // the scale and weight rows are moved by 1-D bulk copies: 16-byte aligned
   // sources, i.e. 16-byte aligned bases and a key row count divisible by 4
@@ -448,7 +474,7 @@ bool index_tc_supported(const IndexParams& P) {
 
 cudaError_t launch_index_tc(const IndexParams& P, cudaStream_t st) {
   CUtensorMap tk, tq;
-  if (!make_rows_map(&tk, P.keys, (int64_t)P.B * P.key_rows, KROW, KT)) return cudaErrorInvalidValue;
+  if (!make_keys_map(&tk, P.keys, (int64_t)P.B * P.key_rows)) return cudaErrorInvalidValue;
   if (!make_rows_map(&tq, P.qI, (int64_t)P.n_q * P.H_I, KROW, P.H_I)) return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
   static unsigned long long configured = 0;

@@ -22,9 +22,11 @@ namespace v4a {
 // Wall-clock limit of every mbarrier wait.  A failed try_wait may suspend the
 // thread for a while, so the bound is in time (%globaltimer), not iterations.
 // On expiry the wait reports failure; the kernel records ST_TIMEOUT in the
-// status word, and every other wait of the grid gives up as soon as it sees
-// that bit, so a stuck kernel ends within about one limit.
-constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s
+// status word, and every other wait of the grid that has lasted kStatusPollNs
+// gives up as soon as it sees that bit, so a stuck kernel ends within about
+// one limit.
+constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s (< 2^32 ns)
+constexpr unsigned long long kStatusPollNs = 20000ull;  // 20 us
 constexpr uint32_t kStatusTimeout = 1u << 8;            // == ST_TIMEOUT
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -77,16 +79,23 @@ __device__ __forceinline__ bool mbar_wait_at(uint64_t* bar, uint32_t parity, uin
 
 // Bounded wait for the phase with the given parity; false on expiry or when
 // `status` (the grid's status word, may be null) already records a timeout.
+// The status word is read only once the wait has lasted kStatusPollNs: a
+// global load on the polling path of every healthy wait would delay noticing
+// the phase by a memory round trip, which under a full HBM stream is several
+// hundred nanoseconds.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           const uint32_t* status = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
+  // elapsed time in 32 bits: it wraps after 4.29 s, well above the limit
+  const uint32_t t0 = (uint32_t)global_ns();
   for (;;) {
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (status && (*reinterpret_cast<const volatile uint32_t*>(status) & kStatusTimeout))
+    const uint32_t dt = (uint32_t)global_ns() - t0;
+    if (dt > (uint32_t)kWaitNs) return false;
+    if (status && dt > (uint32_t)kStatusPollNs &&
+        (*reinterpret_cast<const volatile uint32_t*>(status) & kStatusTimeout))
       return false;
-    if (global_ns() - t0 > kWaitNs) return false;
   }
 }
 __device__ __forceinline__ bool mbar_wait_at(uint64_t* bar, uint32_t parity, uint32_t* status,
@@ -150,6 +159,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 // 1-D bulk copy global -> shared through the TMA engine (16-byte aligned
