@@ -20,11 +20,16 @@ constexpr size_t kAlign = 256;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
-// Workspace: [status header | decode scratch | body].  The body holds either
-// the indexer scores of an index_topk call or the split-K partials of an MQA
-// call; the two never live at the same time (stream order), so they overlap.
+// Workspace: [status header | decode scratch | query images | body].  The
+// query images are the tensor-core MQA's coded queries of one query chunk (none
+// for other KV formats); in a decode step the append kernel writes them before
+// the indexer runs, so they sit outside the body.  The body holds either the
+// indexer scores of an index_topk call or the split-K partials of an MQA call;
+// the two never live at the same time (stream order), so they overlap.  A
+// stand-alone index_topk call, which leaves the images alone, starts its body
+// at the images' offset.
 size_t dec_bytes(int32_t n_q) { return align_up((size_t)n_q * 3 * sizeof(int64_t)); }
-size_t body0(int32_t n_q) { return align_up(sizeof(WsHeader)) + dec_bytes(n_q); }
+size_t qimg_off(int32_t n_q) { return align_up(sizeof(WsHeader)) + dec_bytes(n_q); }
 // index_topk and the MQA calls walk their queries in chunks of kQChunk; the
 // scores / split-K partials of one chunk live in the workspace body, reused
 // by the next chunk in stream order.
@@ -42,12 +47,14 @@ size_t mqa_part_ml_bytes(const v4attn_layer_desc* d, int32_t n_q, int n_split) {
   return align_up((size_t)n_q * n_split * d->H * 2 * sizeof(float));
 }
 size_t mqa_qbuf_bytes(const v4attn_layer_desc* d, int32_t n_q) {
-  return d->kv_dtype == V4A_E4M3_BF16ROPE ? align_up((size_t)n_q * kMqaQImageStride) : 0;
+  return d->kv_dtype == V4A_E4M3_BF16ROPE ? align_up((size_t)q_chunk(n_q) * kMqaQImageStride) : 0;
 }
+// body offset of MQA calls and of every call of a decode step
+size_t body_mqa(const v4attn_layer_desc* d, int32_t n_q) { return qimg_off(n_q) + mqa_qbuf_bytes(d, n_q); }
 size_t mqa_need(const v4attn_layer_desc* d, int32_t n_q, int64_t n_main_max) {
   const int S = mqa_num_splits(d, n_main_max);
   const int32_t c = q_chunk(n_q);
-  return mqa_part_o_bytes(d, c, S) + mqa_part_ml_bytes(d, c, S) + mqa_qbuf_bytes(d, c);
+  return mqa_part_o_bytes(d, c, S) + mqa_part_ml_bytes(d, c, S);
 }
 size_t total_need(const v4attn_layer_desc* d, int32_t n_q, int64_t max_vis) {
   size_t body = mqa_need(d, n_q, max_vis);
@@ -55,7 +62,7 @@ size_t total_need(const v4attn_layer_desc* d, int32_t n_q, int64_t max_vis) {
     body = std::max(body, index_need(n_q, max_vis));
     body = std::max(body, mqa_need(d, n_q, (int64_t)d->top_k));
   }
-  return body0(n_q) + body;
+  return body_mqa(d, n_q) + body;
 }
 
 v4attn_status check_desc(const v4attn_layer_desc* d) {
@@ -143,7 +150,7 @@ v4attn_status run_compress(const v4attn_layer_desc* d, const v4attn_compress_arg
 }
 
 v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args* a, void* ws,
-                             size_t ws_bytes, cudaStream_t st) {
+                             size_t ws_bytes, cudaStream_t st, size_t body_off) {
   if (d->kind != V4A_CSA) return V4A_ERR_INVALID_ARG;
   if (!a || a->n_q < 1 || a->n_q > kMaxQueries || a->B < 1) return V4A_ERR_INVALID_ARG;
   if (!a->qI || !a->w || !a->q_pos || !a->keys || (!a->idx_out && !a->scores_out))
@@ -151,7 +158,7 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
   if (d->idx_dtype == V4A_MXFP4 && (!a->qI_sf || !a->keys_sf)) return V4A_ERR_INVALID_ARG;
   if (a->key_rows < 1 || a->max_vis < 0 || a->max_vis > a->key_rows) return V4A_ERR_INVALID_ARG;
   if (!ws) return V4A_ERR_WORKSPACE;
-  if (ws_bytes < body0(a->n_q) + index_need(a->n_q, a->max_vis)) return V4A_ERR_WORKSPACE;
+  if (ws_bytes < body_off + index_need(a->n_q, a->max_vis)) return V4A_ERR_WORKSPACE;
   uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
   const int64_t ld = std::max<int64_t>(a->max_vis, 1);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
@@ -160,7 +167,7 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
   for (int32_t q0 = 0; q0 < a->n_q; q0 += kQChunk) {
     const int32_t cn = std::min(kQChunk, a->n_q - q0);
     float* scores = a->scores_out ? a->scores_out + (int64_t)q0 * ld
-                                  : reinterpret_cast<float*>(w8 + body0(a->n_q));
+                                  : reinterpret_cast<float*>(w8 + body_off);
     if (a->max_vis > 0) {
       IndexParams P;
       P.n_q = cn;
@@ -200,7 +207,7 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
 }
 
 v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void* ws,
-                      size_t ws_bytes, cudaStream_t st, bool sparse) {
+                      size_t ws_bytes, cudaStream_t st, bool sparse, bool q_ready = false) {
   if (!a || a->n_q < 1 || a->n_q > kMaxQueries || a->B < 1) return V4A_ERR_INVALID_ARG;
   if (!a->Q || !a->q_pos || !a->kv || !a->out) return V4A_ERR_INVALID_ARG;
   if (d->n_win > 0 && (!a->swa || a->swa_rows < d->n_win)) return V4A_ERR_INVALID_ARG;
@@ -215,7 +222,8 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
     return V4A_ERR_INVALID_ARG;
   if (!ws) return V4A_ERR_WORKSPACE;
   const int64_t n_main_max = sparse ? (int64_t)a->n_sel : a->max_vis;
-  if (ws_bytes < body0(a->n_q) + mqa_need(d, a->n_q, n_main_max)) return V4A_ERR_WORKSPACE;
+  const size_t b0 = body_mqa(d, a->n_q);
+  if (ws_bytes < b0 + mqa_need(d, a->n_q, n_main_max)) return V4A_ERR_WORKSPACE;
   uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
   const int32_t c = q_chunk(a->n_q);
   const size_t qb = (size_t)d->H * d->d * (a->q_dtype == V4A_BF16 ? 2 : 4);
@@ -251,12 +259,10 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
     P.sink = a->sink;
     P.split_keys = mqa_split_keys(d);
     P.n_split = mqa_num_splits(d, n_main_max);
-    P.part_o = reinterpret_cast<float*>(w8 + body0(a->n_q));
-    P.part_ml =
-        reinterpret_cast<float*>(w8 + body0(a->n_q) + mqa_part_o_bytes(d, c, P.n_split));
-    P.qbuf = mqa_qbuf_bytes(d, c) ? w8 + body0(a->n_q) + mqa_part_o_bytes(d, c, P.n_split) +
-                                        mqa_part_ml_bytes(d, c, P.n_split)
-                                  : nullptr;
+    P.part_o = reinterpret_cast<float*>(w8 + b0);
+    P.part_ml = reinterpret_cast<float*>(w8 + b0 + mqa_part_o_bytes(d, c, P.n_split));
+    P.qbuf = mqa_qbuf_bytes(d, c) ? w8 + qimg_off(a->n_q) : nullptr;
+    P.q_ready = q_ready ? 1 : 0;
     P.out = reinterpret_cast<uint8_t*>(a->out) + (size_t)q0 * ob;
     P.out_dtype = a->out_dtype;
     P.lse = a->lse ? a->lse + (int64_t)q0 * d->H : nullptr;
@@ -295,7 +301,7 @@ v4attn_status v4attn_index_topk(const v4attn_layer_desc* desc, const v4attn_inde
                                 void* ws, size_t ws_bytes, cudaStream_t stream) {
   v4attn_status s = check_desc(desc);
   if (s != V4A_OK) return s;
-  return run_index_topk(desc, args, ws, ws_bytes, stream);
+  return run_index_topk(desc, args, ws, ws_bytes, stream, args ? qimg_off(args->n_q) : 0);
 }
 
 v4attn_status v4attn_sparse_mqa(const v4attn_layer_desc* desc, const v4attn_mqa_args* args,
@@ -372,6 +378,16 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
   A.keys = csa ? a->keys : nullptr;
   A.keys_sf = csa ? a->keys_sf : nullptr;
   A.key_rows = csa ? a->key_rows : 0;
+  // the tensor-core MQA's query images, coded in the same launch when its
+  // format applies and the step's queries fit one query chunk
+  const bool fuse_q = desc->kv_dtype == V4A_E4M3_BF16ROPE && a->q_dtype == V4A_BF16 &&
+                      d == 512 && desc->d_rope == 64 && desc->H <= 128 && a->B <= kQChunk &&
+                      aligned16(a->Q);
+  if (fuse_q) {
+    A.Q = a->Q;
+    A.H = desc->H;
+    A.qimg = reinterpret_cast<uint8_t*>(ws) + qimg_off(a->B);
+  }
   if (launch_decode_append(A, stream) != cudaSuccess) return V4A_ERR_CUDA;
   if (csa) {
     // 3. indexer + top-k
@@ -388,7 +404,7 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
     ix.key_rows = a->key_rows;
     ix.max_vis = a->max_vis;
     ix.idx_out = a->idx_out;
-    s = run_index_topk(desc, &ix, ws, ws_bytes, stream);
+    s = run_index_topk(desc, &ix, ws, ws_bytes, stream, body_mqa(desc, a->B));
     if (s != V4A_OK) return s;
   }
   // 4. MQA
@@ -413,7 +429,7 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
   q.out = a->out;
   q.out_dtype = a->out_dtype;
   q.lse = a->lse;
-  return run_mqa(desc, &q, ws, ws_bytes, stream, csa);
+  return run_mqa(desc, &q, ws, ws_bytes, stream, csa, fuse_q);
 }
 
 v4attn_status v4attn_project(const v4attn_project_args* a, cudaStream_t stream) {
@@ -489,7 +505,7 @@ extern "C" v4attn_status v4attn_index_topk_noalloc(const v4attn_layer_desc* desc
   if (s != V4A_OK) return s;
   if (!args || args->n_q < 1 || args->max_vis < 0) return V4A_ERR_INVALID_ARG;
   if ((int64_t)args->n_q * std::max<int64_t>(args->max_vis, 1) > V4A_NOALLOC_MAX_SCORES ||
-      body0(args->n_q) + index_need(args->n_q, args->max_vis) > kNoallocBytes)
+      qimg_off(args->n_q) + index_need(args->n_q, args->max_vis) > kNoallocBytes)
     return V4A_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return V4A_ERR_CUDA;
@@ -501,5 +517,5 @@ extern "C" v4attn_status v4attn_index_topk_noalloc(const v4attn_layer_desc* desc
   void* ws = g_noalloc_ptr[dev];
   // the status word must start at zero; the scores are fully rewritten by the call
   if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), stream) != cudaSuccess) return V4A_ERR_CUDA;
-  return run_index_topk(desc, args, ws, kNoallocBytes, stream);
+  return run_index_topk(desc, args, ws, kNoallocBytes, stream, qimg_off(args->n_q));
 }

@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "mqa_qimage.cuh"
 
 namespace v4a {
 
@@ -280,13 +281,21 @@ __device__ __forceinline__ void copy_share(uint8_t* dst, const uint8_t* src, int
   }
 }
 
-__global__ void __launch_bounds__(kAppendThreads) decode_append_kernel(AppendParams A) {
+__global__ void __launch_bounds__(kAppendThreads, 2) decode_append_kernel(AppendParams A) {
   __shared__ float red[32];
   __shared__ float part[2];
   __shared__ float mrg[kAppendThreads * 6];
-  const int nj = A.csa ? 3 : 2;
+  const int nbase = A.csa ? 3 : 2;
+  const int nj = nbase + (A.qimg ? 1 : 0);
   const int job = blockIdx.x / kAppendCluster, rank = blockIdx.x % kAppendCluster;
   const int b = job / nj, t = job % nj;
+  if (t == nbase) {
+    // the tensor-core MQA's query image: CTA `rank` codes head rows 16*rank .. +15
+    __shared__ float qcs[32], qsn[32];
+    qimage_code_rows(reinterpret_cast<const __nv_bfloat16*>(A.Q) + (int64_t)b * A.H * 512, A.H,
+                     A.pos[b], A.theta, A.qimg + (int64_t)b * kMqaQImageStride, rank, qcs, qsn);
+    return;
+  }
   const int elt = A.in_dtype == V4A_F32 ? 4 : 2;
   const int64_t p = A.pos[b];
   const int64_t nb = (int64_t)A.n_arr * A.d * elt;         // bytes of one main input row
@@ -386,7 +395,8 @@ __global__ void __launch_bounds__(kAppendThreads) decode_append_kernel(AppendPar
 }
 
 cudaError_t launch_decode_append(const AppendParams& A, cudaStream_t st) {
-  const int nj = A.csa ? 3 : 2;
+  static_assert(kAppendCluster == 8 && kAppendThreads >= 64, "query image: 8 CTAs of 16 head rows");
+  const int nj = (A.csa ? 3 : 2) + (A.qimg ? 1 : 0);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(A.B * nj * kAppendCluster), 1, 1);
   cfg.blockDim = dim3(kAppendThreads, 1, 1);

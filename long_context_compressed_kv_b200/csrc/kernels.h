@@ -51,6 +51,11 @@ struct AppendParams {
   int64_t kv_rows;
   void *keys, *keys_sf;
   int64_t key_rows;
+  // optional: code each sequence's bf16 query (H heads of 512 dims, RoPE at
+  // pos[b]) into the tensor-core MQA's query image at qimg + b * kMqaQImageStride
+  const void* Q = nullptr;
+  int H = 0;
+  uint8_t* qimg = nullptr;
 };
 
 struct IndexParams {
@@ -105,6 +110,7 @@ struct MqaParams {
   float* part_o;        // [n_q][n_split][H][d]
   float* part_ml;       // [n_q][n_split][H][2]
   uint8_t* qbuf;        // tensor-core path: [n_q] coded query images (kMqaQImageStride bytes)
+  int q_ready = 0;      // the images in qbuf are already coded (decode: by the append kernel)
   void* out;
   int out_dtype;
   float* lse;

@@ -7,10 +7,11 @@
 // "其他稳定性细节" (448 FP8 + 64 BF16 RoPE dims, sink, inverse RoPE on the
 // output, which the combine applies); "拆解 DeepSeekv4", section "细节".
 //
-// Layout of the work.  A small pre-kernel codes each query once (RoPE at its
-// position on dims 448..511, E4M3 with a power-of-two scale on dims 0..447)
-// straight into the swizzled shared-memory image the MMAs read; every CTA of
-// the query copies that image in with bulk copies.  A CTA owns (query, key
+// Layout of the work.  Each query is coded once (RoPE at its position on dims
+// 448..511, E4M3 with a power-of-two scale on dims 0..447) straight into the
+// swizzled shared-memory image the MMAs read, by a small pre-kernel or, in the
+// decode step, by the append kernel that runs before it; every CTA of the
+// query copies that image in with bulk copies.  A CTA owns (query, key
 // chunk of split_keys keys, half of the 512 output dims).  Output dims are
 // split because fp32 O for 128 heads x 512 dims is all of TMEM (512 columns x
 // 128 lanes): each CTA keeps O[128 x 256] in TMEM columns 256..511 and S for
@@ -44,6 +45,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "mqa_qimage.cuh"
 #include "tc_common.cuh"
 #include "tc_kernels.h"
 
@@ -62,11 +64,10 @@ constexpr int SKMAX = 512;      // keys per split, at most
 constexpr int SKMAX_SEL = 128;  // keys per split of a selected-entry (sparse) call
 constexpr int TILE_BYTES = NK * (4 * 128 + 64);
 constexpr float kTau = 4.f;     // lazy-rescale margin of the running score maximum (log2 units)
-// query image: Q nope bytes 0..383 as three K-major SW128 blocks, bytes
-// 384..447 as one K-major SW64 block, the RoPE dims (bf16) as one K-major SW128
-// block, then the per-head E4M3 scale
-constexpr int Q_NOPE3 = 3 * 16384, Q_ROPE = Q_NOPE3 + 8192, QTILE = Q_ROPE + 16384;
-constexpr int QIMG = QTILE + 128 * 4;
+// query image (layout in mqa_qimage.cuh)
+constexpr int Q_NOPE3 = kQImgNope3, Q_ROPE = kQImgRope, QTILE = kQImgTile;
+constexpr int QIMG = kQImgBytes;
+static_assert(kQImgBytes <= kMqaQImageStride, "query image stride");
 constexpr int QCHUNK = QIMG / 4;
 static_assert(QCHUNK % 16 == 0, "bulk copies move multiples of 16 bytes");
 
@@ -126,19 +127,6 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// byte offset of (row, byte c) in a K-major tile of 128-byte rows, 128B swizzle
-__device__ __forceinline__ int sw128(int row, int c) {
-  return (row >> 3) * 1024 + (row & 7) * 128 + ((((c >> 4) ^ (row & 7)) & 7) << 4) + (c & 15);
-}
-// ... of 64-byte rows, 64B swizzle
-__device__ __forceinline__ int sw64(int row, int c) {
-  return (row >> 3) * 512 + (row & 7) * 64 + ((((c >> 4) ^ ((row & 7) >> 1)) & 3) << 4) + (c & 15);
-}
-
-// two floats -> two E4M3 codes (saturating, round to nearest even), low byte = a
-__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
-  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-}
 __device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t c) {
   const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)c, __NV_E4M3);
   return __half22float2(*reinterpret_cast<const __half2*>(&h));
@@ -149,8 +137,6 @@ __device__ __forceinline__ float ex2f(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 struct Geo {
   int b;
@@ -192,75 +178,12 @@ __device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
 }  // namespace
 
 // Eight CTAs per query (16 head rows each, so that a query's 128 KB of bf16 Q
-// is read by eight SMs), four threads per head row (7 of the 28 E4M3 chunks
-// and 2 of the 8 RoPE chunks each): the query image of the main kernel.  Each
-// thread issues all of its loads before the RoPE angles are computed.
+// is read by eight SMs): the query image of the main kernel.
 __global__ void __launch_bounds__(64) mqa_tc_qprep_kernel(MqaParams P) {
   __shared__ float cs[32], sn[32];
   const int q = blockIdx.x;
-  const int h = blockIdx.y * 16 + (threadIdx.x >> 2), part = threadIdx.x & 3;
-  const int64_t p = P.q_pos[q];
-  uint8_t* img = P.qbuf + (int64_t)q * kMqaQImageStride;
-  const bool live = h < P.H;
-  const uint4* src = reinterpret_cast<const uint4*>(
-      reinterpret_cast<const __nv_bfloat16*>(P.Q) + ((int64_t)q * P.H + (live ? h : 0)) * 512);
-  uint4 nope[14], rope[2];
-#pragma unroll
-  for (int i = 0; i < 14; ++i) nope[i] = live ? src[part * 14 + i] : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-  for (int i = 0; i < 2; ++i) rope[i] = live ? src[56 + part * 2 + i] : make_uint4(0u, 0u, 0u, 0u);
-  if (threadIdx.x < 32) {
-    float c = 1.f, sv = 0.f;
-    if (p >= 0) rope_cs(p, threadIdx.x, 64, P.theta, c, sv);
-    cs[threadIdx.x] = c;
-    sn[threadIdx.x] = sv;
-  }
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 14; ++i) {
-    const uint32_t w[4] = {nope[i].x, nope[i].y, nope[i].z, nope[i].w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[k])), fabsf(bf16hi(w[k]))));
-  }
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-  const int se = e4m3_scale_exp(amax);
-  // dims 0..447: 16 E4M3 codes per 16-byte chunk (chunks part*7 .. part*7+6)
-#pragma unroll
-  for (int j = 0; j < 7; ++j) {
-    const uint4 a = nope[2 * j], b = nope[2 * j + 1];
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    uint32_t pk[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t lo = e4m3x2(scale_pow2(bf16lo(w[2 * k]), se), scale_pow2(bf16hi(w[2 * k]), se));
-      const uint32_t hi =
-          e4m3x2(scale_pow2(bf16lo(w[2 * k + 1]), se), scale_pow2(bf16hi(w[2 * k + 1]), se));
-      pk[k] = lo | (hi << 16);
-    }
-    const int c = (part * 7 + j) * 16;
-    uint8_t* dst = (c < 384) ? img + (c >> 7) * 16384 + sw128(h, c & 127)
-                             : img + Q_NOPE3 + sw64(h, c - 384);
-    *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  }
-  __syncthreads();                          // RoPE angles
-  // dims 448..511: RoPE at the query position, kept in bf16
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int c16 = part * 2 + j;
-    const uint32_t w[4] = {rope[j].x, rope[j].y, rope[j].z, rope[j].w};
-    uint32_t pk[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int pr = c16 * 4 + k;
-      const float x0 = bf16lo(w[k]), x1 = bf16hi(w[k]);
-      const float r0 = x0 * cs[pr] - x1 * sn[pr], r1 = x0 * sn[pr] + x1 * cs[pr];
-      pk[k] = (uint32_t)f32_to_bf16_bits(r0) | ((uint32_t)f32_to_bf16_bits(r1) << 16);
-    }
-    *reinterpret_cast<uint4*>(img + Q_ROPE + sw128(h, c16 * 16)) =
-        make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  }
-  if (part == 0) reinterpret_cast<float*>(img + QTILE)[h] = exp2i(se);
+  qimage_code_rows(reinterpret_cast<const __nv_bfloat16*>(P.Q) + (int64_t)q * P.H * 512, P.H,
+                   P.q_pos[q], P.theta, P.qbuf + (int64_t)q * kMqaQImageStride, blockIdx.y, cs, sn);
 }
 
 __global__ void __launch_bounds__(NTHR, 1)
@@ -707,7 +630,7 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   }
   const int64_t grid = (int64_t)P.n_q * P.n_split * 2;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  mqa_tc_qprep_kernel<<<dim3((unsigned)P.n_q, 8), 64, 0, st>>>(P);
+  if (!P.q_ready) mqa_tc_qprep_kernel<<<dim3((unsigned)P.n_q, 8), 64, 0, st>>>(P);
   mqa_tc_kernel<<<(unsigned)grid, NTHR, smem, st>>>(P, m);
   return cudaGetLastError();
 }
