@@ -67,6 +67,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The same test, letting the hardware suspend the thread until the phase
+// completes (or the hint runs out) instead of returning at once: waiting
+// warps then take no issue slots from the warps they wait for (an MMA-issuing
+// warp shares its scheduler with epilogue warps).
+constexpr uint32_t kSuspendHintNs = 1000000;   // 1 ms; completion wakes the thread first
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -89,8 +104,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   // elapsed time in 32 bits: it wraps after 4.29 s, well above the limit
   const uint32_t t0 = (uint32_t)global_ns();
   for (;;) {
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity)) return true;
     const uint32_t dt = (uint32_t)global_ns() - t0;
     if (dt > (uint32_t)kWaitNs) return false;
     if (status && dt > (uint32_t)kStatusPollNs &&
