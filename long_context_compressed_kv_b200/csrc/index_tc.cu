@@ -24,7 +24,10 @@
 // streaming read over one stage per barrier round trip reaches HBM speed only
 // from about 32 KB per stage on, while the work is still split between CTAs
 // tile by tile.  The accumulator has several TMEM stages so the epilogue of
-// tile i overlaps the MMAs of the tiles after it.  Roles: warp 0 TMA producer,
+// tile i overlaps the MMAs of the tiles after it.  The MMA warp commits once
+// per stage (a tcgen05.commit costs hundreds of cycles of issue); the first
+// epilogue warp, once it has seen that commit, hands the ring stage (and at a
+// query's end its query buffer) back to the producer.  Roles: warp 0 TMA producer,
 // warp 1 MMA issuer (one lane), warps 2..5 and 6..9 two epilogue groups on
 // alternate tiles (one thread per key row).  The kernel is HBM-bound: 68 bytes
 // per key against 16384 FP4 FLOP.
@@ -62,7 +65,7 @@ struct Smem {
   alignas(128) uint8_t sfb[2][SF_BYTES];
   alignas(128) uint32_t sfb_raw[2][128];
   alignas(16) float w[2][128];
-  uint64_t full[STAGES], empty[STAGES], qfull[2], qempty[2], accfull[MAX_ACC],
+  uint64_t full[STAGES], empty[STAGES], accstage[STAGES], qfull[2], qempty[2],
       accempty[MAX_ACC], done;
   int tile_prefix[MAXQ + 1];
   uint32_t tmem_base;
@@ -136,16 +139,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     s.abort = 0;
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&s.full[i], 1);    // the producer lane's arrive + TMA / bulk bytes
-      mbar_init(&s.empty[i], 1);
+      mbar_init(&s.empty[i], 1);   // the epilogue's releaser, once the stage's MMAs are done
+      mbar_init(&s.accstage[i], 1);   // one commit after all MMAs of a stage
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.qfull[i], 1);
-      mbar_init(&s.qempty[i], 1 + 4 * EPI_GROUPS);
+      mbar_init(&s.qempty[i], 1 + 4 * EPI_GROUPS);   // releaser + every epilogue warp
     }
-    for (int i = 0; i < MAX_ACC; ++i) {
-      mbar_init(&s.accfull[i], 1);
-      mbar_init(&s.accempty[i], 4);
-    }
+    for (int i = 0; i < MAX_ACC; ++i) mbar_init(&s.accempty[i], 4);
     mbar_init(&s.done, 1);
     fence_mbar_init();
   }
@@ -257,9 +258,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       // every accumulator of the stage free first; then all scale copies, then
-      // the MMAs tile by tile, each tile committed to its own barrier (a copy
-      // issued behind an MMA waits for it, and back-to-back commits to one
-      // barrier serialise)
+      // the MMAs (a copy issued behind an MMA waits for it)
       for (int k = 0; k < n; ++k) {
         const int it = g - g0 + k, a = it % NACC, ua = it / NACC;
         if (ua >= 1 && !mbar_wait_warp(&s.accempty[a], (ua - 1) & 1, P.status)) {
@@ -285,14 +284,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // K = 0..63 (scale bytes 0,1), then K = 64..127 (scale bytes 2,3): +32 B
           mma_mxf4(d, da, db, idesc_mxf4(KT, N, 0, 0), sfa, sfb, 0);
           mma_mxf4(d, da + 2, db + 2, idesc_mxf4(KT, N, 2, 2), sfa, sfb, 1);
-          tc_commit(&s.accfull[a]);
         }
-      }
-      __syncwarp();
-      if (lane == 0) {
-        tc_commit(&s.empty[st]);
-        const bool seg_end = (g + n == g1) || (g + n >= s.tile_prefix[t.q + 1]);
-        if (seg_end) tc_commit(&s.qempty[j]);
+        // one commit for the whole stage: commits are the costly tcgen05
+        // instruction here; the epilogue releases the ring stage and the
+        // query buffer once it has seen this one
+        tc_commit(&s.accstage[st]);
       }
       __syncwarp();
       g += n;
@@ -320,10 +316,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     }
     TileIter t;
-    bool ok = true;
     float wreg[W_IN_REGS ? N : 1];
     int64_t nv = 0;
-    for (int g = g0; ok && g < g1 && !aborted();) {
+    int stg = 0;
+    // warp 2 lane 0 (group 0) is the releaser: it waits for every stage's
+    // commit and then frees the ring stage (and, at a query's last stage, the
+    // query buffer) for the producer
+    const bool releaser = warp == 2 && lane == 0;
+    for (int g = g0; g < g1 && !aborted(); ++stg) {
       const int seg_before = t.seg;
       locate(s, P.n_q, g, t);
       const int n = stage_tiles(s, t, g, g1);
@@ -339,16 +339,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         nv = min((int64_t)(P.q_pos[t.q] + 1) / P.m, min(P.key_rows, P.max_vis));
       }
+      const int st = stg % STAGES;
+      const bool has_tile = n > 1 || ((g - g0) & 1) == grp;
+      const bool seg_end = (g + n == g1) || (g + n >= s.tile_prefix[t.q + 1]);
+      if (grp == 0 || has_tile) {
+        if (!mbar_wait_warp(&s.accstage[st], (stg / STAGES) & 1, P.status)) {
+          fail(s, P.status);
+          break;
+        }
+        if (releaser) {
+          mbar_arrive(&s.empty[st]);
+          if (seg_end) mbar_arrive(&s.qempty[j]);
+        }
+      }
+      tc_fence_after();
       for (int k = 0; k < n; ++k) {
         const int it = g - g0 + k;
         if ((it & 1) != grp) continue;
         const int a = it % NACC;
-        if (!mbar_wait_warp(&s.accfull[a], (it / NACC) & 1, P.status)) {
-          fail(s, P.status);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
         const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + a * N;
         float s0 = 0.f, s1 = 0.f;
         constexpr int CH = N <= 64 ? N : 64;      // columns per TMEM round trip
@@ -375,8 +383,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int64_t i = (int64_t)(t.lt + k) * KT + r;
         if (i < P.max_vis) P.scores[(int64_t)t.q * P.scores_ld + i] = (i < nv) ? score : -INFINITY;
       }
-      if (!ok) break;
-      const bool seg_end = (g + n == g1) || (g + n >= s.tile_prefix[t.q + 1]);
       if (seg_end) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.qempty[j]);
