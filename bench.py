@@ -359,10 +359,11 @@ class Workload:
             return self.kernel_nodes
         n = 0
         for ly in self.w.layers:
-            # prep + window-KV compress + entry compress (+ key compress)
-            # (+ index scores + top-k) (+ query coding) + MQA + combine
+            # fused append (+ index scores + top-k) (+ query coding when the
+            # append cannot do it) + MQA + combine
             tc_mqa = ly.kv_fp8 and ly.d == 512
-            n += 1 + 2 + (3 if ly.kind == "csa" else 0) + (1 if tc_mqa else 0) + 2
+            coded_in_append = tc_mqa and self.w.B <= 1024
+            n += 1 + (2 if ly.kind == "csa" else 0) + (1 if tc_mqa and not coded_in_append else 0) + 2
         return n
 
     # per-step host<->device traffic of the end-to-end measurement
@@ -397,8 +398,8 @@ def run_gpu(args, dist, rank, world):
         flush_sink.copy_(flush_buf.view(torch.int32).amax().view(1))
 
     wl = Workload(args.workload, rank)
-    launches = wl.launches_per_step()
     wl.capture()
+    launches = wl.launches_per_step()
     for _ in range(args.warmup):
         flush()
         wl.replay()
