@@ -88,3 +88,70 @@ def test_csa_workspace_covers_index_and_sparse_mqa():
                        _abi.E4M3_BF16ROPE, _abi.MXFP4, 1e-6)
     n = lib.v4attn_workspace_size(ctypes.byref(d), 4, 262144)
     assert n >= 4 * 262144 * 4                    # fp32 scores of every visible key
+
+
+def _no_gpu():
+    try:
+        import torch
+        return not torch.cuda.is_available()
+    except Exception:
+        return True
+
+
+@pytest.mark.skipif(not _no_gpu(), reason="host-only check with fake device pointers")
+def test_every_entry_point_rejects_a_short_workspace():
+    """Each call checks its workspace on the host before launching: a decode
+    step given one byte less than v4attn_workspace_size, an indexer call
+    without room for its scores, an MQA call without room for its partials
+    all return V4A_ERR_WORKSPACE.  The pointers are fake (never touched: every
+    check here runs before a launch)."""
+    from long_context_compressed_kv_b200 import _abi
+    lib = _abi.load()
+    fake = ctypes.c_void_p(1 << 20)          # 16-byte aligned, never dereferenced
+    B, L = 4, 1 << 20
+    for kind, m, kv, idx in ((_abi.CSA, 4, _abi.E4M3_BF16ROPE, _abi.MXFP4),
+                             (_abi.HCA, 128, _abi.E4M3_BF16ROPE, _abi.MXFP4),
+                             (_abi.CSA, 4, _abi.F32, _abi.F32)):
+        csa = kind == _abi.CSA
+        d = _abi.LayerDesc(kind, m, 128, 128, 512, 64, 160000.0, 0.0, 64 if csa else 0,
+                           128 if csa else 0, 1024 if csa else 0, kv, idx, 1e-6)
+        rows = L // m
+        need = lib.v4attn_workspace_size(ctypes.byref(d), B, rows)
+        assert need > 0
+        a = _abi.DecodeArgs()
+        a.B = B
+        for f in ("pos", "x_main", "tail", "bias", "kv", "kv_scale", "swa", "swa_scale", "Q",
+                  "sink", "out"):
+            setattr(a, f, fake)
+        if csa:
+            for f in ("x_idx", "itail", "ibias", "keys", "keys_sf", "qI", "qI_sf", "w", "idx_out"):
+                setattr(a, f, fake)
+        a.in_dtype = _abi.BF16
+        a.q_dtype = _abi.BF16
+        a.out_dtype = _abi.BF16
+        a.kv_rows = a.key_rows = rows
+        a.swa_rows = 128
+        a.max_vis = rows
+        assert lib.v4attn_decode(ctypes.byref(d), ctypes.byref(a), fake, need - 1, None) == \
+            _abi.ERR_WORKSPACE
+        q = _abi.MqaArgs()
+        q.n_q, q.B = B, B
+        for f in ("Q", "q_pos", "kv", "kv_scale", "swa", "swa_scale", "sink", "out"):
+            setattr(q, f, fake)
+        q.q_dtype = q.out_dtype = _abi.BF16
+        q.kv_rows, q.swa_rows, q.max_vis = rows, 128, rows
+        if csa:
+            q.idx, q.n_sel = fake, 1024
+            assert lib.v4attn_sparse_mqa(ctypes.byref(d), ctypes.byref(q), fake, 1024,
+                                         None) == _abi.ERR_WORKSPACE
+            ix = _abi.IndexArgs()
+            ix.n_q, ix.B = B, B
+            for f in ("qI", "qI_sf", "w", "q_pos", "keys", "keys_sf", "idx_out"):
+                setattr(ix, f, fake)
+            ix.key_rows = ix.max_vis = rows
+            # the scores of every visible key of every query do not fit in 4 MB - 1
+            assert lib.v4attn_index_topk(ctypes.byref(d), ctypes.byref(ix), fake,
+                                         4 * B * rows - 1, None) == _abi.ERR_WORKSPACE
+        else:
+            assert lib.v4attn_dense_mqa(ctypes.byref(d), ctypes.byref(q), fake, 1024,
+                                        None) == _abi.ERR_WORKSPACE
