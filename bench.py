@@ -138,17 +138,28 @@ def graph_kernel_nodes(graph):
         return None
 
 
+def code_digest(paths):
+    """sha256 of C/CUDA sources with comments and whitespace removed, so that a
+    comment edit does not count as a change of the kernel."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for f in paths:
+        text = open(os.path.join(ROOT, f), encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
+    return h.hexdigest()
+
+
 def _index_traffic():
     """DRAM bytes (read + write) per indexer launch from the committed ncu
-    capture, or None when the kernel's sources have changed since."""
-    import hashlib
+    capture, or None when the kernel's code has changed since."""
     path = os.path.join(ROOT, "profiles", "index_tc_pro_pair_1m_counters.json")
     try:
         rec = json.load(open(path))
-        h = hashlib.sha256()
-        for f in rec["sources"]:
-            h.update(open(os.path.join(ROOT, f), "rb").read())
-        return int(rec["dram_bytes_per_launch"]) if h.hexdigest() == rec["source_sha256"] else None
+        same = code_digest(rec["sources"]) == rec["code_sha256"]
+        return int(rec["dram_bytes_per_launch"]) if same else None
     except (OSError, KeyError, ValueError):
         return None
 
