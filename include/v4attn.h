@@ -236,8 +236,10 @@ typedef struct {
  * most max_vis visible entries per query (>= 256; includes the status word).
  * index_topk and the MQA calls process their queries in chunks of 1024 (up to
  * 2^20 queries per call), so the body of the workspace holds the scores or
- * split-K partials of one chunk; the size grows with n_q only by 24 bytes per
- * query beyond that. */
+ * split-K partials of one chunk; for a V4A_E4M3_BF16ROPE layer it also holds
+ * the coded queries of one chunk (74,752 bytes a query) that the tensor-core
+ * MQA reads.  The size grows with n_q only by 24 bytes per query beyond 1024.
+ * Its layout is internal to the library; one workspace serves one stream. */
 size_t v4attn_workspace_size(const v4attn_layer_desc* desc, int32_t n_q, int64_t max_vis);
 
 /* Zero the workspace's status word (stream-ordered). */
