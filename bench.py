@@ -81,6 +81,181 @@ def build_decode_layer(w, li, inp, in_dtype=None):
     return lay
 
 
+class PrefillPair:
+    """Chunked prefill of a CSA + HCA layer pair (one sequence): ``w.n_queries``
+    new tokens on a prefix of ``w.prefix`` tokens.  ``prefix_state()`` builds
+    the caches of the prefix (untimed); ``step()`` is the timed chunk: the
+    projection of the new tokens' raw activations into every compressor input
+    (one GEMM), the CSA entries, CSA indexer keys and HCA entries their blocks
+    complete, every new token's window KV in both layers, then for every new
+    token the indexer + top-k, the sparse MQA (CSA) and the dense MQA (HCA).
+    Every device buffer is allocated here; every computation runs in the
+    library."""
+
+    CHUNK = 4096                       # host-side generation chunk (rows)
+
+    def __init__(self, w):
+        import torch
+        import long_context_compressed_kv_b200 as v
+        self.v, self.w = v, w
+        csa, hca = w.layers
+        self.csa, self.hca = csa, hca
+        L, P, n = w.L, w.prefix, w.n_queries
+        assert P + n == L
+        # projection columns: CSA (Ca, Cb, Za, Zb), CSA indexer (ICa, ICb, IZa, IZb), HCA (C, Z)
+        names = list(synth.PREFILL_CSA_COLS) + list(synth.PREFILL_IDX_COLS) + \
+            list(synth.PREFILL_HCA_COLS)
+        widths = [csa.d] * 4 + [csa.d_I] * 4 + [hca.d] * 2
+        self.cols, c0 = {}, 0
+        for nm, wd in zip(names, widths):
+            self.cols[nm] = (c0, c0 + wd)
+            c0 += wd
+        self.ncol = c0
+        dev = "cuda"
+        self.x = torch.empty(L, w.d_model, dtype=torch.bfloat16, device=dev)
+        for r0 in range(0, L, self.CHUNK):
+            rows = np.arange(r0, min(L, r0 + self.CHUNK))
+            self.x[r0:r0 + len(rows)] = torch.from_numpy(synth.prefill_x(w, rows)).to(dev)
+        self.W = torch.from_numpy(synth.prefill_weight(w)).to(dev).to(torch.bfloat16)
+        self.Y = torch.empty(L, self.ncol, dtype=torch.float32, device=dev)
+        self.dc, self.dh = desc_for(csa), desc_for(hca)
+        self.rows_c = (L // csa.m + 127) // 128 * 128
+        self.rows_h = max(128, (L // hca.m + 127) // 128 * 128)
+
+        def rows_of(fmt, c, nr, d_rope=64):
+            out = torch.zeros(1, nr, v.row_bytes(fmt, c, d_rope), dtype=torch.uint8, device=dev)
+            sc = (torch.zeros(1, nr, dtype=torch.float32, device=dev) if fmt == v.E4M3_BF16ROPE
+                  else torch.zeros(1, nr, c // 32, dtype=torch.uint8, device=dev))
+            return out, sc
+        self.kv_c, self.kvs_c = rows_of(v.E4M3_BF16ROPE, csa.d, self.rows_c)
+        self.keys, self.keys_sf = rows_of(v.MXFP4, csa.d_I, self.rows_c, 0)
+        self.kv_h, self.kvs_h = rows_of(v.E4M3_BF16ROPE, hca.d, self.rows_h)
+        # window KV of every token (token t at row t)
+        self.swa_c, self.swas_c = rows_of(v.E4M3_BF16ROPE, csa.d, L)
+        self.swa_h, self.swas_h = rows_of(v.E4M3_BF16ROPE, hca.d, L)
+        # per-query inputs of the new tokens
+        self.Q_c = torch.empty(n, csa.H, csa.d, dtype=torch.bfloat16, device=dev)
+        self.Q_h = torch.empty(n, hca.H, hca.d, dtype=torch.bfloat16, device=dev)
+        self.qI = torch.zeros(n, csa.H_I, csa.d_I // 2, dtype=torch.uint8, device=dev)
+        self.qI_sf = torch.zeros(n, csa.H_I, csa.d_I // 32, dtype=torch.uint8, device=dev)
+        self.wI = torch.empty(n, csa.H_I, dtype=torch.float32, device=dev)
+        for r0 in range(0, n, self.CHUNK):
+            rows = np.arange(r0, min(n, r0 + self.CHUNK))
+            q0 = synth.prefill_queries(w, 0, rows=rows)
+            q1 = synth.prefill_queries(w, 1, rows=rows)
+            sl = slice(r0, r0 + len(rows))
+            self.Q_c[sl] = torch.from_numpy(q0["Q"]).to(dev)
+            self.Q_h[sl] = torch.from_numpy(q1["Q"]).to(dev)
+            self.wI[sl] = torch.from_numpy(q0["w"]).to(dev)
+            vals = torch.from_numpy(q0["qI"]).to(dev).reshape(1, -1, csa.d_I)
+            qrows = self.qI[sl].reshape(1, -1, csa.d_I // 2)
+            qsf = self.qI_sf[sl].reshape(1, -1, csa.d_I // 32)
+            from long_context_compressed_kv_b200.decode import code_rows as _code_rows
+            _code_rows(self.dc, vals, v.MXFP4, qrows, qsf, 0)
+            self.qI[sl] = qrows.reshape(len(rows), csa.H_I, -1)
+            self.qI_sf[sl] = qsf.reshape(len(rows), csa.H_I, -1)
+        q0 = synth.prefill_queries(w, 0, rows=np.arange(1))
+        q1 = synth.prefill_queries(w, 1, rows=np.arange(1))
+        self.bias_c = torch.from_numpy(q0["bias"]).to(dev)
+        self.ibias = torch.from_numpy(q0["ibias"]).to(dev)
+        self.bias_h = torch.from_numpy(q1["bias"]).to(dev)
+        self.sink_c = torch.from_numpy(q0["sink"]).to(dev)
+        self.sink_h = torch.from_numpy(q1["sink"]).to(dev)
+        self.pos = torch.arange(P, L, dtype=torch.int64, device=dev)
+        self.seq = torch.zeros(n, dtype=torch.int32, device=dev)
+        self.idx = torch.full((n, csa.top_k), -1, dtype=torch.int32, device=dev)
+        self.out_c = torch.zeros(n, csa.H, csa.d, dtype=torch.bfloat16, device=dev)
+        self.lse_c = torch.zeros(n, csa.H, dtype=torch.float32, device=dev)
+        self.out_h = torch.zeros(n, hca.H, hca.d, dtype=torch.bfloat16, device=dev)
+        self.lse_h = torch.zeros(n, hca.H, dtype=torch.float32, device=dev)
+        self.ws_c = v.workspace(self.dc, n, self.rows_c)
+        self.ws_h = v.workspace(self.dh, n, self.rows_h)
+        self._one = lambda val: torch.full((1,), val, dtype=torch.int64, device=dev)
+        self.L_t = self._one(L)
+
+    def _col(self, nm):
+        c0, _ = self.cols[nm]
+        return self.Y[:, c0:]
+
+    def _compress_tokens(self, t0, t1, seq_len):
+        """Entries and keys whose blocks complete in tokens [t0, t1) (a block
+        that straddles t0 was skipped as incomplete before), and the window
+        rows of tokens [t0, t1)."""
+        v, csa, hca, L = self.v, self.csa, self.hca, self.w.L
+        common = dict(in_rows=L, in_seq_stride=L * self.ncol, in_row_stride=self.ncol,
+                      seq_len=seq_len)
+        e0, ne = t0 // csa.m, t1 // csa.m - t0 // csa.m
+        v.compress(self.dc, m=csa.m, overlap=True, c=csa.d, Ca=self._col("Ca"),
+                   Za=self._col("Za"), Cb=self._col("Cb"), Zb=self._col("Zb"), bias=self.bias_c,
+                   entry_begin=self._one(e0), n_entries=ne, complete_only=True,
+                   out_dtype=v.E4M3_BF16ROPE, out=self.kv_c, out_scale=self.kvs_c,
+                   out_rows=self.rows_c, **common)
+        v.compress(self.dc, m=csa.m, overlap=True, c=csa.d_I, Ca=self._col("ICa"),
+                   Za=self._col("IZa"), Cb=self._col("ICb"), Zb=self._col("IZb"),
+                   bias=self.ibias, entry_begin=self._one(e0), n_entries=ne, complete_only=True,
+                   out_dtype=v.MXFP4, out=self.keys, out_scale=self.keys_sf, out_rows=self.rows_c,
+                   apply_rmsnorm=False, apply_rope=False, **common)
+        h0, nh = t0 // hca.m, t1 // hca.m - t0 // hca.m
+        v.compress(self.dh, m=hca.m, overlap=False, c=hca.d, Ca=self._col("C"),
+                   Za=self._col("Z"), bias=self.bias_h, entry_begin=self._one(h0), n_entries=nh,
+                   complete_only=True, out_dtype=v.E4M3_BF16ROPE, out=self.kv_h,
+                   out_scale=self.kvs_h, out_rows=self.rows_h, **common)
+        for desc, col, out, sc in ((self.dc, "Ca", self.swa_c, self.swas_c),
+                                   (self.dh, "C", self.swa_h, self.swas_h)):
+            v.compress(desc, m=1, overlap=False, c=csa.d, Ca=self._col(col), Za=None,
+                       entry_begin=self._one(t0), n_entries=t1 - t0, out_dtype=v.E4M3_BF16ROPE,
+                       out=out, out_scale=sc, out_rows=L, **common)
+
+    def prefix_state(self):
+        """The caches of the prefix tokens (not part of the timed step)."""
+        P = self.w.prefix
+        if P:
+            self.v.project(self.x[:P], self.W, self.Y[:P])
+            self._compress_tokens(0, P, self._one(P))
+
+    def step(self):
+        """The timed chunked-prefill step of the new tokens."""
+        for _, f in self.phases():
+            f()
+
+    def phases(self):
+        """The step's calls as (name, callable), in step order."""
+        v, csa, hca, w = self.v, self.csa, self.hca, self.w
+        P, L = w.prefix, w.L
+        return [
+            ("project (a0)", lambda: v.project(self.x[P:], self.W, self.Y[P:])),
+            ("compress (a1)", lambda: self._compress_tokens(P, L, self.L_t)),
+            ("index_topk (a3, a4)", lambda: v.index_topk(
+                self.dc, qI=self.qI, qI_sf=self.qI_sf, w=self.wI, q_pos=self.pos, q_seq=self.seq,
+                B=1, keys=self.keys, keys_sf=self.keys_sf, key_rows=self.rows_c,
+                max_vis=L // csa.m, idx_out=self.idx, ws=self.ws_c)),
+            ("sparse_mqa (a2, a5-a7)", lambda: v.sparse_mqa(
+                self.dc, Q=self.Q_c, q_pos=self.pos, q_seq=self.seq, B=1, kv=self.kv_c,
+                kv_scale=self.kvs_c, kv_rows=self.rows_c, swa=self.swa_c, swa_scale=self.swas_c,
+                swa_rows=L, idx=self.idx, out=self.out_c, ws=self.ws_c, sink=self.sink_c,
+                lse=self.lse_c)),
+            ("dense_mqa (a2, a5-a7)", lambda: v.dense_mqa(
+                self.dh, Q=self.Q_h, q_pos=self.pos, q_seq=self.seq, B=1, kv=self.kv_h,
+                kv_scale=self.kvs_h, kv_rows=self.rows_h, swa=self.swa_h, swa_scale=self.swas_h,
+                swa_rows=L, max_vis=L // hca.m, out=self.out_h, ws=self.ws_h, sink=self.sink_h,
+                lse=self.lse_h)),
+        ]
+
+    def flops(self):
+        """Algorithmic FLOPs of one step by tensor-core format."""
+        csa, hca, w = self.csa, self.hca, self.w
+        P, L, n = w.prefix, w.L, w.n_queries
+        pos = np.arange(P, L, dtype=np.float64)
+        nv_c = np.floor((pos + 1) / csa.m)
+        nv_h = np.floor((pos + 1) / hca.m)
+        win = np.minimum(pos + 1, csa.n_win)
+        proj = 2.0 * n * w.d_model * self.ncol
+        idx = float(np.sum(nv_c)) * 2 * csa.H_I * csa.d_I
+        mqa_c = float(np.sum(np.minimum(nv_c, csa.top_k) + win)) * 4 * csa.H * csa.d
+        mqa_h = float(np.sum(nv_h + np.minimum(pos + 1, hca.n_win))) * 4 * hca.H * hca.d
+        return {"bf16": proj, "fp4": idx, "fp8": mqa_c + mqa_h}
+
+
 def algorithmic_bytes(w):
     """Bytes one decode step must move (per the method), per layer: visible or
     selected entries x 580 B, indexer keys x 68 B, window tokens x 580 B, Q in
@@ -461,23 +636,42 @@ def run_gpu(args, dist, rank, world):
                  "achieved_gbs": round(step_bytes / (ms / 1e3) / 1e9, 1),
                  "frac_hbm": round(step_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers: every step
+    # copies its inputs from pinned host memory, runs the step, and reads the
+    # outputs back; the step itself as the captured graph (how a serving loop
+    # runs it) and, separately, as eager calls through the Python binding
     ins, outs = wl.host_io()
     h2d = sum(h.numel() * h.element_size() for h, _ in ins)
     d2h = sum(h.numel() * h.element_size() for h, _ in outs)
 
-    def e2e_step():
-        for h, d in ins:
-            d.copy_(h, non_blocking=True)
-        wl.step()
-        for h, d in outs:
-            h.copy_(d, non_blocking=True)
-    for _ in range(args.warmup):
-        flush()
-        e2e_step()
-    barrier(dist)
-    e2e_ms = max_over_ranks(float(np.mean(timed_device(e2e_step, flush, args.steps, stream))), dist)
+    def with_copies(run):
+        def f():
+            for h, d in ins:
+                d.copy_(h, non_blocking=True)
+            run()
+            for h, d in outs:
+                h.copy_(d, non_blocking=True)
+        return f
+    e2e = {}
+    for name, run in (("graph", wl.replay), ("eager", wl.step)):
+        f = with_copies(run)
+        for _ in range(args.warmup):
+            flush()
+            f()
+        barrier(dist)
+        e2e[name] = max_over_ranks(float(np.mean(timed_device(f, flush, args.steps, stream))), dist)
+    e2e_ms = e2e["graph"]
     e2e_val = world * q_step / (e2e_ms / 1e3)
+    e2e_eager = world * q_step / (e2e["eager"] / 1e3)
+    peaks_tc = measure_tc_peaks(stream)
+    if roof is not None:
+        fp4 = abytes["csa"]["keys"] * 2 * csa[0].desc.H_I * csa[0].desc.d_I
+        ach_t = fp4 / (t_idx / 1e3) / 1e12
+        roof["tensor"] = {"format": "mxfp4", "flops_per_launch": int(fp4),
+                          "achieved_tflops": round(ach_t, 1),
+                          "peak_tflops": peaks_tc["fp4_mxf4_tflops"],
+                          "frac": round(ach_t / peaks_tc["fp4_mxf4_tflops"], 4),
+                          "peak_source": "measured in this run (tcgen05 probe)"}
 
     also = {}
     if not args.no_also and world == 1:
@@ -498,9 +692,123 @@ def run_gpu(args, dist, rank, world):
             del w2
             torch.cuda.empty_cache()
     return dict(value=value, ms=ms, roof=roof, step_roof=step_roof, clocks=clk.summary(),
-                e2e=dict(value=e2e_val, h2d=h2d, d2h=d2h, ms=e2e_ms), also=also,
+                e2e=dict(value=e2e_val, h2d=h2d, d2h=d2h, ms=e2e_ms, eager_value=e2e_eager,
+                         eager_ms=e2e["eager"]), also=also, tc_peaks=peaks_tc,
                 launches=launches, q_step=q_step,
                 per_step=per_step)
+
+
+def measure_tc_peaks(stream, reps=5, n_iter=16384):
+    """Dense MMA rate of the three tcgen05 kinds the kernels use (bf16, E4M3,
+    block-scaled MXFP4), from the library's probe: one CTA per SM issuing
+    128 x 256 MMAs over shared-memory operands; best of ``reps`` launches timed
+    with CUDA events on ``stream``, with the SM clock sampled meanwhile."""
+    import torch
+    import long_context_compressed_kv_b200 as v
+    out = {}
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for kind, name in ((0, "bf16"), (1, "fp8_e4m3"), (2, "fp4_mxf4")):
+            v.tc_peak_probe(kind, 64, stream=stream)          # warm-up
+            best = 0.0
+            clk.start()
+            for _ in range(reps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                flops, ctas = v.tc_peak_probe(kind, n_iter, stream=stream)
+                b.record(stream)
+                b.synchronize()
+                best = max(best, flops / (a.elapsed_time(b) / 1e3) / 1e12)
+            clk.stop()
+            out[name + "_tflops"] = round(best, 1)
+    out["ctas"] = ctas
+    out["shape"] = "M=128 N=256 per instruction, 1 CTA per SM, operands in shared memory"
+    out["clocks"] = clk.summary()
+    return out
+
+
+def run_prefill(args, dist, rank, world):
+    """The chunked-prefill workload: one step = the whole chunk of new tokens
+    through both layers (bench.PrefillPair.step), tokens/s."""
+    import torch
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    stream = torch.cuda.current_stream()
+    w = rank_workload(args.workload, rank)
+    pp = PrefillPair(w)
+    pp.prefix_state()
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_sink = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def flush():
+        flush_buf.zero_()
+        flush_sink.copy_(flush_buf.view(torch.int32).amax().view(1))
+    steps = min(args.steps, 10)
+    for _ in range(args.warmup):
+        flush()
+        pp.step()
+    barrier(dist)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        barrier(dist)
+        clk.start()
+        per_step = timed_device(pp.step, flush, steps, stream)
+        clk.stop()
+        barrier(dist)
+    ms = max_over_ranks(float(np.mean(per_step)), dist)
+    n = w.n_queries
+    value = world * n / (ms / 1e3)
+    # per-phase device time (each phase alone, after an L2 flush)
+    phases = {}
+    for name, f in pp.phases():
+        phases[name] = round(float(np.mean(timed_device(f, flush, 3, stream))), 4)
+    peaks = measure_tc_peaks(stream)
+    fl = pp.flops()
+    pk = {"bf16": peaks["bf16_tflops"], "fp4": peaks["fp4_mxf4_tflops"],
+          "fp8": peaks["fp8_e4m3_tflops"]}
+    t_roof = sum(fl[k] / (pk[k] * 1e12) for k in fl)       # seconds at the measured peaks
+    total = sum(fl.values())
+    dom = max(phases, key=phases.get)
+    dom_fl = {"project (a0)": ("bf16", fl["bf16"]), "index_topk (a3, a4)": ("fp4", fl["fp4"])}
+    roof = {"bound": "tensor", "achieved": round(total / (ms / 1e3) / 1e12, 2),
+            "peak": round(total / t_roof / 1e12, 1), "unit": "TFLOP/s",
+            "frac": round(t_roof / (ms / 1e3), 5), "traffic": None,
+            "note": "step FLOPs over the sum of each format's FLOPs at its measured tcgen05 "
+                    "peak (bf16 projection, MXFP4 indexer, E4M3/bf16 MQA)",
+            "flops": {k: float(v_) for k, v_ in fl.items()}, "dominant_phase": dom}
+    if dom in dom_fl:
+        fmt, f_ = dom_fl[dom]
+        roof["dominant"] = {"phase": dom, "format": fmt,
+                            "achieved_tflops": round(f_ / (phases[dom] / 1e3) / 1e12, 2),
+                            "peak_tflops": pk[fmt],
+                            "frac": round(f_ / (phases[dom] / 1e3) / 1e12 / pk[fmt], 5)}
+    # end to end: the chunk's raw tokens and per-query inputs copied in from
+    # pinned memory, the step, both layers' outputs and LSE read back
+    e2e = None
+    try:
+        P = w.prefix
+        ins = [(torch.empty(t.shape, dtype=t.dtype, pin_memory=True), t)
+               for t in (pp.x[P:], pp.Q_c, pp.Q_h, pp.qI, pp.qI_sf, pp.wI)]
+        outs = [(torch.empty(t.shape, dtype=t.dtype, pin_memory=True), t)
+                for t in (pp.out_c, pp.out_h, pp.lse_c, pp.lse_h, pp.idx)]
+        for h, d in ins:
+            h.copy_(d)
+
+        def e2e_step():
+            for h, d in ins:
+                d.copy_(h, non_blocking=True)
+            pp.step()
+            for h, d in outs:
+                h.copy_(d, non_blocking=True)
+        e2e_step()
+        barrier(dist)
+        e_ms = max_over_ranks(float(np.mean(timed_device(e2e_step, flush, min(steps, 3),
+                                                         stream))), dist)
+        e2e = {"value": round(world * n / (e_ms / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(sum(h.numel() * h.element_size() for h, _ in ins)),
+               "d2h_bytes_per_step": int(sum(h.numel() * h.element_size() for h, _ in outs)),
+               "ms_per_step": round(e_ms, 4)}
+    except RuntimeError as ex:              # pinned host memory refused
+        e2e = {"value": None, "unavailable": str(ex).splitlines()[0][:200]}
+    return dict(value=value, ms=ms, roof=roof, phases=phases, clocks=clk.summary(), e2e=e2e,
+                tc_peaks=peaks, steps=steps, w=w)
 
 
 def _peaks():
@@ -514,6 +822,19 @@ def _peaks():
 
 
 # ------------------------------------------------------------------ the oracle (CPU) arm
+
+def _cpu_info():
+    """(logical CPUs of this host, CPU model string)."""
+    model = None
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return os.cpu_count(), model
+
 
 def _blas_threads():
     try:
@@ -545,6 +866,63 @@ def oracle_sample(name, seconds_target=12.0, max_seqs=None):
     return n / t_total, f"{n} sequence(s) x {len(w.layers)} layer(s) of {name}", t_total
 
 
+def oracle_prefill_sample(name, seconds_target=12.0):
+    """Time the CPU oracle's per-token work of the chunked-prefill workload on
+    a bounded sample: for consecutive new tokens at the end of the chunk, the
+    token's projection row, its share of the pooling (one CSA entry + indexer
+    key per 4 tokens, one HCA entry per 128), the indexer scores over every
+    visible key, top-k, and both layers' attention.  The cached keys and
+    entries it reads are synthetic stand-ins of the right shapes (the time of
+    these steps does not depend on their values).  Returns (tokens/s,
+    description, seconds)."""
+    from oracle import compress as ocomp, indexer as oidx, mqa as omqa, pipeline
+    w = synth.WORKLOADS[name]
+    csa, hca = w.layers
+    W = synth.prefill_weight(w).astype(np.float64)
+    rng = np.random.default_rng(0)
+    nk = w.L // csa.m
+    keys = rng.standard_normal((nk, csa.d_I))
+    ents_c = rng.standard_normal((nk, csa.d))
+    ents_h = rng.standard_normal((w.L // hca.m, hca.d))
+    win = rng.standard_normal((csa.n_win, csa.d))
+    n, t_total, r = 0, 0.0, w.n_queries - 1
+    blk = synth.ROWS_PER_BLOCK
+    cache = {}
+    while t_total < seconds_target and r >= 0:
+        b0 = r // blk * blk
+        if b0 not in cache:                # one generator block of rows at a time
+            rows = np.arange(b0, min(w.n_queries, b0 + blk))
+            cache = {b0: (synth.prefill_queries(w, 0, rows=rows),
+                          synth.prefill_queries(w, 1, rows=rows),
+                          synth.prefill_x(w, rows=rows + w.prefix).astype(np.float64))}
+        Q0, Q1, X = cache[b0]
+        j = r - b0
+        q0 = {k: (v_[j:j + 1] if k in ("Q", "qI", "w") else v_) for k, v_ in Q0.items()}
+        q1 = {k: (v_[j:j + 1] if k == "Q" else v_) for k, v_ in Q1.items()}
+        x = X[j:j + 1]
+        t0 = time.perf_counter()
+        p = w.prefix + r
+        y = x @ W                                             # a0
+        if p % csa.m == 0:                                    # a1 (amortised shares)
+            i = np.array([p // csa.m])
+            ocomp.pool(i, csa.m, True, w.L, lambda t: np.repeat(y[:, :csa.d], t.size, 0).reshape(
+                t.shape + (csa.d,)), lambda t: np.zeros(t.shape + (csa.d,)), q0["bias"],
+                lambda t: np.zeros(t.shape + (csa.d,)), lambda t: np.zeros(t.shape + (csa.d,)))
+        nv = (p + 1) // csa.m
+        s = oidx.scores(pipeline.store_key(q0["qI"][0], csa)[1], q0["w"][0], keys[:nv])  # a3
+        sel = oidx.topk(s, nv, csa.top_k)                     # a4
+        kc = np.concatenate([ents_c[sel[sel >= 0]], win], 0)
+        qc = omqa.prepare_query(q0["Q"][0], p, csa.d_rope, csa.rope_theta, True)
+        omqa.attend(qc, kc, 1 / np.sqrt(csa.d), q0["sink"])   # a6 CSA
+        kh = np.concatenate([ents_h[:(p + 1) // hca.m], win], 0)
+        qh = omqa.prepare_query(q1["Q"][0], p, hca.d_rope, hca.rope_theta, True)
+        omqa.attend(qh, kh, 1 / np.sqrt(hca.d), q1["sink"])   # a6 HCA
+        t_total += time.perf_counter() - t0
+        n += 1
+        r -= 1
+    return n / t_total, f"{n} consecutive new tokens at the end of the chunk of {name}", t_total
+
+
 def run_reference(args):
     """The reference arm: the fp64 CPU oracle, as it stands, on host cores."""
     from oracle import pipeline
@@ -569,6 +947,7 @@ def run_reference(args):
             "config": {"workload": args.workload, "batch": w.B, "context": w.L,
                        "layers": [ly.kind for ly in w.layers], "l2": "n/a (CPU)"},
             "cpu_baseline": {"value": round(value, 4), "unit": "queries/s", "cores": cores,
+                             "nproc": _cpu_info()[0], "cpu_model": _cpu_info()[1],
                              "kind": "oracle",
                              "sample": f"per step: 1 sequence through every layer of {args.workload}"},
             "e2e": {"value": round(value, 4), "unit": "queries/s", "h2d_bytes_per_step": 0,
@@ -581,7 +960,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="v4attn", choices=["v4attn", "reference"])
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(synth.WORKLOADS))
@@ -605,6 +984,39 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
+    if synth.WORKLOADS[args.workload].prefix > 0:
+        res = run_prefill(args, dist, rank, world)
+        if rank == 0:
+            w = res["w"]
+            line = {
+                "metric": "chunked-prefill tokens/s of a V4-Flash CSA + HCA layer pair; "
+                          "% of FP4/FP8/BF16-TC roofline",
+                "value": round(res["value"], 1), "unit": "tokens/s", "n_gpus": world,
+                "steps": res["steps"], "warmup": args.warmup, "ms_per_step": round(res["ms"], 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16 projection, e4m3+bf16 KV, mxfp4 indexer, f32 accumulate",
+                "data": "synthetic",
+                "config": {"workload": args.workload, "new_tokens": w.n_queries,
+                           "prefix": w.prefix, "d_model": w.d_model,
+                           "layers": [f"{ly.kind} m={ly.m} H={ly.H} d={ly.d}" +
+                                      (f" top_k={ly.top_k} H_I={ly.H_I}x{ly.d_I}"
+                                       if ly.kind == "csa" else "") for ly in w.layers],
+                           "l2": "flushed between steps (320 MB write, then read back)"},
+                "e2e": res["e2e"], "roofline": res["roof"], "phases_ms": res["phases"],
+                "tc_peaks": res["tc_peaks"], "clocks": res["clocks"], "cpu_baseline": None,
+            }
+            if world == 1 and not args.no_cpu_baseline:
+                val, sample, secs = oracle_prefill_sample(args.workload)
+                ncpu, model = _cpu_info()
+                line["cpu_baseline"] = {"value": round(val, 3), "unit": "tokens/s",
+                                        "cores": _blas_threads(), "nproc": ncpu,
+                                        "cpu_model": model, "kind": "oracle", "sample": sample,
+                                        "seconds": round(secs, 1)}
+            print(json.dumps(line), flush=True)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     res = run_gpu(args, dist, rank, world)
     if res.get("profile"):
         if rank == 0:
@@ -616,8 +1028,11 @@ def main():
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             val, sample, secs = oracle_sample(args.workload)
+            ncpu, model = _cpu_info()
             cpu = {"value": round(val, 4), "unit": "queries/s", "cores": _blas_threads(),
-                   "kind": "oracle", "sample": sample, "seconds": round(secs, 1)}
+                   "kind": "oracle", "sample": sample, "seconds": round(secs, 1),
+                   "nproc": ncpu, "cpu_model": model,
+                   "threads": "numpy/BLAS threads of the fp64 matrix products (cores)"}
         line = {
             "metric": METRIC, "value": round(res["value"], 1), "unit": "queries/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -634,7 +1049,13 @@ def main():
             "e2e": {"value": round(res["e2e"]["value"], 1), "unit": "queries/s",
                     "h2d_bytes_per_step": int(res["e2e"]["h2d"]),
                     "d2h_bytes_per_step": int(res["e2e"]["d2h"]),
-                    "ms_per_step": round(res["e2e"]["ms"], 5)},
+                    "ms_per_step": round(res["e2e"]["ms"], 5),
+                    "how": "pinned H2D of the step's inputs + captured-graph step + D2H of "
+                           "the outputs, every step",
+                    "eager": {"value": round(res["e2e"]["eager_value"], 1),
+                              "ms_per_step": round(res["e2e"]["eager_ms"], 5),
+                              "how": "the same copies around eager calls through the binding"}},
+            "tc_peaks": res["tc_peaks"],
             "gpu_launches": res["launches"] * args.steps,
             "roofline": res["roof"],
             "step_roofline": res["step_roof"],

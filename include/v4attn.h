@@ -136,7 +136,12 @@ typedef struct {
  * "FP4 QAT、可恢复 rollout 与百万 Token RL" for the MXFP4 QK path):
  *   s_i = sum_h w_h * max(0, q_h . k_i)   for i < n_vis(p)
  * then the top_k largest s_i (exact ties to the lower index), written in
- * ascending index order, -1 padded when n_vis < top_k.  */
+ * ascending index order, -1 padded when n_vis < top_k.
+ * Formats: V4A_F32 (d_I 32, 64 or 128, any H_I <= 128) runs on CUDA cores;
+ * V4A_MXFP4 runs on the tcgen05 block-scaled tensor-core kernel only and needs
+ * d_I = 128, H_I in {32, 64, 128} and key_rows % 4 == 0 (else
+ * V4A_ERR_UNSUPPORTED), with qI, qI_sf, w, keys, keys_sf 16-byte aligned
+ * (else V4A_ERR_INVALID_ARG).  */
 typedef struct {
   int32_t n_q;                /* queries, 1 .. 2^20 */
   int32_t B;                  /* sequences */
@@ -163,7 +168,11 @@ typedef struct {
  *           sparse: entries idx[q][0..n_sel) (-1 skipped) + window tokens,
  *           dense:  entries 0..n_vis(p)-1 + window tokens;
  *   o_h   = sum_j exp(s_hj) k_j / (exp(sink_h) + sum_j exp(s_hj))   (V = K)
- *   out   = o_h with its RoPE dims rotated by -p;  lse_h = log of the denominator.  */
+ *   out   = o_h with its RoPE dims rotated by -p;  lse_h = log of the denominator.
+ * Formats: V4A_F32 caches run on CUDA cores; V4A_E4M3_BF16ROPE caches run on
+ * the tcgen05 tensor-core kernel only and need a bf16 Q (else
+ * V4A_ERR_UNSUPPORTED), 16-byte aligned Q, kv, swa and out (else
+ * V4A_ERR_INVALID_ARG), and B * kv_rows, B * swa_rows < 2^31.  */
 typedef struct {
   int32_t n_q;                /* queries, 1 .. 2^20 */
   int32_t B;
@@ -266,8 +275,9 @@ v4attn_status v4attn_project(const v4attn_project_args* args, cudaStream_t strea
  *   - The scratch it needs (a status word and the fp32 scores) is one array
  *     compiled into the library, so every GPU that loads libv4attn holds it
  *     (about 8.4 MB) until the process exits.
- *   - Limit: n_q * max(max_vis, 1) <= V4A_NOALLOC_MAX_SCORES and n_q <= 1365;
- *     a larger call returns V4A_ERR_UNSUPPORTED before launching anything.
+ *   - Limits: n_q * max(max_vis, 1) <= V4A_NOALLOC_MAX_SCORES and
+ *     n_q <= V4A_NOALLOC_MAX_QUERIES; a larger call returns
+ *     V4A_ERR_UNSUPPORTED before launching anything.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
@@ -276,14 +286,51 @@ v4attn_status v4attn_project(const v4attn_project_args* args, cudaStream_t strea
  *     the call clears the status word and rewrites every score it reads, but
  *     two calls whose work overlaps on the GPU (unordered streams, or several
  *     host threads) race on the array; the caller must order them.
- *   - Device-side check bits land in the array's status word, which the API
- *     does not expose; out-of-range positions are skipped as in
- *     v4attn_index_topk.
+ *   - Device-side check bits (out-of-range positions, which are skipped as in
+ *     v4attn_index_topk, and a bounded wait that ran out, after which the
+ *     selection is not valid) land in the array's status word; each call
+ *     clears it first.  v4attn_noalloc_device_status reads it.
  * Arguments and results are those of v4attn_index_topk (scores_out may be
  * given; idx_out may be NULL only when scores_out is given). */
 #define V4A_NOALLOC_MAX_SCORES 2097152
+#define V4A_NOALLOC_MAX_QUERIES 1365
 v4attn_status v4attn_index_topk_noalloc(const v4attn_layer_desc* desc,
                                         const v4attn_index_args* args, cudaStream_t stream);
+/* Status word of the last v4attn_index_topk_noalloc call on the current
+ * device, read and mapped as v4attn_device_status does (it synchronises
+ * `stream`; order it after the call). */
+v4attn_status v4attn_noalloc_device_status(cudaStream_t stream, uint32_t* bits);
+
+/* Failure-detection test hook (no counterpart in the pages): v4attn_index_topk
+ * on the MXFP4 tensor-core indexer with one of its waits made to run out.  The
+ * kernel's MMA-issuing warp first waits on a barrier that nothing ever
+ * completes, with every bounded wait of the launch limited to `wait_ns`
+ * (1e5 .. 1e9 ns).  That wait gives up before any MMA is issued, records
+ * V4A_ERR_TIMEOUT (status bit 8, and bit 16 + 12 for this wait site) in the
+ * workspace's status word, and the kernel's other warps stop at their next
+ * wait; the launch returns with no copy in flight and its tensor memory
+ * released.  Read the result with v4attn_device_status; clear the word with
+ * v4attn_workspace_init before the next call.  Arguments as v4attn_index_topk
+ * (scores written by the stalled launch are undefined).  Returns
+ * V4A_ERR_UNSUPPORTED for a layer whose indexer is not MXFP4. */
+v4attn_status v4attn_debug_index_stall(const v4attn_layer_desc* desc,
+                                       const v4attn_index_args* args, void* ws, size_t ws_bytes,
+                                       uint32_t wait_ns, cudaStream_t stream);
+
+/* Tensor-core throughput probe (measurement support; no counterpart in the
+ * pages).  Launches one CTA per SM, each issuing n_iter x 4 back-to-back
+ * tcgen05 MMAs of M = 128 x N = 256 with operands resident in shared memory
+ * and fp32 accumulators in tensor memory, of kind
+ *   0: kind::f16 bf16 x bf16 (K = 16),  1: kind::f8f6f4 E4M3 x E4M3 (K = 32),
+ *   2: kind::mxf4 block-scaled E2M1 x E2M1, E8M0 per 32 elements (K = 64).
+ * Time the launch on `stream` (e.g. with CUDA events) and divide *flops (the
+ * dense FLOPs the launch performs, 2*M*N*K per MMA) by it for the GPU's MMA
+ * rate of that format.  *n_ctas receives the CTA count.  `ws`: a workspace
+ * whose status word receives V4A_ERR_TIMEOUT's bit if the final wait runs
+ * out, or NULL.  Nothing is read or written in global memory otherwise.
+ * n_iter in 1 .. 2^24, else V4A_ERR_INVALID_ARG. */
+v4attn_status v4attn_tc_peak_probe(int32_t kind, int32_t n_iter, int32_t* n_ctas, double* flops,
+                                   void* ws, cudaStream_t stream);
 
 /* Synchronise `stream`, read the status word the kernels left in `ws` and
  * map it: 0 -> V4A_OK, a bounds / argument check -> V4A_ERR_DEVICE_CHECK,

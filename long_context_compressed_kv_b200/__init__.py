@@ -21,7 +21,9 @@ from ._abi import (BF16, CSA, E4M3_BF16ROPE, F32, HCA, MXFP4, CompressArgs, Deco
 _lib = _abi.load()
 
 __all__ = ["F32", "BF16", "E4M3_BF16ROPE", "MXFP4", "CSA", "HCA", "V4AttnError", "layer_desc",
-           "workspace", "workspace_size", "compress", "index_topk", "index_topk_noalloc",
+           "workspace", "workspace_size", "workspace_init", "compress", "index_topk",
+           "index_topk_noalloc", "noalloc_device_status", "debug_index_stall",
+           "device_status_code", "tc_peak_probe",
            "sparse_mqa", "dense_mqa",
            "decode", "project", "device_status", "build_info", "row_bytes"]
 
@@ -126,6 +128,52 @@ def index_topk_noalloc(desc: LayerDesc, *, qI, w, q_pos, keys, key_rows: int, ma
                   _p(scores_out))
     _check("v4attn_index_topk_noalloc",
            _lib.v4attn_index_topk_noalloc(ctypes.byref(desc), ctypes.byref(a), _stream(stream)))
+
+
+def noalloc_device_status(stream=None) -> int:
+    """Raw status word of the last index_topk_noalloc call on this device
+    (synchronises); raises on a device-side error."""
+    bits = ctypes.c_uint32(0)
+    st = _lib.v4attn_noalloc_device_status(_stream(stream), ctypes.byref(bits))
+    _check("v4attn_noalloc_device_status", st)
+    return bits.value
+
+
+def debug_index_stall(desc: LayerDesc, *, qI, w, q_pos, keys, key_rows: int, max_vis: int, ws,
+                      wait_ns: int, qI_sf=None, keys_sf=None, q_seq=None, B=None,
+                      scores_out=None, idx_out=None, stream=None):
+    """Failure-detection hook: index_topk with one wait of the tensor-core
+    indexer made to run out after ``wait_ns`` (see include/v4attn.h)."""
+    n_q = int(q_pos.numel())
+    a = IndexArgs(n_q, B if B is not None else n_q, _p(qI), _p(qI_sf), _p(w), _p(q_seq),
+                  _p(q_pos), _p(keys), _p(keys_sf), key_rows, max_vis, _p(idx_out),
+                  _p(scores_out))
+    _check("v4attn_debug_index_stall",
+           _lib.v4attn_debug_index_stall(ctypes.byref(desc), ctypes.byref(a), _p(ws), ws.numel(),
+                                         int(wait_ns), _stream(stream)))
+
+
+def tc_peak_probe(kind: int, n_iter: int, ws=None, stream=None):
+    """Launch the tensor-core throughput probe (see include/v4attn.h);
+    returns (dense FLOPs of the launch, CTAs)."""
+    n = ctypes.c_int32(0)
+    f = ctypes.c_double(0.0)
+    _check("v4attn_tc_peak_probe",
+           _lib.v4attn_tc_peak_probe(int(kind), int(n_iter), ctypes.byref(n), ctypes.byref(f),
+                                     _p(ws), _stream(stream)))
+    return f.value, n.value
+
+
+def device_status_code(ws, stream=None):
+    """(status code, raw word) of a workspace, without raising."""
+    bits = ctypes.c_uint32(0)
+    st = _lib.v4attn_device_status(_p(ws), _stream(stream), ctypes.byref(bits))
+    return st, bits.value
+
+
+def workspace_init(ws, stream=None):
+    _check("v4attn_workspace_init", _lib.v4attn_workspace_init(_p(ws), ws.numel(),
+                                                                _stream(stream)))
 
 
 def _mqa(fn, desc, Q, q_pos, kv, kv_rows, swa, swa_rows, out, ws, kv_scale, swa_scale, q_seq, B,

@@ -12,6 +12,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_
 # dtypes
 F32, BF16, E4M3_BF16ROPE, MXFP4 = range(4)
 NOALLOC_MAX_SCORES = 2097152   # V4A_NOALLOC_MAX_SCORES
+NOALLOC_MAX_QUERIES = 1365     # V4A_NOALLOC_MAX_QUERIES
 # layer kinds
 CSA, HCA = 0, 1
 
@@ -88,6 +89,12 @@ SIGNATURES = {
     "v4attn_project": (ctypes.c_int, [ctypes.POINTER(ProjectArgs), c_ptr]),
     "v4attn_index_topk_noalloc": (ctypes.c_int, [ctypes.POINTER(LayerDesc),
                                                  ctypes.POINTER(IndexArgs), c_ptr]),
+    "v4attn_noalloc_device_status": (ctypes.c_int, [c_ptr, ctypes.POINTER(ctypes.c_uint32)]),
+    "v4attn_debug_index_stall": (ctypes.c_int, [ctypes.POINTER(LayerDesc),
+                                                ctypes.POINTER(IndexArgs), c_ptr, c_sz,
+                                                ctypes.c_uint32, c_ptr]),
+    "v4attn_tc_peak_probe": (ctypes.c_int, [c_i32, c_i32, ctypes.POINTER(c_i32),
+                                            ctypes.POINTER(ctypes.c_double), c_ptr, c_ptr]),
     "v4attn_device_status": (ctypes.c_int, [c_ptr, c_ptr, ctypes.POINTER(ctypes.c_uint32)]),
     "v4attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "v4attn_build_info": (ctypes.c_char_p, []),

@@ -149,8 +149,18 @@ v4attn_status run_compress(const v4attn_layer_desc* d, const v4attn_compress_arg
   return cuda_status(launch_compress(P, a->B, a->n_entries, st));
 }
 
+// Checks of the tensor-core paths, taken on the host before anything is
+// launched: an E4M3 / MXFP4 call either runs on its tcgen05 kernel or is
+// refused (there is no slower fallback for these formats).
+v4attn_status tc_status(int code) {
+  return code == 0 ? V4A_OK : (code == 1 ? V4A_ERR_INVALID_ARG : V4A_ERR_UNSUPPORTED);
+}
+
+// `dry`: validate and return without launching.  `wait_ns` / `stall`: the
+// failure-detection test hook (see v4attn_debug_index_stall).
 v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args* a, void* ws,
-                             size_t ws_bytes, cudaStream_t st, size_t body_off) {
+                             size_t ws_bytes, cudaStream_t st, size_t body_off, bool dry = false,
+                             uint32_t wait_ns = 0, int stall = 0) {
   if (d->kind != V4A_CSA) return V4A_ERR_INVALID_ARG;
   if (!a || a->n_q < 1 || a->n_q > kMaxQueries || a->B < 1) return V4A_ERR_INVALID_ARG;
   if (!a->qI || !a->w || !a->q_pos || !a->keys || (!a->idx_out && !a->scores_out))
@@ -164,6 +174,27 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
   const bool fp4 = d->idx_dtype == V4A_MXFP4;
   const size_t qrow = fp4 ? (size_t)d->d_I / 2 : (size_t)d->d_I * sizeof(float);
+  if (fp4) {
+    // the first chunk's pointers stand for every chunk: chunk offsets are
+    // multiples of 64-byte query rows, H_I scale rows and H_I weights
+    IndexParams P;
+    P.n_q = std::min(kQChunk, a->n_q);
+    P.B = a->B;
+    P.m = d->m;
+    P.H_I = d->H_I;
+    P.d_I = d->d_I;
+    P.idx_dtype = d->idx_dtype;
+    P.qI = a->qI;
+    P.qI_sf = a->qI_sf;
+    P.w = a->w;
+    P.keys = a->keys;
+    P.keys_sf = a->keys_sf;
+    P.key_rows = a->key_rows;
+    P.max_vis = a->max_vis;
+    const v4attn_status s = tc_status(index_tc_check(P));
+    if (s != V4A_OK) return s;
+  }
+  if (dry) return V4A_OK;
   for (int32_t q0 = 0; q0 < a->n_q; q0 += kQChunk) {
     const int32_t cn = std::min(kQChunk, a->n_q - q0);
     float* scores = a->scores_out ? a->scores_out + (int64_t)q0 * ld
@@ -189,6 +220,8 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
       P.scores = scores;
       P.scores_ld = ld;
       P.status = status;
+      P.wait_ns = wait_ns;
+      P.stall = stall;
       if (index_scores_dispatch(P, st) != cudaSuccess) return V4A_ERR_CUDA;
     }
     if (!a->idx_out) continue;   // scores-only call
@@ -207,7 +240,8 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
 }
 
 v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void* ws,
-                      size_t ws_bytes, cudaStream_t st, bool sparse, bool q_ready = false) {
+                      size_t ws_bytes, cudaStream_t st, bool sparse, bool q_ready = false,
+                      bool dry = false) {
   if (!a || a->n_q < 1 || a->n_q > kMaxQueries || a->B < 1) return V4A_ERR_INVALID_ARG;
   if (!a->Q || !a->q_pos || !a->kv || !a->out) return V4A_ERR_INVALID_ARG;
   if (d->n_win > 0 && (!a->swa || a->swa_rows < d->n_win)) return V4A_ERR_INVALID_ARG;
@@ -229,6 +263,7 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
   const size_t qb = (size_t)d->H * d->d * (a->q_dtype == V4A_BF16 ? 2 : 4);
   const size_t ob = (size_t)d->H * d->d * (a->out_dtype == V4A_BF16 ? 2 : 4);
   for (int32_t q0 = 0; q0 < a->n_q; q0 += kQChunk) {
+    if (dry && q0 > 0) break;
     MqaParams P;
     P.n_q = std::min(kQChunk, a->n_q - q0);
     P.B = a->B;
@@ -267,6 +302,11 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
     P.out_dtype = a->out_dtype;
     P.lse = a->lse ? a->lse + (int64_t)q0 * d->H : nullptr;
     P.status = reinterpret_cast<uint32_t*>(ws);
+    if (q0 == 0 && d->kv_dtype == V4A_E4M3_BF16ROPE) {
+      const v4attn_status s = tc_status(mqa_tc_check(P));
+      if (s != V4A_OK) return s;
+    }
+    if (dry) return V4A_OK;
     if (mqa_dispatch(P, st) != cudaSuccess) return V4A_ERR_CUDA;
     if (launch_mqa_combine(P, st) != cudaSuccess) return V4A_ERR_CUDA;
   }
@@ -388,10 +428,11 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
     A.H = desc->H;
     A.qimg = reinterpret_cast<uint8_t*>(ws) + qimg_off(a->B);
   }
-  if (launch_decode_append(A, stream) != cudaSuccess) return V4A_ERR_CUDA;
+  // 3. indexer + top-k, 4. MQA: arguments built and validated before the
+  // first launch, so that a refused step leaves the caches untouched
+  v4attn_index_args ix{};
+  v4attn_mqa_args q{};
   if (csa) {
-    // 3. indexer + top-k
-    v4attn_index_args ix{};
     ix.n_q = a->B;
     ix.B = a->B;
     ix.qI = a->qI;
@@ -404,11 +445,9 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
     ix.key_rows = a->key_rows;
     ix.max_vis = a->max_vis;
     ix.idx_out = a->idx_out;
-    s = run_index_topk(desc, &ix, ws, ws_bytes, stream, body_mqa(desc, a->B));
+    s = run_index_topk(desc, &ix, ws, ws_bytes, stream, body_mqa(desc, a->B), true);
     if (s != V4A_OK) return s;
   }
-  // 4. MQA
-  v4attn_mqa_args q{};
   q.n_q = a->B;
   q.B = a->B;
   q.Q = a->Q;
@@ -429,6 +468,14 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
   q.out = a->out;
   q.out_dtype = a->out_dtype;
   q.lse = a->lse;
+  s = run_mqa(desc, &q, ws, ws_bytes, stream, csa, fuse_q, true);
+  if (s != V4A_OK) return s;
+  if (launch_decode_append(A, stream) != cudaSuccess) return V4A_ERR_CUDA;
+  if (csa) {
+    s = run_index_topk(desc, &ix, ws, ws_bytes, stream, body_mqa(desc, a->B));
+    if (s != V4A_OK) return s;
+  }
+  // 4. MQA
   return run_mqa(desc, &q, ws, ws_bytes, stream, csa, fuse_q);
 }
 
@@ -482,6 +529,17 @@ const char* v4attn_status_string(v4attn_status s) {
 
 const char* v4attn_build_info(void) { return build_info_string(); }
 
+v4attn_status v4attn_debug_index_stall(const v4attn_layer_desc* desc,
+                                       const v4attn_index_args* args, void* ws, size_t ws_bytes,
+                                       uint32_t wait_ns, cudaStream_t stream) {
+  v4attn_status s = check_desc(desc);
+  if (s != V4A_OK) return s;
+  if (desc->idx_dtype != V4A_MXFP4) return V4A_ERR_UNSUPPORTED;   // the tcgen05 kernel only
+  if (wait_ns < 100000u || wait_ns > 1000000000u) return V4A_ERR_INVALID_ARG;
+  return run_index_topk(desc, args, ws, ws_bytes, stream, args ? qimg_off(args->n_q) : 0, false,
+                        wait_ns, 1);
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------- no-allocation variant
@@ -498,15 +556,8 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocBytes];
 void* g_noalloc_ptr[64] = {nullptr};
 }  // namespace
 
-extern "C" v4attn_status v4attn_index_topk_noalloc(const v4attn_layer_desc* desc,
-                                                   const v4attn_index_args* args,
-                                                   cudaStream_t stream) {
-  v4attn_status s = check_desc(desc);
-  if (s != V4A_OK) return s;
-  if (!args || args->n_q < 1 || args->max_vis < 0) return V4A_ERR_INVALID_ARG;
-  if ((int64_t)args->n_q * std::max<int64_t>(args->max_vis, 1) > V4A_NOALLOC_MAX_SCORES ||
-      qimg_off(args->n_q) + index_need(args->n_q, args->max_vis) > kNoallocBytes)
-    return V4A_ERR_UNSUPPORTED;
+// The array's device address on the current device (looked up on first use).
+static v4attn_status noalloc_scratch(void** ws) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return V4A_ERR_CUDA;
   if (!g_noalloc_ptr[dev]) {
@@ -514,8 +565,32 @@ extern "C" v4attn_status v4attn_index_topk_noalloc(const v4attn_layer_desc* desc
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return V4A_ERR_CUDA;
     g_noalloc_ptr[dev] = p;
   }
-  void* ws = g_noalloc_ptr[dev];
+  *ws = g_noalloc_ptr[dev];
+  return V4A_OK;
+}
+
+extern "C" v4attn_status v4attn_index_topk_noalloc(const v4attn_layer_desc* desc,
+                                                   const v4attn_index_args* args,
+                                                   cudaStream_t stream) {
+  v4attn_status s = check_desc(desc);
+  if (s != V4A_OK) return s;
+  if (!args || args->n_q < 1 || args->max_vis < 0) return V4A_ERR_INVALID_ARG;
+  // both limits of the header, checked as stated (the byte check follows from them)
+  if (args->n_q > V4A_NOALLOC_MAX_QUERIES ||
+      (int64_t)args->n_q * std::max<int64_t>(args->max_vis, 1) > V4A_NOALLOC_MAX_SCORES ||
+      qimg_off(args->n_q) + index_need(args->n_q, args->max_vis) > kNoallocBytes)
+    return V4A_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  s = noalloc_scratch(&ws);
+  if (s != V4A_OK) return s;
   // the status word must start at zero; the scores are fully rewritten by the call
   if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), stream) != cudaSuccess) return V4A_ERR_CUDA;
   return run_index_topk(desc, args, ws, kNoallocBytes, stream, qimg_off(args->n_q));
+}
+
+extern "C" v4attn_status v4attn_noalloc_device_status(cudaStream_t stream, uint32_t* bits) {
+  void* ws = nullptr;
+  const v4attn_status s = noalloc_scratch(&ws);
+  if (s != V4A_OK) return s;
+  return v4attn_device_status(ws, stream, bits);
 }

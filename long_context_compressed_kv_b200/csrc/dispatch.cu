@@ -17,8 +17,11 @@ int mqa_num_splits(const v4attn_layer_desc* d, int64_t n_main_max) {
   return (int)std::max<int64_t>(1, (keys + sk - 1) / sk);
 }
 
+// MXFP4 runs on the tensor-core kernel only, F32 on CUDA cores only; the
+// C-ABI has refused any MXFP4 call the tensor-core kernel does not take.
 cudaError_t index_scores_dispatch(const IndexParams& P, cudaStream_t st) {
-  if (index_tc_supported(P)) return launch_index_tc(P, st);
+  if (P.idx_dtype == V4A_MXFP4)
+    return index_tc_check(P) == 0 ? launch_index_tc(P, st) : cudaErrorNotSupported;
   return launch_index_scores(P, st);
 }
 
@@ -27,8 +30,10 @@ cudaError_t topk_dispatch(const TopkParams& P, cudaStream_t st) {
   return launch_topk(P, st);
 }
 
+// E4M3 caches run on the tensor-core kernel only, F32 caches on CUDA cores.
 cudaError_t mqa_dispatch(const MqaParams& P, cudaStream_t st) {
-  if (mqa_tc_supported(P)) return launch_mqa_tc(P, st);
+  if (P.kv_dtype == V4A_E4M3_BF16ROPE)
+    return mqa_tc_check(P) == 0 ? launch_mqa_tc(P, st) : cudaErrorNotSupported;
   return launch_mqa_simt(P, st);
 }
 
@@ -37,7 +42,7 @@ cudaError_t project_dispatch(const ProjectParams& P, cudaStream_t st) {
 }
 
 const char* build_info_string() {
-  return "v4attn sm_100a: compress(simt) index(tcgen05 mxf4 | simt) topk(cluster radix | radix) mqa(tcgen05 fp8/bf16 | simt) project(simt)";
+  return "v4attn sm_100a: compress(simt) index(mxfp4: tcgen05 mxf4; f32: simt) topk(cluster radix | radix) mqa(e4m3: tcgen05 fp8/bf16; f32: simt) project(simt)";
 }
 
 }  // namespace v4a

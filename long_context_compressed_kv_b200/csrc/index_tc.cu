@@ -67,7 +67,7 @@ struct Smem {
   alignas(128) uint32_t sfb_raw[2][128];
   alignas(16) float w[2][128];
   uint64_t full[STAGES], empty[STAGES], accstage[STAGES], qfull[2], qempty[2],
-      accempty[MAX_ACC], done;
+      accempty[MAX_ACC], done, never;
   int tile_prefix[MAXQ + 1];
   uint32_t tmem_base;
   int abort;
@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   constexpr int NACC = n_acc(N);
   static_assert(NACC >= 2 && NACC * (N + 4) + 8 <= (int)TM_COLS, "TMEM budget");
   constexpr bool W_IN_REGS = N <= 64;
+  const uint32_t lim = P.wait_ns ? P.wait_ns : (uint32_t)kWaitNs;   // bound of every wait
 
   // tiles per query, loaded in parallel, then a serial prefix over shared memory
   for (int q = threadIdx.x; q < P.n_q; q += NTHREADS) {
@@ -149,6 +150,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int i = 0; i < MAX_ACC; ++i) mbar_init(&s.accempty[i], 4);
     mbar_init(&s.done, 1);
+    mbar_init(&s.never, 1);   // debug stall site: nothing ever arrives on it
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(&s.tmem_base, TM_COLS);
@@ -176,6 +178,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t* ksf32 = reinterpret_cast<const uint32_t*>(P.keys_sf);
     const int64_t total_rows = (int64_t)P.B * P.key_rows;
     int stg = 0;
+    int qissued = 0;                            // query-buffer loads issued
     int b = 0;                                  // sequence of the current query
     for (int g = g0; g < g1 && !aborted(); ++stg) {
       const int seg_before = t.seg;
@@ -185,7 +188,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // read once per query: a global load per stage would sit on the issue path
         b = P.q_seq ? P.q_seq[t.q] : P.q_base + t.q;
         const int j = t.seg & 1, uq = t.seg >> 1;
-        if (uq >= 1 && !mbar_wait_warp(&s.qempty[j], (uq - 1) & 1, P.status)) {
+        if (uq >= 1 && !mbar_wait_warp(&s.qempty[j], (uq - 1) & 1, P.status, -1, lim)) {
           fail(s, P.status);
           break;
         }
@@ -197,9 +200,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     N * 4, &s.qfull[j]);
           bulk_load(s.w[j], P.w + (int64_t)t.q * P.H_I, N * 4, &s.qfull[j]);
         }
+        ++qissued;
       }
       const int st = stg % STAGES, u = stg / STAGES;
-      if (u >= 1 && !mbar_wait_warp(&s.empty[st], (u - 1) & 1, P.status)) {
+      if (u >= 1 && !mbar_wait_warp(&s.empty[st], (u - 1) & 1, P.status, -1, lim)) {
         fail(s, P.status);
         break;
       }
@@ -220,11 +224,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       g += n;
     }
-    // drain: no load may still be landing in shared memory when the CTA exits
-    if (s.abort && lane == 0) {
+    // drain: no load may still be landing in shared memory when the CTA exits.
+    // The last use of every ring slot and query buffer is waited for (on a
+    // normal run those phases completed long ago; after an abort their
+    // consumers may never have waited on them)
+    if (lane == 0) {
       for (int k = 0; k < STAGES && k < stg; ++k) {
         const int i2 = stg - 1 - k;
         mbar_wait(&s.full[i2 % STAGES], (i2 / STAGES) & 1);   // time bound only
+      }
+      for (int k = 0; k < 2 && k < qissued; ++k) {
+        const int sg = qissued - 1 - k;
+        mbar_wait(&s.qfull[sg & 1], (sg >> 1) & 1);
       }
     }
   } else if (warp == 1) {
@@ -232,6 +243,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     TileIter t;
     int stg = 0;
     bool ok = true;
+    if (P.stall && !mbar_wait_warp(&s.never, 0, P.status, 12, lim)) {
+      // debug: a wait that nothing completes runs out here, before any MMA is
+      // issued; the other roles see the status bit and return
+      fail(s, P.status);
+      ok = false;
+    }
     const uint64_t kdesc_bits = smem_desc_bits(16, 8 * KROW, 4);    // K-major, 64B swizzle
     const uint64_t sf_bits = smem_desc_bits(16, 128, 0);            // 32 rows x 16 B
     for (int g = g0; ok && g < g1 && !aborted(); ++stg) {
@@ -240,7 +257,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int n = stage_tiles(s, t, g, g1);
       const int j = t.seg & 1;
       if (t.seg != seg_before) {
-        if (!mbar_wait_warp(&s.qfull[j], (t.seg >> 1) & 1, P.status)) {
+        if (!mbar_wait_warp(&s.qfull[j], (t.seg >> 1) & 1, P.status, -1, lim)) {
           fail(s, P.status);
           break;
         }
@@ -254,7 +271,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) tmem_cp_32x128b_warpx4(tmem + col_sfb + 4 * j, smem_desc(s.sfb[j], sf_bits));
       }
       const int st = stg % STAGES;
-      if (!mbar_wait_warp(&s.full[st], (stg / STAGES) & 1, P.status)) {
+      if (!mbar_wait_warp(&s.full[st], (stg / STAGES) & 1, P.status, -1, lim)) {
         fail(s, P.status);
         break;
       }
@@ -262,7 +279,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // the MMAs (a copy issued behind an MMA waits for it)
       for (int k = 0; k < n; ++k) {
         const int it = g - g0 + k, a = it % NACC, ua = it / NACC;
-        if (ua >= 1 && !mbar_wait_warp(&s.accempty[a], (ua - 1) & 1, P.status)) {
+        if (ua >= 1 && !mbar_wait_warp(&s.accempty[a], (ua - 1) & 1, P.status, -1, lim)) {
           fail(s, P.status);
           ok = false;
           break;
@@ -330,7 +347,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int n = stage_tiles(s, t, g, g1);
       const int j = t.seg & 1;
       if (t.seg != seg_before) {
-        if (!mbar_wait_warp(&s.qfull[j], (t.seg >> 1) & 1, P.status)) {
+        if (!mbar_wait_warp(&s.qfull[j], (t.seg >> 1) & 1, P.status, -1, lim)) {
           fail(s, P.status);
           break;
         }
@@ -344,7 +361,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const bool has_tile = n > 1 || ((g - g0) & 1) == grp;
       const bool seg_end = (g + n == g1) || (g + n >= s.tile_prefix[t.q + 1]);
       if (grp == 0 || has_tile) {
-        if (!mbar_wait_warp(&s.accstage[st], (stg / STAGES) & 1, P.status)) {
+        if (!mbar_wait_warp(&s.accstage[st], (stg / STAGES) & 1, P.status, -1, lim)) {
           fail(s, P.status);
           break;
         }
@@ -468,15 +485,18 @@ static bool make_keys_map(CUtensorMap* map, const void* base, int64_t rows) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool index_tc_supported(const IndexParams& P) {
+int index_tc_check(const IndexParams& P) {
+  if (P.idx_dtype != V4A_MXFP4 || P.d_I != 128 || !(P.H_I == 32 || P.H_I == 64 || P.H_I == 128) ||
+      P.n_q > MAXQ)
+    return 2;
   // the scale and weight rows are moved by 1-D bulk copies: 16-byte aligned
   // sources, i.e. 16-byte aligned bases and a key row count divisible by 4
-  return P.idx_dtype == V4A_MXFP4 && P.d_I == 128 &&
-         (P.H_I == 32 || P.H_I == 64 || P.H_I == 128) && P.n_q <= MAXQ &&
-         encode_fn() != nullptr && P.key_rows % 4 == 0 &&
-         ((uintptr_t)P.keys & 15) == 0 && ((uintptr_t)P.qI & 15) == 0 &&
-         ((uintptr_t)P.keys_sf & 15) == 0 && ((uintptr_t)P.qI_sf & 15) == 0 &&
-         ((uintptr_t)P.w & 15) == 0;
+  // (the 3-D key view needs the latter too)
+  if (P.key_rows % 4 != 0 || (int64_t)P.B * P.key_rows > (1ll << 31)) return 2;
+  if (((uintptr_t)P.keys & 15) || ((uintptr_t)P.qI & 15) || ((uintptr_t)P.keys_sf & 15) ||
+      ((uintptr_t)P.qI_sf & 15) || ((uintptr_t)P.w & 15))
+    return 1;
+  return encode_fn() != nullptr ? 0 : 2;   // the driver's tensor-map encoder
 }
 
 cudaError_t launch_index_tc(const IndexParams& P, cudaStream_t st) {

@@ -72,6 +72,9 @@ struct IndexParams {
   float* scores;        // [n_q][max_vis]
   int64_t scores_ld;
   uint32_t* status;
+  uint32_t wait_ns = 0; // bound of the tensor-core kernel's waits (0: the default, 1 s)
+  int stall = 0;        // debug: the tensor-core kernel's MMA warp waits on a barrier
+                        // nothing completes, so that its bounded wait runs out
 };
 
 struct TopkParams {

@@ -37,14 +37,16 @@ __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w <
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // Codes head rows 16*hblk .. 16*hblk+15 of one query (bf16 rows of 512 dims,
-// `Qrow0` = its head 0, H heads) at position p into `img`.  Threads 0..63 of
+// `Qrow0` = its head 0, H heads) at position p into `img`, after a per-head
+// RMSNorm (unit weight, epsilon eps) when `rmsnorm` is set.  Threads 0..63 of
 // the block work, four per head row (7 of the 28 E4M3 chunks and 2 of the 8
 // RoPE chunks each), and issue all of their loads before the RoPE angles are
 // computed; every thread of the block must call this (one __syncthreads).
 // cs / sn: 32 floats of shared memory each.
 __device__ __forceinline__ void qimage_code_rows(const __nv_bfloat16* Qrow0, int H, int64_t p,
                                                  float theta, uint8_t* img, int hblk,
-                                                 float* cs, float* sn) {
+                                                 float* cs, float* sn, bool rmsnorm = false,
+                                                 float eps = 0.f) {
   const int tid = threadIdx.x;
   const bool worker = tid < 64;
   const int h = hblk * 16 + ((tid & 63) >> 2), part = tid & 3;
@@ -61,12 +63,32 @@ __device__ __forceinline__ void qimage_code_rows(const __nv_bfloat16* Qrow0, int
     cs[tid] = c;
     sn[tid] = sv;
   }
+  // RMSNorm factor of the row (the four threads of a row are adjacent lanes)
+  float inv = 1.f;
+  if (rmsnorm) {
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint4 u = i < 14 ? nope[i] : rope[i - 14];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float a = bf16lo(w[k]), b = bf16hi(w[k]);
+        ss = fmaf(a, a, fmaf(b, b, ss));
+      }
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    const float den = ss / 512.f + eps;
+    inv = den > 0.f ? 1.0f / sqrtf(den) : 0.f;     // an all-zero row stays zero
+  }
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < 14; ++i) {
     const uint32_t w[4] = {nope[i].x, nope[i].y, nope[i].z, nope[i].w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[k])), fabsf(bf16hi(w[k]))));
+    for (int k = 0; k < 4; ++k)
+      amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[k]) * inv), fabsf(bf16hi(w[k]) * inv)));
   }
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
@@ -80,9 +102,10 @@ __device__ __forceinline__ void qimage_code_rows(const __nv_bfloat16* Qrow0, int
       uint32_t pk[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const uint32_t lo = e4m3x2(scale_pow2(bf16lo(w[2 * k]), se), scale_pow2(bf16hi(w[2 * k]), se));
-        const uint32_t hi =
-            e4m3x2(scale_pow2(bf16lo(w[2 * k + 1]), se), scale_pow2(bf16hi(w[2 * k + 1]), se));
+        const uint32_t lo = e4m3x2(scale_pow2(bf16lo(w[2 * k]) * inv, se),
+                                   scale_pow2(bf16hi(w[2 * k]) * inv, se));
+        const uint32_t hi = e4m3x2(scale_pow2(bf16lo(w[2 * k + 1]) * inv, se),
+                                   scale_pow2(bf16hi(w[2 * k + 1]) * inv, se));
         pk[k] = lo | (hi << 16);
       }
       const int c = (part * 7 + j) * 16;
@@ -102,7 +125,7 @@ __device__ __forceinline__ void qimage_code_rows(const __nv_bfloat16* Qrow0, int
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int pr = c16 * 4 + k;
-        const float x0 = bf16lo(w[k]), x1 = bf16hi(w[k]);
+        const float x0 = bf16lo(w[k]) * inv, x1 = bf16hi(w[k]) * inv;
         const float r0 = x0 * cs[pr] - x1 * sn[pr], r1 = x0 * sn[pr] + x1 * cs[pr];
         pk[k] = (uint32_t)f32_to_bf16_bits(r0) | ((uint32_t)f32_to_bf16_bits(r1) << 16);
       }

@@ -183,7 +183,8 @@ __global__ void __launch_bounds__(64) mqa_tc_qprep_kernel(MqaParams P) {
   __shared__ float cs[32], sn[32];
   const int q = blockIdx.x;
   qimage_code_rows(reinterpret_cast<const __nv_bfloat16*>(P.Q) + (int64_t)q * P.H * 512, P.H,
-                   P.q_pos[q], P.theta, P.qbuf + (int64_t)q * kMqaQImageStride, blockIdx.y, cs, sn);
+                   P.q_pos[q], P.theta, P.qbuf + (int64_t)q * kMqaQImageStride, blockIdx.y, cs, sn,
+                   P.q_rmsnorm != 0, P.eps);
 }
 
 __global__ void __launch_bounds__(NTHR, 1)
@@ -596,13 +597,16 @@ __global__ void __launch_bounds__(NTHR, 1)
 bool make_rows_map_sw(CUtensorMap* map, const void* base, int64_t rows, int row_bytes,
                       int box_bytes, int box_rows, int swizzle_bytes);
 
-bool mqa_tc_supported(const MqaParams& P) {
-  return P.kv_dtype == V4A_E4M3_BF16ROPE && P.d == 512 && P.d_rope == 64 && P.H <= 128 &&
-         P.q_dtype == V4A_BF16 && !P.q_rmsnorm && P.split_keys % NK == 0 &&
-         P.qbuf != nullptr && ((uintptr_t)P.qbuf & 15) == 0 &&
-         P.split_keys <= SKMAX && (!P.idx || P.split_keys <= SKMAX_SEL) && P.n_win <= 1024 && ((uintptr_t)P.kv & 15) == 0 &&
-         (P.n_win == 0 || ((uintptr_t)P.swa & 15) == 0) && ((uintptr_t)P.Q & 15) == 0 &&
-         (int64_t)P.B * P.kv_rows < (1ll << 31) && (int64_t)P.B * P.swa_rows < (1ll << 31);
+int mqa_tc_check(const MqaParams& P) {
+  if (P.kv_dtype != V4A_E4M3_BF16ROPE || P.d != 512 || P.d_rope != 64 || P.H > 128 ||
+      P.q_dtype != V4A_BF16 || P.split_keys % NK != 0 || P.split_keys > SKMAX ||
+      (P.idx && P.split_keys > SKMAX_SEL) || P.n_win > 1024 || P.qbuf == nullptr ||
+      (int64_t)P.B * P.kv_rows >= (1ll << 31) || (int64_t)P.B * P.swa_rows >= (1ll << 31))
+    return 2;
+  if (((uintptr_t)P.qbuf & 15) || ((uintptr_t)P.kv & 15) ||
+      (P.n_win > 0 && ((uintptr_t)P.swa & 15)) || ((uintptr_t)P.Q & 15))
+    return 1;
+  return 0;
 }
 
 cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {

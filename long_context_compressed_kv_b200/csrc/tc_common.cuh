@@ -90,7 +90,7 @@ __device__ __forceinline__ unsigned long long global_ns() {
 // Bounded wait that, on expiry, also records its call site (bit 16 + site of
 // the status word) so a report says which wait gave up.
 __device__ __forceinline__ bool mbar_wait_at(uint64_t* bar, uint32_t parity, uint32_t* status,
-                                             int site);
+                                             int site, uint32_t limit_ns = (uint32_t)kWaitNs);
 
 // Bounded wait for the phase with the given parity; false on expiry or when
 // `status` (the grid's status word, may be null) already records a timeout.
@@ -98,23 +98,25 @@ __device__ __forceinline__ bool mbar_wait_at(uint64_t* bar, uint32_t parity, uin
 // global load on the polling path of every healthy wait would delay noticing
 // the phase by a memory round trip, which under a full HBM stream is several
 // hundred nanoseconds.
+// `limit_ns` (default kWaitNs) is the wall-clock bound of this wait.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          const uint32_t* status = nullptr) {
+                                          const uint32_t* status = nullptr,
+                                          uint32_t limit_ns = (uint32_t)kWaitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   // elapsed time in 32 bits: it wraps after 4.29 s, well above the limit
   const uint32_t t0 = (uint32_t)global_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity)) return true;
     const uint32_t dt = (uint32_t)global_ns() - t0;
-    if (dt > (uint32_t)kWaitNs) return false;
+    if (dt > limit_ns) return false;
     if (status && dt > (uint32_t)kStatusPollNs &&
         (*reinterpret_cast<const volatile uint32_t*>(status) & kStatusTimeout))
       return false;
   }
 }
 __device__ __forceinline__ bool mbar_wait_at(uint64_t* bar, uint32_t parity, uint32_t* status,
-                                             int site) {
-  if (mbar_wait(bar, parity, status)) return true;
+                                             int site, uint32_t limit_ns) {
+  if (mbar_wait(bar, parity, status, limit_ns)) return true;
   if (status) atomicOr(status, kStatusTimeout | (1u << (16 + (site & 15))));
   return false;
 }
@@ -123,9 +125,10 @@ __device__ __forceinline__ bool mbar_wait_at(uint64_t* bar, uint32_t parity, uin
 // them: a warp never splits at a timeout, so the warp-wide (.sync.aligned)
 // tcgen05 loads and stores that follow always see every lane.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, uint32_t* status,
-                                               int site = -1) {
-  const bool ok = site >= 0 ? mbar_wait_at(bar, parity, status, site)
-                            : mbar_wait(bar, parity, status);
+                                               int site = -1,
+                                               uint32_t limit_ns = (uint32_t)kWaitNs) {
+  const bool ok = site >= 0 ? mbar_wait_at(bar, parity, status, site, limit_ns)
+                            : mbar_wait(bar, parity, status, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 

@@ -18,11 +18,13 @@ cudaError_t mqa_dispatch(const MqaParams& P, cudaStream_t st);
 cudaError_t project_dispatch(const ProjectParams& P, cudaStream_t st);
 const char* build_info_string();
 
-bool index_tc_supported(const IndexParams& P);
+// 0: the tensor-core kernel takes these arguments; 1: a pointer is not
+// 16-byte aligned; 2: a shape or format the kernel does not cover.
+int index_tc_check(const IndexParams& P);
 bool topk_cluster_supported(const TopkParams& P);
 cudaError_t launch_topk_cluster(const TopkParams& P, cudaStream_t st);
 cudaError_t topk_dispatch(const TopkParams& P, cudaStream_t st);
-bool mqa_tc_supported(const MqaParams& P);
+int mqa_tc_check(const MqaParams& P);   // as index_tc_check
 cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st);
 cudaError_t launch_index_tc(const IndexParams& P, cudaStream_t st);
 

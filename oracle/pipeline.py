@@ -57,8 +57,9 @@ def decode_layer(inp: dict, ly, seqs, need_scores: bool = False) -> dict:
     i_new = (p + 1) // m - 1
     n_vis = int(n_visible(p, m))
     scale = 1.0 / np.sqrt(ly.d)
-    out = {k: [] for k in ("entry_new", "entry_new_val", "key_new", "key_new_val", "swa_new",
-                           "swa_new_val", "scores", "idx", "out", "lse")}
+    out = {k: [] for k in ("entry_new", "entry_new_val", "entry_new_raw", "key_new",
+                           "key_new_val", "key_new_raw", "swa_new", "swa_new_val", "swa_new_raw",
+                           "scores", "idx", "out", "lse")}
     for b in seqs:
         hist = inp["hist_entries"][b]
         n_hist = hist.shape[0]
@@ -72,6 +73,7 @@ def decode_layer(inp: dict, ly, seqs, need_scores: bool = False) -> dict:
                 e = pool(np.array([i_new]), m, False, p + 1, tail("C"), tail("Z"), inp["bias"])
             e = finish_main(e, np.array([i_new]), m, ly.d_rope, ly.rope_theta)
             st, new_val = store_kv(e, ly)
+            out["entry_new_raw"].append(e[0])
             out["entry_new"].append(st)
             out["entry_new_val"].append(new_val[0])
 
@@ -87,7 +89,9 @@ def decode_layer(inp: dict, ly, seqs, need_scores: bool = False) -> dict:
             return res
         # window: synthetic history rows for tokens p-n_win+1 .. p-1, then token p
         ca_p = inp["tail_Ca" if ly.kind == "csa" else "tail_C"][b][ring - 1]
-        st, swa_p = store_kv(token_kv(ca_p[None, :], np.array([p]), ly), ly)
+        swa_raw = token_kv(ca_p[None, :], np.array([p]), ly)
+        st, swa_p = store_kv(swa_raw, ly)
+        out["swa_new_raw"].append(swa_raw[0])
         out["swa_new"].append(st)
         out["swa_new_val"].append(swa_p[0])
         toks = window_tokens(p, ly.n_win)
@@ -101,6 +105,7 @@ def decode_layer(inp: dict, ly, seqs, need_scores: bool = False) -> dict:
                 k = pool(np.array([i_new]), m, True, p + 1, itail("Ca"), itail("Za"), inp["ibias"],
                          itail("Cb"), itail("Zb"))
                 kst, kv = store_key(k, ly)
+                out["key_new_raw"].append(k[0])
                 out["key_new"].append(kst)
                 out["key_new_val"].append(kv[0])
                 kval = np.concatenate([kval, kv], axis=0)
@@ -139,7 +144,7 @@ def tiny_layer(inp: dict, w, query_rows=None) -> dict:
     swa = token_kv(C, np.arange(L), ly)
     positions = inp["positions"] if query_rows is None else inp["positions"][query_rows]
     res = dict(entries=ents, keys=keys, swa=swa, scores=[], idx=[], out=[], lse=[], qI=[], w=[],
-               Q=[])
+               Q=[], q=[])
     scale = 1.0 / np.sqrt(ly.d)
     for p in positions:
         xp = x[p]
@@ -159,6 +164,7 @@ def tiny_layer(inp: dict, w, query_rows=None) -> dict:
         res["qI"].append(qI)
         res["w"].append(wh)
         res["Q"].append(Q)
+        res["q"].append(q)
     return res
 
 

@@ -1,20 +1,25 @@
 """Helpers shared by the GPU parity tests: moving seeded inputs to the
-device, building decode state through the C-ABI, reading stored rows back and
-the tolerance checks (from the stated parity bar: top-k sets exact except
-swaps within 1e-3 relative of the k-th oracle score; entries and outputs
-within max-abs 1e-4 for the fp32 layer and 2e-2 relative-to-RMS for the
-FP8/BF16/FP4 layers)."""
+device, building decode state through the C-ABI, reading stored rows back,
+and the stage-wise checks (tests/parity.py states the tolerances and why).
+
+Stage-wise: every stage is checked on the GPU's own checked output of the
+stage before.  Stored rows (entries, indexer keys, window KV) are checked as
+valid codings of the oracle's values; then the oracle's indexer scores the
+keys the GPU stored, and the oracle's attention runs over the rows the GPU
+stored and the entries the GPU selected."""
 from __future__ import annotations
 
 import numpy as np
 import torch
 
 import synth
-from oracle import codecs
+from oracle import codecs, indexer as oidx, mqa as omqa, pipeline
+from tests.parity import (F32_ABS_TOL, LSE_ABS_TOL, R16_TOL, TOPK_REL_TOL, check_e4m3_rows,
+                          check_mxfp4_rows, check_topk, r16)
 
-TOPK_REL_TOL = 1e-3
-R16_TOL = 2e-2
-F32_ABS_TOL = 1e-4
+__all__ = ["F32_ABS_TOL", "LSE_ABS_TOL", "R16_TOL", "TOPK_REL_TOL", "check_topk", "r16", "v4",
+           "dev", "desc_for", "code_rows", "read_kv", "read_keys", "check_stored_kv",
+           "check_stored_keys", "oracle_attention", "DecodeState", "compare_decode"]
 
 
 def v4():
@@ -24,13 +29,6 @@ def v4():
 
 def dev(x, dtype=torch.float32):
     return torch.from_numpy(np.ascontiguousarray(x)).to(dtype).cuda()
-
-
-def r16(gpu, ref):
-    """max-abs error over the RMS of the reference."""
-    gpu = np.asarray(gpu, dtype=np.float64)
-    ref = np.asarray(ref, dtype=np.float64)
-    return float(np.max(np.abs(gpu - ref)) / np.sqrt(np.mean(ref * ref)))
 
 
 def desc_for(ly, kv_fp8=None):
@@ -66,101 +64,76 @@ def code_rows(desc, vals, fmt, rows=None, first_row=0, d_rope=64):
     return out, sc
 
 
+def _np(x):
+    return x.cpu().numpy() if isinstance(x, torch.Tensor) else np.asarray(x)
+
+
 def read_kv(rows, scale, fmt, d=512, d_rope=64):
-    """Stored KV rows (numpy uint8 [..., rb]) -> float64 values [..., d]."""
-    rows = np.asarray(rows)
+    """Stored KV rows (uint8 [..., rb]) -> float64 values [..., d]."""
+    rows = _np(rows)
     v = v4()
     if fmt == v.F32:
         return rows.view(np.float32).astype(np.float64)
     dn = d - d_rope
     codes = rows[..., :dn]
     rbits = rows[..., dn:].copy().view(np.uint16)
-    return codecs.dequantize_kv(codes, rbits, np.asarray(scale))
+    return codecs.dequantize_kv(codes, rbits, _np(scale))
 
 
 def read_keys(rows, sf, fmt):
     v = v4()
-    rows = np.asarray(rows)
+    rows = _np(rows)
     if fmt == v.F32:
         return rows.view(np.float32).astype(np.float64)
-    return codecs.dequantize_mxfp4(codecs.unpack_e2m1(rows), np.asarray(sf))
+    return codecs.dequantize_mxfp4(codecs.unpack_e2m1(rows), _np(sf))
 
 
-def check_topk(gpu_idx, oracle_scores, n_vis, k, extra_tol=None):
-    """GPU selection vs the oracle: ascending, -1 padded, and the same set up
-    to swaps among entries whose oracle score is within 1e-3 relative of the
-    k-th oracle score (plus ``extra_tol[i]`` where the two sides' stored keys
-    differ by a coding decision).  Returns the number of swaps."""
-    gpu_idx = np.asarray(gpu_idx, dtype=np.int64)
-    s = np.asarray(oracle_scores, dtype=np.float64)[:n_vis]
-    kk = min(k, n_vis)
-    sel = gpu_idx[:kk]
-    assert np.all(gpu_idx[kk:] == -1), "padding"
-    assert np.all(sel >= 0) and np.all(sel < n_vis), "range"
-    assert np.all(np.diff(sel) > 0), "ascending, distinct"
-    if kk == 0:
+def check_stored_kv(rows, scale, fmt, raw, d=512, d_rope=64, what=""):
+    """Stored KV rows [n, rb] (+ scales [n]) against the oracle's values before
+    coding raw [n, d]: valid codings (E4M3 + bf16), or within F32_ABS_TOL (fp32)."""
+    v = v4()
+    rows = _np(rows).reshape(-1, _np(rows).shape[-1])
+    raw = np.asarray(raw, dtype=np.float64).reshape(len(rows), -1)
+    if fmt == v.F32:
+        got = rows.view(np.float32).astype(np.float64)
+        assert np.max(np.abs(got - raw)) <= F32_ABS_TOL, (what, np.max(np.abs(got - raw)))
         return 0
-    order = np.lexsort((np.arange(n_vis), -s))
-    want = set(order[:kk].tolist())
-    got = set(sel.tolist())
-    kth = s[order[kk - 1]]
-    diff = want ^ got
-    for i in diff:
-        tol = TOPK_REL_TOL * abs(kth) + (0.0 if extra_tol is None else extra_tol[i])
-        assert abs(s[i] - kth) <= tol, (i, s[i], kth)
-    return len(diff) // 2
+    dn = d - d_rope
+    return check_e4m3_rows(rows[:, :dn], rows[:, dn:].copy().view(np.uint16),
+                           _np(scale).reshape(-1), raw, d_rope, what)
 
 
-def check_coded_row(got, ref, ref_raw, d_rope=64, what=""):
-    """One stored E4M3 + bf16 row against the oracle's coded row.  Codes may
-    differ only where the two sides took a rounding decision differently: the
-    oracle's value before coding lies within 1e-4 relative of the midpoint of
-    the two decoded values (fp32 pooling against fp64 pooling), and such
-    flips are rare; a changed power-of-two scale is allowed only when the
-    oracle's amax / 448 lies within 1e-4 (log2) of a power of two."""
-    got, ref, raw = (np.asarray(a, dtype=np.float64) for a in (got, ref, ref_raw))
-    if r16(got, ref) <= R16_TOL:
-        return
-    dn = len(raw) - d_rope
-    t = np.max(np.abs(raw[:dn])) / codecs.E4M3_MAX
-    if t > 0 and abs(np.log2(t) - np.round(np.log2(t))) < 1e-4:
-        assert r16(got, ref) <= 8 * R16_TOL, (what, "scale boundary", r16(got, ref))
-        return
-    d = got != ref
-    mid = 0.5 * (got + ref)
-    near = np.abs(raw - mid) <= 1e-4 * np.maximum(np.abs(raw), 1e-6)
-    assert np.all(near[d]), (what, "code differs away from a rounding midpoint",
-                             np.flatnonzero(d & ~near)[:8])
-    assert d.mean() < 0.01, (what, "too many flipped codes", int(d.sum()))
+def check_stored_keys(rows, sf, fmt, raw, what=""):
+    """Stored indexer keys [n, rb] (+ E8M0 [n, c/32]) against raw [n, c]."""
+    v = v4()
+    rows = _np(rows).reshape(-1, _np(rows).shape[-1])
+    raw = np.asarray(raw, dtype=np.float64).reshape(len(rows), -1)
+    if fmt == v.F32:
+        got = rows.view(np.float32).astype(np.float64)
+        assert np.max(np.abs(got - raw)) <= F32_ABS_TOL, (what, np.max(np.abs(got - raw)))
+        return 0
+    return check_mxfp4_rows(rows, _np(sf), raw, what)
 
 
-def coding_bound(keys_ref, keys_gpu, a, q, o, scale, d_rope=64):
-    """First-order bound on how much the MQA output of one query moves when
-    its key rows change from the oracle's codes (keys_ref [n, d]) to the
-    codes the GPU stored (keys_gpu), both valid roundings of nearly equal
-    values: |do_h| <= sum_j a_hj |dk_j| + sum_j a_hj |k_j - o_h| scale |q_h . dk_j|
-    (V = K), with a [H, n] the oracle's attention weights and o [H, d] its
-    output before the inverse RoPE.  The RoPE dims are rotated afterwards, so
-    a pair gets the larger bound of its two dims times sqrt(2).  [H, d]."""
-    dk = np.asarray(keys_gpu, np.float64) - np.asarray(keys_ref, np.float64)
-    rows = np.flatnonzero(np.any(dk != 0, axis=1))
-    b = np.zeros_like(np.asarray(o, np.float64))
-    if len(rows) == 0:
-        return b
-    dk, kr, ar = dk[rows], np.asarray(keys_ref, np.float64)[rows], np.asarray(a)[:, rows]
-    ds = scale * np.abs(np.asarray(q, np.float64) @ dk.T)                 # [H, m]
-    b = ar @ np.abs(dk) + np.einsum("hm,hmd->hd", ar * ds, np.abs(kr[None] - o[:, None, :]))
-    dn = b.shape[1] - d_rope
-    pair = np.maximum(b[:, dn::2], b[:, dn + 1::2]) * np.sqrt(2.0)
-    b[:, dn::2] = pair
-    b[:, dn + 1::2] = pair
-    return b
+def oracle_attention(Q_h, p, keys, sink, ly, fp8, q_rmsnorm=False):
+    """The oracle's attention of one query (raw Q [H, d]) at position p over
+    the given key rows (the GPU's stored rows, decoded): (out [H, d], lse [H])."""
+    q = omqa.prepare_query(Q_h, p, ly.d_rope, ly.rope_theta, fp8, apply_rmsnorm=q_rmsnorm)
+    o, lse = omqa.attend(q, keys, 1.0 / np.sqrt(ly.d), sink)
+    return omqa.finish_output(o, p, ly.d_rope, ly.rope_theta), lse
 
 
-def r16_excess(got, ref, bound):
-    """max(|got - ref| - bound, 0) over the RMS of ref."""
-    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
-    return float(np.max(np.maximum(np.abs(got - ref) - bound, 0.0)) / np.sqrt(np.mean(ref * ref)))
+def check_output(got, want, lse_got, lse_want, fp32, what=""):
+    if fp32:
+        err = float(np.max(np.abs(np.asarray(got, np.float64) - want)))
+        assert err <= F32_ABS_TOL, (what, "out", err)
+    else:
+        err = r16(got, want)
+        assert err <= R16_TOL, (what, "out", err)
+    if lse_got is not None:
+        le = float(np.max(np.abs(np.asarray(lse_got, np.float64) - lse_want)))
+        assert le <= LSE_ABS_TOL, (what, "lse", le)
+    return err
 
 
 class DecodeState:
@@ -178,55 +151,63 @@ class DecodeState:
         self.max_vis = lay.max_vis
         if self.csa:
             self.kfmt, self.keys, self.keys_sf = lay.kfmt, lay.keys, lay.keys_sf
-            self.idx, self.qI = lay.idx, lay.qI
+            self.idx, self.qI, self.qI_sf, self.w = lay.idx, lay.qI, lay.qI_sf, lay.w
 
     def step(self, stream=None):
         self.lay.step(self.max_vis, stream=stream)
 
 
-def compare_decode(st: DecodeState, ref: dict, seqs, strict_keys=True):
-    """Check one decode step of ``seqs`` against ``oracle.pipeline.decode_layer``."""
+def compare_decode(st: DecodeState, seqs):
+    """Stage-wise check of one decode step of sequences ``seqs``:
+      a1  the new window row, and on a block boundary the new entry (and the
+          new indexer key), are valid codings of the oracle's values
+          (``oracle.pipeline.decode_layer``);
+      a3  the oracle's scores of the keys the GPU stored, with the indexer
+          query the GPU stored, select what the GPU selected (a4);
+      a6  the oracle's attention over the rows the GPU stored (the selected /
+          visible entries and the window tokens) gives the GPU's output and LSE."""
     v = v4()
-    ly, p = st.ly, st.inp["p"]
+    ly, inp = st.ly, st.inp
+    p = inp["p"]
     torch.cuda.synchronize()
     assert v.device_status(st.ws) == 0
-    i_new = (p + 1) // ly.m - 1
+    ref = pipeline.decode_layer(inp, ly, seqs)
+    n_vis = (p + 1) // ly.m
+    i_new = n_vis - 1
     complete = (p + 1) % ly.m == 0
-    report = {}
+    fp32 = st.fmt == v.F32
+    report = {"out_err": [], "swaps": []}
     for n, b in enumerate(seqs):
+        sr = p % st.swa_rows
+        check_stored_kv(st.swa[b, sr:sr + 1], None if fp32 else st.swa_scale[b, sr:sr + 1],
+                        st.fmt, ref["swa_new_raw"][n][None], ly.d, ly.d_rope, ("window row", b))
         if complete:
-            row = st.kv[b, i_new].cpu().numpy()
-            sc = None if st.kv_scale is None else st.kv_scale[b, i_new].cpu().numpy()
-            got = read_kv(row, sc, st.fmt, ly.d, ly.d_rope)
-            err = r16(got, ref["entry_new_val"][n])
-            assert err <= R16_TOL, ("new entry", b, err)
-        srow = st.swa[b, p % st.swa_rows].cpu().numpy()
-        ssc = None if st.swa_scale is None else st.swa_scale[b, p % st.swa_rows].cpu().numpy()
-        assert r16(read_kv(srow, ssc, st.fmt, ly.d, ly.d_rope), ref["swa_new_val"][n]) <= R16_TOL
-        extra = None
+            check_stored_kv(st.kv[b, i_new:i_new + 1],
+                            None if fp32 else st.kv_scale[b, i_new:i_new + 1], st.fmt,
+                            ref["entry_new_raw"][n][None], ly.d, ly.d_rope, ("new entry", b))
         if st.csa:
             if complete:
-                krow = st.keys[b, i_new].cpu().numpy()
-                ksf = None if st.keys_sf is None else st.keys_sf[b, i_new].cpu().numpy()
-                kgot = read_keys(krow, ksf, st.kfmt)
-                kref = ref["key_new_val"][n]
-                assert r16(kgot, kref) <= R16_TOL
-                if not np.array_equal(kgot, kref):
-                    # a coding decision taken differently on the two sides (values
-                    # within fp32 rounding of a grid midpoint): bound its effect
-                    from oracle import codecs as C
-                    qv = C.dequantize_mxfp4(*C.quantize_mxfp4(st.inp["qI"][b])) \
-                        if ly.idx_fp4 else st.inp["qI"][b]
-                    bound = float(np.abs(qv) @ np.abs(kgot - kref) @ st.inp["w"][b])
-                    extra = np.zeros(len(ref["scores"][n]))
-                    extra[i_new] = bound
-            nsw = check_topk(st.idx[b].cpu().numpy(), ref["scores"][n], (p + 1) // ly.m,
-                             ly.top_k, extra)
-            report.setdefault("swaps", []).append(nsw)
-        got = st.out[b].float().cpu().numpy()
-        err = r16(got, ref["out"][n])
-        report.setdefault("out_r16", []).append(err)
-        assert err <= R16_TOL, ("out", b, err)
-        lse_err = np.max(np.abs(st.lse[b].cpu().numpy() - ref["lse"][n]))
-        assert lse_err <= 5e-2, ("lse", b, lse_err)
+                check_stored_keys(st.keys[b, i_new:i_new + 1],
+                                  None if st.keys_sf is None else st.keys_sf[b, i_new:i_new + 1],
+                                  st.kfmt, ref["key_new_raw"][n][None], ("new key", b))
+            kv = read_keys(st.keys[b, :n_vis], None if st.keys_sf is None
+                           else st.keys_sf[b, :n_vis], st.kfmt)
+            qv = read_keys(st.qI[b], None if st.qI_sf is None else st.qI_sf[b], st.kfmt)
+            s = oidx.scores(qv, _np(st.w[b]), kv)
+            gidx = _np(st.idx[b])
+            report["swaps"].append(check_topk(gidx, s, n_vis, ly.top_k))
+            sel = gidx[gidx >= 0]
+        else:
+            sel = np.arange(n_vis)
+        ent = read_kv(st.kv[b][torch.from_numpy(sel).long().cuda()],
+                      None if fp32 else st.kv_scale[b][torch.from_numpy(sel).long().cuda()],
+                      st.fmt, ly.d, ly.d_rope)
+        toks = omqa.window_tokens(p, ly.n_win)
+        rr = torch.from_numpy(toks % st.swa_rows).long().cuda()
+        win = read_kv(st.swa[b][rr], None if fp32 else st.swa_scale[b][rr], st.fmt, ly.d,
+                      ly.d_rope)
+        o, lse = oracle_attention(inp["Q"][b], p, np.concatenate([ent, win], 0), inp["sink"], ly,
+                                  ly.kv_fp8)
+        report["out_err"].append(check_output(_np(st.out[b].float()), o, _np(st.lse[b]), lse,
+                                              fp32, ("output", b)))
     return report

@@ -155,3 +155,60 @@ def test_every_entry_point_rejects_a_short_workspace():
         else:
             assert lib.v4attn_dense_mqa(ctypes.byref(d), ctypes.byref(q), fake, 1024,
                                         None) == _abi.ERR_WORKSPACE
+
+
+@pytest.mark.skipif(not _no_gpu(), reason="host-only check with fake device pointers")
+def test_tensor_core_formats_are_refused_not_downgraded():
+    """An MXFP4 indexer or E4M3 MQA call that the tensor-core kernel does not
+    take is refused before any launch (no slower fallback runs): an MXFP4
+    indexer with d_I = 64 or a key row count not divisible by 4 ->
+    V4A_ERR_UNSUPPORTED, a misaligned pointer -> V4A_ERR_INVALID_ARG; an E4M3
+    MQA with an fp32 Q -> V4A_ERR_UNSUPPORTED; a decode step whose indexer is
+    refused launches nothing either (fake pointers, never dereferenced)."""
+    from long_context_compressed_kv_b200 import _abi
+    lib = _abi.load()
+    fake = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(1 << 21)
+    big = 1 << 40
+
+    def index_call(d_I, key_rows, qI=fake):
+        d = _abi.LayerDesc(_abi.CSA, 4, 128, 64, 512, 64, 160000.0, 0.0, 64, d_I, 512,
+                           _abi.E4M3_BF16ROPE, _abi.MXFP4, 1e-6)
+        ix = _abi.IndexArgs()
+        ix.n_q = ix.B = 2
+        for f in ("qI_sf", "w", "q_pos", "keys", "keys_sf", "idx_out"):
+            setattr(ix, f, fake)
+        ix.qI = qI
+        ix.key_rows = ix.max_vis = key_rows
+        return lib.v4attn_index_topk(ctypes.byref(d), ctypes.byref(ix), ws, big, None)
+    assert index_call(64, 4096) == _abi.ERR_UNSUPPORTED
+    assert index_call(128, 4098) == _abi.ERR_UNSUPPORTED
+    assert index_call(128, 4096, ctypes.c_void_p((1 << 20) + 8)) == _abi.ERR_INVALID_ARG
+    d = _abi.LayerDesc(_abi.HCA, 128, 128, 64, 512, 64, 160000.0, 0.0, 0, 0, 0,
+                       _abi.E4M3_BF16ROPE, _abi.MXFP4, 1e-6)
+    q = _abi.MqaArgs()
+    q.n_q, q.B = 2, 2
+    for f in ("Q", "q_pos", "kv", "kv_scale", "swa", "swa_scale", "sink", "out"):
+        setattr(q, f, fake)
+    q.q_dtype, q.out_dtype = _abi.F32, _abi.BF16
+    q.kv_rows, q.swa_rows, q.max_vis = 1024, 128, 1024
+    assert lib.v4attn_dense_mqa(ctypes.byref(d), ctypes.byref(q), ws, big, None) == \
+        _abi.ERR_UNSUPPORTED
+    q.q_dtype = _abi.BF16
+    q.Q = ctypes.c_void_p((1 << 20) + 2)
+    assert lib.v4attn_dense_mqa(ctypes.byref(d), ctypes.byref(q), ws, big, None) == \
+        _abi.ERR_INVALID_ARG
+    # decode: the indexer of this step is refused before the append launch
+    dc = _abi.LayerDesc(_abi.CSA, 4, 128, 64, 512, 64, 160000.0, 0.0, 64, 64, 512,
+                        _abi.E4M3_BF16ROPE, _abi.MXFP4, 1e-6)
+    a = _abi.DecodeArgs()
+    a.B = 2
+    for f in ("pos", "x_main", "tail", "bias", "kv", "kv_scale", "swa", "swa_scale", "Q", "sink",
+              "out", "x_idx", "itail", "ibias", "keys", "keys_sf", "qI", "qI_sf", "w", "idx_out"):
+        setattr(a, f, fake)
+    a.in_dtype = a.q_dtype = a.out_dtype = _abi.BF16
+    a.kv_rows = a.key_rows = 4096
+    a.swa_rows = 128
+    a.max_vis = 4096
+    assert lib.v4attn_decode(ctypes.byref(dc), ctypes.byref(a), ws, big, None) == \
+        _abi.ERR_UNSUPPORTED

@@ -100,3 +100,51 @@ def test_decode_window_holds_own_token():
     kv = pipeline.token_kv(inp["tail_C"][0][-1][None, :], np.array([p]), ly)
     _, kv_val = pipeline.store_kv(kv, ly)
     assert np.allclose(kv_val[0], r["swa_new_val"][0])
+
+
+def test_tiny_layer_query_construction_closed_form():
+    """The low-rank indexer query x_p W_dq W_uq reshaped to [H_I, d_I] (head
+    major), the head weights x_p W_w and the MQA query x_p W_q reshaped to
+    [H, d], pinned with one-hot weights: with x_p = e_0, W_dq = e_0 -> e_j,
+    W_uq = e_j -> e_(h0*d_I + c0), W_w = 0.75 e_0 -> e_h0 and
+    W_q = e_0 -> e_(h1*d + c1), the indexer query is the one-hot at (h0, c0),
+    the scores are 0.75 * max(0, k_i[c0]) for every visible key, and the MQA
+    query before RMSNorm is the one-hot at (h1, c1) (after RMSNorm,
+    1/sqrt(1/d + eps) there; RoPE leaves a non-RoPE dim alone).  A transposed reshape or a
+    swapped head / dim order lands the one-hot elsewhere."""
+    w, inp = _tiny(L=200, nq=3)
+    ly = w.layers[0]
+    r, h0, c0, h1, c1 = 5, 2, 11, 9, 17
+    assert c1 < ly.d - ly.d_rope
+    inp = dict(inp)
+    x = inp["x"].copy()
+    for p in inp["positions"]:
+        x[p] = 0.0
+        x[p, 0] = 1.0
+    inp["x"] = x
+    W_dq = np.zeros_like(inp["W_dq"])
+    W_dq[0, r] = 1.0
+    W_uq = np.zeros_like(inp["W_uq"])
+    W_uq[r, h0 * ly.d_I + c0] = 1.0
+    W_w = np.zeros_like(inp["W_w"])
+    W_w[0, h0] = 0.75
+    W_q = np.zeros_like(inp["W_q"])
+    W_q[0, h1 * ly.d + c1] = 1.0
+    inp.update(W_dq=W_dq, W_uq=W_uq, W_w=W_w, W_q=W_q)
+    res = pipeline.tiny_layer(inp, w)
+    for n, p in enumerate(inp["positions"]):
+        want_q = np.zeros((ly.H_I, ly.d_I))
+        want_q[h0, c0] = 1.0
+        assert np.array_equal(res["qI"][n], want_q)
+        want_w = np.zeros(ly.H_I)
+        want_w[h0] = 0.75
+        assert np.allclose(res["w"][n], want_w, rtol=0, atol=1e-15)
+        nv = int(compress.n_visible(p, ly.m))
+        assert np.allclose(res["scores"][n], 0.75 * np.maximum(res["keys"][:nv, c0], 0.0),
+                           rtol=0, atol=1e-12)
+        want_Q = np.zeros((ly.H, ly.d))
+        want_Q[h1, c1] = 1.0
+        assert np.array_equal(res["Q"][n], want_Q)
+        q = res["q"][n]
+        assert abs(q[h1, c1] - 1.0 / np.sqrt(1.0 / ly.d + 1e-6)) < 1e-12     # RMSNorm, eps 1e-6
+        assert np.count_nonzero(np.abs(q) > 1e-9) == 1
