@@ -74,7 +74,10 @@ __global__ void __launch_bounds__(128, 1) tc_peak_kernel(int n_iter, uint32_t* s
 }
 
 cudaError_t launch_tc_peak(int kind, int n_iter, uint32_t* status, cudaStream_t st) {
-  const size_t smem = A_BYTES + B_BYTES + 1024;
+  // more shared memory than two CTAs can share, so that every CTA has an SM
+  // (and its tensor memory) to itself
+  const size_t smem = 120 * 1024;
+  static_assert(A_BYTES + B_BYTES + 1024 <= 120 * 1024, "operands fit");
   static unsigned long long configured = 0;
   int dev = 0;
   cudaGetDevice(&dev);
