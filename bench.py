@@ -706,22 +706,29 @@ def measure_tc_peaks(stream, reps=5, n_iter=16384):
     import torch
     import long_context_compressed_kv_b200 as v
     out = {}
+    narrow = {}
     with ClockSampler(torch.cuda.current_device()) as clk:
         for kind, name in ((0, "bf16"), (1, "fp8_e4m3"), (2, "fp4_mxf4")):
-            v.tc_peak_probe(kind, 64, stream=stream)          # warm-up
-            best = 0.0
-            clk.start()
-            for _ in range(reps):
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                flops, ctas = v.tc_peak_probe(kind, n_iter, stream=stream)
-                b.record(stream)
-                b.synchronize()
-                best = max(best, flops / (a.elapsed_time(b) / 1e3) / 1e12)
-            clk.stop()
-            out[name + "_tflops"] = round(best, 1)
+            for n_cols in (256, 128, 64):
+                v.tc_peak_probe(kind, 64, n_cols, stream=stream)          # warm-up
+                best = 0.0
+                clk.start()
+                for _ in range(reps):
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    flops, ctas = v.tc_peak_probe(kind, n_iter, n_cols, stream=stream)
+                    b.record(stream)
+                    b.synchronize()
+                    best = max(best, flops / (a.elapsed_time(b) / 1e3) / 1e12)
+                clk.stop()
+                if n_cols == 256:
+                    out[name + "_tflops"] = round(best, 1)
+                else:
+                    narrow[f"{name}_n{n_cols}_tflops"] = round(best, 1)
     out["ctas"] = ctas
     out["shape"] = "M=128 N=256 per instruction, 1 CTA per SM, operands in shared memory"
+    out["narrow_n"] = narrow
     out["clocks"] = clk.summary()
     return out
 

@@ -319,7 +319,8 @@ v4attn_status v4attn_debug_index_stall(const v4attn_layer_desc* desc,
 
 /* Tensor-core throughput probe (measurement support; no counterpart in the
  * pages).  Launches one CTA per SM, each issuing n_iter x 4 back-to-back
- * tcgen05 MMAs of M = 128 x N = 256 with operands resident in shared memory
+ * tcgen05 MMAs of M = 128 x N = n_cols (64, 128 or 256) with operands
+ * resident in shared memory
  * and fp32 accumulators in tensor memory, of kind
  *   0: kind::f16 bf16 x bf16 (K = 16),  1: kind::f8f6f4 E4M3 x E4M3 (K = 32),
  *   2: kind::mxf4 block-scaled E2M1 x E2M1, E8M0 per 32 elements (K = 64).
@@ -328,9 +329,9 @@ v4attn_status v4attn_debug_index_stall(const v4attn_layer_desc* desc,
  * rate of that format.  *n_ctas receives the CTA count.  `ws`: a workspace
  * whose status word receives V4A_ERR_TIMEOUT's bit if the final wait runs
  * out, or NULL.  Nothing is read or written in global memory otherwise.
- * n_iter in 1 .. 2^24, else V4A_ERR_INVALID_ARG. */
-v4attn_status v4attn_tc_peak_probe(int32_t kind, int32_t n_iter, int32_t* n_ctas, double* flops,
-                                   void* ws, cudaStream_t stream);
+ * n_iter in 1 .. 2^24 and n_cols in {64, 128, 256}, else V4A_ERR_INVALID_ARG. */
+v4attn_status v4attn_tc_peak_probe(int32_t kind, int32_t n_cols, int32_t n_iter, int32_t* n_ctas,
+                                   double* flops, void* ws, cudaStream_t stream);
 
 /* Synchronise `stream`, read the status word the kernels left in `ws` and
  * map it: 0 -> V4A_OK, a bounds / argument check -> V4A_ERR_DEVICE_CHECK,

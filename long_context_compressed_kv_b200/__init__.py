@@ -153,14 +153,14 @@ def debug_index_stall(desc: LayerDesc, *, qI, w, q_pos, keys, key_rows: int, max
                                          int(wait_ns), _stream(stream)))
 
 
-def tc_peak_probe(kind: int, n_iter: int, ws=None, stream=None):
+def tc_peak_probe(kind: int, n_iter: int, n_cols: int = 256, ws=None, stream=None):
     """Launch the tensor-core throughput probe (see include/v4attn.h);
     returns (dense FLOPs of the launch, CTAs)."""
     n = ctypes.c_int32(0)
     f = ctypes.c_double(0.0)
     _check("v4attn_tc_peak_probe",
-           _lib.v4attn_tc_peak_probe(int(kind), int(n_iter), ctypes.byref(n), ctypes.byref(f),
-                                     _p(ws), _stream(stream)))
+           _lib.v4attn_tc_peak_probe(int(kind), int(n_cols), int(n_iter), ctypes.byref(n),
+                                     ctypes.byref(f), _p(ws), _stream(stream)))
     return f.value, n.value
 
 

@@ -93,7 +93,7 @@ SIGNATURES = {
     "v4attn_debug_index_stall": (ctypes.c_int, [ctypes.POINTER(LayerDesc),
                                                 ctypes.POINTER(IndexArgs), c_ptr, c_sz,
                                                 ctypes.c_uint32, c_ptr]),
-    "v4attn_tc_peak_probe": (ctypes.c_int, [c_i32, c_i32, ctypes.POINTER(c_i32),
+    "v4attn_tc_peak_probe": (ctypes.c_int, [c_i32, c_i32, c_i32, ctypes.POINTER(c_i32),
                                             ctypes.POINTER(ctypes.c_double), c_ptr, c_ptr]),
     "v4attn_device_status": (ctypes.c_int, [c_ptr, c_ptr, ctypes.POINTER(ctypes.c_uint32)]),
     "v4attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
