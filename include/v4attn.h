@@ -233,7 +233,10 @@ typedef struct {
  * Y[M][N] = X[M][K] . W[K][N] with fp32 accumulation: the linear maps that
  * produce the compressor inputs C, Z from raw tokens ([deep-read] "CSA 与 HCA":
  * per-channel learned gating of token KV) and, in the small fp32 layer, the
- * queries.  X, W, Y row-major with the given leading dimensions (elements). */
+ * queries.  X, W, Y row-major with the given leading dimensions (elements).
+ * bf16 X and W run on the tcgen05 tensor-core GEMM only (X, W 16-byte aligned
+ * with ldx, ldw multiples of 8 elements, else V4A_ERR_INVALID_ARG); fp32 X and
+ * W run on CUDA cores.  K >= 1 (V4A_ERR_INVALID_ARG otherwise). */
 typedef struct {
   int64_t M, N, K;
   const void* X; int32_t x_dtype; int64_t ldx;   /* V4A_F32 or V4A_BF16 */

@@ -487,6 +487,7 @@ v4attn_status v4attn_project(const v4attn_project_args* a, cudaStream_t stream) 
   if (a->ldx < a->K || a->ldw < a->N || a->ldy < a->N) return V4A_ERR_INVALID_ARG;
   if (a->M == 0 || a->N == 0) return V4A_OK;
   if (a->M > 65535LL * 64) return V4A_ERR_UNSUPPORTED;
+  if ((int64_t)a->K < 1) return V4A_ERR_INVALID_ARG;
   ProjectParams P;
   P.M = a->M;
   P.N = a->N;
@@ -499,6 +500,10 @@ v4attn_status v4attn_project(const v4attn_project_args* a, cudaStream_t stream) 
   P.Y = a->Y;
   P.y_dtype = a->y_dtype;
   P.ldy = a->ldy;
+  if (P.x_dtype == V4A_BF16) {
+    const v4attn_status s = tc_status(project_tc_check(P));
+    if (s != V4A_OK) return s;
+  }
   return cuda_status(project_dispatch(P, stream));
 }
 

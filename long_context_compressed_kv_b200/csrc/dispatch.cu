@@ -37,12 +37,15 @@ cudaError_t mqa_dispatch(const MqaParams& P, cudaStream_t st) {
   return launch_mqa_simt(P, st);
 }
 
+// bf16 projections run on the tensor-core GEMM only, fp32 ones on CUDA cores.
 cudaError_t project_dispatch(const ProjectParams& P, cudaStream_t st) {
+  if (P.x_dtype == V4A_BF16)
+    return project_tc_check(P) == 0 ? launch_project_tc(P, st) : cudaErrorNotSupported;
   return launch_project(P, st);
 }
 
 const char* build_info_string() {
-  return "v4attn sm_100a: compress(simt) index(mxfp4: tcgen05 mxf4; f32: simt) topk(cluster radix | radix) mqa(e4m3: tcgen05 fp8/bf16; f32: simt) project(simt)";
+  return "v4attn sm_100a: compress(simt) index(mxfp4: tcgen05 mxf4; f32: simt) topk(cluster radix | radix) mqa(e4m3: tcgen05 fp8/bf16; f32: simt) project(bf16: tcgen05 f16; f32: simt)";
 }
 
 }  // namespace v4a

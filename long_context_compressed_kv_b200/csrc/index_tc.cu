@@ -436,6 +436,8 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
+void* tensor_map_encoder() { return reinterpret_cast<void*>(encode_fn()); }
+
 // 2-D uint8 tensor map: rows of `row_bytes`, box of `box_rows` rows, 64B swizzle.
 bool make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int row_bytes, int box_rows) {
   EncodeTiledFn enc = encode_fn();

@@ -25,6 +25,10 @@ bool topk_cluster_supported(const TopkParams& P);
 cudaError_t launch_topk_cluster(const TopkParams& P, cudaStream_t st);
 cudaError_t topk_dispatch(const TopkParams& P, cudaStream_t st);
 int mqa_tc_check(const MqaParams& P);   // as index_tc_check
+int project_tc_check(const ProjectParams& P);   // as index_tc_check
+cudaError_t launch_project_tc(const ProjectParams& P, cudaStream_t st);
+// the driver's cuTensorMapEncodeTiled (nullptr when the driver lacks it)
+void* tensor_map_encoder();
 cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st);
 cudaError_t launch_index_tc(const IndexParams& P, cudaStream_t st);
 

@@ -436,3 +436,26 @@ def test_full_csa_flash_128k():
 
 def test_full_pro_pair_1m():
     _full_decode("pro_pair_1m", [0, 3])
+
+
+# ------------------------------------------------------------------ projection (a0)
+
+@pytest.mark.parametrize("M,N,K,y_bf16", [(300, 700, 200, False), (1024, 3584, 4096, False),
+                                          (129, 257, 64, True), (5, 40, 1000, False)])
+def test_projection_tensor_core(M, N, K, y_bf16):
+    """bf16 x bf16 -> fp32 / bf16 on the tcgen05 GEMM, ragged in every dim
+    (partial 128 x 256 tiles, a k tail that the loads zero-fill), against the
+    float64 product of the same bf16 values."""
+    v = v4()
+    rng = np.random.default_rng(M + N + K)
+    X = synth.bf16_values(rng.standard_normal((M, K)).astype(np.float32))
+    W = synth.bf16_values((rng.standard_normal((K, N)) / np.sqrt(K)).astype(np.float32))
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16 if y_bf16 else torch.float32,
+                   device="cuda")
+    v.project(dev(X, torch.bfloat16), dev(W, torch.bfloat16), Y)
+    torch.cuda.synchronize()
+    want = X.astype(np.float64) @ W.astype(np.float64)
+    got = Y.float().cpu().numpy().astype(np.float64)
+    # fp32 accumulation of exact bf16 products over K terms; bf16 output rounding
+    tol = (2.0 ** -8 if y_bf16 else 1e-4) * np.maximum(np.abs(want), 1.0)
+    assert np.all(np.abs(got - want) <= tol)
