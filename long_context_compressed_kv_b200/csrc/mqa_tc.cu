@@ -473,16 +473,26 @@ __global__ void __launch_bounds__(NTHR, 1)
           (K_new == -1000) ? 0.f : exp2i(min(126, max(-126, 8 - (int)kTau - K_new)));
       const float ak = (cu > 0.f && cu_new != cu) ? cu_new / cu : 1.f;   // exact: powers of two
       const float ms_ref = (Ms_new == -INFINITY) ? 0.f : Ms_new;
+      // The weight each key really gets is its coded value: (hi + lo) / (k_scale cu)
+      // on the FP8 dims (exact in fp32: hi and lo carry 4 significant bits each,
+      // k_scale cu is a power of two) and that weight rounded to bf16 on the RoPE
+      // dims.  The row sum is taken over the coded weights, so that O / l is a
+      // convex combination with exactly the weights the MMAs used.
       float lsum = 0.f;
       uint32_t phi[KPG / 4], plo[KPG / 4], pbf[KPG / 2];
 #pragma unroll
       for (int j = 0; j < KPG; j += 2) {
         const float p0 = ex2f(s2[j] - ms_ref), p1 = ex2f(s2[j + 1] - ms_ref);   // 0 for -inf
-        lsum += p0 + p1;
-        const float u0 = p0 * ksc[j] * cu_new, u1 = p1 * ksc[j + 1] * cu_new;   // P' = P k_scale cu
+        const float kc0 = ksc[j] * cu_new, kc1 = ksc[j + 1] * cu_new;          // powers of two (or 0)
+        const float u0 = p0 * kc0, u1 = p1 * kc1;                               // P' = P k_scale cu
         const uint32_t hi = e4m3x2(u0, u1);
         const float2 hf = e4m3x2_to_f32(hi);
         const uint32_t lo = e4m3x2(u0 - hf.x, u1 - hf.y);
+        const float2 lf = e4m3x2_to_f32(lo);
+        // 1 / (k_scale cu) by exponent arithmetic (exact for a normal power of two)
+        const float w0 = kc0 != 0.f ? (hf.x + lf.x) * __int_as_float((254 << 23) - __float_as_int(kc0)) : 0.f;
+        const float w1 = kc1 != 0.f ? (hf.y + lf.y) * __int_as_float((254 << 23) - __float_as_int(kc1)) : 0.f;
+        lsum += w0 + w1;
         if ((j & 3) == 0) {
           phi[j >> 2] = hi;
           plo[j >> 2] = lo;
@@ -490,7 +500,7 @@ __global__ void __launch_bounds__(NTHR, 1)
           phi[j >> 2] |= hi << 16;
           plo[j >> 2] |= lo << 16;
         }
-        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+        const __nv_bfloat162 pb = __floats2bfloat162_rn(w0, w1);
         pbf[j >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
       }
       l = l * as + lsum;
