@@ -52,6 +52,9 @@ size_t mqa_qbuf_bytes(const v4attn_layer_desc* d, int32_t n_q) {
 // body offset of MQA calls and of every call of a decode step
 size_t body_mqa(const v4attn_layer_desc* d, int32_t n_q) { return qimg_off(n_q) + mqa_qbuf_bytes(d, n_q); }
 size_t mqa_need(const v4attn_layer_desc* d, int32_t n_q, int64_t n_main_max) {
+  // the tensor-core MQA (E4M3 caches) merges its key splits inside a thread-block
+  // cluster and writes the output directly: no split-K partials
+  if (d->kv_dtype == V4A_E4M3_BF16ROPE) return 0;
   const int S = mqa_num_splits(d, n_main_max);
   const int32_t c = q_chunk(n_q);
   return mqa_part_o_bytes(d, c, S) + mqa_part_ml_bytes(d, c, S);
@@ -308,7 +311,8 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
     }
     if (dry) return V4A_OK;
     if (mqa_dispatch(P, st) != cudaSuccess) return V4A_ERR_CUDA;
-    if (launch_mqa_combine(P, st) != cudaSuccess) return V4A_ERR_CUDA;
+    if (d->kv_dtype != V4A_E4M3_BF16ROPE && launch_mqa_combine(P, st) != cudaSuccess)
+      return V4A_ERR_CUDA;
   }
   return V4A_OK;
 }

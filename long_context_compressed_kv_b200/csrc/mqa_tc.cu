@@ -41,6 +41,7 @@
 // per TMEM lane quarter, one per 16-key group of each tile, exchanging row
 // maxima through shared memory.  Every cross-warp hand-off is an mbarrier with a
 // bounded, warp-uniform wait, so a stalled kernel ends with a status bit.
+#include <cooperative_groups.h>
 #include <cstddef>
 
 #include "common.cuh"
@@ -60,8 +61,6 @@ constexpr int KPG = 64 / KG;    // keys per group
 constexpr int NSM = 4 * KG;     // softmax / epilogue warps
 constexpr int NTHR = 64 + 32 * NSM;
 constexpr int ROWB = 576;       // stored row: 448 E4M3 + 64 bf16
-constexpr int SKMAX = 512;      // keys per split, at most
-constexpr int SKMAX_SEL = 128;  // keys per split of a selected-entry (sparse) call
 constexpr int TILE_BYTES = NK * (4 * 128 + 64);
 constexpr float kTau = 4.f;     // lazy-rescale margin of the running score maximum (log2 units)
 // query image (layout in mqa_qimage.cuh)
@@ -80,8 +79,14 @@ struct Smem {
   alignas(1024) uint8_t p_lo[128 * 64];       // P' low part
   alignas(1024) uint8_t p_bf[128 * 128];      // P for the RoPE dims, bf16, K-major SW128
   float kscale[KST][NK];
-  int idx[SKMAX_SEL];
-  float xmax[2][KG][2][128];                  // [tile parity][key group][M_s, M_u][row]
+  union {
+    float xmax[2][KG][2][128];                // tile loop: [tile parity][key group][M_s, M_u][row]
+    struct {                                  // merge (the loop is over for every warp):
+      float rms[128], rl[128], rfn[128];      // this split's row max (log2), row sum, 1 / cu
+      float fself[128], invl[128];            // merge factor of this split, 1 / denominator
+      float rcs[32], rsn[32];                 // RoPE angles of the query position
+    } mg;
+  };
   float xl[KG - 1][128];                      // the other groups' row sums, for the epilogue
   uint64_t full[KST], empty[KST], sfull[2], sfree[2], xbar[2];
   uint64_t pfull, pempty, qready, ofinal, done, lbar;
@@ -90,6 +95,10 @@ struct Smem {
 
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory per CTA");
 static_assert(offsetof(Smem, qsc) == QTILE, "the query image is one contiguous copy");
+// the merge stages this split's O (fp32, 128 rows of SST floats) over the key
+// stages and P buffers, which are free once the last P.V has completed
+constexpr int SST = 260;                     // row stride (floats): conflict-free float4 rows
+static_assert(offsetof(Smem, kscale) - offsetof(Smem, kv) >= 128 * SST * 4, "merge stage fits");
 
 struct Maps {
   CUtensorMap kv128, kv64;      // tile mode, boxes {128 B | 64 B} x NK rows
@@ -169,9 +178,11 @@ __device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
   if (g.n_swa < 0) g.n_swa = 0;
   g.nmp = (g.n_main + NK - 1) / NK * NK;
   g.total = g.nmp + (g.n_swa + NK - 1) / NK * NK;
-  g.s0 = split * P.split_keys;
-  const int len = min(P.split_keys, g.total - g.s0);
-  g.T = len > 0 ? len / NK : 0;
+  // split `split` of C takes tiles [T * split / C, T * (split + 1) / C) of the query's T
+  const int T = g.total / NK, C = P.n_split;
+  const int t0 = (int)((int64_t)T * split / C), t1 = (int)((int64_t)T * (split + 1) / C);
+  g.s0 = t0 * NK;
+  g.T = t1 - t0;
   return g;
 }
 
@@ -193,20 +204,14 @@ __global__ void __launch_bounds__(NTHR, 1)
   Smem& s = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int dh = blockIdx.x & 1;
-  const int rest = blockIdx.x >> 1;
-  const int split = rest % P.n_split, q = rest / P.n_split;
+  // the C = n_split CTAs of a cluster are the key splits of one (query, half);
+  // cluster rank == split
+  const int C = P.n_split;
+  const int split = (int)(blockIdx.x % (unsigned)C);
+  const int unit = (int)(blockIdx.x / (unsigned)C);
+  const int dh = unit & 1, q = unit >> 1;
   const Geo g = geometry(P, q, split);
-  const int64_t pbase = ((int64_t)q * P.n_split + split) * P.H;
-
-  if (g.T == 0) {                     // nothing in this chunk: an empty partial
-    if (dh == 0)
-      for (int h = threadIdx.x; h < P.H; h += NTHR) {
-        P.part_ml[(pbase + h) * 2] = -INFINITY;
-        P.part_ml[(pbase + h) * 2 + 1] = 0.f;
-      }
-    return;
-  }
+  // every CTA, also one with no tiles (T = 0), takes part in the merge below
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < KST; ++i) {
@@ -225,13 +230,6 @@ __global__ void __launch_bounds__(NTHR, 1)
     mbar_init(&s.done, 1);
     mbar_init(&s.lbar, NSM - 4);
     fence_mbar_init();
-  }
-  if (warp == 0 && P.idx) {
-    // this chunk's selected entries (-1 marks an empty slot)
-    for (int i = lane; i < P.split_keys; i += 32) {
-      const int j = g.s0 + i;
-      s.idx[i] = (j < g.n_main) ? P.idx[(int64_t)q * P.n_sel + j] : -1;
-    }
   }
   if (warp == 1) tmem_alloc(&s.tmem_base, 512);
   tc_fence_before();
@@ -258,7 +256,7 @@ __global__ void __launch_bounds__(NTHR, 1)
       if (main_tile) {
         const int jj = vk + r;
         if (jj >= g.n_main) return -1;
-        const int e = P.idx ? s.idx[jj - g.s0] : jj;
+        const int e = P.idx ? P.idx[(int64_t)q * P.n_sel + jj] : jj;   // -1: an empty slot
         if (e < 0) return -1;
         if (e >= g.n_vis) {
           flag(P.status, ST_BAD_INDEX);
@@ -272,12 +270,14 @@ __global__ void __launch_bounds__(NTHR, 1)
       return sw_base + tok % P.swa_rows;
     };
     bool issued_ok = true;
+    int issued = 0;
     for (int t = 0; t < g.T; ++t) {
       const int st = t % KST, u = t / KST;
       if (u >= 1 && !mbar_wait_warp(&s.empty[st], (u - 1) & 1, P.status, 0)) {
         issued_ok = false;
         break;
       }
+      issued = t + 1;
       const int vk = g.s0 + t * NK;
       const bool main_tile = vk < g.nmp;
       const bool contiguous = main_tile && !P.idx && vk + NK <= g.n_main;
@@ -323,6 +323,16 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     cp_async_wait<0>();
     if (!issued_ok) flag(P.status, ST_TIMEOUT);
+    // drain: no copy may still be landing when the merge reuses the stages (or
+    // the CTA exits); on a normal run these phases completed long ago
+    if (lane == 0) {
+      mbar_wait(&s.qready, 0);                                      // time bound only
+      for (int k = 0; k < KST && k < issued; ++k) {
+        const int i2 = issued - 1 - k;
+        mbar_wait(&s.full[i2 % KST], (i2 / KST) & 1);
+      }
+    }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     const uint64_t kq128 = smem_desc_bits(16, 1024, 2);   // K-major, 128B swizzle
@@ -398,7 +408,7 @@ __global__ void __launch_bounds__(NTHR, 1)
       __syncwarp();
       if (t >= 1 && !pv(t - 1)) { ok = false; break; }
     }
-    if (ok) ok = pv(g.T - 1);
+    if (ok && g.T > 0) ok = pv(g.T - 1);
     if (!ok) flag(P.status, ST_TIMEOUT);
     if (lane == 0) {
       tc_commit(&s.ofinal);
@@ -565,37 +575,119 @@ __global__ void __launch_bounds__(NTHR, 1)
       for (int o = 0; o < KG - 1; ++o) l += s.xl[o][h];
     }
     fin = fin && live;
-    // O_nope is in units of cu exp2(. - Ms); express it in units of exp2(. - Ms)
-    const float fn = (Ms == -INFINITY || cu == 0.f) ? 0.f : 1.f / cu;
-    // O rows leave through a per-warp 32 x 32 staging block in shared memory
-    // (the key stages are free once ofinal has fired), so that every global
-    // store writes one 128-byte row segment.
-    const uint32_t ob = tmem + lane_off + 256;
-    float* stg = reinterpret_cast<float*>(&s.kv[0][0][0]) + (warp - 2) * (32 * 33);
-    const int64_t row0 = pbase + quad * 32;
+    // this split's per-row results for the merge: the row maximum (log2 units;
+    // -inf for no key), the row sum in units of exp2(. - Ms), and 1 / cu, the
+    // factor that brings O_nope (kept in units of cu exp2(. - Ms)) to those units
+    if (grp == 0) {
+      const bool any = fin && Ms != -INFINITY;
+      s.mg.rms[h] = any ? Ms : -INFINITY;
+      s.mg.rl[h] = any ? l : 0.f;
+      s.mg.rfn[h] = (any && cu != 0.f) ? 1.f / cu : 0.f;
+    }
+  }
+
+  // ------------------------------------------------------------ merge the C splits
+  // Every thread of every CTA of the cluster passes the cluster barriers below
+  // exactly once (the roles above have no early exit), so none can hang.
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  const int tid = threadIdx.x;
+  tc_fence_before();
+  __syncthreads();
+  cl.sync();                                    // every split's rms / rl / rfn published
+  const float log2e = 1.4426950408889634f;
+  if (tid < 128) {
+    // the merged row maximum (with the sink, in log2 units) and denominator
+    const int hh = tid;
+    const float z = (P.sink && hh < P.H) ? P.sink[hh] * log2e : -INFINITY;
+    float M = z;
+    for (int r = 0; r < C; ++r) M = fmaxf(M, cl.map_shared_rank(s.mg.rms, (unsigned)r)[hh]);
+    float den = 0.f;
+    if (M != -INFINITY) {
+      for (int r = 0; r < C; ++r) {
+        const float mr = cl.map_shared_rank(s.mg.rms, (unsigned)r)[hh];
+        if (mr != -INFINITY) den += ex2f(mr - M) * cl.map_shared_rank(s.mg.rl, (unsigned)r)[hh];
+      }
+      if (z != -INFINITY) den += ex2f(z - M);
+    }
+    s.mg.fself[hh] = (s.mg.rms[hh] == -INFINITY) ? 0.f : ex2f(s.mg.rms[hh] - M);
+    s.mg.invl[hh] = den > 0.f ? 1.f / den : 0.f;
+    if (P.lse && dh == 0 && split == 0 && hh < P.H)
+      P.lse[(int64_t)q * P.H + hh] = den > 0.f ? M * 0.6931471805599453f + logf(den) : -INFINITY;
+  } else if (tid < 160 && dh == 1) {
+    // rotation by -p of the output's RoPE dims: the angles of the 32 pairs
+    float c = 1.f, sv = 0.f;
+    if (g.p >= 0) rope_cs(g.p, tid - 128, 64, P.theta, c, sv);
+    s.mg.rcs[tid - 128] = c;
+    s.mg.rsn[tid - 128] = sv;
+  }
+  __syncthreads();
+  // stage this split's O, scaled to the merged units, as fp32 rows in shared memory
+  float* stage = reinterpret_cast<float*>(&s.kv[0][0][0]);
+  if (warp >= 2) {
+    const int quad = warp & 3, grp = (warp - 2) >> 2;
+    const int hh = quad * 32 + lane;
+    const uint32_t ob = tmem + ((uint32_t)(quad * 32) << 16) + 256;
+    const float fs = s.mg.fself[hh], fnn = fs * s.mg.rfn[hh];
+#pragma unroll 1
     for (int cc = 0; cc < 256 / KG; cc += 32) {
       const int c = grp * (256 / KG) + cc;
       uint32_t r[32];
       tmem_ld32_nowait(ob + c, r);
       tmem_ld_wait();
-      const float f = (dh == 1 && c >= 192) ? (Ms == -INFINITY ? 0.f : 1.f) : fn;
-      if (fin) {
+      const float f = (dh == 1 && c >= 192) ? fs : fnn;   // RoPE dims carry no cu
+      float4* dst = reinterpret_cast<float4*>(stage + hh * SST + c);
 #pragma unroll
-        for (int k = 0; k < 32; ++k) stg[lane * 33 + k] = __uint_as_float(r[k]) * f;
-        __syncwarp();
-        for (int rr = 0; rr < 32; ++rr)
-          if (quad * 32 + rr < P.H)
-            P.part_o[(row0 + rr) * 512 + dh * 256 + c + lane] = stg[rr * 33 + lane];
-        __syncwarp();
-      }
-    }
-    if (dh == 0 && grp == 0 && h < P.H) {
-      P.part_ml[(pbase + h) * 2] = (Ms == -INFINITY) ? -INFINITY : Ms * 0.6931471805599453f;
-      P.part_ml[(pbase + h) * 2 + 1] = l;
+      for (int k = 0; k < 8; ++k)
+        dst[k] = make_float4(__uint_as_float(r[4 * k]) * f, __uint_as_float(r[4 * k + 1]) * f,
+                             __uint_as_float(r[4 * k + 2]) * f, __uint_as_float(r[4 * k + 3]) * f);
     }
   }
   tc_fence_before();
   __syncthreads();
+  cl.sync();                                    // every split's O staged
+  {
+    // this CTA writes output columns [c0, c1) of its half: the sum over the
+    // splits (distributed shared memory), / denominator, R(-p) on RoPE dims
+    const int c0 = 256 * split / C, c1 = 256 * (split + 1) / C;
+    const int ng = (c1 - c0) / 4;
+    const int64_t obase = (int64_t)q * P.H * 512 + dh * 256;
+    for (int it = tid; it < 128 * ng; it += NTHR) {
+      const int hh = it / ng, col = c0 + 4 * (it % ng);
+      if (hh >= P.H) continue;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int r = 0; r < C; ++r) {
+        const float4 b = *reinterpret_cast<const float4*>(
+            cl.map_shared_rank(stage, (unsigned)r) + hh * SST + col);
+        a.x += b.x;
+        a.y += b.y;
+        a.z += b.z;
+        a.w += b.w;
+      }
+      const float il = s.mg.invl[hh];
+      float o[4] = {a.x * il, a.y * il, a.z * il, a.w * il};
+      if (dh == 1 && col >= 192) {
+#pragma unroll
+        for (int e = 0; e < 4; e += 2) {
+          const int k = (col + e - 192) >> 1;
+          const float cs = s.mg.rcs[k], sn = s.mg.rsn[k];
+          const float r0 = o[e] * cs + o[e + 1] * sn, r1 = -o[e] * sn + o[e + 1] * cs;
+          o[e] = r0;
+          o[e + 1] = r1;
+        }
+      }
+      const int64_t off = obase + (int64_t)hh * 512 + col;
+      if (P.out_dtype == V4A_F32) {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) + off) =
+            make_float4(o[0], o[1], o[2], o[3]);
+      } else {
+        const uint32_t w0 = (uint32_t)f32_to_bf16_bits(o[0]) | ((uint32_t)f32_to_bf16_bits(o[1]) << 16);
+        const uint32_t w1 = (uint32_t)f32_to_bf16_bits(o[2]) | ((uint32_t)f32_to_bf16_bits(o[3]) << 16);
+        *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(P.out) + off) = make_uint2(w0, w1);
+      }
+    }
+  }
+  cl.sync();                                    // no CTA leaves while its stage is read
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -609,8 +701,7 @@ bool make_rows_map_sw(CUtensorMap* map, const void* base, int64_t rows, int row_
 
 int mqa_tc_check(const MqaParams& P) {
   if (P.kv_dtype != V4A_E4M3_BF16ROPE || P.d != 512 || P.d_rope != 64 || P.H > 128 ||
-      P.q_dtype != V4A_BF16 || P.split_keys % NK != 0 || P.split_keys > SKMAX ||
-      (P.idx && P.split_keys > SKMAX_SEL) || P.n_win > 1024 || P.qbuf == nullptr ||
+      P.q_dtype != V4A_BF16 || P.n_win > 1024 || P.qbuf == nullptr ||
       (int64_t)P.B * P.kv_rows >= (1ll << 31) || (int64_t)P.B * P.swa_rows >= (1ll << 31))
     return 2;
   if (((uintptr_t)P.qbuf & 15) || ((uintptr_t)P.kv & 15) ||
@@ -633,20 +724,67 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
       !make_rows_map_sw(&m.swg64, swa, swr, ROWB, 64, 1, 64))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
-  static unsigned long long configured = 0;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !(configured & (1ull << dev))) {
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  // per device: the largest cluster size whose clusters can all be resident
+  // for a given cluster count (queried once per size)
+  static int max_active[64][5];                  // sizes 1, 2, 4, 8, 16; 0 = not queried
+  static bool configured[64] = {false};
+  if (!configured[dev]) {
     cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    configured |= 1ull << dev;
+    if (cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+        cudaSuccess)
+      cudaGetLastError();                        // 16-CTA clusters then report 0 below
+    for (int k = 0; k < 5; ++k) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(1u << k, 1, 1);
+      cfg.blockDim = dim3(NTHR, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 1u << k;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, mqa_tc_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+      max_active[dev][k] = n;
+    }
+    configured[dev] = true;
   }
-  const int64_t grid = (int64_t)P.n_q * P.n_split * 2;
+  // key splits per (query, half) = CTAs per cluster: the largest power of two
+  // that keeps every cluster of the launch resident at once on this GPU (one
+  // CTA per SM), at most the query's key tiles, at least 1
+  MqaParams Q = P;
+  const int64_t n_main = P.idx ? (int64_t)P.n_sel : P.max_vis;
+  const int64_t tiles = (n_main + NK - 1) / NK + (P.n_win + NK - 1) / NK;
+  const int64_t units = 2 * (int64_t)P.n_q;
+  int k = 4;
+  while (k > 0 && ((1ll << k) > tiles || max_active[dev][k] < units)) --k;
+  Q.n_split = 1 << k;
+  const int64_t grid = units * Q.n_split;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
   if (!P.q_ready) mqa_tc_qprep_kernel<<<dim3((unsigned)P.n_q, 8), 64, 0, st>>>(P);
-  mqa_tc_kernel<<<(unsigned)grid, NTHR, smem, st>>>(P, m);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(NTHR, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)Q.n_split;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mqa_tc_kernel, Q, m);
 }
 
 }  // namespace v4a
