@@ -48,7 +48,7 @@ def desc_for(ly):
                         idx_dtype=v.MXFP4 if ly.idx_fp4 else v.F32)
 
 
-def build_decode_layer(w, li, inp, in_dtype=None):
+def build_decode_layer(w, li, inp, in_dtype=None, out_dtype=None):
     """A DecodeLayer holding the coded synthetic history of ``synth.decode_layer_inputs``
     and the new token's inputs, ready for ``step``."""
     import torch
@@ -56,7 +56,7 @@ def build_decode_layer(w, li, inp, in_dtype=None):
     ly = w.layers[li]
     p, ring = inp["p"], inp["ring"]
     lay = DecodeLayer(desc_for(ly), w.B, kv_rows=inp["n_hist"] + 1, swa_rows=ly.n_win,
-                      in_dtype=in_dtype or torch.float32)
+                      in_dtype=in_dtype or torch.float32, out_dtype=out_dtype or torch.bfloat16)
     lay.load_entries(inp["hist_entries"])
     lay.load_window(inp["swa_hist"], first_token=p - (ly.n_win - 1))
     names = ["Ca", "Za", "Cb", "Zb"] if ly.kind == "csa" else ["C", "Z"]
@@ -94,7 +94,7 @@ class PrefillPair:
 
     CHUNK = 4096                       # host-side generation chunk (rows)
 
-    def __init__(self, w):
+    def __init__(self, w, out_dtype=None):
         import torch
         import long_context_compressed_kv_b200 as v
         self.v, self.w = v, w
@@ -164,9 +164,10 @@ class PrefillPair:
         self.pos = torch.arange(P, L, dtype=torch.int64, device=dev)
         self.seq = torch.zeros(n, dtype=torch.int32, device=dev)
         self.idx = torch.full((n, csa.top_k), -1, dtype=torch.int32, device=dev)
-        self.out_c = torch.zeros(n, csa.H, csa.d, dtype=torch.bfloat16, device=dev)
+        od = out_dtype or torch.bfloat16
+        self.out_c = torch.zeros(n, csa.H, csa.d, dtype=od, device=dev)
         self.lse_c = torch.zeros(n, csa.H, dtype=torch.float32, device=dev)
-        self.out_h = torch.zeros(n, hca.H, hca.d, dtype=torch.bfloat16, device=dev)
+        self.out_h = torch.zeros(n, hca.H, hca.d, dtype=od, device=dev)
         self.lse_h = torch.zeros(n, hca.H, dtype=torch.float32, device=dev)
         self.ws_c = v.workspace(self.dc, n, self.rows_c)
         self.ws_h = v.workspace(self.dh, n, self.rows_h)

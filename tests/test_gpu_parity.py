@@ -11,8 +11,8 @@ import synth
 from oracle import codecs, compress as ocomp, indexer as oidx, mqa as omqa, pipeline
 from tests.gpu_util import (F32_ABS_TOL, LSE_ABS_TOL, R16_TOL, DecodeState, check_output,
                             check_stored_keys, check_stored_kv, check_topk, code_rows,
-                            compare_decode, desc_for, dev, oracle_attention, r16, read_keys,
-                            read_kv, v4)
+                            check_bf16_output_is_rounded_fp32, compare_decode, desc_for, dev,
+                            oracle_attention, r16, read_keys, read_kv, v4)
 
 pytestmark = pytest.mark.gpu
 
@@ -253,19 +253,27 @@ def test_mqa_parity(sparse, fp8, H, d, d_rope, q_rmsnorm):
         nv = int(ocomp.n_visible(positions[q], m))
         sel = np.sort(rng.choice(nv, size=min(k, nv), replace=False)) if nv else np.zeros(0, int)
         idx[q, : len(sel)] = sel
-    out = torch.zeros(nq, H, d, dtype=torch.float32 if not fp8 else torch.bfloat16, device="cuda")
+    # parity on the fp32 output; the bf16 output is checked to be its rounding
+    out = torch.zeros(nq, H, d, dtype=torch.float32, device="cuda")
     lse = torch.zeros(nq, H, dtype=torch.float32, device="cuda")
     ws = v.workspace(desc, nq, N)
     kw = dict(Q=dev(Q, torch.bfloat16), q_pos=dev(positions, torch.int64),
               q_seq=dev(q_seq, torch.int32), B=B, kv=kv, kv_scale=kv_sc, kv_rows=N, swa=swa,
               swa_scale=swa_sc, swa_rows=swa_rows, out=out, ws=ws, sink=dev(sink), lse=lse,
               q_rmsnorm=q_rmsnorm)
-    if sparse:
-        v.sparse_mqa(desc, idx=dev(idx, torch.int32), **kw)
-    else:
-        v.dense_mqa(desc, max_vis=N, **kw)
+    def run(**extra):
+        if sparse:
+            v.sparse_mqa(desc, idx=dev(idx, torch.int32), **{**kw, **extra})
+        else:
+            v.dense_mqa(desc, max_vis=N, **{**kw, **extra})
+    run()
     torch.cuda.synchronize()
     assert v.device_status(ws) == 0
+    if fp8:
+        ob = torch.zeros(nq, H, d, dtype=torch.bfloat16, device="cuda")
+        run(out=ob)
+        torch.cuda.synchronize()
+        assert torch.equal(ob, out.to(torch.bfloat16))
     g_out, g_lse = out.float().cpu().numpy(), lse.cpu().numpy()
     e_val = read_kv(kv, kv_sc, fmt, d, d_rope)
     s_val = read_kv(swa, swa_sc, fmt, d, d_rope)
@@ -290,7 +298,7 @@ def test_mqa_no_sink_and_empty_selection():
                             rows=128)
     Q = synth.bf16_values(rng.standard_normal((1, 64, 512)).astype(np.float32))
     idx = torch.full((1, 32), -1, dtype=torch.int32, device="cuda")     # nothing selected
-    out = torch.zeros(1, 64, 512, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(1, 64, 512, dtype=torch.float32, device="cuda")
     ws = v.workspace(desc, 1, 50)
     v.sparse_mqa(desc, Q=dev(Q, torch.bfloat16), q_pos=dev(np.array([40]), torch.int64), kv=kv,
                  kv_scale=kv_sc, kv_rows=50, swa=swa, swa_scale=swa_sc, swa_rows=128, idx=idx,
@@ -316,6 +324,7 @@ def test_decode_step_small(kind, L):
     st = DecodeState(w, 0, inp)
     st.step()
     compare_decode(st, [0, 1, 2])
+    check_bf16_output_is_rounded_fp32(st)
 
 
 def test_decode_is_deterministic_and_batch_invariant():
@@ -421,6 +430,7 @@ def _full_decode(name, seqs):
         st = DecodeState(w, li, inp)
         st.step()
         rep = compare_decode(st, seqs)
+        check_bf16_output_is_rounded_fp32(st)
         print(name, li, rep)
         del st
         torch.cuda.empty_cache()
@@ -452,7 +462,13 @@ def test_projection_tensor_core(M, N, K, y_bf16):
     W = synth.bf16_values((rng.standard_normal((K, N)) / np.sqrt(K)).astype(np.float32))
     Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16 if y_bf16 else torch.float32,
                    device="cuda")
-    v.project(dev(X, torch.bfloat16), dev(W, torch.bfloat16), Y)
+    # row strides of X and W must be multiples of 16 bytes: views of padded buffers
+    ldx, ldw = (K + 7) // 8 * 8, (N + 7) // 8 * 8
+    Xd = torch.zeros(M, ldx, dtype=torch.bfloat16, device="cuda")
+    Wd = torch.zeros(K, ldw, dtype=torch.bfloat16, device="cuda")
+    Xd[:, :K] = dev(X, torch.bfloat16)
+    Wd[:, :N] = dev(W, torch.bfloat16)
+    v.project(Xd[:, :K], Wd[:, :N], Y)
     torch.cuda.synchronize()
     want = X.astype(np.float64) @ W.astype(np.float64)
     got = Y.float().cpu().numpy().astype(np.float64)

@@ -36,7 +36,7 @@ def _run(w):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from bench import PrefillPair
-    pp = PrefillPair(w)
+    pp = PrefillPair(w, out_dtype=torch.float32)     # parity on the fp32 outputs
     pp.prefix_state()
     pp.step()
     torch.cuda.synchronize()
@@ -186,6 +186,19 @@ def test_scaled_entries_keys_and_window(scaled):
 def test_scaled_every_query(scaled):
     check_queries(scaled, np.arange(scaled.w.n_queries))
     check_selection_valid(scaled)
+
+
+def test_scaled_bf16_outputs_are_rounded_fp32(scaled):
+    """The same step with bf16 outputs gives the bf16 rounding of the fp32
+    outputs, bit for bit (the step is idempotent)."""
+    f32 = (scaled.out_c.clone(), scaled.out_h.clone())
+    scaled.out_c = torch.zeros(f32[0].shape, dtype=torch.bfloat16, device="cuda")
+    scaled.out_h = torch.zeros(f32[1].shape, dtype=torch.bfloat16, device="cuda")
+    scaled.step()
+    torch.cuda.synchronize()
+    assert torch.equal(scaled.out_c, f32[0].to(torch.bfloat16))
+    assert torch.equal(scaled.out_h, f32[1].to(torch.bfloat16))
+    scaled.out_c, scaled.out_h = f32
 
 
 # ------------------------------------------------------------------ full size (sampled)
