@@ -206,7 +206,10 @@ typedef struct {
  *   2. if (p+1) % m == 0 the completed block is pooled into entry (p+1)/m-1
  *      of the main cache (and, for CSA, of the indexer-key cache);
  *   3. CSA: indexer + top-k over the visible keys;
- *   4. MQA over the selected (CSA) or all visible (HCA) entries + window.  */
+ *   4. MQA over the selected (CSA) or all visible (HCA) entries + window.
+ * x_main, tail, x_idx, itail must be aligned to 4 elements and bias, ibias
+ * to 16 bytes (else V4A_ERR_INVALID_ARG); the pooling window (ring rows)
+ * times d must not exceed 65536 (V4A_ERR_UNSUPPORTED).  */
 typedef struct {
   int32_t B;
   const int64_t* pos;         /* device [B] position p of each sequence's new token */

@@ -383,12 +383,16 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
   const int d = desc->d;
   const int elt = a->in_dtype == V4A_F32 ? 4 : 2;
   {
-    // channel pairs are read as one 2-element load
-    const uintptr_t al = 2 * (uintptr_t)elt;
+    // the append kernel reads four channels per load: bases aligned to 4 elements,
+    // biases to 16 bytes
+    const uintptr_t al = 4 * (uintptr_t)elt;
     for (const void* p : {a->x_main, (const void*)a->tail, a->x_idx, (const void*)a->itail})
       if (p && (reinterpret_cast<uintptr_t>(p) % al)) return V4A_ERR_INVALID_ARG;
     for (const void* p : {(const void*)a->bias, (const void*)a->ibias})
-      if (p && (reinterpret_cast<uintptr_t>(p) % 8)) return V4A_ERR_INVALID_ARG;
+      if (p && (reinterpret_cast<uintptr_t>(p) % 16)) return V4A_ERR_INVALID_ARG;
+    // a pooling window of at most 65536 / d rows per entry (8 rows per thread
+    // over the d / 8 channels of each of the job's 8 CTAs)
+    if ((int64_t)ring * d > 65536) return V4A_ERR_UNSUPPORTED;
   }
   // 1.-2. tail rings, the new token's window KV (RMSNorm, RoPE at p), the
   // entry (and indexer key) its block completes: one launch

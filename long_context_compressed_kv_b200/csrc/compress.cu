@@ -25,7 +25,6 @@
 
 #include "common.cuh"
 #include "kernels.h"
-#include "mqa_qimage.cuh"
 
 namespace v4a {
 
@@ -251,165 +250,6 @@ __global__ void __launch_bounds__(512) compress_kernel(CompressParams P, int n_e
     compress_entry(P, b, e0 + e, red, mrg, part, PT, RS, CH, chunk);
     __syncthreads();
   }
-}
-
-// One decode step's appends for every sequence b, in one launch: job (b, t)
-// is one cluster of kAppendCluster CTAs; t = 0 codes the new token's window
-// KV (and copies its raw inputs into the main tail ring), t = 1 pools the
-// entry its block completes, t = 2 (CSA) pools the indexer key (and copies
-// the indexer inputs into the indexer tail ring).  The pooling jobs read the
-// new token from its input row, so the ring copies run concurrently with them.
-constexpr int kAppendCluster = 8;
-constexpr int kAppendThreads = 256;
-
-__device__ __forceinline__ int chunks_for(int c) {
-  int CH = kAppendCluster;
-  while (CH > 1 && (c % (32 * CH) != 0 || c / CH < 64)) CH >>= 1;
-  return CH;
-}
-
-__device__ __forceinline__ void copy_share(uint8_t* dst, const uint8_t* src, int64_t n, int rank) {
-  // rank's share of an n-byte copy, 16 bytes at a time where both ends allow it
-  const int64_t per = (n / kAppendCluster + 15) / 16 * 16;
-  const int64_t lo = min(n, per * rank), hi = min(n, lo + per);
-  if ((((uintptr_t)(dst + lo)) | ((uintptr_t)(src + lo)) | (uintptr_t)(hi - lo)) % 16 == 0) {
-    const uint4* s4 = reinterpret_cast<const uint4*>(src + lo);
-    uint4* d4 = reinterpret_cast<uint4*>(dst + lo);
-    for (int64_t e = threadIdx.x; e < (hi - lo) / 16; e += blockDim.x) d4[e] = s4[e];
-  } else {
-    for (int64_t e = lo + threadIdx.x; e < hi; e += blockDim.x) dst[e] = src[e];
-  }
-}
-
-__global__ void __launch_bounds__(kAppendThreads, 2) decode_append_kernel(AppendParams A) {
-  __shared__ float red[32];
-  __shared__ float part[2];
-  __shared__ float mrg[kAppendThreads * 6];
-  const int nbase = A.csa ? 3 : 2;
-  const int nj = nbase + (A.qimg ? 1 : 0);
-  const int job = blockIdx.x / kAppendCluster, rank = blockIdx.x % kAppendCluster;
-  const int b = job / nj, t = job % nj;
-  if (t == nbase) {
-    // the tensor-core MQA's query image: CTA `rank` codes head rows 16*rank .. +15
-    __shared__ float qcs[32], qsn[32];
-    qimage_code_rows(reinterpret_cast<const __nv_bfloat16*>(A.Q) + (int64_t)b * A.H * 512, A.H,
-                     A.pos[b], A.theta, A.qimg + (int64_t)b * kMqaQImageStride, rank, qcs, qsn);
-    return;
-  }
-  const int elt = A.in_dtype == V4A_F32 ? 4 : 2;
-  const int64_t p = A.pos[b];
-  const int64_t nb = (int64_t)A.n_arr * A.d * elt;         // bytes of one main input row
-  const uint8_t* xm = reinterpret_cast<const uint8_t*>(A.x_main);
-  const uint8_t* tl = reinterpret_cast<const uint8_t*>(A.tail);
-  CompressParams P;
-  P.in_dtype = A.in_dtype;
-  P.d_rope = A.d_rope;
-  P.theta = A.theta;
-  P.eps = A.eps;
-  P.seq_len = nullptr;
-  P.entry_begin = nullptr;
-  P.new_pos = A.pos;
-  int64_t i;
-  if (t == 0) {
-    if (p >= 0)
-      copy_share(reinterpret_cast<uint8_t*>(A.tail) + ((int64_t)b * A.ring + p % A.ring) * nb,
-                 xm + b * nb, nb, rank);
-    P.m = 1;
-    P.overlap = 0;
-    P.c = A.d;
-    P.Ca = A.x_main;
-    P.Za = P.Cb = P.Zb = nullptr;
-    P.Ca_new = A.x_main;
-    P.in_seq_stride = P.in_row_stride = P.new_seq_stride = (int64_t)A.n_arr * A.d;
-    P.in_rows = 1;
-    P.bias = nullptr;
-    P.complete_only = 0;
-    P.apply_rmsnorm = 1;
-    P.apply_rope = 1;
-    P.out_dtype = A.kv_dtype;
-    P.out = A.swa;
-    P.out_scale = A.swa_scale;
-    P.out_rows = A.swa_rows;
-    i = p;
-  } else if (t == 1) {
-    const int64_t da = (int64_t)A.d * elt;
-    P.m = A.m;
-    P.overlap = A.csa;
-    P.c = A.d;
-    P.Ca = tl;
-    P.Za = tl + da;
-    P.Cb = A.csa ? tl + 2 * da : nullptr;
-    P.Zb = A.csa ? tl + 3 * da : nullptr;
-    P.Ca_new = xm;
-    P.Za_new = xm + da;
-    P.Cb_new = A.csa ? xm + 2 * da : nullptr;
-    P.Zb_new = A.csa ? xm + 3 * da : nullptr;
-    P.in_seq_stride = (int64_t)A.ring * A.n_arr * A.d;
-    P.in_row_stride = P.new_seq_stride = (int64_t)A.n_arr * A.d;
-    P.in_rows = A.ring;
-    P.bias = A.bias;
-    P.complete_only = 1;
-    P.apply_rmsnorm = 1;
-    P.apply_rope = 1;
-    P.out_dtype = A.kv_dtype;
-    P.out = A.kv;
-    P.out_scale = A.kv_scale;
-    P.out_rows = A.kv_rows;
-    i = p / A.m;
-  } else {
-    const int64_t ni = (int64_t)4 * A.dI * elt;
-    const uint8_t* xi = reinterpret_cast<const uint8_t*>(A.x_idx);
-    const uint8_t* it = reinterpret_cast<const uint8_t*>(A.itail);
-    if (p >= 0)
-      copy_share(reinterpret_cast<uint8_t*>(A.itail) + ((int64_t)b * A.ring + p % A.ring) * ni,
-                 xi + b * ni, ni, rank);
-    const int64_t da = (int64_t)A.dI * elt;
-    P.m = A.m;
-    P.overlap = 1;
-    P.c = A.dI;
-    P.Ca = it;
-    P.Za = it + da;
-    P.Cb = it + 2 * da;
-    P.Zb = it + 3 * da;
-    P.Ca_new = xi;
-    P.Za_new = xi + da;
-    P.Cb_new = xi + 2 * da;
-    P.Zb_new = xi + 3 * da;
-    P.in_seq_stride = (int64_t)A.ring * 4 * A.dI;
-    P.in_row_stride = P.new_seq_stride = (int64_t)4 * A.dI;
-    P.in_rows = A.ring;
-    P.bias = A.ibias;
-    P.complete_only = 1;
-    P.apply_rmsnorm = 0;
-    P.apply_rope = 0;
-    P.out_dtype = A.idx_dtype;
-    P.out = A.keys;
-    P.out_scale = A.keys_sf;
-    P.out_rows = A.key_rows;
-    i = p / A.m;
-  }
-  const int CH = chunks_for(P.c);
-  int PT = ((P.c / CH / 2 + 31) / 32) * 32;
-  if (PT < 32) PT = 32;
-  compress_entry(P, b, i, red, mrg, part, PT, kAppendThreads / PT, CH, rank);
-}
-
-cudaError_t launch_decode_append(const AppendParams& A, cudaStream_t st) {
-  static_assert(kAppendCluster == 8 && kAppendThreads >= 64, "query image: 8 CTAs of 16 head rows");
-  const int nj = (A.csa ? 3 : 2) + (A.qimg ? 1 : 0);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(A.B * nj * kAppendCluster), 1, 1);
-  cfg.blockDim = dim3(kAppendThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kAppendCluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_append_kernel, A);
 }
 
 cudaError_t launch_compress(const CompressParams& P, int B, int n_entries, cudaStream_t st) {
