@@ -75,9 +75,6 @@ struct Smem {
   float qsc[128];                             // contiguous with q: one image
   alignas(1024) uint8_t kv[KST][4][NK * 128]; // nope blocks 0..2 and the rope block, SW128
   alignas(1024) uint8_t kv3[KST][NK * 64];    // nope bytes 384..447, SW64
-  alignas(1024) uint8_t p_hi[128 * 64];       // P' high part, E4M3, K-major SW64
-  alignas(1024) uint8_t p_lo[128 * 64];       // P' low part
-  alignas(1024) uint8_t p_bf[128 * 128];      // P for the RoPE dims, bf16, K-major SW128
   float kscale[KST][NK];
   union {
     float xmax[2][KG][2][128];                // tile loop: [tile parity][key group][M_s, M_u][row]
@@ -88,17 +85,22 @@ struct Smem {
     } mg;
   };
   float xl[KG - 1][128];                      // the other groups' row sums, for the epilogue
-  uint64_t full[KST], empty[KST], sfull[2], sfree[2], xbar[2];
-  uint64_t pfull, pempty, qready, ofinal, done, lbar;
+  uint64_t full[KST], empty[KST], sfull[2], pfull[2], pdone[2], xbar[2];
+  uint64_t qready, ofinal, done, lbar;
   uint32_t tmem_base;
 };
 
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory per CTA");
 static_assert(offsetof(Smem, qsc) == QTILE, "the query image is one contiguous copy");
-// the merge stages this split's O (fp32, 128 rows of SST floats) over the key
-// stages and P buffers, which are free once the last P.V has completed
-constexpr int SST = 260;                     // row stride (floats): conflict-free float4 rows
-static_assert(offsetof(Smem, kscale) - offsetof(Smem, kv) >= 128 * SST * 4, "merge stage fits");
+// the merge stages half of this split's O (fp32, 128 rows of SSTH floats) over
+// the key stages, which are free once the last P.V has completed
+constexpr int SSTH = 132;                    // row stride (floats): conflict-free float4 rows
+static_assert(offsetof(Smem, kscale) - offsetof(Smem, kv) >= 128 * SSTH * 4, "merge stage fits");
+// TMEM columns of the coded P inside a tile's 128-column S buffer (written
+// after the buffer's S has been read): E4M3 hi / mid / lo parts at
+// PC_E4 + 16 part (64 keys, 4 a column), bf16 hi / lo parts at PC_BF + 32 part
+// (2 keys a column)
+constexpr uint32_t PC_E4 = 0, PC_BF = 48;
 
 struct Maps {
   CUtensorMap kv128, kv64;      // tile mode, boxes {128 B | 64 B} x NK rows
@@ -134,6 +136,37 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 }
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// 32 lanes x 4 / 8 consecutive columns from registers
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                   taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
+// MMAs whose A operand is read from tensor memory (M = 128 rows at lanes
+// 0..127, K along the columns: four 8-bit or two 16-bit elements a column)
+__device__ __forceinline__ void mma_f8f6f4_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 __device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t c) {
@@ -198,7 +231,9 @@ __global__ void __launch_bounds__(64) mqa_tc_qprep_kernel(MqaParams P) {
                    P.q_rmsnorm != 0, P.eps);
 }
 
-__global__ void __launch_bounds__(NTHR, 1)
+// 576 threads: at most 113 registers a thread; 112 keeps the softmax loop
+// free of spills (the default launch-bound heuristic chose 96)
+__global__ void __maxnreg__(112)
     mqa_tc_kernel(MqaParams P, const __grid_constant__ Maps maps) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>(
@@ -219,12 +254,11 @@ __global__ void __launch_bounds__(NTHR, 1)
       mbar_init(&s.empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s.sfull[i], 1);
-      mbar_init(&s.sfree[i], NSM);
+      mbar_init(&s.sfull[i], 1);     // QK of the buffer's tile done (one commit)
+      mbar_init(&s.pfull[i], NSM);   // every softmax warp wrote its P of the tile
+      mbar_init(&s.pdone[i], 1);     // PV of the buffer's tile done (one commit)
       mbar_init(&s.xbar[i], NSM);
     }
-    mbar_init(&s.pfull, NSM);
-    mbar_init(&s.pempty, 1);
     mbar_init(&s.qready, 1);
     mbar_init(&s.ofinal, 1);
     mbar_init(&s.done, 1);
@@ -347,46 +381,52 @@ __global__ void __launch_bounds__(NTHR, 1)
     const uint32_t id_pvr = idesc_f(1, 1, 128, 64, false, true);
     const uint32_t O = tmem + 256;
     bool ok = mbar_wait_warp(&s.qready, 0, P.status, 1);
+    // P.V of tile tt: A = the coded P of the tile, read from its TMEM buffer
+    // (tt & 1, written there by the softmax), B = V (= K) in shared memory
     auto pv = [&](int tt) -> bool {
-      const int st = tt % KST;
-      if (!mbar_wait_warp(&s.pfull, tt & 1, P.status, 2)) return false;
+      const int st = tt % KST, a = tt & 1;
+      if (!mbar_wait_warp(&s.pfull[a], (tt >> 1) & 1, P.status, 2)) return false;
       tc_fence_after();
       if (lane == 0) {
-        const uint64_t ahi = smem_desc(s.p_hi, kq64), alo = smem_desc(s.p_lo, kq64);
+        const uint32_t pb = tmem + a * 128;
         if (dh == 0) {
           const uint64_t bv = smem_desc(s.kv[st][0], mn128);
-          for (int ks = 0; ks < 2; ++ks) {
+          for (int ks = 0; ks < 2; ++ks) {                    // 32 keys (8 columns) a step
             const uint64_t bk = bv + (uint64_t)(ks * 32 * 128 >> 4);
-            mma_f8f6f4(O, ahi + 2 * ks, bk, id_pv256, (tt | ks) != 0);
-            mma_f8f6f4(O, alo + 2 * ks, bk, id_pv256, 1);
+            for (int pt = 0; pt < 3; ++pt)                    // E4M3 hi, mid, lo parts of P'
+              mma_f8f6f4_ts(O, pb + PC_E4 + 16 * pt + 8 * ks, bk, id_pv256, (tt | ks | pt) != 0);
           }
         } else {
           const uint64_t b2 = smem_desc(s.kv[st][2], mn128);
           const uint64_t b3 = smem_desc(s.kv3[st], mn64);
           const uint64_t br = smem_desc(s.kv[st][3], mn128);
-          const uint64_t apb = smem_desc(s.p_bf, kq128);
           for (int ks = 0; ks < 2; ++ks) {
             const uint64_t bk2 = b2 + (uint64_t)(ks * 32 * 128 >> 4);
             const uint64_t bk3 = b3 + (uint64_t)(ks * 32 * 64 >> 4);
-            mma_f8f6f4(O, ahi + 2 * ks, bk2, id_pv128, (tt | ks) != 0);
-            mma_f8f6f4(O, alo + 2 * ks, bk2, id_pv128, 1);
-            mma_f8f6f4(O + 128, ahi + 2 * ks, bk3, id_pv64, (tt | ks) != 0);
-            mma_f8f6f4(O + 128, alo + 2 * ks, bk3, id_pv64, 1);
+            for (int pt = 0; pt < 3; ++pt) {
+              const uint32_t pa = pb + PC_E4 + 16 * pt + 8 * ks;
+              mma_f8f6f4_ts(O, pa, bk2, id_pv128, (tt | ks | pt) != 0);
+              mma_f8f6f4_ts(O + 128, pa, bk3, id_pv64, (tt | ks | pt) != 0);
+            }
           }
-          for (int ks = 0; ks < 4; ++ks)
-            mma_f16(O + 192, apb + 2 * ks, br + (uint64_t)(ks * 16 * 128 >> 4), id_pvr,
-                    (tt | ks) != 0);
+          for (int ks = 0; ks < 4; ++ks)                      // 16 keys (8 columns) a step
+            for (int pt = 0; pt < 2; ++pt)                    // bf16 hi, lo parts of the weight
+              mma_f16_ts(O + 192, pb + PC_BF + 32 * pt + 8 * ks,
+                         br + (uint64_t)(ks * 16 * 128 >> 4), id_pvr, (tt | ks | pt) != 0);
         }
-        tc_commit(&s.pempty);
         tc_commit(&s.empty[st]);
+        tc_commit(&s.pdone[a]);
       }
       __syncwarp();
       return true;
     };
+    // Issue order QK(t), PV(t-1), QK(t+1), PV(t), ...: the tensor pipe runs
+    // QK(t+1) while the softmax works on tile t.  QK(t) overwrites the TMEM
+    // buffer of tile t-2, whose PV was issued earlier by this thread (tcgen05
+    // MMAs of one thread execute in issue order).
     for (int t = 0; t < g.T && ok; ++t) {
-      const int st = t % KST, a = t & 1, ua = t >> 1;
+      const int st = t % KST, a = t & 1;
       if (!mbar_wait_warp(&s.full[st], (t / KST) & 1, P.status, 3)) { ok = false; break; }
-      if (ua >= 1 && !mbar_wait_warp(&s.sfree[a], (ua - 1) & 1, P.status, 4)) { ok = false; break; }
       tc_fence_after();
       if (lane == 0) {
         const uint32_t Sn = tmem + a * 128, Sr = Sn + 64;
@@ -417,7 +457,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax, epilogue
+    // ------------------------------------------------------------ softmax
     const int quad = warp & 3;
     const int grp = (warp - 2) >> 2;          // keys grp*KPG .. +KPG-1 of each tile
     const int h = quad * 32 + lane;           // head row == TMEM lane
@@ -441,13 +481,10 @@ __global__ void __launch_bounds__(NTHR, 1)
       }
       tc_fence_after();
       uint32_t sn_[KPG], sr_[KPG];
-      const uint32_t ta = tmem + lane_off + a * 128 + grp * KPG;
-      tmem_ld16_nowait(ta, sn_);
-      tmem_ld16_nowait(ta + 64, sr_);
+      const uint32_t tb = tmem + lane_off + a * 128;     // this tile's TMEM buffer
+      tmem_ld16_nowait(tb + grp * KPG, sn_);
+      tmem_ld16_nowait(tb + 64 + grp * KPG, sr_);
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.sfree[a]);
       const float* ksc = &s.kscale[st][grp * KPG];
       float s2[KPG];
       float ms = -INFINITY;
@@ -460,7 +497,9 @@ __global__ void __launch_bounds__(NTHR, 1)
         ms = fmaxf(ms, s2[j]);
         kbits = max(kbits, __float_as_uint(kj));
       }
-      // tile maxima (row score, scale exponent): exchange with the other key groups
+      // tile maxima (row score, scale exponent): exchange with the other key
+      // groups; past this exchange every group has read its S columns, so the
+      // coded P may overwrite the buffer
       s.xmax[xb][grp][0][h] = ms;
       s.xmax[xb][grp][1][h] = __uint_as_float(kbits);
       __syncwarp();
@@ -483,51 +522,57 @@ __global__ void __launch_bounds__(NTHR, 1)
           (K_new == -1000) ? 0.f : exp2i(min(126, max(-126, 8 - (int)kTau - K_new)));
       const float ak = (cu > 0.f && cu_new != cu) ? cu_new / cu : 1.f;   // exact: powers of two
       const float ms_ref = (Ms_new == -INFINITY) ? 0.f : Ms_new;
-      // The weight each key really gets is its coded value: (hi + lo) / (k_scale cu)
-      // on the FP8 dims (exact in fp32: hi and lo carry 4 significant bits each,
-      // k_scale cu is a power of two) and that weight rounded to bf16 on the RoPE
-      // dims.  The row sum is taken over the coded weights, so that O / l is a
-      // convex combination with exactly the weights the MMAs used.
+      // P' = P k_scale cu coded as three E4M3 parts (hi + mid + lo: 12
+      // significant bits) for the FP8 dims; the weight each key then really
+      // gets, w = (hi + mid + lo) / (k_scale cu) (exact in fp32), coded as two
+      // bf16 parts for the RoPE dims; the row sum is taken over the w.
       float lsum = 0.f;
-      uint32_t phi[KPG / 4], plo[KPG / 4], pbf[KPG / 2];
+      uint32_t phi[KPG / 4], pmd[KPG / 4], plo[KPG / 4], pbh[KPG / 2], pbl[KPG / 2];
 #pragma unroll
       for (int j = 0; j < KPG; j += 2) {
         const float p0 = ex2f(s2[j] - ms_ref), p1 = ex2f(s2[j + 1] - ms_ref);   // 0 for -inf
         const float kc0 = ksc[j] * cu_new, kc1 = ksc[j + 1] * cu_new;          // powers of two (or 0)
-        const float u0 = p0 * kc0, u1 = p1 * kc1;                               // P' = P k_scale cu
+        const float u0 = p0 * kc0, u1 = p1 * kc1;
         const uint32_t hi = e4m3x2(u0, u1);
         const float2 hf = e4m3x2_to_f32(hi);
-        const uint32_t lo = e4m3x2(u0 - hf.x, u1 - hf.y);
+        const float r0 = u0 - hf.x, r1 = u1 - hf.y;
+        const uint32_t md = e4m3x2(r0, r1);
+        const float2 mf = e4m3x2_to_f32(md);
+        const uint32_t lo = e4m3x2(r0 - mf.x, r1 - mf.y);
         const float2 lf = e4m3x2_to_f32(lo);
-        // 1 / (k_scale cu) by exponent arithmetic (exact for a normal power of two)
-        const float w0 = kc0 != 0.f ? (hf.x + lf.x) * __int_as_float((254 << 23) - __float_as_int(kc0)) : 0.f;
-        const float w1 = kc1 != 0.f ? (hf.y + lf.y) * __int_as_float((254 << 23) - __float_as_int(kc1)) : 0.f;
+        const float w0 = kc0 != 0.f ? ((hf.x + mf.x) + lf.x) * __int_as_float((254 << 23) - __float_as_int(kc0)) : 0.f;
+        const float w1 = kc1 != 0.f ? ((hf.y + mf.y) + lf.y) * __int_as_float((254 << 23) - __float_as_int(kc1)) : 0.f;
         lsum += w0 + w1;
         if ((j & 3) == 0) {
           phi[j >> 2] = hi;
+          pmd[j >> 2] = md;
           plo[j >> 2] = lo;
         } else {
           phi[j >> 2] |= hi << 16;
+          pmd[j >> 2] |= md << 16;
           plo[j >> 2] |= lo << 16;
         }
-        const __nv_bfloat162 pb = __floats2bfloat162_rn(w0, w1);
-        pbf[j >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
+        const __nv_bfloat162 bh = __floats2bfloat162_rn(w0, w1);
+        const float2 bhf = __bfloat1622float2(bh);
+        const __nv_bfloat162 bl = __floats2bfloat162_rn(w0 - bhf.x, w1 - bhf.y);
+        pbh[j >> 1] = *reinterpret_cast<const uint32_t*>(&bh);
+        pbl[j >> 1] = *reinterpret_cast<const uint32_t*>(&bl);
       }
       l = l * as + lsum;
-      // PV of the previous tile must be done before O or P change
-      if (t >= 1 && !mbar_wait_warp(&s.pempty, (t - 1) & 1, P.status, 8)) {
-        live = false;
-        break;
-      }
-      tc_fence_after();
-      // Rescale this warp's share of O (columns grp*64 .. +63): the FP8 part
-      // by as*ak, the RoPE part by as.  tcgen05.ld / st are warp-wide
+      // Rescale this warp's share of O (columns grp*64 .. +63) when the row's
+      // reference moved: the FP8 part by as*ak, the RoPE part by as, after the
+      // previous tile's P.V has completed.  tcgen05.ld / st are warp-wide
       // (.sync.aligned): the decision is taken per warp, every lane takes part
       // with its own factor.
       const float an = as * ak;
       const bool grow_n = __any_sync(0xffffffffu, wrote && an < 1.f);
       const bool grow_r = __any_sync(0xffffffffu, wrote && dh == 1 && as < 1.f);
       if (grow_n || grow_r) {
+        if (t >= 1 && !mbar_wait_warp(&s.pdone[(t - 1) & 1], ((t - 1) >> 1) & 1, P.status, 8)) {
+          live = false;
+          break;
+        }
+        tc_fence_after();
         const uint32_t ob = tmem + lane_off + 256;
         for (int cc = 0; cc < 256 / KG; cc += 32) {
           const int c = grp * (256 / KG) + cc;
@@ -546,22 +591,23 @@ __global__ void __launch_bounds__(NTHR, 1)
       Ms = Ms_new;
       K = K_new;
       cu = cu_new;
-      *reinterpret_cast<uint4*>(s.p_hi + sw64(h, grp * KPG)) = make_uint4(phi[0], phi[1], phi[2], phi[3]);
-      *reinterpret_cast<uint4*>(s.p_lo + sw64(h, grp * KPG)) = make_uint4(plo[0], plo[1], plo[2], plo[3]);
+      // the coded P of this group's 16 keys into the tile's TMEM buffer:
+      // E4M3 parts at columns PC_E4 + 16 * part + 4 * grp (4 keys a column),
+      // bf16 parts at PC_BF + 32 * part + 8 * grp (2 keys a column)
+      tmem_st4(tb + PC_E4 + 4 * grp, phi);
+      tmem_st4(tb + PC_E4 + 16 + 4 * grp, pmd);
+      tmem_st4(tb + PC_E4 + 32 + 4 * grp, plo);
       if (dh == 1) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          *reinterpret_cast<uint4*>(s.p_bf + sw128(h, grp * 2 * KPG + 16 * c)) =
-              make_uint4(pbf[4 * c], pbf[4 * c + 1], pbf[4 * c + 2], pbf[4 * c + 3]);
+        tmem_st8(tb + PC_BF + 8 * grp, pbh);
+        tmem_st8(tb + PC_BF + 32 + 8 * grp, pbl);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.pfull);
+      if (lane == 0) mbar_arrive(&s.pfull[a]);
       wrote = true;
     }
     if (!live) flag(P.status, ST_TIMEOUT);
-    // ------------------------------------------------------------ epilogue
     bool fin = mbar_wait_warp(&s.ofinal, 0, P.status, 9);
     tc_fence_after();
     // row sums of all key groups
@@ -622,72 +668,98 @@ __global__ void __launch_bounds__(NTHR, 1)
     s.mg.rsn[tid - 128] = sv;
   }
   __syncthreads();
-  // stage this split's O, scaled to the merged units, as fp32 rows in shared memory
-  float* stage = reinterpret_cast<float*>(&s.kv[0][0][0]);
-  if (warp >= 2) {
-    const int quad = warp & 3, grp = (warp - 2) >> 2;
-    const int hh = quad * 32 + lane;
-    const uint32_t ob = tmem + ((uint32_t)(quad * 32) << 16) + 256;
-    const float fs = s.mg.fself[hh], fnn = fs * s.mg.rfn[hh];
-#pragma unroll 1
-    for (int cc = 0; cc < 256 / KG; cc += 32) {
-      const int c = grp * (256 / KG) + cc;
-      uint32_t r[32];
-      tmem_ld32_nowait(ob + c, r);
-      tmem_ld_wait();
-      const float f = (dh == 1 && c >= 192) ? fs : fnn;   // RoPE dims carry no cu
-      float4* dst = reinterpret_cast<float4*>(stage + hh * SST + c);
+  const int64_t obase = (int64_t)q * P.H * 512 + dh * 256;
+  // the final value of output column `col` (this half) of row hh from its
+  // merged (summed, scaled) value: / denominator, R(-p) on RoPE pairs, stored
+  auto emit4 = [&](int hh, int col, float4 a) {
+    const float il = s.mg.invl[hh];
+    float o[4] = {a.x * il, a.y * il, a.z * il, a.w * il};
+    if (dh == 1 && col >= 192) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        dst[k] = make_float4(__uint_as_float(r[4 * k]) * f, __uint_as_float(r[4 * k + 1]) * f,
-                             __uint_as_float(r[4 * k + 2]) * f, __uint_as_float(r[4 * k + 3]) * f);
+      for (int e = 0; e < 4; e += 2) {
+        const int k = (col + e - 192) >> 1;
+        const float cs = s.mg.rcs[k], sn = s.mg.rsn[k];
+        const float r0 = o[e] * cs + o[e + 1] * sn, r1 = -o[e] * sn + o[e + 1] * cs;
+        o[e] = r0;
+        o[e + 1] = r1;
+      }
+    }
+    const int64_t off = obase + (int64_t)hh * 512 + col;
+    if (P.out_dtype == V4A_F32) {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) + off) = make_float4(o[0], o[1], o[2], o[3]);
+    } else {
+      const uint32_t w0 = (uint32_t)f32_to_bf16_bits(o[0]) | ((uint32_t)f32_to_bf16_bits(o[1]) << 16);
+      const uint32_t w1 = (uint32_t)f32_to_bf16_bits(o[2]) | ((uint32_t)f32_to_bf16_bits(o[3]) << 16);
+      *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(P.out) + off) = make_uint2(w0, w1);
+    }
+  };
+  if (C == 1) {
+    // one split: the output straight from TMEM (each thread 32 columns of its row)
+    if (warp >= 2) {
+      const int quad = warp & 3, grp = (warp - 2) >> 2;
+      const int hh = quad * 32 + lane;
+      const uint32_t ob = tmem + ((uint32_t)(quad * 32) << 16) + 256;
+      const float fs = s.mg.fself[hh], fnn = fs * s.mg.rfn[hh];
+#pragma unroll 1
+      for (int cc = 0; cc < 256 / KG; cc += 32) {
+        const int c = grp * (256 / KG) + cc;
+        uint32_t r[32];
+        tmem_ld32_nowait(ob + c, r);
+        tmem_ld_wait();
+        const float f = (dh == 1 && c >= 192) ? fs : fnn;   // RoPE dims carry no cu
+        if (hh < P.H)
+#pragma unroll
+          for (int k = 0; k < 32; k += 4)
+            emit4(hh, c + k, make_float4(__uint_as_float(r[k]) * f, __uint_as_float(r[k + 1]) * f,
+                                         __uint_as_float(r[k + 2]) * f, __uint_as_float(r[k + 3]) * f));
+      }
+    }
+  } else {
+    // the splits' O, scaled to the merged units, staged as fp32 rows in shared
+    // memory (over the key stages, free now), one half of the columns at a
+    // time; CTA `split` then writes columns [128 split / C, 128 (split+1) / C)
+    // of each half: the sum over the splits read through distributed shared memory
+    float* stage = reinterpret_cast<float*>(&s.kv[0][0][0]);
+    for (int half = 0; half < 2; ++half) {
+      if (warp >= 2) {
+        const int quad = warp & 3, grp = (warp - 2) >> 2;
+        const int hh = quad * 32 + lane;
+        const uint32_t ob = tmem + ((uint32_t)(quad * 32) << 16) + 256;
+        const float fs = s.mg.fself[hh], fnn = fs * s.mg.rfn[hh];
+        const int c = half * 128 + grp * 32;
+        uint32_t r[32];
+        tmem_ld32_nowait(ob + c, r);
+        tmem_ld_wait();
+        const float f = (dh == 1 && c >= 192) ? fs : fnn;
+        float4* dst = reinterpret_cast<float4*>(stage + hh * SSTH + grp * 32);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          dst[k] = make_float4(__uint_as_float(r[4 * k]) * f, __uint_as_float(r[4 * k + 1]) * f,
+                               __uint_as_float(r[4 * k + 2]) * f, __uint_as_float(r[4 * k + 3]) * f);
+      }
+      __syncthreads();
+      cl.sync();                                  // every split's half staged
+      const int c0 = 128 * split / C, c1 = 128 * (split + 1) / C;
+      const int ng = (c1 - c0) / 4;
+      for (int it = tid; it < 128 * ng; it += NTHR) {
+        const int hh = it / ng, col = c0 + 4 * (it % ng);
+        if (hh >= P.H) continue;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < C; ++r) {
+          const float4 b = *reinterpret_cast<const float4*>(
+              cl.map_shared_rank(stage, (unsigned)r) + hh * SSTH + col);
+          a.x += b.x;
+          a.y += b.y;
+          a.z += b.z;
+          a.w += b.w;
+        }
+        emit4(hh, half * 128 + col, a);
+      }
+      cl.sync();                                  // the stage is read before it is reused
     }
   }
   tc_fence_before();
   __syncthreads();
-  cl.sync();                                    // every split's O staged
-  {
-    // this CTA writes output columns [c0, c1) of its half: the sum over the
-    // splits (distributed shared memory), / denominator, R(-p) on RoPE dims
-    const int c0 = 256 * split / C, c1 = 256 * (split + 1) / C;
-    const int ng = (c1 - c0) / 4;
-    const int64_t obase = (int64_t)q * P.H * 512 + dh * 256;
-    for (int it = tid; it < 128 * ng; it += NTHR) {
-      const int hh = it / ng, col = c0 + 4 * (it % ng);
-      if (hh >= P.H) continue;
-      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int r = 0; r < C; ++r) {
-        const float4 b = *reinterpret_cast<const float4*>(
-            cl.map_shared_rank(stage, (unsigned)r) + hh * SST + col);
-        a.x += b.x;
-        a.y += b.y;
-        a.z += b.z;
-        a.w += b.w;
-      }
-      const float il = s.mg.invl[hh];
-      float o[4] = {a.x * il, a.y * il, a.z * il, a.w * il};
-      if (dh == 1 && col >= 192) {
-#pragma unroll
-        for (int e = 0; e < 4; e += 2) {
-          const int k = (col + e - 192) >> 1;
-          const float cs = s.mg.rcs[k], sn = s.mg.rsn[k];
-          const float r0 = o[e] * cs + o[e + 1] * sn, r1 = -o[e] * sn + o[e + 1] * cs;
-          o[e] = r0;
-          o[e + 1] = r1;
-        }
-      }
-      const int64_t off = obase + (int64_t)hh * 512 + col;
-      if (P.out_dtype == V4A_F32) {
-        *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) + off) =
-            make_float4(o[0], o[1], o[2], o[3]);
-      } else {
-        const uint32_t w0 = (uint32_t)f32_to_bf16_bits(o[0]) | ((uint32_t)f32_to_bf16_bits(o[1]) << 16);
-        const uint32_t w1 = (uint32_t)f32_to_bf16_bits(o[2]) | ((uint32_t)f32_to_bf16_bits(o[3]) << 16);
-        *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(P.out) + off) = make_uint2(w0, w1);
-      }
-    }
-  }
-  cl.sync();                                    // no CTA leaves while its stage is read
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
