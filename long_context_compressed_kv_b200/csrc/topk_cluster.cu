@@ -5,8 +5,9 @@
 // query; Flash k = 512, Pro k = 1024).  Ties go to the lower index and the
 // selection is written in ascending index order, -1 padded.
 //
-// The 16 (or, where a 16-CTA cluster cannot be resident, 8) CTAs of a
-// cluster split the query's visible scores into slices and
+// The CTAs of a cluster (16 for a few queries, fewer for many: the largest
+// power of two whose clusters for all the call's queries fit on the GPU at
+// once, down to one CTA a query) split the query's visible scores into slices and
 // keep their slice in shared memory (as order-preserving uint32 keys).  A
 // cluster-wide min / max first finds the key bits that every visible score
 // shares; an exact radix select then resolves the remaining bits 8 at a time.
@@ -33,7 +34,6 @@
 namespace v4a {
 
 namespace {
-constexpr int CL_MAX = 16;        // CTAs per cluster = slices per query (8 or 16, set at launch)
 constexpr int TPB = 512;          // threads per CTA
 constexpr int CACHE = 32768;      // keys a CTA keeps in shared memory (+1/64 padding)
 constexpr int PAD_CACHE = CACHE + CACHE / 64;
@@ -358,36 +358,46 @@ bool topk_cluster_supported(const TopkParams& P) { return P.n_q <= (1 << 20); }
 
 cudaError_t launch_topk_cluster(const TopkParams& P, cudaStream_t st) {
   const size_t smem = SMEM_WORDS * sizeof(uint32_t);
-  static int cluster_size[64] = {0};                 // per device: 16 if it can be resident, else 8
+  // per device: how many clusters of 1, 2, 4, 8, 16 CTAs can be resident at once
+  static int max_active[64][5];
+  static bool configured[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 64) return cudaErrorInvalidDevice;
-  if (!cluster_size[dev]) {
+  if (!configured[dev]) {
     cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    int cs = 8;
     if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed,
-                             1) == cudaSuccess) {
+                             1) != cudaSuccess)
+      cudaGetLastError();                            // 16-CTA clusters then report 0 below
+    for (int k = 0; k < 5; ++k) {
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(CL_MAX, 1, 1);
+      cfg.gridDim = dim3(1u << k, 1, 1);
       cfg.blockDim = dim3(TPB, 1, 1);
       cfg.dynamicSmemBytes = smem;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = CL_MAX;
+      attr[0].val.clusterDim.x = 1u << k;
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel, &cfg) == cudaSuccess && n >= 1)
-        cs = CL_MAX;
+      if (cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+      max_active[dev][k] = n;
     }
-    cudaGetLastError();                              // a refused query leaves the portable size
-    cluster_size[dev] = cs;
+    configured[dev] = true;
   }
-  const int CL = cluster_size[dev];
+  // CTAs per query: the largest power of two <= 16 whose clusters for all the
+  // queries are resident at once (few queries: wide clusters over long score
+  // rows; many queries, as in prefill: one CTA each)
+  int k = 4;
+  while (k > 0 && max_active[dev][k] < P.n_q) --k;
+  const int CL = 1 << k;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(P.n_q * CL), 1, 1);
   cfg.blockDim = dim3(TPB, 1, 1);
