@@ -347,6 +347,10 @@ v4attn_status v4attn_device_status(const void* ws, cudaStream_t stream, uint32_t
 
 const char* v4attn_status_string(v4attn_status s);
 
+/* The description of the last CUDA error behind a V4A_ERR_CUDA return on the
+ * calling host thread ("no error" when there was none). */
+const char* v4attn_last_cuda_error(void);
+
 /* Library build identification (kernel variants compiled in). */
 const char* v4attn_build_info(void);
 

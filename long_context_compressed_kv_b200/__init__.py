@@ -31,6 +31,8 @@ __all__ = ["F32", "BF16", "E4M3_BF16ROPE", "MXFP4", "CSA", "HCA", "V4AttnError",
 class V4AttnError(RuntimeError):
     def __init__(self, fn: str, status: int):
         msg = _lib.v4attn_status_string(status).decode()
+        if status == _abi.ERR_CUDA:
+            msg += ": " + _lib.v4attn_last_cuda_error().decode()
         super().__init__(f"{fn}: {msg} (status {status})")
         self.status = status
 

@@ -98,6 +98,7 @@ SIGNATURES = {
     "v4attn_device_status": (ctypes.c_int, [c_ptr, c_ptr, ctypes.POINTER(ctypes.c_uint32)]),
     "v4attn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "v4attn_build_info": (ctypes.c_char_p, []),
+    "v4attn_last_cuda_error": (ctypes.c_char_p, []),
 }
 
 _lib = None

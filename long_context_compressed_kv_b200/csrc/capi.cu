@@ -94,7 +94,13 @@ float softmax_scale(const v4attn_layer_desc* d) {
   return d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)d->d);
 }
 
-v4attn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? V4A_OK : V4A_ERR_CUDA; }
+// the last CUDA error an entry point met on this host thread (v4attn_last_cuda_error)
+thread_local cudaError_t t_last_cuda = cudaSuccess;
+v4attn_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return V4A_OK;
+  t_last_cuda = e;
+  return V4A_ERR_CUDA;
+}
 
 v4attn_status run_compress(const v4attn_layer_desc* d, const v4attn_compress_args* a,
                            cudaStream_t st) {
@@ -225,7 +231,7 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
       P.status = status;
       P.wait_ns = wait_ns;
       P.stall = stall;
-      if (index_scores_dispatch(P, st) != cudaSuccess) return V4A_ERR_CUDA;
+      if (const cudaError_t e = index_scores_dispatch(P, st)) return cuda_status(e);
     }
     if (!a->idx_out) continue;   // scores-only call
     TopkParams T;
@@ -237,7 +243,7 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
     T.max_vis = a->max_vis;
     T.q_pos = a->q_pos + q0;
     T.idx_out = a->idx_out + (int64_t)q0 * d->top_k;
-    if (topk_dispatch(T, st) != cudaSuccess) return V4A_ERR_CUDA;
+    if (const cudaError_t e = topk_dispatch(T, st)) return cuda_status(e);
   }
   return V4A_OK;
 }
@@ -310,9 +316,9 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
       if (s != V4A_OK) return s;
     }
     if (dry) return V4A_OK;
-    if (mqa_dispatch(P, st) != cudaSuccess) return V4A_ERR_CUDA;
-    if (d->kv_dtype != V4A_E4M3_BF16ROPE && launch_mqa_combine(P, st) != cudaSuccess)
-      return V4A_ERR_CUDA;
+    if (const cudaError_t e = mqa_dispatch(P, st)) return cuda_status(e);
+    if (d->kv_dtype != V4A_E4M3_BF16ROPE)
+      if (const cudaError_t e = launch_mqa_combine(P, st)) return cuda_status(e);
   }
   return V4A_OK;
 }
@@ -478,7 +484,7 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
   q.lse = a->lse;
   s = run_mqa(desc, &q, ws, ws_bytes, stream, csa, fuse_q, true);
   if (s != V4A_OK) return s;
-  if (launch_decode_append(A, stream) != cudaSuccess) return V4A_ERR_CUDA;
+  if (const cudaError_t e = launch_decode_append(A, stream)) return cuda_status(e);
   if (csa) {
     s = run_index_topk(desc, &ix, ws, ws_bytes, stream, body_mqa(desc, a->B));
     if (s != V4A_OK) return s;
@@ -541,6 +547,8 @@ const char* v4attn_status_string(v4attn_status s) {
 }
 
 const char* v4attn_build_info(void) { return build_info_string(); }
+
+const char* v4attn_last_cuda_error(void) { return cudaGetErrorString(t_last_cuda); }
 
 v4attn_status v4attn_debug_index_stall(const v4attn_layer_desc* desc,
                                        const v4attn_index_args* args, void* ws, size_t ws_bytes,

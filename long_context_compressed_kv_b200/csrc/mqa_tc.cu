@@ -231,9 +231,9 @@ __global__ void __launch_bounds__(64) mqa_tc_qprep_kernel(MqaParams P) {
                    P.q_rmsnorm != 0, P.eps);
 }
 
-// 576 threads: at most 113 registers a thread; 112 keeps the softmax loop
-// free of spills (the default launch-bound heuristic chose 96)
-__global__ void __maxnreg__(112)
+// 576 threads = 18 warps: on the SM sub-partition that holds five of them at
+// most 16384 / 5 registers a warp, hence 96 registers a thread
+__global__ void __launch_bounds__(NTHR, 1)
     mqa_tc_kernel(MqaParams P, const __grid_constant__ Maps maps) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>(
