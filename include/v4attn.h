@@ -172,7 +172,11 @@ typedef struct {
  * Formats: V4A_F32 caches run on CUDA cores; V4A_E4M3_BF16ROPE caches run on
  * the tcgen05 tensor-core kernel only and need a bf16 Q (else
  * V4A_ERR_UNSUPPORTED), 16-byte aligned Q, kv, swa and out (else
- * V4A_ERR_INVALID_ARG), and B * kv_rows, B * swa_rows < 2^31.  */
+ * V4A_ERR_INVALID_ARG), and B * kv_rows, B * swa_rows < 2^31.  That kernel
+ * takes P V in f16: stored values (entry scale x code, RoPE dims) must lie
+ * below 65504 in magnitude (values below 2^-14 lose bits; an RMSNorm'ed row
+ * is at most sqrt(d) = 22.6), and the softmax weights carry 11 significant
+ * bits.  */
 typedef struct {
   int32_t n_q;                /* queries, 1 .. 2^20 */
   int32_t B;
@@ -208,8 +212,9 @@ typedef struct {
  *   3. CSA: indexer + top-k over the visible keys;
  *   4. MQA over the selected (CSA) or all visible (HCA) entries + window.
  * x_main, tail, x_idx, itail must be aligned to 4 elements and bias, ibias
- * to 16 bytes (else V4A_ERR_INVALID_ARG); the pooling window (ring rows)
- * times d must not exceed 65536 (V4A_ERR_UNSUPPORTED).  */
+ * to 16 bytes (else V4A_ERR_INVALID_ARG); d must be 64, 128, 256 or 512 and
+ * the pooling window (ring rows) times d must not exceed 65536 (else
+ * V4A_ERR_UNSUPPORTED).  */
 typedef struct {
   int32_t B;
   const int64_t* pos;         /* device [B] position p of each sequence's new token */
@@ -253,11 +258,16 @@ typedef struct {
  * 2^20 queries per call), so the body of the workspace holds the scores or
  * split-K partials of one chunk; for a V4A_E4M3_BF16ROPE layer it also holds
  * the coded queries of one chunk (74,752 bytes a query) that the tensor-core
- * MQA reads.  The size grows with n_q only by 24 bytes per query beyond 1024.
+ * MQA reads, and, when n_q <= 40, room for that MQA's split-K partials
+ * (160 CTAs x 129 KiB: a call of few queries spreads each (query, half of the
+ * output dims) over up to 64 resident CTAs that meet at one grid barrier).
+ * The size grows with n_q only by 24 bytes per query beyond 1024.
  * Its layout is internal to the library; one workspace serves one stream. */
 size_t v4attn_workspace_size(const v4attn_layer_desc* desc, int32_t n_q, int64_t max_vis);
 
-/* Zero the workspace's status word (stream-ordered). */
+/* Zero the workspace's header: the status word and the tensor-core MQA's grid
+ * barrier state (stream-ordered).  Call it once before the first call and
+ * again after a call has reported V4A_ERR_TIMEOUT. */
 v4attn_status v4attn_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream);
 
 v4attn_status v4attn_compress(const v4attn_layer_desc* desc, const v4attn_compress_args* args,

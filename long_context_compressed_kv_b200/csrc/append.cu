@@ -18,14 +18,16 @@
 //   K  (CSA) when the token completes a block: its indexer key (same pooling,
 //      no RMSNorm / RoPE, MXFP4), 32 channels per CTA;
 //   Q  (optional) the tensor-core MQA's query image, 16 head rows per CTA.
-// The pooling loads every window row a thread needs before it computes, so a
-// job waits for memory once; the row slices of each channel are merged in
-// shared memory.  Only E synchronises its cluster (twice).
+// The pooling issues the loads of every window row a thread needs (the biases
+// by asynchronous copies) before it computes, so a job waits for memory once,
+// and computes its RoPE angles while they are in flight; the row slices of
+// each channel are merged by shuffles.  Only E synchronises its cluster (once).
 #include <cooperative_groups.h>
 
 #include "common.cuh"
 #include "kernels.h"
 #include "mqa_qimage.cuh"
+#include "tc_common.cuh"
 
 namespace v4a {
 
@@ -67,100 +69,139 @@ struct PoolArgs {
   const void* xnew;       // the new token's row: [n_arr][d_row]
   int dtype, ring, n_arr, d_row;
   int ia, iz, ib, izb;    // array index of C^a, Z^a, C^b, Z^b in a row
-  int m, R;               // stride, window rows (2m overlapped, m otherwise)
+  int m, R;               // stride, window rows (2m overlapped, m otherwise; R <= ring)
   bool overlap;
   const float* bias;      // [R][d_row]
   int64_t p, i;           // the new token's position, the entry index
 };
 
+// RoPE angles a job needs (pair k of a vector at position pos), or none
+struct RopeReq {
+  bool on;
+  int64_t pos;
+  int k, d_rope;
+  float theta;
+};
+
 // Softmax-gated pooling of channels [c_lo, c_lo + CW) of entry i (CW a
-// multiple of 4, CW / 4 threads per row): e[c - c_lo] in shared memory.
-__device__ void pool_channels(const PoolArgs& a, int c_lo, int CW, float* e, float* part) {
+// multiple of 4, CW / 4 threads per row): e[c - c_lo] in shared memory.  Each
+// thread issues the loads of all its rows (the biases by asynchronous copies
+// into its own slots of `bsm`) before any arithmetic, computes the RoPE angle
+// `rq` asks for while they are in flight (into rc / rs), then pools; the
+// slices of each channel are merged by kThr / CW adjacent threads, four
+// slices each.
+__device__ void pool_channels(const PoolArgs& a, int c_lo, int CW, float* e, float* part,
+                              float4* bsm, const RopeReq& rq, float& rc, float& rs) {
   const int PT = CW / 4, NS = kThr / PT;
   const int t = threadIdx.x, cg = t % PT, sl = t / PT;
   const int c0 = c_lo + 4 * cg;
   const int64_t j0 = a.overlap ? (int64_t)a.m * (a.i - 1) : (int64_t)a.m * a.i;
   const int64_t row_el = (int64_t)a.n_arr * a.d_row;
-  // every row of this thread's slice first (one wait for memory), then the math
-  float4 cv[kMaxRps], zv[kMaxRps];
+  // ring slot of window row 0; row r sits r slots later (R <= ring: one wrap at most)
+  const int s0 = (int)(((j0 % a.ring) + a.ring) % a.ring);
   bool ok[kMaxRps];
 #pragma unroll
   for (int k = 0; k < kMaxRps; ++k) {
     const int r = sl + k * NS;
     const int64_t j = j0 + r;
     ok[k] = r < a.R && j >= 0 && j <= a.p;
+    if (a.bias)
+      cp_async16(&bsm[k * kThr + t], a.bias + (ok[k] ? (int64_t)r * a.d_row + c0 : 0), ok[k]);
+  }
+  cp_async_commit();
+  float4 cv[kMaxRps], zv[kMaxRps];
+#pragma unroll
+  for (int k = 0; k < kMaxRps; ++k) {
     cv[k] = zv[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (ok[k]) {
+      const int r = sl + k * NS;
       const bool br_a = !a.overlap || r >= a.m;
       const int ic = br_a ? a.ia : a.ib, iz = br_a ? a.iz : a.izb;
-      const void* src = j == a.p ? a.xnew : a.tail;
-      const int64_t rb = j == a.p ? 0 : (j % a.ring) * row_el;
+      const bool is_new = j0 + r == a.p;
+      int slot = s0 + r;
+      slot -= slot >= a.ring ? a.ring : 0;
+      const void* src = is_new ? a.xnew : a.tail;
+      const int64_t rb = is_new ? 0 : (int64_t)slot * row_el;
       cv[k] = ld4(src, a.dtype, rb + (int64_t)ic * a.d_row + c0);
       zv[k] = ld4(src, a.dtype, rb + (int64_t)iz * a.d_row + c0);
-      if (a.bias) {
-        const float4 bb = *reinterpret_cast<const float4*>(a.bias + (int64_t)r * a.d_row + c0);
-        zv[k].x += bb.x;
-        zv[k].y += bb.y;
-        zv[k].z += bb.z;
-        zv[k].w += bb.w;
-      }
+    }
+  }
+  rc = 1.f;
+  rs = 0.f;
+  if (rq.on) rope_cs(rq.pos, rq.k, rq.d_rope, rq.theta, rc, rs);
+  cp_async_wait<0>();                                // this thread's own bias copies
+  if (a.bias) {
+#pragma unroll
+    for (int k = 0; k < kMaxRps; ++k) {
+      const float4 bb = bsm[k * kThr + t];
+      zv[k].x += bb.x;
+      zv[k].y += bb.y;
+      zv[k].z += bb.z;
+      zv[k].w += bb.w;
     }
   }
   // this slice's (max, sum, weighted sum) of each of its 4 channels
-  float mx[4], sm[4], ac[4];
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     float m = -INFINITY;
 #pragma unroll
     for (int k = 0; k < kMaxRps; ++k)
       if (ok[k]) m = fmaxf(m, f4(zv[k], c));
-    float s = 0.f, acc = 0.f;
+    float sm = 0.f, acc = 0.f;
     if (m != -INFINITY) {
 #pragma unroll
       for (int k = 0; k < kMaxRps; ++k)
         if (ok[k]) {
           const float w = __expf(f4(zv[k], c) - m);
-          s += w;
+          sm += w;
           acc = fmaf(w, f4(cv[k], c), acc);
         }
     }
-    mx[c] = m;
-    sm[c] = s;
-    ac[c] = acc;
-  }
-  // merge the slices: part[slice][channel][3]
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    float* q = part + ((int64_t)sl * CW + 4 * cg + c) * 3;
-    q[0] = mx[c];
-    q[1] = sm[c];
-    q[2] = ac[c];
+    float* q = part + ((int64_t)sl * CW + 4 * cg + c) * 3;   // part[slice][channel][3]
+    q[0] = m;
+    q[1] = sm;
+    q[2] = acc;
   }
   __syncthreads();
-  if (t < CW) {
-    float M = -INFINITY;
-    for (int s2 = 0; s2 < NS; ++s2) M = fmaxf(M, part[((int64_t)s2 * CW + t) * 3]);
-    float S = 0.f, A = 0.f;
-    if (M != -INFINITY)
-      for (int s2 = 0; s2 < NS; ++s2) {
-        const float* q = part + ((int64_t)s2 * CW + t) * 3;
-        if (q[0] != -INFINITY) {
-          const float f = __expf(q[0] - M);
-          S = fmaf(f, q[1], S);
-          A = fmaf(f, q[2], A);
-        }
-      }
-    e[t] = S > 0.f ? A / S : 0.f;
+  // merge: channel t / TPC, slices 4 (t % TPC) .. + 3, then across the TPC lanes
+  const int TPC = kThr / CW, ch = t / TPC, sub = t % TPC;
+  float ms[4], ss[4], as[4];
+  float M = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float* q = part + ((int64_t)(4 * sub + u) * CW + ch) * 3;
+    ms[u] = q[0];
+    ss[u] = q[1];
+    as[u] = q[2];
+    M = fmaxf(M, ms[u]);
   }
+  for (int o = 1; o < TPC; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float S = 0.f, A = 0.f;
+  if (M != -INFINITY) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (ms[u] != -INFINITY) {
+        const float f = __expf(ms[u] - M);
+        S = fmaf(f, ss[u], S);
+        A = fmaf(f, as[u], A);
+      }
+  }
+  for (int o = 1; o < TPC; o <<= 1) {
+    S += __shfl_xor_sync(0xffffffffu, S, o);
+    A += __shfl_xor_sync(0xffffffffu, A, o);
+  }
+  if (sub == 0) e[ch] = S > 0.f ? A / S : 0.f;
   __syncthreads();
 }
 
-// RMSNorm (over all d channels of the vector, CH CTAs of CW each), RoPE at
-// `rope_pos` on the last d_rope channels, and the stored format of channels
-// [c_lo, c_lo + CW) of one row: E4M3 + bf16 (scale written by rank 0) or fp32.
-// All threads call; with CH > 1 the CTAs of the cluster call it together.
+// RMSNorm (over all d channels of the vector, CH CTAs of CW each), RoPE on the
+// last d_rope channels with this thread's pair angle (rc, rs), and the stored
+// format of channels [c_lo, c_lo + CW) of one row: E4M3 + bf16 (scale written
+// by the CTA holding channel 0) or fp32.  All threads call; with CH > 1 the
+// CTAs of the cluster call it together and meet at one cluster barrier (each
+// pushes its partial sum / amax into every CTA's xch[2 rank ..]).
 __device__ void finish_main(const float* e, int c_lo, int CW, int d, int d_rope, bool norm,
-                            bool rope, int64_t rope_pos, float theta, float eps, int out_dtype,
+                            bool rope, float rc, float rs, float eps, int out_dtype,
                             uint8_t* out_row, float* out_scale, int CH, float* red, float* xch) {
   namespace cg = cooperative_groups;
   const int t = threadIdx.x;
@@ -169,35 +210,23 @@ __device__ void finish_main(const float* e, int c_lo, int CW, int d, int d_rope,
   float e0 = act ? e[2 * t] : 0.f, e1 = act ? e[2 * t + 1] : 0.f;
   const int dn = d - d_rope;
   const bool e4 = out_dtype == V4A_E4M3_BF16ROPE;
-  // the rotation angle of this pair, computed while the reductions run
-  float rc = 1.f, rs = 0.f;
-  if (act && rope && c >= dn) rope_cs(rope_pos, (c - dn) / 2, d_rope, theta, rc, rs);
   float2 sa = cta_sum_max(e0 * e0 + e1 * e1,
                           (act && c < dn) ? fmaxf(fabsf(e0), fabsf(e1)) : 0.f, red);
   if (CH > 1) {
     cg::cluster_group cl = cg::this_cluster();
-    if (t == 0) {
-      xch[0] = sa.x;
-      xch[1] = sa.y;
+    const unsigned rank = cl.block_rank();
+    if (t < CH) {
+      float* rp = cl.map_shared_rank(xch, (unsigned)t);
+      rp[2 * rank] = sa.x;
+      rp[2 * rank + 1] = sa.y;
     }
-    cl.sync();                                       // every CTA's partial published
-    if (t < 32) {
-      float s2 = 0.f, a2 = 0.f;
-      if (t < CH) {
-        const float* rp = cl.map_shared_rank(xch, (unsigned)t);
-        s2 = rp[0];
-        a2 = rp[1];
-      }
-      s2 = warp_sum(s2);
-      a2 = warp_max(a2);
-      if (t == 0) {
-        red[64] = s2;
-        red[65] = a2;
-      }
+    cl.sync();                                       // every CTA's partial in every xch
+    float s2 = 0.f, a2 = 0.f;
+    for (int r = 0; r < CH; ++r) {                   // the same order in every CTA
+      s2 += xch[2 * r];
+      a2 = fmaxf(a2, xch[2 * r + 1]);
     }
-    __syncthreads();
-    sa = make_float2(red[64], red[65]);
-    cl.sync();                                       // no CTA rewrites xch while it is read
+    sa = make_float2(s2, a2);
   }
   float amax = sa.y;
   if (norm) {
@@ -259,9 +288,10 @@ __device__ __forceinline__ void copy_share(uint8_t* dst, const uint8_t* src, int
 
 __global__ void __launch_bounds__(kThr, 2) decode_append_kernel(AppendParams A) {
   __shared__ float red[72];
-  __shared__ float xch[2];
-  __shared__ float ebuf[512];
+  __shared__ float xch[2 * kCl];
+  __shared__ __align__(16) float ebuf[512];
   __shared__ float part[kThr * 4 * 3];               // slices x channels x (max, sum, acc)
+  __shared__ float4 bsm[kMaxRps * kThr];             // each thread's pooling biases
   const int nbase = A.csa ? 3 : 2;
   const int nj = nbase + (A.qimg ? 1 : 0);
   const int job = blockIdx.x / kCl, rank = blockIdx.x % kCl;
@@ -280,18 +310,16 @@ __global__ void __launch_bounds__(kThr, 2) decode_append_kernel(AppendParams A) 
   const uint8_t* xm = reinterpret_cast<const uint8_t*>(A.x_main) + b * nb;
   if (t == 0) {
     if (rank == 0) {
-      // W: the new token's window KV = RMSNorm(C^a_p) with RoPE at p
-      for (int c = threadIdx.x * 4; c < A.d; c += kThr * 4) {
-        const float4 v = ld4(xm, A.in_dtype, c);
-        ebuf[c] = v.x;
-        ebuf[c + 1] = v.y;
-        ebuf[c + 2] = v.z;
-        ebuf[c + 3] = v.w;
-      }
+      // W: the new token's window KV = RMSNorm(C^a_p) with RoPE at p (d <= 4 kThr)
+      const int c4 = threadIdx.x * 4, c2 = threadIdx.x * 2, dn = A.d - A.d_rope;
+      const float4 v = c4 < A.d ? ld4(xm, A.in_dtype, c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float rc = 1.f, rs = 0.f;                      // this thread's pair in finish_main
+      if (c2 >= dn && c2 < A.d) rope_cs(p, (c2 - dn) / 2, A.d_rope, A.theta, rc, rs);
+      if (c4 < A.d) *reinterpret_cast<float4*>(&ebuf[c4]) = v;
       __syncthreads();
       const int64_t rb = row_bytes(A.kv_dtype, A.d, A.d_rope);
       const int64_t row = (int64_t)b * A.swa_rows + p % A.swa_rows;
-      finish_main(ebuf, 0, A.d, A.d, A.d_rope, true, true, p, A.theta, A.eps, A.kv_dtype,
+      finish_main(ebuf, 0, A.d, A.d, A.d_rope, true, true, rc, rs, A.eps, A.kv_dtype,
                   reinterpret_cast<uint8_t*>(A.swa) + row * rb,
                   A.swa_scale ? reinterpret_cast<float*>(A.swa_scale) + row : nullptr, 1, red, xch);
     } else {
@@ -329,14 +357,18 @@ __global__ void __launch_bounds__(kThr, 2) decode_append_kernel(AppendParams A) 
     a.d_row = A.d;
     a.bias = A.bias;
     const int CW = A.d / kCl, c_lo = rank * CW;
-    pool_channels(a, c_lo, CW, ebuf, part);
+    // the RoPE angle of this thread's pair in finish_main (entry position m i)
+    const int c2 = c_lo + 2 * (int)threadIdx.x, dn = A.d - A.d_rope;
+    RopeReq rq{2 * (int)threadIdx.x < CW && c2 >= dn, (int64_t)A.m * i, (c2 - dn) / 2, A.d_rope,
+               A.theta};
+    float rc, rs;
+    pool_channels(a, c_lo, CW, ebuf, part, bsm, rq, rc, rs);
     const int64_t rb = row_bytes(A.kv_dtype, A.d, A.d_rope);
     const int64_t row = (int64_t)b * A.kv_rows + i % A.kv_rows;
     uint8_t* orow = reinterpret_cast<uint8_t*>(A.kv) + row * rb;
     // this CTA's channels, offset so that finish_main writes them in place
-    finish_main(ebuf, c_lo, CW, A.d, A.d_rope, true, true, (int64_t)A.m * i, A.theta, A.eps,
-                A.kv_dtype, orow, A.kv_scale ? reinterpret_cast<float*>(A.kv_scale) + row : nullptr,
-                kCl, red, xch);
+    finish_main(ebuf, c_lo, CW, A.d, A.d_rope, true, true, rc, rs, A.eps, A.kv_dtype, orow,
+                A.kv_scale ? reinterpret_cast<float*>(A.kv_scale) + row : nullptr, kCl, red, xch);
     return;
   }
   // K (CSA): the indexer key this token completes; 32 channels per CTA
@@ -347,7 +379,9 @@ __global__ void __launch_bounds__(kThr, 2) decode_append_kernel(AppendParams A) 
   a.xnew = reinterpret_cast<const uint8_t*>(A.x_idx) + b * ni;
   a.d_row = A.dI;
   a.bias = A.ibias;
-  pool_channels(a, c_lo, CW, ebuf, part);
+  RopeReq none{false, 0, 0, 0, 0.f};
+  float rc, rs;
+  pool_channels(a, c_lo, CW, ebuf, part, bsm, none, rc, rs);
   const int64_t row = (int64_t)b * A.key_rows + i % A.key_rows;
   if (A.idx_dtype == V4A_MXFP4) {
     finish_mxfp4(ebuf, c_lo, reinterpret_cast<uint8_t*>(A.keys) + row * (A.dI / 2),

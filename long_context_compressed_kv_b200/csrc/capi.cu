@@ -52,9 +52,10 @@ size_t mqa_qbuf_bytes(const v4attn_layer_desc* d, int32_t n_q) {
 // body offset of MQA calls and of every call of a decode step
 size_t body_mqa(const v4attn_layer_desc* d, int32_t n_q) { return qimg_off(n_q) + mqa_qbuf_bytes(d, n_q); }
 size_t mqa_need(const v4attn_layer_desc* d, int32_t n_q, int64_t n_main_max) {
-  // the tensor-core MQA (E4M3 caches) merges its key splits inside a thread-block
-  // cluster and writes the output directly: no split-K partials
-  if (d->kv_dtype == V4A_E4M3_BF16ROPE) return 0;
+  // the tensor-core MQA (E4M3 caches) splits a (query, half) over several
+  // CTAs only when at least two CTAs per (query, half) fit kMqaTcMaxCtas
+  if (d->kv_dtype == V4A_E4M3_BF16ROPE)
+    return 4 * (int64_t)q_chunk(n_q) <= kMqaTcMaxCtas ? align_up(kMqaTcPartBytes) : 0;
   const int S = mqa_num_splits(d, n_main_max);
   const int32_t c = q_chunk(n_q);
   return mqa_part_o_bytes(d, c, S) + mqa_part_ml_bytes(d, c, S);
@@ -304,7 +305,10 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
     P.split_keys = mqa_split_keys(d);
     P.n_split = mqa_num_splits(d, n_main_max);
     P.part_o = reinterpret_cast<float*>(w8 + b0);
-    P.part_ml = reinterpret_cast<float*>(w8 + b0 + mqa_part_o_bytes(d, c, P.n_split));
+    P.part_ml = d->kv_dtype == V4A_E4M3_BF16ROPE
+                    ? P.part_o + kMqaTcPartFloats
+                    : reinterpret_cast<float*>(w8 + b0 + mqa_part_o_bytes(d, c, P.n_split));
+    P.grid_bar = &reinterpret_cast<WsHeader*>(ws)->bar_count;
     P.qbuf = mqa_qbuf_bytes(d, c) ? w8 + qimg_off(a->n_q) : nullptr;
     P.q_ready = q_ready ? 1 : 0;
     P.out = reinterpret_cast<uint8_t*>(a->out) + (size_t)q0 * ob;
@@ -397,8 +401,10 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
     for (const void* p : {(const void*)a->bias, (const void*)a->ibias})
       if (p && (reinterpret_cast<uintptr_t>(p) % 16)) return V4A_ERR_INVALID_ARG;
     // a pooling window of at most 65536 / d rows per entry (8 rows per thread
-    // over the d / 8 channels of each of the job's 8 CTAs)
+    // over the d / 8 channels of each of the job's 8 CTAs, whose row slices
+    // are merged by 2048 / d adjacent lanes)
     if ((int64_t)ring * d > 65536) return V4A_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128 && d != 256 && d != 512) return V4A_ERR_UNSUPPORTED;
   }
   // 1.-2. tail rings, the new token's window KV (RMSNorm, RoPE at p), the
   // entry (and indexer key) its block completes: one launch

@@ -26,8 +26,12 @@ enum : uint32_t {
 
 struct WsHeader {
   uint32_t status;
-  uint32_t pad[63];
+  // the tensor-core MQA's grid barrier (arrivals, generation): zero after
+  // workspace init, the count back at zero after every completed barrier
+  uint32_t bar_count, bar_gen;
+  uint32_t pad[61];
 };
+static_assert(sizeof(WsHeader) == 256, "workspace header");
 
 __device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {
   if (status) atomicOr(status, bit);

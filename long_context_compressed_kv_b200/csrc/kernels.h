@@ -88,6 +88,12 @@ struct TopkParams {
 // Bytes per query of the tensor-core MQA's coded query image (73728 bytes of
 // swizzled E4M3 / bf16 tiles + 512 bytes of per-head scales, 1024-aligned).
 constexpr int64_t kMqaQImageStride = 74752;
+// The tensor-core MQA's split-K partials (launches of a few queries split each
+// (query, half) over several resident CTAs): at most kMqaTcMaxCtas CTAs, each
+// 128 x 256 fp32 of O and 2 x 128 row statistics.
+constexpr int kMqaTcMaxCtas = 160;
+constexpr size_t kMqaTcPartFloats = (size_t)kMqaTcMaxCtas * 128 * 256;
+constexpr size_t kMqaTcPartBytes = (kMqaTcPartFloats + (size_t)kMqaTcMaxCtas * 256) * sizeof(float);
 
 struct MqaParams {
   int n_q, B, H, d, d_rope, n_win, m;
@@ -110,8 +116,9 @@ struct MqaParams {
   const float* sink;
   int n_split;          // splits per query
   int split_keys;       // keys per split
-  float* part_o;        // [n_q][n_split][H][d]
-  float* part_ml;       // [n_q][n_split][H][2]
+  float* part_o;        // [n_q][n_split][H][d]; tensor-core path: [CTA][128][256]
+  float* part_ml;       // [n_q][n_split][H][2]; tensor-core path: [CTA][2][128]
+  uint32_t* grid_bar = nullptr;   // tensor-core path: [count, generation] in the workspace header
   uint8_t* qbuf;        // tensor-core path: [n_q] coded query images (kMqaQImageStride bytes)
   int q_ready = 0;      // the images in qbuf are already coded (decode: by the append kernel)
   void* out;

@@ -1,47 +1,48 @@
-// Shared-KV MQA on the 5th-generation tensor cores (tcgen05), decode form:
-// one query's H heads against a chunk of selected (CSA) or visible (HCA)
-// compressed entries and its window tokens, split-K partials out.
+// Shared-KV MQA on the 5th-generation tensor cores (tcgen05): each query's H
+// heads against its selected (CSA) or visible (HCA) compressed entries and its
+// window tokens, softmax with a per-head sink, inverse RoPE on the output.
 //
 // Method: "DeepSeek-V4 深读" (ricardokevins.github.io), model-spec table (64 /
 // 128 query heads of dim 512 over one shared KV head) and section
 // "其他稳定性细节" (448 FP8 + 64 BF16 RoPE dims, sink, inverse RoPE on the
-// output, which the combine applies); "拆解 DeepSeekv4", section "细节".
+// output); "拆解 DeepSeekv4", section "细节".
 //
 // Layout of the work.  Each query is coded once (RoPE at its position on dims
 // 448..511, E4M3 with a power-of-two scale on dims 0..447) straight into the
 // swizzled shared-memory image the MMAs read, by a small pre-kernel or, in the
 // decode step, by the append kernel that runs before it; every CTA of the
-// query copies that image in with bulk copies.  A CTA owns (query, key
-// chunk of split_keys keys, half of the 512 output dims).  Output dims are
-// split because fp32 O for 128 heads x 512 dims is all of TMEM (512 columns x
-// 128 lanes): each CTA keeps O[128 x 256] in TMEM columns 256..511 and S for
-// two 64-key tiles in columns 0..255, and recomputes S = Q K^T (the two
-// halves of a chunk run on neighbouring CTAs, so the second read of the
-// chunk's rows comes from L2).
+// query copies that image in with bulk copies.  A CTA owns (query, one of C
+// key splits, half of the 512 output dims).  Output dims are split because
+// fp32 O for 128 heads x 512 dims is all of TMEM (512 columns x 128 lanes):
+// each CTA keeps O[128 x 256] in TMEM columns 256..511 and S for two 64-key
+// tiles in columns 0..255, and recomputes S = Q K^T (the two halves of a split
+// run on neighbouring CTAs, so the second read of its rows comes from L2).
+// With few queries C > 1 key splits per (query, half) keep every SM busy; the
+// launch is then cooperative and the splits merge through L2 after one grid
+// barrier.
 //
 // Per 64-key tile:
 //   S_nope = Q_nope(E4M3) . K_nope(E4M3)^T   14 x tcgen05.mma kind::f8f6f4, K=32
 //   S_rope = Q_rope(BF16) . K_rope(BF16)^T    4 x tcgen05.mma kind::f16,   K=16
 //   s_j    = scale * (q_scale * k_scale_j * S_nope + S_rope)       (log2 units)
-//   P_j    = exp2(s_j - M_s)                                        (BF16, RoPE dims)
-//   P'_j   = P_j * k_scale_j * 2^(8 - tau - K)                      (E4M3 hi + lo parts)
-//   O_nope += P'_hi V_nope + P'_lo V_nope                           kind::f8f6f4, V MN-major
-//   O_rope += P V_rope                                              kind::f16, V MN-major
-// The entry scale k_scale_j (a power of two) of the FP8 dims is folded into
-// P'; K is the CTA's running maximum of log2 k_scale, the same for every head
-// row.  M_s is the row's running score maximum, moved only when a tile beats
-// it by more than tau = 4, so P <= 2^tau and P' <= 2^8 (inside E4M3's range);
-// O is rescaled in TMEM only when M_s or K moves.  The same shared-memory tile serves as the K-major B operand
-// of Q K^T and the MN-major B operand of P V.
+//   P_j    = exp2(s_j - M_s)                                        (f16, in TMEM)
+//   V_j    = k_scale_j * code_j (dims < 448), bf16 RoPE dims        (f16, in smem)
+//   O     += P V                                 4 x tcgen05.mma kind::f16, K=16, N=256
+// M_s is the row's running score maximum, moved only when a tile beats it by
+// more than tau = 4, so P <= 2^tau; O is rescaled in TMEM only when M_s moves.
+// V in f16 is exact for stored values of magnitude 2^-14 .. 65504 (an entry
+// scale times an E4M3 code has four significant bits); P in f16 carries 11
+// significant bits, and the row sum is taken over those f16 values.
 //
 // Rows arrive by TMA: tile mode for contiguous HCA entries, tile::gather4 (4
 // rows per instruction) for selected entries and window tokens; the entry
 // scales by 4-byte cp.async.  Roles: warp 0 loads, warp 1 issues the
-// MMAs (one lane), warps 2..17 run the softmax and the epilogue: four warps
-// per TMEM lane quarter, one per 16-key group of each tile, exchanging row
-// maxima through shared memory.  Every cross-warp hand-off is an mbarrier with a
-// bounded, warp-uniform wait, so a stalled kernel ends with a status bit.
-#include <cooperative_groups.h>
+// MMAs (one lane), warps 2..17 run the softmax, the conversion of V to f16
+// and the epilogue: four warps per TMEM lane quarter, one per 16-key group of
+// each tile, exchanging row maxima through shared memory.  Every cross-warp
+// hand-off is an mbarrier with a bounded, warp-uniform wait, and the grid
+// barrier is bounded too, so a stalled kernel ends with a status bit.
+#include <algorithm>
 #include <cstddef>
 
 #include "common.cuh"
@@ -75,11 +76,15 @@ struct Smem {
   float qsc[128];                             // contiguous with q: one image
   alignas(1024) uint8_t kv[KST][4][NK * 128]; // nope blocks 0..2 and the rope block, SW128
   alignas(1024) uint8_t kv3[KST][NK * 64];    // nope bytes 384..447, SW64
+  // V of the tile in f16 (values = code x entry scale; RoPE dims converted
+  // from bf16) for this CTA's 256 output dims: four MN-major SW128 blocks of
+  // 64 dims x NK keys, the B operand of P V
+  alignas(1024) uint8_t v16[4][NK * 128];
   float kscale[KST][NK];
   union {
-    float xmax[2][KG][2][128];                // tile loop: [tile parity][key group][M_s, M_u][row]
+    float xmax[2][KG][128];                   // tile loop: [tile parity][key group][row]
     struct {                                  // merge (the loop is over for every warp):
-      float rms[128], rl[128], rfn[128];      // this split's row max (log2), row sum, 1 / cu
+      float rms[128], rl[128];                // this split's row max (log2), row sum
       float fself[128], invl[128];            // merge factor of this split, 1 / denominator
       float rcs[32], rsn[32];                 // RoPE angles of the query position
     } mg;
@@ -92,15 +97,15 @@ struct Smem {
 
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory per CTA");
 static_assert(offsetof(Smem, qsc) == QTILE, "the query image is one contiguous copy");
-// the merge stages half of this split's O (fp32, 128 rows of SSTH floats) over
-// the key stages, which are free once the last P.V has completed
-constexpr int SSTH = 132;                    // row stride (floats): conflict-free float4 rows
-static_assert(offsetof(Smem, kscale) - offsetof(Smem, kv) >= 128 * SSTH * 4, "merge stage fits");
-// TMEM columns of the coded P inside a tile's 128-column S buffer (written
-// after the buffer's S has been read): E4M3 hi / mid / lo parts at
-// PC_E4 + 16 part (64 keys, 4 a column), bf16 hi / lo parts at PC_BF + 32 part
-// (2 keys a column)
-constexpr uint32_t PC_E4 = 0, PC_BF = 48;
+// the merge stages this split's O (fp32, 128 rows of SST floats) over the query
+// image and the key stages, which are free once the last P.V has completed
+constexpr int SST = 260;                     // row stride (floats): conflict-free float4 rows
+constexpr int kMaxSplit = 64;                // key splits per (query, half), at most
+static_assert(offsetof(Smem, kscale) >= 128 * SST * 4, "merge stage fits");
+static_assert(offsetof(Smem, kscale) >= 2 * kMaxSplit * 128 * 4, "merge factors fit");
+// TMEM column of P (f16, two keys a column, 32 columns) inside a tile's
+// 128-column S buffer, written after the buffer's S has been read
+constexpr uint32_t PC_F16 = 0;
 
 struct Maps {
   CUtensorMap kv128, kv64;      // tile mode, boxes {128 B | 64 B} x NK rows
@@ -137,12 +142,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
-// 32 lanes x 4 / 8 consecutive columns from registers
-__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t* r) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr),
-               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
-               : "memory");
-}
+// 32 lanes x 8 consecutive columns from registers
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
                    taddr),
@@ -150,16 +150,8 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
                "r"(r[7])
                : "memory");
 }
-// MMAs whose A operand is read from tensor memory (M = 128 rows at lanes
-// 0..127, K along the columns: four 8-bit or two 16-bit elements a column)
-__device__ __forceinline__ void mma_f8f6f4_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
-                                              uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
+// MMA whose A operand is read from tensor memory (M = 128 rows at lanes
+// 0..127, K along the columns: two 16-bit elements a column)
 __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
                                            uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -169,15 +161,80 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
       : "memory");
 }
 
-__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t c) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)c, __NV_E4M3);
-  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+// two E4M3 codes (low byte first) -> f16x2, exact, times the f16x2 scale
+__device__ __forceinline__ uint32_t e4m3x2_f16x2_scaled(uint32_t c, __half2 sc) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(c & 0xFFFFu), __NV_E4M3);
+  const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&h), sc);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+// two bf16 (low half first) -> f16x2 (round to nearest even)
+__device__ __forceinline__ uint32_t bf16x2_f16x2(uint32_t w) {
+  const __half2 v = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+// 16 E4M3 codes (one 16-byte chunk) -> 16 f16 values scaled by sc, as 2 x 16 bytes
+__device__ __forceinline__ void e4m3x16_f16(const uint4 c, __half2 sc, uint4& lo, uint4& hi) {
+  lo.x = e4m3x2_f16x2_scaled(c.x, sc);
+  lo.y = e4m3x2_f16x2_scaled(c.x >> 16, sc);
+  lo.z = e4m3x2_f16x2_scaled(c.y, sc);
+  lo.w = e4m3x2_f16x2_scaled(c.y >> 16, sc);
+  hi.x = e4m3x2_f16x2_scaled(c.z, sc);
+  hi.y = e4m3x2_f16x2_scaled(c.z >> 16, sc);
+  hi.z = e4m3x2_f16x2_scaled(c.w, sc);
+  hi.w = e4m3x2_f16x2_scaled(c.w >> 16, sc);
 }
 // 2^x by the SFU (ex2.approx, flush to zero; 2^-inf = 0)
 __device__ __forceinline__ float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// V of the tile in stage st into s.v16 for this CTA's 256 output dims
+// (dh * 256 ..), by the 512 softmax threads (ctid = 0..511), one 16-byte
+// source chunk (16 E4M3 codes or 8 bf16 of one key) at a time.  The E4M3 codes
+// are scaled by the entry's scale (a power of two; zero for an empty slot).
+template <typename SmemT>
+__device__ __forceinline__ void convert_v(SmemT& s, int st, int dh, int ctid) {
+  if (dh == 0) {
+    // dims 0..255: blocks 0 and 1 of the stage, 16 chunks a key
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int u = ctid + 512 * i;
+      const int k = u >> 4, c16 = u & 15;
+      const uint4 c = *reinterpret_cast<const uint4*>(s.kv[st][c16 >> 3] + sw128(k, (c16 & 7) * 16));
+      const __half2 sc = __float2half2_rn(s.kscale[st][k]);
+      uint4 lo, hi;
+      e4m3x16_f16(c, sc, lo, hi);
+      uint8_t* blk = s.v16[c16 >> 2];            // output dims 16 c16 .. + 15
+      const int nb = (c16 & 3) * 32;
+      *reinterpret_cast<uint4*>(blk + sw128(k, nb)) = lo;
+      *reinterpret_cast<uint4*>(blk + sw128(k, nb + 16)) = hi;
+    }
+  } else {
+    // dims 256..383 (block 2), 384..447 (the SW64 block), RoPE 448..511
+    // (block 3, bf16): 20 chunks a key
+    for (int u = ctid; u < NK * 20; u += 512) {
+      const int k = u / 20, w = u - k * 20;
+      if (w < 12) {
+        const uint4 c = w < 8 ? *reinterpret_cast<const uint4*>(s.kv[st][2] + sw128(k, w * 16))
+                              : *reinterpret_cast<const uint4*>(s.kv3[st] + sw64(k, (w - 8) * 16));
+        const __half2 sc = __float2half2_rn(s.kscale[st][k]);
+        uint4 lo, hi;
+        e4m3x16_f16(c, sc, lo, hi);
+        uint8_t* blk = s.v16[w >> 2];            // output dims 16 w .. + 15
+        const int nb = (w & 3) * 32;
+        *reinterpret_cast<uint4*>(blk + sw128(k, nb)) = lo;
+        *reinterpret_cast<uint4*>(blk + sw128(k, nb + 16)) = hi;
+      } else {
+        const int r = w - 12;                    // dims 448 + 8 r .. + 7
+        const uint4 b = *reinterpret_cast<const uint4*>(s.kv[st][3] + sw128(k, r * 16));
+        const uint4 o = make_uint4(bf16x2_f16x2(b.x), bf16x2_f16x2(b.y), bf16x2_f16x2(b.z),
+                                   bf16x2_f16x2(b.w));
+        *reinterpret_cast<uint4*>(s.v16[3] + sw128(k, r * 16)) = o;
+      }
+    }
+  }
 }
 
 struct Geo {
@@ -239,13 +296,14 @@ __global__ void __launch_bounds__(NTHR, 1)
   Smem& s = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // the C = n_split CTAs of a cluster are the key splits of one (query, half);
-  // cluster rank == split
+  // CTAs unit * C .. unit * C + C - 1 are the key splits of one (query, half)
   const int C = P.n_split;
   const int split = (int)(blockIdx.x % (unsigned)C);
   const int unit = (int)(blockIdx.x / (unsigned)C);
   const int dh = unit & 1, q = unit >> 1;
   const Geo g = geometry(P, q, split);
+  // the grid barrier's generation before this CTA arrives (merging launches)
+  const uint32_t bar_gen0 = (C > 1 && threadIdx.x == 0) ? ld_acquire_gpu(P.grid_bar + 1) : 0u;
   // every CTA, also one with no tiles (T = 0), takes part in the merge below
 
   if (threadIdx.x == 0) {
@@ -371,49 +429,24 @@ __global__ void __launch_bounds__(NTHR, 1)
     // ------------------------------------------------------------ MMA issue
     const uint64_t kq128 = smem_desc_bits(16, 1024, 2);   // K-major, 128B swizzle
     const uint64_t kq64 = smem_desc_bits(16, 512, 4);     // K-major, 64B swizzle
-    const uint64_t mn128 = smem_desc_bits(NK * 128, 1024, 2);  // MN-major, 128B swizzle
-    const uint64_t mn64 = smem_desc_bits(16, 512, 4);      // MN-major, 64B swizzle
+    const uint64_t mn128 = smem_desc_bits(NK * 128, 1024, 2);  // MN-major, 128B swizzle, 8 KB blocks
     const uint32_t id_qk8 = idesc_f(0, 0, 128, NK, false, false);
     const uint32_t id_qk16 = idesc_f(1, 1, 128, NK, false, false);
-    const uint32_t id_pv256 = idesc_f(0, 0, 128, 256, false, true);
-    const uint32_t id_pv128 = idesc_f(0, 0, 128, 128, false, true);
-    const uint32_t id_pv64 = idesc_f(0, 0, 128, 64, false, true);
-    const uint32_t id_pvr = idesc_f(1, 1, 128, 64, false, true);
+    const uint32_t id_pv = idesc_f(0, 0, 128, 256, false, true);   // f16 x f16, B MN-major
     const uint32_t O = tmem + 256;
     bool ok = mbar_wait_warp(&s.qready, 0, P.status, 1);
-    // P.V of tile tt: A = the coded P of the tile, read from its TMEM buffer
-    // (tt & 1, written there by the softmax), B = V (= K) in shared memory
+    // P.V of tile tt: A = P (f16) of the tile, read from its TMEM buffer
+    // (tt & 1, written there by the softmax), B = the tile's V in f16
+    // (s.v16, converted by the softmax warps), N = this CTA's 256 dims
     auto pv = [&](int tt) -> bool {
       const int st = tt % KST, a = tt & 1;
       if (!mbar_wait_warp(&s.pfull[a], (tt >> 1) & 1, P.status, 2)) return false;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t pb = tmem + a * 128;
-        if (dh == 0) {
-          const uint64_t bv = smem_desc(s.kv[st][0], mn128);
-          for (int ks = 0; ks < 2; ++ks) {                    // 32 keys (8 columns) a step
-            const uint64_t bk = bv + (uint64_t)(ks * 32 * 128 >> 4);
-            for (int pt = 0; pt < 3; ++pt)                    // E4M3 hi, mid, lo parts of P'
-              mma_f8f6f4_ts(O, pb + PC_E4 + 16 * pt + 8 * ks, bk, id_pv256, (tt | ks | pt) != 0);
-          }
-        } else {
-          const uint64_t b2 = smem_desc(s.kv[st][2], mn128);
-          const uint64_t b3 = smem_desc(s.kv3[st], mn64);
-          const uint64_t br = smem_desc(s.kv[st][3], mn128);
-          for (int ks = 0; ks < 2; ++ks) {
-            const uint64_t bk2 = b2 + (uint64_t)(ks * 32 * 128 >> 4);
-            const uint64_t bk3 = b3 + (uint64_t)(ks * 32 * 64 >> 4);
-            for (int pt = 0; pt < 3; ++pt) {
-              const uint32_t pa = pb + PC_E4 + 16 * pt + 8 * ks;
-              mma_f8f6f4_ts(O, pa, bk2, id_pv128, (tt | ks | pt) != 0);
-              mma_f8f6f4_ts(O + 128, pa, bk3, id_pv64, (tt | ks | pt) != 0);
-            }
-          }
-          for (int ks = 0; ks < 4; ++ks)                      // 16 keys (8 columns) a step
-            for (int pt = 0; pt < 2; ++pt)                    // bf16 hi, lo parts of the weight
-              mma_f16_ts(O + 192, pb + PC_BF + 32 * pt + 8 * ks,
-                         br + (uint64_t)(ks * 16 * 128 >> 4), id_pvr, (tt | ks | pt) != 0);
-        }
+        const uint32_t pb = tmem + a * 128 + PC_F16;
+        const uint64_t bv = smem_desc(s.v16[0], mn128);
+        for (int ks = 0; ks < 4; ++ks)                        // 16 keys (8 columns) a step
+          mma_f16_ts(O, pb + 8 * ks, bv + (uint64_t)(ks * 16 * 128 >> 4), id_pv, (tt | ks) != 0);
         tc_commit(&s.empty[st]);
         tc_commit(&s.pdone[a]);
       }
@@ -464,14 +497,12 @@ __global__ void __launch_bounds__(NTHR, 1)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const float sl2 = P.scale * 1.4426950408889634f;     // softmax scale x log2(e)
     // Ms: the row's running score maximum (log2 units), moved only when a tile
-    // exceeds it by more than kTau, so P <= 2^kTau; K: the CTA's running
-    // maximum entry-scale exponent, so P' = P k_scale 2^(8 - kTau - K) <= 2^8.
+    // exceeds it by more than kTau, so P <= 2^kTau (well inside f16's range).
     float Ms = -INFINITY, l = 0.f;
-    int K = -1000;                                       // no key seen yet
-    float cu = 0.f;                                      // 2^(8 - kTau - K), exponent clamped
     bool wrote = false;                                  // O holds a PV result
     bool live = mbar_wait_warp(&s.qready, 0, P.status, 1);
     const float qs = s.qsc[h];
+    const int ctid = (warp - 2) * 32 + lane;             // 0 .. 511: share of the V conversion
     for (int t = 0; t < g.T && live; ++t) {
       const int a = t & 1, st = t % KST, xb = t & 1;
       if (!mbar_wait_warp(&s.sfull[a], (t >> 1) & 1, P.status, 6) ||
@@ -488,20 +519,16 @@ __global__ void __launch_bounds__(NTHR, 1)
       const float* ksc = &s.kscale[st][grp * KPG];
       float s2[KPG];
       float ms = -INFINITY;
-      uint32_t kbits = 0;                                // largest scale bits of the group's keys
 #pragma unroll
       for (int j = 0; j < KPG; ++j) {
         const float kj = ksc[j];
         const float v = (qs * kj * __uint_as_float(sn_[j]) + __uint_as_float(sr_[j])) * sl2;
-        s2[j] = (kj != 0.f) ? v : -INFINITY;
+        s2[j] = (kj != 0.f) ? v : -INFINITY;             // a zero scale marks an empty slot
         ms = fmaxf(ms, s2[j]);
-        kbits = max(kbits, __float_as_uint(kj));
       }
-      // tile maxima (row score, scale exponent): exchange with the other key
-      // groups; past this exchange every group has read its S columns, so the
-      // coded P may overwrite the buffer
-      s.xmax[xb][grp][0][h] = ms;
-      s.xmax[xb][grp][1][h] = __uint_as_float(kbits);
+      // the tile's row maximum: exchanged with the other key groups; past this
+      // exchange every group has read its S columns, so P may overwrite them
+      s.xmax[xb][grp][h] = ms;
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.xbar[xb]);
       if (!mbar_wait_warp(&s.xbar[xb], (t >> 1) & 1, P.status, 10)) {
@@ -509,98 +536,52 @@ __global__ void __launch_bounds__(NTHR, 1)
         break;
       }
 #pragma unroll
-      for (int o = 0; o < KG; ++o) {
-        ms = fmaxf(ms, s.xmax[xb][o][0][h]);
-        kbits = max(kbits, __float_as_uint(s.xmax[xb][o][1][h]));
-      }
-      const int kt = (int)((kbits >> 23) & 0xFF) - 127;      // exponent of the tile's largest scale
+      for (int o = 0; o < KG; ++o) ms = fmaxf(ms, s.xmax[xb][o][h]);
       const bool upd = ms > Ms + kTau;
       const float Ms_new = upd ? ms : Ms;
-      const int K_new = (kbits != 0 && kt > K) ? kt : K;
       const float as = (upd && Ms != -INFINITY) ? ex2f(Ms - Ms_new) : 1.f;
-      const float cu_new =
-          (K_new == -1000) ? 0.f : exp2i(min(126, max(-126, 8 - (int)kTau - K_new)));
-      const float ak = (cu > 0.f && cu_new != cu) ? cu_new / cu : 1.f;   // exact: powers of two
       const float ms_ref = (Ms_new == -INFINITY) ? 0.f : Ms_new;
-      // P' = P k_scale cu coded as three E4M3 parts (hi + mid + lo: 12
-      // significant bits) for the FP8 dims; the weight each key then really
-      // gets, w = (hi + mid + lo) / (k_scale cu) (exact in fp32), coded as two
-      // bf16 parts for the RoPE dims; the row sum is taken over the w.
+      // P = exp2(s - Ms) in f16 (the A operand of P V); the row sum is taken
+      // over the f16 values, i.e. the weights P V really applies
       float lsum = 0.f;
-      uint32_t phi[KPG / 4], pmd[KPG / 4], plo[KPG / 4], pbh[KPG / 2], pbl[KPG / 2];
+      uint32_t ph[KPG / 2];
 #pragma unroll
       for (int j = 0; j < KPG; j += 2) {
-        const float p0 = ex2f(s2[j] - ms_ref), p1 = ex2f(s2[j + 1] - ms_ref);   // 0 for -inf
-        const float kc0 = ksc[j] * cu_new, kc1 = ksc[j + 1] * cu_new;          // powers of two (or 0)
-        const float u0 = p0 * kc0, u1 = p1 * kc1;
-        const uint32_t hi = e4m3x2(u0, u1);
-        const float2 hf = e4m3x2_to_f32(hi);
-        const float r0 = u0 - hf.x, r1 = u1 - hf.y;
-        const uint32_t md = e4m3x2(r0, r1);
-        const float2 mf = e4m3x2_to_f32(md);
-        const uint32_t lo = e4m3x2(r0 - mf.x, r1 - mf.y);
-        const float2 lf = e4m3x2_to_f32(lo);
-        const float w0 = kc0 != 0.f ? ((hf.x + mf.x) + lf.x) * __int_as_float((254 << 23) - __float_as_int(kc0)) : 0.f;
-        const float w1 = kc1 != 0.f ? ((hf.y + mf.y) + lf.y) * __int_as_float((254 << 23) - __float_as_int(kc1)) : 0.f;
-        lsum += w0 + w1;
-        if ((j & 3) == 0) {
-          phi[j >> 2] = hi;
-          pmd[j >> 2] = md;
-          plo[j >> 2] = lo;
-        } else {
-          phi[j >> 2] |= hi << 16;
-          pmd[j >> 2] |= md << 16;
-          plo[j >> 2] |= lo << 16;
-        }
-        const __nv_bfloat162 bh = __floats2bfloat162_rn(w0, w1);
-        const float2 bhf = __bfloat1622float2(bh);
-        const __nv_bfloat162 bl = __floats2bfloat162_rn(w0 - bhf.x, w1 - bhf.y);
-        pbh[j >> 1] = *reinterpret_cast<const uint32_t*>(&bh);
-        pbl[j >> 1] = *reinterpret_cast<const uint32_t*>(&bl);
+        const __half2 hp = __floats2half2_rn(ex2f(s2[j] - ms_ref), ex2f(s2[j + 1] - ms_ref));
+        const float2 pf = __half22float2(hp);
+        lsum += pf.x + pf.y;
+        ph[j >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
       }
       l = l * as + lsum;
+      // the previous tile's P.V has completed: O may be rescaled and the
+      // f16 V buffer rewritten
+      if (t >= 1 && !mbar_wait_warp(&s.pdone[(t - 1) & 1], ((t - 1) >> 1) & 1, P.status, 8)) {
+        live = false;
+        break;
+      }
+      tc_fence_after();
       // Rescale this warp's share of O (columns grp*64 .. +63) when the row's
-      // reference moved: the FP8 part by as*ak, the RoPE part by as, after the
-      // previous tile's P.V has completed.  tcgen05.ld / st are warp-wide
-      // (.sync.aligned): the decision is taken per warp, every lane takes part
-      // with its own factor.
-      const float an = as * ak;
-      const bool grow_n = __any_sync(0xffffffffu, wrote && an < 1.f);
-      const bool grow_r = __any_sync(0xffffffffu, wrote && dh == 1 && as < 1.f);
-      if (grow_n || grow_r) {
-        if (t >= 1 && !mbar_wait_warp(&s.pdone[(t - 1) & 1], ((t - 1) >> 1) & 1, P.status, 8)) {
-          live = false;
-          break;
-        }
-        tc_fence_after();
+      // reference moved.  tcgen05.ld / st are warp-wide (.sync.aligned): the
+      // decision is taken per warp, every lane takes part with its own factor.
+      if (__any_sync(0xffffffffu, wrote && as < 1.f)) {
         const uint32_t ob = tmem + lane_off + 256;
+#pragma unroll 1
         for (int cc = 0; cc < 256 / KG; cc += 32) {
           const int c = grp * (256 / KG) + cc;
-          const bool rope_cols = dh == 1 && c >= 192;
-          if (rope_cols ? !grow_r : !grow_n) continue;     // uniform across the warp
-          const float f = rope_cols ? as : an;
           uint32_t r[32];
           tmem_ld32_nowait(ob + c, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * f);
+          for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * as);
           tmem_st32(ob + c, r);
         }
-        tmem_st_wait();
       }
       Ms = Ms_new;
-      K = K_new;
-      cu = cu_new;
-      // the coded P of this group's 16 keys into the tile's TMEM buffer:
-      // E4M3 parts at columns PC_E4 + 16 * part + 4 * grp (4 keys a column),
-      // bf16 parts at PC_BF + 32 * part + 8 * grp (2 keys a column)
-      tmem_st4(tb + PC_E4 + 4 * grp, phi);
-      tmem_st4(tb + PC_E4 + 16 + 4 * grp, pmd);
-      tmem_st4(tb + PC_E4 + 32 + 4 * grp, plo);
-      if (dh == 1) {
-        tmem_st8(tb + PC_BF + 8 * grp, pbh);
-        tmem_st8(tb + PC_BF + 32 + 8 * grp, pbl);
-      }
+      // this group's 16 keys of P into the tile's TMEM buffer (columns
+      // PC_F16 + 8 grp ..), and this thread's share of the tile's V in f16
+      tmem_st8(tb + PC_F16 + 8 * grp, ph);
+      convert_v(s, st, dh, ctid);
+      fence_proxy_async_smem();                          // V16 visible to the tensor core
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -622,50 +603,115 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     fin = fin && live;
     // this split's per-row results for the merge: the row maximum (log2 units;
-    // -inf for no key), the row sum in units of exp2(. - Ms), and 1 / cu, the
-    // factor that brings O_nope (kept in units of cu exp2(. - Ms)) to those units
+    // -inf for no key) and the row sum, O and the sum both in units of exp2(. - Ms)
     if (grp == 0) {
       const bool any = fin && Ms != -INFINITY;
       s.mg.rms[h] = any ? Ms : -INFINITY;
       s.mg.rl[h] = any ? l : 0.f;
-      s.mg.rfn[h] = (any && cu != 0.f) ? 1.f / cu : 0.f;
     }
   }
 
   // ------------------------------------------------------------ merge the C splits
-  // Every thread of every CTA of the cluster passes the cluster barriers below
-  // exactly once (the roles above have no early exit), so none can hang.
-  namespace cg = cooperative_groups;
-  cg::cluster_group cl = cg::this_cluster();
+  // C == 1: the output straight from TMEM.  C > 1 (a cooperative launch, every
+  // CTA resident): each split writes its O, in units of exp2(. - its row
+  // maximum), and its row maxima / sums to the workspace (L2-resident), all
+  // CTAs meet at one grid barrier, then CTA `split` reduces column groups
+  // [64 split / C, 64 (split + 1) / C) (four columns each) of its (query, half)
+  // over the C partials and writes them.  Every thread passes the barriers
+  // below exactly once (the roles above have no early exit).
   const int tid = threadIdx.x;
   tc_fence_before();
   __syncthreads();
-  cl.sync();                                    // every split's rms / rl / rfn published
   const float log2e = 1.4426950408889634f;
+  float* stage = reinterpret_cast<float*>(&s.q[0]);    // q .. kv3: free, every MMA / copy is done
+  float* fac = stage;                                   // [C][128] row factors (after the copy-out)
+  float* lsp = stage + C * 128;                         // [C][128] row sums
+  bool merge_ok = true;
+  if (C > 1) {
+    // (1) this split's O as fp32 rows of SST floats
+    if (warp >= 2) {
+      const int quad = warp & 3, grp = (warp - 2) >> 2;
+      const int hh = quad * 32 + lane;
+      const uint32_t ob = tmem + ((uint32_t)(quad * 32) << 16) + 256;
+#pragma unroll 1
+      for (int cc = 0; cc < 256 / KG; cc += 32) {
+        const int c = grp * (256 / KG) + cc;
+        uint32_t r[32];
+        tmem_ld32_nowait(ob + c, r);
+        tmem_ld_wait();
+        float4* dst = reinterpret_cast<float4*>(stage + hh * SST + c);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          dst[k] = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
+                               __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
+      }
+    }
+    __syncthreads();
+    // (2) to this CTA's partial: [128][256] fp32, then [row max | row sum][128]
+    float* po = P.part_o + (int64_t)blockIdx.x * (128 * 256);
+    float* pm = P.part_ml + (int64_t)blockIdx.x * 256;
+    for (int i = tid; i < 128 * 64; i += NTHR)
+      __stcg(reinterpret_cast<float4*>(po) + i,
+             *reinterpret_cast<const float4*>(stage + (i >> 6) * SST + (i & 63) * 4));
+    if (tid < 128) {
+      __stcg(pm + tid, s.mg.rms[tid]);
+      __stcg(pm + 128 + tid, s.mg.rl[tid]);
+    }
+    __syncthreads();
+    // (3) every split of every (query, half) written
+    if (tid == 0) {
+      const bool ok = grid_barrier(P.grid_bar, P.grid_bar + 1, bar_gen0, gridDim.x, P.status);
+      if (!ok) flag(P.status, ST_TIMEOUT | (1u << (16 + 13)));
+      s.mg.rcs[0] = ok ? 1.f : 0.f;                      // the verdict, for the whole CTA
+    }
+    __syncthreads();
+    merge_ok = s.mg.rcs[0] != 0.f;
+    __syncthreads();
+    // (4) the C splits' row maxima and sums of this (query, half)
+    if (merge_ok) {
+      const float* pm0 = P.part_ml + (int64_t)(blockIdx.x - split) * 256;
+      for (int i = tid; i < C * 128; i += NTHR) {
+        const int r = i >> 7, hh = i & 127;
+        fac[i] = __ldcg(pm0 + r * 256 + hh);
+        lsp[i] = __ldcg(pm0 + r * 256 + 128 + hh);
+      }
+    }
+    __syncthreads();
+  }
   if (tid < 128) {
-    // the merged row maximum (with the sink, in log2 units) and denominator
+    // the merged row maximum (with the sink, log2 units) and denominator; the
+    // factor exp2(max_r - M) of each split
     const int hh = tid;
     const float z = (P.sink && hh < P.H) ? P.sink[hh] * log2e : -INFINITY;
     float M = z;
-    for (int r = 0; r < C; ++r) M = fmaxf(M, cl.map_shared_rank(s.mg.rms, (unsigned)r)[hh]);
-    float den = 0.f;
-    if (M != -INFINITY) {
-      for (int r = 0; r < C; ++r) {
-        const float mr = cl.map_shared_rank(s.mg.rms, (unsigned)r)[hh];
-        if (mr != -INFINITY) den += ex2f(mr - M) * cl.map_shared_rank(s.mg.rl, (unsigned)r)[hh];
-      }
-      if (z != -INFINITY) den += ex2f(z - M);
+    if (C == 1) {
+      M = fmaxf(M, s.mg.rms[hh]);
+    } else {
+      for (int r = 0; r < C; ++r) M = fmaxf(M, fac[r * 128 + hh]);
     }
-    s.mg.fself[hh] = (s.mg.rms[hh] == -INFINITY) ? 0.f : ex2f(s.mg.rms[hh] - M);
+    float den = 0.f;
+    if (C == 1) {
+      const float f = (M != -INFINITY && s.mg.rms[hh] != -INFINITY) ? ex2f(s.mg.rms[hh] - M) : 0.f;
+      s.mg.fself[hh] = f;
+      den = f * s.mg.rl[hh];
+    } else {
+      for (int r = 0; r < C; ++r) {
+        const float mr = fac[r * 128 + hh];
+        const float f = (M != -INFINITY && mr != -INFINITY) ? ex2f(mr - M) : 0.f;
+        fac[r * 128 + hh] = f;
+        den += f * lsp[r * 128 + hh];
+      }
+    }
+    if (M != -INFINITY && z != -INFINITY) den += ex2f(z - M);
     s.mg.invl[hh] = den > 0.f ? 1.f / den : 0.f;
-    if (P.lse && dh == 0 && split == 0 && hh < P.H)
+    if (P.lse && dh == 0 && split == 0 && hh < P.H && merge_ok)
       P.lse[(int64_t)q * P.H + hh] = den > 0.f ? M * 0.6931471805599453f + logf(den) : -INFINITY;
-  } else if (tid < 160 && dh == 1) {
+  } else if (tid >= 160 && tid < 192 && dh == 1) {
     // rotation by -p of the output's RoPE dims: the angles of the 32 pairs
     float c = 1.f, sv = 0.f;
-    if (g.p >= 0) rope_cs(g.p, tid - 128, 64, P.theta, c, sv);
-    s.mg.rcs[tid - 128] = c;
-    s.mg.rsn[tid - 128] = sv;
+    if (g.p >= 0) rope_cs(g.p, tid - 160, 64, P.theta, c, sv);
+    s.mg.rcs[tid - 160] = c;
+    s.mg.rsn[tid - 160] = sv;
   }
   __syncthreads();
   const int64_t obase = (int64_t)q * P.H * 512 + dh * 256;
@@ -694,19 +740,18 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
   };
   if (C == 1) {
-    // one split: the output straight from TMEM (each thread 32 columns of its row)
+    // each epilogue thread 64 columns of its row
     if (warp >= 2) {
       const int quad = warp & 3, grp = (warp - 2) >> 2;
       const int hh = quad * 32 + lane;
       const uint32_t ob = tmem + ((uint32_t)(quad * 32) << 16) + 256;
-      const float fs = s.mg.fself[hh], fnn = fs * s.mg.rfn[hh];
+      const float f = s.mg.fself[hh];
 #pragma unroll 1
       for (int cc = 0; cc < 256 / KG; cc += 32) {
         const int c = grp * (256 / KG) + cc;
         uint32_t r[32];
         tmem_ld32_nowait(ob + c, r);
         tmem_ld_wait();
-        const float f = (dh == 1 && c >= 192) ? fs : fnn;   // RoPE dims carry no cu
         if (hh < P.H)
 #pragma unroll
           for (int k = 0; k < 32; k += 4)
@@ -714,48 +759,38 @@ __global__ void __launch_bounds__(NTHR, 1)
                                          __uint_as_float(r[k + 2]) * f, __uint_as_float(r[k + 3]) * f));
       }
     }
-  } else {
-    // the splits' O, scaled to the merged units, staged as fp32 rows in shared
-    // memory (over the key stages, free now), one half of the columns at a
-    // time; CTA `split` then writes columns [128 split / C, 128 (split+1) / C)
-    // of each half: the sum over the splits read through distributed shared memory
-    float* stage = reinterpret_cast<float*>(&s.kv[0][0][0]);
-    for (int half = 0; half < 2; ++half) {
-      if (warp >= 2) {
-        const int quad = warp & 3, grp = (warp - 2) >> 2;
-        const int hh = quad * 32 + lane;
-        const uint32_t ob = tmem + ((uint32_t)(quad * 32) << 16) + 256;
-        const float fs = s.mg.fself[hh], fnn = fs * s.mg.rfn[hh];
-        const int c = half * 128 + grp * 32;
-        uint32_t r[32];
-        tmem_ld32_nowait(ob + c, r);
-        tmem_ld_wait();
-        const float f = (dh == 1 && c >= 192) ? fs : fnn;
-        float4* dst = reinterpret_cast<float4*>(stage + hh * SSTH + grp * 32);
+  } else if (merge_ok) {
+    // (5) this CTA's column groups of every row, summed over the C partials
+    const int g0 = 64 * split / C, g1 = 64 * (split + 1) / C, ng = g1 - g0;
+    const float* po0 = P.part_o + (int64_t)(blockIdx.x - split) * (128 * 256);
+    for (int it = tid; it < 128 * ng; it += NTHR) {
+      const int hh = it / ng, col = 4 * (g0 + it % ng);
+      if (hh >= P.H) continue;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      int r = 0;
+      for (; r + 4 <= C; r += 4) {                     // four loads in flight
+        float4 b[4];
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          dst[k] = make_float4(__uint_as_float(r[4 * k]) * f, __uint_as_float(r[4 * k + 1]) * f,
-                               __uint_as_float(r[4 * k + 2]) * f, __uint_as_float(r[4 * k + 3]) * f);
-      }
-      __syncthreads();
-      cl.sync();                                  // every split's half staged
-      const int c0 = 128 * split / C, c1 = 128 * (split + 1) / C;
-      const int ng = (c1 - c0) / 4;
-      for (int it = tid; it < 128 * ng; it += NTHR) {
-        const int hh = it / ng, col = c0 + 4 * (it % ng);
-        if (hh >= P.H) continue;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int r = 0; r < C; ++r) {
-          const float4 b = *reinterpret_cast<const float4*>(
-              cl.map_shared_rank(stage, (unsigned)r) + hh * SSTH + col);
-          a.x += b.x;
-          a.y += b.y;
-          a.z += b.z;
-          a.w += b.w;
+        for (int u = 0; u < 4; ++u)
+          b[u] = __ldcg(reinterpret_cast<const float4*>(po0 + (int64_t)(r + u) * (128 * 256) + hh * 256 + col));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float f = fac[(r + u) * 128 + hh];
+          a.x = fmaf(f, b[u].x, a.x);
+          a.y = fmaf(f, b[u].y, a.y);
+          a.z = fmaf(f, b[u].z, a.z);
+          a.w = fmaf(f, b[u].w, a.w);
         }
-        emit4(hh, half * 128 + col, a);
       }
-      cl.sync();                                  // the stage is read before it is reused
+      for (; r < C; ++r) {
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(po0 + (int64_t)r * (128 * 256) + hh * 256 + col));
+        const float f = fac[r * 128 + hh];
+        a.x = fmaf(f, b.x, a.x);
+        a.y = fmaf(f, b.y, a.y);
+        a.z = fmaf(f, b.z, a.z);
+        a.w = fmaf(f, b.w, a.w);
+      }
+      emit4(hh, col, a);
     }
   }
   tc_fence_before();
@@ -799,49 +834,32 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 64) return cudaErrorInvalidDevice;
-  // per device: the largest cluster size whose clusters can all be resident
-  // for a given cluster count (queried once per size)
-  static int max_active[64][5];                  // sizes 1, 2, 4, 8, 16; 0 = not queried
-  static bool configured[64] = {false};
-  if (!configured[dev]) {
+  // per device: CTAs that can be resident at once (one per SM)
+  static int resident[64] = {0};
+  if (resident[dev] == 0) {
     cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    if (cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-        cudaSuccess)
-      cudaGetLastError();                        // 16-CTA clusters then report 0 below
-    for (int k = 0; k < 5; ++k) {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(1u << k, 1, 1);
-      cfg.blockDim = dim3(NTHR, 1, 1);
-      cfg.dynamicSmemBytes = smem;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = 1u << k;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, mqa_tc_kernel, &cfg) != cudaSuccess) {
-        cudaGetLastError();
-        n = 0;
-      }
-      max_active[dev][k] = n;
-    }
-    configured[dev] = true;
+    int per_sm = 0, n_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mqa_tc_kernel, NTHR, smem);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    resident[dev] = std::max(1, per_sm * n_sm);
   }
-  // key splits per (query, half) = CTAs per cluster: the largest power of two
-  // that keeps every cluster of the launch resident at once on this GPU (one
-  // CTA per SM), at most the query's key tiles, at least 1
+  // key splits per (query, half): as many as keep every CTA of the launch
+  // resident (at most kMqaTcMaxCtas, kMaxSplit, the query's key tiles); one
+  // when fewer than two fit, which needs no partials and no grid barrier
   MqaParams Q = P;
   const int64_t n_main = P.idx ? (int64_t)P.n_sel : P.max_vis;
   const int64_t tiles = (n_main + NK - 1) / NK + (P.n_win + NK - 1) / NK;
   const int64_t units = 2 * (int64_t)P.n_q;
-  int k = 4;
-  while (k > 0 && ((1ll << k) > tiles || max_active[dev][k] < units)) --k;
-  Q.n_split = 1 << k;
-  const int64_t grid = units * Q.n_split;
+  const int64_t cap = std::min<int64_t>(resident[dev], kMqaTcMaxCtas);
+  int64_t C = 1;
+  if (units * 2 <= cap) C = std::max<int64_t>(1, std::min<int64_t>({cap / units, tiles, (int64_t)kMaxSplit}));
+  Q.n_split = (int)C;
+  if (C > 1 && (Q.part_o == nullptr || Q.part_ml == nullptr || Q.grid_bar == nullptr))
+    return cudaErrorInvalidValue;
+  const int64_t grid = units * C;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
   if (!P.q_ready) mqa_tc_qprep_kernel<<<dim3((unsigned)P.n_q, 8), 64, 0, st>>>(P);
   cudaLaunchConfig_t cfg = {};
@@ -850,12 +868,10 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)Q.n_split;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  attr[0].id = cudaLaunchAttributeCooperative;        // the grid barrier needs every CTA resident
+  attr[0].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = C > 1 ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, mqa_tc_kernel, Q, m);
 }
 

@@ -121,6 +121,42 @@ __device__ __forceinline__ bool mbar_wait_at(uint64_t* bar, uint32_t parity, uin
   return false;
 }
 
+// Barrier of all n CTAs of a cooperative launch (co-resident by construction),
+// taken by one thread of each CTA after a __syncthreads that follows the CTA's
+// writes; the CTA's other threads wait at a __syncthreads after it.  `count`
+// and `gen` are words of the workspace header; gen0 is `gen` as the CTA read it
+// when it started (a barrier completes only after every CTA has arrived, so
+// no CTA can read the new generation there).  The last CTA to arrive returns
+// the count to zero and publishes the next generation; the others poll it.
+// Bounded like mbar_wait: false on expiry or when `status` records a timeout.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ bool grid_barrier(uint32_t* count, uint32_t* gen, uint32_t gen0,
+                                             uint32_t n, const uint32_t* status,
+                                             uint32_t limit_ns = (uint32_t)kWaitNs) {
+  __threadfence();
+  uint32_t old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(count) : "memory");
+  if (old == n - 1) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(count) : "memory");
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(gen), "r"(gen0 + 1u) : "memory");
+    return true;
+  }
+  const uint32_t t0 = (uint32_t)global_ns();
+  for (;;) {
+    if (ld_acquire_gpu(gen) != gen0) return true;
+    const uint32_t dt = (uint32_t)global_ns() - t0;
+    if (dt > limit_ns) return false;
+    if (status && dt > (uint32_t)kStatusPollNs &&
+        (*reinterpret_cast<const volatile uint32_t*>(status) & kStatusTimeout))
+      return false;
+    __nanosleep(32);
+  }
+}
+
 // The same wait taken by all 32 lanes of a warp, with one answer for all of
 // them: a warp never splits at a timeout, so the warp-wide (.sync.aligned)
 // tcgen05 loads and stores that follow always see every lane.
