@@ -80,28 +80,31 @@ struct Smem {
   // from bf16) for this CTA's 256 output dims: four MN-major SW128 blocks of
   // 64 dims x NK keys, the B operand of P V
   alignas(1024) uint8_t v16[4][NK * 128];
-  float kscale[KST][NK];
+  alignas(16) float kscale[KST][NK];
   union {
     float xmax[2][KG][128];                   // tile loop: [tile parity][key group][row]
     struct {                                  // merge (the loop is over for every warp):
       float rms[128], rl[128];                // this split's row max (log2), row sum
       float fself[128], invl[128];            // merge factor of this split, 1 / denominator
-      float rcs[32], rsn[32];                 // RoPE angles of the query position
     } mg;
   };
+  float rcs[32], rsn[32];                     // RoPE angles of the query position (dh = 1)
+  int verdict;                                // the grid barrier's outcome, for the whole CTA
   float xl[KG - 1][128];                      // the other groups' row sums, for the epilogue
-  uint64_t full[KST], empty[KST], sfull[2], pfull[2], pdone[2], xbar[2];
+  uint64_t full[KST], empty[KST], sfull[2], pfull[2], pdone[2], xbar[4][2];
   uint64_t qready, ofinal, done, lbar;
   uint32_t tmem_base;
 };
 
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory per CTA");
 static_assert(offsetof(Smem, qsc) == QTILE, "the query image is one contiguous copy");
-// the merge stages this split's O (fp32, 128 rows of SST floats) over the query
-// image and the key stages, which are free once the last P.V has completed
-constexpr int SST = 260;                     // row stride (floats): conflict-free float4 rows
+// the merge stages this split's O / l (f16, 128 rows of SSTB bytes) over the
+// query image and the key stages, which are free once the last P.V has completed
+constexpr int SSTB = 528;                    // staged f16 row stride (bytes): conflict-free 16-byte rows
 constexpr int kMaxSplit = 64;                // key splits per (query, half), at most
-static_assert(offsetof(Smem, kscale) >= 128 * SST * 4, "merge stage fits");
+constexpr int kMinSplitTiles = 3;            // dense calls: key tiles per split, at least
+constexpr int kWinCost = 2;                  // a gathered window tile costs about two contiguous ones
+static_assert(offsetof(Smem, kscale) >= 128 * SSTB, "merge stage fits");
 static_assert(offsetof(Smem, kscale) >= 2 * kMaxSplit * 128 * 4, "merge factors fit");
 // TMEM column of P (f16, two keys a column, 32 columns) inside a tile's
 // 128-column S buffer, written after the buffer's S has been read
@@ -268,9 +271,18 @@ __device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
   if (g.n_swa < 0) g.n_swa = 0;
   g.nmp = (g.n_main + NK - 1) / NK * NK;
   g.total = g.nmp + (g.n_swa + NK - 1) / NK * NK;
-  // split `split` of C takes tiles [T * split / C, T * (split + 1) / C) of the query's T
-  const int T = g.total / NK, C = P.n_split;
-  const int t0 = (int)((int64_t)T * split / C), t1 = (int)((int64_t)T * (split + 1) / C);
+  // The query's tiles, entries first then window tokens, are split by cost:
+  // a window tile (rows gathered from the ring) counts kWinCost entry tiles
+  // of a dense call (contiguous rows, one tile-mode copy each); in a sparse
+  // call every tile is gathered and counts one.  Split `split` of C takes
+  // the tiles whose cost prefix starts in [W split / C, W (split + 1) / C).
+  const int mt = g.nmp / NK, wt = (g.total - g.nmp) / NK, C = P.n_split;
+  const int wc = P.idx ? 1 : kWinCost;
+  const int64_t W = mt + (int64_t)wc * wt;
+  auto tile_at = [&](int64_t x) -> int {        // first tile whose cost prefix is >= x
+    return (int)(x <= mt ? x : mt + (x - mt + wc - 1) / wc);
+  };
+  const int t0 = tile_at(W * split / C), t1 = tile_at(W * (split + 1) / C);
   g.s0 = t0 * NK;
   g.T = t1 - t0;
   return g;
@@ -309,13 +321,13 @@ __global__ void __launch_bounds__(NTHR, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < KST; ++i) {
       mbar_init(&s.full[i], 32);   // the producer lanes' scale arrivals + TMA bytes
-      mbar_init(&s.empty[i], 1);
+      mbar_init(&s.empty[i], NSM);   // every softmax warp, done with the stage
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.sfull[i], 1);     // QK of the buffer's tile done (one commit)
       mbar_init(&s.pfull[i], NSM);   // every softmax warp wrote its P of the tile
       mbar_init(&s.pdone[i], 1);     // PV of the buffer's tile done (one commit)
-      mbar_init(&s.xbar[i], NSM);
+      for (int qd = 0; qd < 4; ++qd) mbar_init(&s.xbar[qd][i], KG);   // the quarter's key groups
     }
     mbar_init(&s.qready, 1);
     mbar_init(&s.ofinal, 1);
@@ -425,6 +437,14 @@ __global__ void __launch_bounds__(NTHR, 1)
       }
     }
     __syncwarp();
+    // the angles of the output's inverse RoPE (dims 448..511, one pair a
+    // lane), computed here while the other warps still work through the tiles
+    if (dh == 1) {
+      float c = 1.f, sv = 0.f;
+      if (g.p >= 0) rope_cs(g.p, lane, 64, P.theta, c, sv);
+      s.rcs[lane] = c;
+      s.rsn[lane] = sv;
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     const uint64_t kq128 = smem_desc_bits(16, 1024, 2);   // K-major, 128B swizzle
@@ -439,7 +459,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     // (tt & 1, written there by the softmax), B = the tile's V in f16
     // (s.v16, converted by the softmax warps), N = this CTA's 256 dims
     auto pv = [&](int tt) -> bool {
-      const int st = tt % KST, a = tt & 1;
+      const int a = tt & 1;
       if (!mbar_wait_warp(&s.pfull[a], (tt >> 1) & 1, P.status, 2)) return false;
       tc_fence_after();
       if (lane == 0) {
@@ -447,7 +467,6 @@ __global__ void __launch_bounds__(NTHR, 1)
         const uint64_t bv = smem_desc(s.v16[0], mn128);
         for (int ks = 0; ks < 4; ++ks)                        // 16 keys (8 columns) a step
           mma_f16_ts(O, pb + 8 * ks, bv + (uint64_t)(ks * 16 * 128 >> 4), id_pv, (tt | ks) != 0);
-        tc_commit(&s.empty[st]);
         tc_commit(&s.pdone[a]);
       }
       __syncwarp();
@@ -515,8 +534,12 @@ __global__ void __launch_bounds__(NTHR, 1)
       const uint32_t tb = tmem + lane_off + a * 128;     // this tile's TMEM buffer
       tmem_ld16_nowait(tb + grp * KPG, sn_);
       tmem_ld16_nowait(tb + 64 + grp * KPG, sr_);
+      float ksc[KPG];
+#pragma unroll
+      for (int j = 0; j < KPG; j += 4)
+        *reinterpret_cast<float4*>(&ksc[j]) =
+            *reinterpret_cast<const float4*>(&s.kscale[st][grp * KPG + j]);
       tmem_ld_wait();
-      const float* ksc = &s.kscale[st][grp * KPG];
       float s2[KPG];
       float ms = -INFINITY;
 #pragma unroll
@@ -526,12 +549,13 @@ __global__ void __launch_bounds__(NTHR, 1)
         s2[j] = (kj != 0.f) ? v : -INFINITY;             // a zero scale marks an empty slot
         ms = fmaxf(ms, s2[j]);
       }
-      // the tile's row maximum: exchanged with the other key groups; past this
-      // exchange every group has read its S columns, so P may overwrite them
+      // the tile's row maximum: exchanged with the other key groups of the
+      // same TMEM lane quarter (the same head rows); past this exchange every
+      // group has read its S columns, so P may overwrite them
       s.xmax[xb][grp][h] = ms;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.xbar[xb]);
-      if (!mbar_wait_warp(&s.xbar[xb], (t >> 1) & 1, P.status, 10)) {
+      if (lane == 0) mbar_arrive(&s.xbar[quad][xb]);
+      if (!mbar_wait_warp(&s.xbar[quad][xb], (t >> 1) & 1, P.status, 10)) {
         live = false;
         break;
       }
@@ -553,8 +577,8 @@ __global__ void __launch_bounds__(NTHR, 1)
         ph[j >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
       }
       l = l * as + lsum;
-      // the previous tile's P.V has completed: O may be rescaled and the
-      // f16 V buffer rewritten
+      // the previous tile's P.V has completed: O may be rescaled and the f16
+      // V buffer rewritten
       if (t >= 1 && !mbar_wait_warp(&s.pdone[(t - 1) & 1], ((t - 1) >> 1) & 1, P.status, 8)) {
         live = false;
         break;
@@ -578,9 +602,12 @@ __global__ void __launch_bounds__(NTHR, 1)
       }
       Ms = Ms_new;
       // this group's 16 keys of P into the tile's TMEM buffer (columns
-      // PC_F16 + 8 grp ..), and this thread's share of the tile's V in f16
+      // PC_F16 + 8 grp ..), and this thread's share of the tile's V in f16;
+      // then the stage goes back to the producer (V converted, scales read)
       tmem_st8(tb + PC_F16 + 8 * grp, ph);
       convert_v(s, st, dh, ctid);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.empty[st]);
       fence_proxy_async_smem();                          // V16 visible to the tensor core
       tmem_st_wait();
       tc_fence_before();
@@ -623,36 +650,43 @@ __global__ void __launch_bounds__(NTHR, 1)
   tc_fence_before();
   __syncthreads();
   const float log2e = 1.4426950408889634f;
-  float* stage = reinterpret_cast<float*>(&s.q[0]);    // q .. kv3: free, every MMA / copy is done
-  float* fac = stage;                                   // [C][128] row factors (after the copy-out)
-  float* lsp = stage + C * 128;                         // [C][128] row sums
+  uint8_t* stage = &s.q[0];                             // q .. kv3: free, every MMA / copy is done
+  float* fac = reinterpret_cast<float*>(stage);         // [C][128] row factors (after the copy-out)
+  float* lsp = fac + C * 128;                           // [C][128] row sums
   bool merge_ok = true;
   if (C > 1) {
-    // (1) this split's O as fp32 rows of SST floats
+    // (1) this split's O / l (a weighted mean of V rows: inside f16's range)
+    // as f16 rows of SSTB bytes
     if (warp >= 2) {
       const int quad = warp & 3, grp = (warp - 2) >> 2;
       const int hh = quad * 32 + lane;
       const uint32_t ob = tmem + ((uint32_t)(quad * 32) << 16) + 256;
+      const float lr = s.mg.rl[hh];
+      const float il = lr > 0.f ? 1.f / lr : 0.f;
 #pragma unroll 1
       for (int cc = 0; cc < 256 / KG; cc += 32) {
         const int c = grp * (256 / KG) + cc;
         uint32_t r[32];
         tmem_ld32_nowait(ob + c, r);
         tmem_ld_wait();
-        float4* dst = reinterpret_cast<float4*>(stage + hh * SST + c);
+        uint32_t hv[16];
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          dst[k] = make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
-                               __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
+        for (int k = 0; k < 16; ++k) {
+          const __half2 hp = __floats2half2_rn(__uint_as_float(r[2 * k]) * il,
+                                               __uint_as_float(r[2 * k + 1]) * il);
+          hv[k] = *reinterpret_cast<const uint32_t*>(&hp);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(stage + hh * SSTB + c * 2);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dst[k] = make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
       }
     }
     __syncthreads();
-    // (2) to this CTA's partial: [128][256] fp32, then [row max | row sum][128]
-    float* po = P.part_o + (int64_t)blockIdx.x * (128 * 256);
+    // (2) to this CTA's partial: [128][256] f16, then [row max | row sum][128] fp32
+    uint4* po = reinterpret_cast<uint4*>(P.part_o) + (int64_t)blockIdx.x * (128 * 256 / 8);
     float* pm = P.part_ml + (int64_t)blockIdx.x * 256;
-    for (int i = tid; i < 128 * 64; i += NTHR)
-      __stcg(reinterpret_cast<float4*>(po) + i,
-             *reinterpret_cast<const float4*>(stage + (i >> 6) * SST + (i & 63) * 4));
+    for (int i = tid; i < 128 * 32; i += NTHR)
+      __stcg(po + i, *reinterpret_cast<const uint4*>(stage + (i >> 5) * SSTB + (i & 31) * 16));
     if (tid < 128) {
       __stcg(pm + tid, s.mg.rms[tid]);
       __stcg(pm + 128 + tid, s.mg.rl[tid]);
@@ -662,25 +696,39 @@ __global__ void __launch_bounds__(NTHR, 1)
     if (tid == 0) {
       const bool ok = grid_barrier(P.grid_bar, P.grid_bar + 1, bar_gen0, gridDim.x, P.status);
       if (!ok) flag(P.status, ST_TIMEOUT | (1u << (16 + 13)));
-      s.mg.rcs[0] = ok ? 1.f : 0.f;                      // the verdict, for the whole CTA
+      s.verdict = ok ? 1 : 0;
     }
     __syncthreads();
-    merge_ok = s.mg.rcs[0] != 0.f;
-    __syncthreads();
-    // (4) the C splits' row maxima and sums of this (query, half)
+    merge_ok = s.verdict != 0;
+    // (4) the C splits' row maxima and sums of this (query, half): every
+    // thread's loads issued before its stores (C <= 64: at most 15 a thread)
     if (merge_ok) {
       const float* pm0 = P.part_ml + (int64_t)(blockIdx.x - split) * 256;
-      for (int i = tid; i < C * 128; i += NTHR) {
-        const int r = i >> 7, hh = i & 127;
-        fac[i] = __ldcg(pm0 + r * 256 + hh);
-        lsp[i] = __ldcg(pm0 + r * 256 + 128 + hh);
+      constexpr int PER = (kMaxSplit * 128 + NTHR - 1) / NTHR;
+      float mv[PER], lv[PER];
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int i = tid + u * NTHR;
+        if (i < C * 128) {
+          mv[u] = __ldcg(pm0 + (i >> 7) * 256 + (i & 127));
+          lv[u] = __ldcg(pm0 + (i >> 7) * 256 + 128 + (i & 127));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int i = tid + u * NTHR;
+        if (i < C * 128) {
+          fac[i] = mv[u];
+          lsp[i] = lv[u];
+        }
       }
     }
     __syncthreads();
   }
   if (tid < 128) {
     // the merged row maximum (with the sink, log2 units) and denominator; the
-    // factor exp2(max_r - M) of each split
+    // factor of each split: exp2(max_r - M) for O (C = 1), times l_r for the
+    // normalised partials O_r / l_r (C > 1)
     const int hh = tid;
     const float z = (P.sink && hh < P.H) ? P.sink[hh] * log2e : -INFINITY;
     float M = z;
@@ -697,21 +745,15 @@ __global__ void __launch_bounds__(NTHR, 1)
     } else {
       for (int r = 0; r < C; ++r) {
         const float mr = fac[r * 128 + hh];
-        const float f = (M != -INFINITY && mr != -INFINITY) ? ex2f(mr - M) : 0.f;
+        const float f = (M != -INFINITY && mr != -INFINITY) ? ex2f(mr - M) * lsp[r * 128 + hh] : 0.f;
         fac[r * 128 + hh] = f;
-        den += f * lsp[r * 128 + hh];
+        den += f;
       }
     }
     if (M != -INFINITY && z != -INFINITY) den += ex2f(z - M);
     s.mg.invl[hh] = den > 0.f ? 1.f / den : 0.f;
     if (P.lse && dh == 0 && split == 0 && hh < P.H && merge_ok)
       P.lse[(int64_t)q * P.H + hh] = den > 0.f ? M * 0.6931471805599453f + logf(den) : -INFINITY;
-  } else if (tid >= 160 && tid < 192 && dh == 1) {
-    // rotation by -p of the output's RoPE dims: the angles of the 32 pairs
-    float c = 1.f, sv = 0.f;
-    if (g.p >= 0) rope_cs(g.p, tid - 160, 64, P.theta, c, sv);
-    s.mg.rcs[tid - 160] = c;
-    s.mg.rsn[tid - 160] = sv;
   }
   __syncthreads();
   const int64_t obase = (int64_t)q * P.H * 512 + dh * 256;
@@ -724,7 +766,7 @@ __global__ void __launch_bounds__(NTHR, 1)
 #pragma unroll
       for (int e = 0; e < 4; e += 2) {
         const int k = (col + e - 192) >> 1;
-        const float cs = s.mg.rcs[k], sn = s.mg.rsn[k];
+        const float cs = s.rcs[k], sn = s.rsn[k];
         const float r0 = o[e] * cs + o[e + 1] * sn, r1 = -o[e] * sn + o[e + 1] * cs;
         o[e] = r0;
         o[e + 1] = r1;
@@ -762,33 +804,27 @@ __global__ void __launch_bounds__(NTHR, 1)
   } else if (merge_ok) {
     // (5) this CTA's column groups of every row, summed over the C partials
     const int g0 = 64 * split / C, g1 = 64 * (split + 1) / C, ng = g1 - g0;
-    const float* po0 = P.part_o + (int64_t)(blockIdx.x - split) * (128 * 256);
+    const uint2* po0 = reinterpret_cast<const uint2*>(P.part_o) + (int64_t)(blockIdx.x - split) * (128 * 64);
     for (int it = tid; it < 128 * ng; it += NTHR) {
       const int hh = it / ng, col = 4 * (g0 + it % ng);
       if (hh >= P.H) continue;
       float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-      int r = 0;
-      for (; r + 4 <= C; r += 4) {                     // four loads in flight
-        float4 b[4];
+      for (int r0 = 0; r0 < C; r0 += 8) {              // eight loads in flight
+        uint2 b[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          b[u] = __ldcg(reinterpret_cast<const float4*>(po0 + (int64_t)(r + u) * (128 * 256) + hh * 256 + col));
+        for (int u = 0; u < 8; ++u)
+          if (r0 + u < C) b[u] = __ldcg(po0 + (int64_t)(r0 + u) * (128 * 64) + hh * 64 + (col >> 2));
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float f = fac[(r + u) * 128 + hh];
-          a.x = fmaf(f, b[u].x, a.x);
-          a.y = fmaf(f, b[u].y, a.y);
-          a.z = fmaf(f, b[u].z, a.z);
-          a.w = fmaf(f, b[u].w, a.w);
-        }
-      }
-      for (; r < C; ++r) {
-        const float4 b = __ldcg(reinterpret_cast<const float4*>(po0 + (int64_t)r * (128 * 256) + hh * 256 + col));
-        const float f = fac[r * 128 + hh];
-        a.x = fmaf(f, b.x, a.x);
-        a.y = fmaf(f, b.y, a.y);
-        a.z = fmaf(f, b.z, a.z);
-        a.w = fmaf(f, b.w, a.w);
+        for (int u = 0; u < 8; ++u)
+          if (r0 + u < C) {
+            const float f = fac[(r0 + u) * 128 + hh];
+            const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&b[u].x));
+            const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&b[u].y));
+            a.x = fmaf(f, lo.x, a.x);
+            a.y = fmaf(f, lo.y, a.y);
+            a.z = fmaf(f, hi.x, a.z);
+            a.w = fmaf(f, hi.y, a.w);
+          }
       }
       emit4(hh, col, a);
     }
@@ -847,15 +883,21 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
     resident[dev] = std::max(1, per_sm * n_sm);
   }
   // key splits per (query, half): as many as keep every CTA of the launch
-  // resident (at most kMqaTcMaxCtas, kMaxSplit, the query's key tiles); one
-  // when fewer than two fit, which needs no partials and no grid barrier
+  // resident (at most kMqaTcMaxCtas and kMaxSplit) while each split keeps at
+  // least kMinSplitTiles key tiles in a dense call (a split's fixed cost, its
+  // start and its share of the merge, is worth about that many contiguous
+  // tiles; gathered tiles are bound by the copy engine of their SM, so a
+  // sparse call spreads them over as many SMs as it can); one when fewer
+  // than two fit, which needs no partials and no grid barrier
   MqaParams Q = P;
   const int64_t n_main = P.idx ? (int64_t)P.n_sel : P.max_vis;
   const int64_t tiles = (n_main + NK - 1) / NK + (P.n_win + NK - 1) / NK;
   const int64_t units = 2 * (int64_t)P.n_q;
   const int64_t cap = std::min<int64_t>(resident[dev], kMqaTcMaxCtas);
   int64_t C = 1;
-  if (units * 2 <= cap) C = std::max<int64_t>(1, std::min<int64_t>({cap / units, tiles, (int64_t)kMaxSplit}));
+  if (units * 2 <= cap)
+    C = std::max<int64_t>(1, std::min<int64_t>({cap / units, P.idx ? tiles : tiles / kMinSplitTiles,
+                                               (int64_t)kMaxSplit}));
   Q.n_split = (int)C;
   if (C > 1 && (Q.part_o == nullptr || Q.part_ml == nullptr || Q.grid_bar == nullptr))
     return cudaErrorInvalidValue;
