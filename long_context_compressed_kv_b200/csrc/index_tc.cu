@@ -95,15 +95,21 @@ __device__ __forceinline__ void locate(const Smem& s, int n_q, int g, TileIter& 
   t.lt = g - s.tile_prefix[t.q];
 }
 
-// Tiles in the stage that starts at tile g: up to TPS, all of one query, all
-// inside this CTA's range.  Every role walks the stages with this same rule.
-__device__ __forceinline__ int stage_tiles(const Smem& s, const TileIter& t, int g, int g1) {
+// Tiles in the stage that starts at tile g: up to `tps` (at most TPS and at
+// most the accumulator count, so that the tiles of one stage never wait for
+// each other's accumulator: the epilogue frees a stage's accumulators only
+// after that stage's single commit), all of one query group, all inside this
+// CTA's range.  Every role walks the stages with this same rule.
+__device__ __forceinline__ int stage_tiles(const Smem& s, const TileIter& t, int g, int g1, int tps) {
   const int to_seg = s.tile_prefix[t.q + 1] - g, to_end = g1 - g;
   const int n = to_seg < to_end ? to_seg : to_end;
-  return n < TPS ? n : TPS;
+  return n < tps ? n : tps;
 }
 
-template <int N>   // indexer heads = MMA N
+// N = MMA N: the indexer heads, or with PAIR two consecutive queries of one
+// sequence side by side (2 x H_I columns), so that every key tile serves both:
+// half the MMAs per score where many queries share their keys (prefill)
+template <int N, bool PAIR>
 __global__ void __launch_bounds__(NTHREADS, 1)
     index_tc_kernel(IndexParams P, const __grid_constant__ CUtensorMap tm_keys,
                     const __grid_constant__ CUtensorMap tm_q) {
@@ -113,11 +119,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int NACC = n_acc(N);
   static_assert(NACC >= 2 && NACC * (N + 4) + 8 <= (int)TM_COLS, "TMEM budget");
+  constexpr int TPS_N = NACC < TPS ? NACC : TPS;        // tiles per stage for this N
   constexpr bool W_IN_REGS = N <= 64;
+  constexpr int QPG = PAIR ? 2 : 1;                     // queries per MMA group
+  constexpr int HG = N / QPG;                           // heads of one query
+  const int n_g = P.n_q / QPG;                          // query groups (n_q even with PAIR)
   const uint32_t lim = P.wait_ns ? P.wait_ns : (uint32_t)kWaitNs;   // bound of every wait
 
-  // tiles per query, loaded in parallel, then a serial prefix over shared memory
-  for (int q = threadIdx.x; q < P.n_q; q += NTHREADS) {
+  // visible keys of query q (checked); a group's tiles cover its largest
+  auto visible = [&](int q) -> int64_t {
     int64_t nv = (P.q_pos[q] + 1) / P.m;
     const int b = P.q_seq ? P.q_seq[q] : P.q_base + q;
     if (b < 0 || b >= P.B) {
@@ -128,13 +138,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       flag(P.status, ST_BAD_POSITION);
       nv = min(P.key_rows, P.max_vis);
     }
+    return nv;
+  };
+  // tiles per query group, loaded in parallel, then a serial prefix over shared memory
+  for (int q = threadIdx.x; q < n_g; q += NTHREADS) {
+    int64_t nv = visible(q * QPG);
+    if (PAIR) nv = max(nv, visible(q * QPG + 1));
     s.tile_prefix[q + 1] = (int)((nv + KT - 1) / KT);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     int acc = 0;
     s.tile_prefix[0] = 0;
-    for (int q = 0; q < P.n_q; ++q) {
+    for (int q = 0; q < n_g; ++q) {
       acc += s.tile_prefix[q + 1];
       s.tile_prefix[q + 1] = acc;
     }
@@ -158,7 +174,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
 
-  const int total = s.tile_prefix[P.n_q];
+  const int total = s.tile_prefix[n_g];
   const int g0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
   const int g1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
   const uint32_t tmem = s.tmem_base;
@@ -182,11 +198,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int b = 0;                                  // sequence of the current query
     for (int g = g0; g < g1 && !aborted(); ++stg) {
       const int seg_before = t.seg;
-      locate(s, P.n_q, g, t);
-      const int n = stage_tiles(s, t, g, g1);
+      locate(s, n_g, g, t);
+      const int n = stage_tiles(s, t, g, g1, TPS_N);
       if (t.seg != seg_before) {
         // read once per query: a global load per stage would sit on the issue path
-        b = P.q_seq ? P.q_seq[t.q] : P.q_base + t.q;
+        b = P.q_seq ? P.q_seq[t.q * QPG] : P.q_base + t.q * QPG;
         const int j = t.seg & 1, uq = t.seg >> 1;
         if (uq >= 1 && !mbar_wait_warp(&s.qempty[j], (uq - 1) & 1, P.status, -1, lim)) {
           fail(s, P.status);
@@ -195,10 +211,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) {
           // query codes (TMA), query scales and head weights (bulk copies)
           mbar_arrive_expect_tx(&s.qfull[j], (uint32_t)(N * KROW + 2 * N * 4));
-          tma_load_2d(s.q[j], &tm_q, &s.qfull[j], 0, t.q * P.H_I);
-          bulk_load(s.sfb_raw[j], reinterpret_cast<const uint32_t*>(P.qI_sf) + (int64_t)t.q * P.H_I,
+          tma_load_2d(s.q[j], &tm_q, &s.qfull[j], 0, t.q * N);
+          bulk_load(s.sfb_raw[j], reinterpret_cast<const uint32_t*>(P.qI_sf) + (int64_t)t.q * N,
                     N * 4, &s.qfull[j]);
-          bulk_load(s.w[j], P.w + (int64_t)t.q * P.H_I, N * 4, &s.qfull[j]);
+          bulk_load(s.w[j], P.w + (int64_t)t.q * N, N * 4, &s.qfull[j]);
         }
         ++qissued;
       }
@@ -253,8 +269,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint64_t sf_bits = smem_desc_bits(16, 128, 0);            // 32 rows x 16 B
     for (int g = g0; ok && g < g1 && !aborted(); ++stg) {
       const int seg_before = t.seg;
-      locate(s, P.n_q, g, t);
-      const int n = stage_tiles(s, t, g, g1);
+      locate(s, n_g, g, t);
+      const int n = stage_tiles(s, t, g, g1, TPS_N);
       const int j = t.seg & 1;
       if (t.seg != seg_before) {
         if (!mbar_wait_warp(&s.qfull[j], (t.seg >> 1) & 1, P.status, -1, lim)) {
@@ -325,17 +341,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int quad = warp & 3;
     const int r = 4 * lane + quad;              // key of TMEM lane 32 * quad + lane
     {
-      // keys beyond the last tile of each query: -inf
+      // keys beyond the last tile of each query (group): -inf
       const int et = threadIdx.x - 64;
-      for (int q = blockIdx.x; q < P.n_q; q += gridDim.x) {
+      for (int q = blockIdx.x; q < n_g; q += gridDim.x) {
         const int64_t from = (int64_t)(s.tile_prefix[q + 1] - s.tile_prefix[q]) * KT;
-        for (int64_t i = from + et; i < P.max_vis; i += EPI_GROUPS * 128)
-          P.scores[(int64_t)q * P.scores_ld + i] = -INFINITY;
+        for (int u = 0; u < QPG; ++u)
+          for (int64_t i = from + et; i < P.max_vis; i += EPI_GROUPS * 128)
+            P.scores[(int64_t)(q * QPG + u) * P.scores_ld + i] = -INFINITY;
       }
     }
     TileIter t;
     float wreg[W_IN_REGS ? N : 1];
-    int64_t nv = 0;
+    int64_t nv = 0, nv2 = 0;                    // visible keys of the group's queries
     int stg = 0;
     // warp 2 lane 0 (group 0) is the releaser: it waits for every stage's
     // commit and then frees the ring stage (and, at a query's last stage, the
@@ -343,8 +360,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const bool releaser = warp == 2 && lane == 0;
     for (int g = g0; g < g1 && !aborted(); ++stg) {
       const int seg_before = t.seg;
-      locate(s, P.n_q, g, t);
-      const int n = stage_tiles(s, t, g, g1);
+      locate(s, n_g, g, t);
+      const int n = stage_tiles(s, t, g, g1, TPS_N);
       const int j = t.seg & 1;
       if (t.seg != seg_before) {
         if (!mbar_wait_warp(&s.qfull[j], (t.seg >> 1) & 1, P.status, -1, lim)) {
@@ -355,7 +372,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int h = 0; h < N; ++h) wreg[h] = s.w[j][h];
         }
-        nv = min((int64_t)(P.q_pos[t.q] + 1) / P.m, min(P.key_rows, P.max_vis));
+        nv = min((int64_t)(P.q_pos[t.q * QPG] + 1) / P.m, min(P.key_rows, P.max_vis));
+        if (PAIR) nv2 = min((int64_t)(P.q_pos[t.q * QPG + 1] + 1) / P.m, min(P.key_rows, P.max_vis));
       }
       const int st = stg % STAGES;
       const bool has_tile = n > 1 || ((g - g0) & 1) == grp;
@@ -376,7 +394,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if ((it & 1) != grp) continue;
         const int a = it % NACC;
         const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + a * N;
-        float s0 = 0.f, s1 = 0.f;
+        float s0 = 0.f, s1 = 0.f, u0 = 0.f, u1 = 0.f;   // even / odd heads; u: the second query
         constexpr int CH = N <= 64 ? N : 64;      // columns per TMEM round trip
 #pragma unroll
         for (int c0 = 0; c0 < N; c0 += CH) {
@@ -393,13 +411,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int h = 0; h < CH; h += 2) {
             const float w0 = W_IN_REGS ? wreg[(c0 + h) % (W_IN_REGS ? N : 1)] : s.w[j][c0 + h];
             const float w1 = W_IN_REGS ? wreg[(c0 + h + 1) % (W_IN_REGS ? N : 1)] : s.w[j][c0 + h + 1];
-            s0 = fmaf(w0, fmaxf(__uint_as_float(v[h]), 0.f), s0);
-            s1 = fmaf(w1, fmaxf(__uint_as_float(v[h + 1]), 0.f), s1);
+            if (c0 + h < HG) {
+              s0 = fmaf(w0, fmaxf(__uint_as_float(v[h]), 0.f), s0);
+              s1 = fmaf(w1, fmaxf(__uint_as_float(v[h + 1]), 0.f), s1);
+            } else {
+              u0 = fmaf(w0, fmaxf(__uint_as_float(v[h]), 0.f), u0);
+              u1 = fmaf(w1, fmaxf(__uint_as_float(v[h + 1]), 0.f), u1);
+            }
           }
         }
-        const float score = s0 + s1;
         const int64_t i = (int64_t)(t.lt + k) * KT + r;
-        if (i < P.max_vis) P.scores[(int64_t)t.q * P.scores_ld + i] = (i < nv) ? score : -INFINITY;
+        if (i < P.max_vis) {
+          P.scores[(int64_t)(t.q * QPG) * P.scores_ld + i] = (i < nv) ? s0 + s1 : -INFINITY;
+          if (PAIR)
+            P.scores[(int64_t)(t.q * QPG + 1) * P.scores_ld + i] = (i < nv2) ? u0 + u1 : -INFINITY;
+        }
       }
       if (seg_end) {
         __syncwarp();
@@ -504,28 +530,34 @@ int index_tc_check(const IndexParams& P) {
 cudaError_t launch_index_tc(const IndexParams& P, cudaStream_t st) {
   CUtensorMap tk, tq;
   if (!make_keys_map(&tk, P.keys, (int64_t)P.B * P.key_rows)) return cudaErrorInvalidValue;
-  if (!make_rows_map(&tq, P.qI, (int64_t)P.n_q * P.H_I, KROW, P.H_I)) return cudaErrorInvalidValue;
+  // two consecutive queries per MMA (N = 2 H_I) when every query belongs to
+  // the one sequence of the call and they pair up evenly
+  const bool pair = P.B == 1 && P.n_q >= 2 && P.n_q % 2 == 0 && P.H_I <= 64;
+  const int nmma = pair ? 2 * P.H_I : P.H_I;
+  if (!make_rows_map(&tq, P.qI, (int64_t)P.n_q * P.H_I, KROW, nmma)) return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
   static unsigned long long configured = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !(configured & (1ull << dev))) {
     cudaError_t e = cudaSuccess;
-    e = cudaFuncSetAttribute(index_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(index_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(index_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    for (const void* f : {(const void*)index_tc_kernel<32, false>, (const void*)index_tc_kernel<64, false>,
+                          (const void*)index_tc_kernel<128, false>, (const void*)index_tc_kernel<64, true>,
+                          (const void*)index_tc_kernel<128, true>})
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured |= 1ull << dev;
   }
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = sms;   // persistent: one CTA per SM, contiguous tile ranges
-  switch (P.H_I) {
-    case 32: index_tc_kernel<32><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
-    case 64: index_tc_kernel<64><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
-    case 128: index_tc_kernel<128><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
+  switch (nmma * (pair ? -1 : 1)) {
+    case 32: index_tc_kernel<32, false><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
+    case 64: index_tc_kernel<64, false><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
+    case 128: index_tc_kernel<128, false><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
+    case -64: index_tc_kernel<64, true><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
+    case -128: index_tc_kernel<128, true><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

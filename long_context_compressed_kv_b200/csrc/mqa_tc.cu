@@ -104,6 +104,7 @@ constexpr int SSTB = 528;                    // staged f16 row stride (bytes): c
 constexpr int kMaxSplit = 64;                // key splits per (query, half), at most
 constexpr int kMinSplitTiles = 3;            // dense calls: key tiles per split, at least
 constexpr int kWinCost = 2;                  // a gathered window tile costs about two contiguous ones
+constexpr int kFastSplits = 24;              // merges of at most this many splits load in one flight
 static_assert(offsetof(Smem, kscale) >= 128 * SSTB, "merge stage fits");
 static_assert(offsetof(Smem, kscale) >= 2 * kMaxSplit * 128 * 4, "merge factors fit");
 // TMEM column of P (f16, two keys a column, 32 columns) inside a tile's
@@ -700,9 +701,44 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     __syncthreads();
     merge_ok = s.verdict != 0;
+  }
+  // this CTA's column groups [g0, g1) of every row (four columns each); with
+  // few splits and at most one (row, group) item a thread, every partial the
+  // thread will sum is loaded together with the row statistics, so the whole
+  // merge waits for L2 once
+  const int g0 = 64 * split / C, g1 = 64 * (split + 1) / C, ng = g1 - g0;
+  const bool fast = C > 1 && C <= kFastSplits && 128 * ng <= NTHR;
+  const uint2* po0 = reinterpret_cast<const uint2*>(P.part_o) + (int64_t)(blockIdx.x - split) * (128 * 64);
+  const int f_hh = fast ? tid / max(ng, 1) : 0, f_col = fast ? 4 * (g0 + tid % max(ng, 1)) : 0;
+  const bool f_item = fast && tid < 128 * ng && f_hh < P.H;
+  uint2 pre[kFastSplits];
+  if (C > 1) {
     // (4) the C splits' row maxima and sums of this (query, half): every
     // thread's loads issued before its stores (C <= 64: at most 15 a thread)
-    if (merge_ok) {
+    if (merge_ok && fast) {
+#pragma unroll
+      for (int r = 0; r < kFastSplits; ++r)
+        if (r < C && f_item) pre[r] = __ldcg(po0 + (int64_t)r * (128 * 64) + f_hh * 64 + (f_col >> 2));
+      const float* pm0 = P.part_ml + (int64_t)(blockIdx.x - split) * 256;
+      constexpr int PERF = (kFastSplits * 128 + NTHR - 1) / NTHR;
+      float mv[PERF], lv[PERF];
+#pragma unroll
+      for (int u = 0; u < PERF; ++u) {
+        const int i = tid + u * NTHR;
+        if (i < C * 128) {
+          mv[u] = __ldcg(pm0 + (i >> 7) * 256 + (i & 127));
+          lv[u] = __ldcg(pm0 + (i >> 7) * 256 + 128 + (i & 127));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < PERF; ++u) {
+        const int i = tid + u * NTHR;
+        if (i < C * 128) {
+          fac[i] = mv[u];
+          lsp[i] = lv[u];
+        }
+      }
+    } else if (merge_ok) {
       const float* pm0 = P.part_ml + (int64_t)(blockIdx.x - split) * 256;
       constexpr int PER = (kMaxSplit * 128 + NTHR - 1) / NTHR;
       float mv[PER], lv[PER];
@@ -803,8 +839,23 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
   } else if (merge_ok) {
     // (5) this CTA's column groups of every row, summed over the C partials
-    const int g0 = 64 * split / C, g1 = 64 * (split + 1) / C, ng = g1 - g0;
-    const uint2* po0 = reinterpret_cast<const uint2*>(P.part_o) + (int64_t)(blockIdx.x - split) * (128 * 64);
+    if (fast) {
+      if (f_item) {
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < kFastSplits; ++r)
+          if (r < C) {
+            const float f = fac[r * 128 + f_hh];
+            const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&pre[r].x));
+            const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&pre[r].y));
+            a.x = fmaf(f, lo.x, a.x);
+            a.y = fmaf(f, lo.y, a.y);
+            a.z = fmaf(f, hi.x, a.z);
+            a.w = fmaf(f, hi.y, a.w);
+          }
+        emit4(f_hh, f_col, a);
+      }
+    } else
     for (int it = tid; it < 128 * ng; it += NTHR) {
       const int hh = it / ng, col = 4 * (g0 + it % ng);
       if (hh >= P.H) continue;

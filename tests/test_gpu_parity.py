@@ -168,6 +168,46 @@ def test_index_topk_parity(fp4, d_I, H_I):
         check_topk(g_idx[q], s, nv, k)
 
 
+@pytest.mark.parametrize("H_I,nq", [(64, 8), (32, 6), (64, 7), (128, 6)])
+def test_index_topk_one_sequence_pairs(H_I, nq):
+    """Queries of one sequence (B = 1): the tensor-core indexer scores two
+    consecutive queries per key tile when their count is even (7: every
+    query alone; H_I = 128: alone, N = 128).  Positions differ inside a pair,
+    down to one key.  16384 keys give every CTA several tiles, so that its
+    stages fill up to their tile limit (the accumulator count at N = 128)."""
+    v = v4()
+    rng = np.random.default_rng(H_I + nq)
+    N, k, d_I = 16384, 64, 128
+    keys = rng.standard_normal((1, N, d_I)).astype(np.float32)
+    positions = np.array([4 * N - 1, 4 * N - 5, 4 * 700 + 3, 4 * 700 + 4, 9, 4 * 129,
+                          4 * 1000 + 1, 4 * 1000 + 2])[:nq]
+    qI = rng.standard_normal((nq, H_I, d_I)).astype(np.float32)
+    w = rng.uniform(-0.2, 1, (nq, H_I)).astype(np.float32)
+    ly = synth.Layer("csa", 4, 16, 512, 64, 128, H_I, d_I, k, idx_fp4=True)
+    desc = desc_for(ly)
+    krows, ksf = code_rows(desc, dev(keys), v.MXFP4)
+    qrows, qsf = code_rows(desc, dev(qI.reshape(1, nq * H_I, d_I)), v.MXFP4)
+    qrows, qsf = qrows.reshape(nq, H_I, -1), qsf.reshape(nq, H_I, -1)
+    idx = torch.full((nq, k), -9, dtype=torch.int32, device="cuda")
+    scores = torch.zeros(nq, N, dtype=torch.float32, device="cuda")
+    ws = v.workspace(desc, nq, N)
+    v.index_topk(desc, qI=qrows, qI_sf=qsf, w=dev(w), q_pos=dev(positions, torch.int64),
+                 q_seq=dev(np.zeros(nq), torch.int32), B=1, keys=krows, keys_sf=ksf,
+                 key_rows=N, max_vis=N, idx_out=idx, scores_out=scores, ws=ws)
+    torch.cuda.synchronize()
+    assert v.device_status(ws) == 0
+    kd = read_keys(krows, ksf, v.MXFP4)
+    qd = read_keys(qrows, qsf, v.MXFP4)
+    g_idx, g_s = idx.cpu().numpy(), scores.cpu().numpy()
+    for q in range(nq):
+        nv = int(ocomp.n_visible(positions[q], 4))
+        s = oidx.scores(qd[q], w[q], kd[0, :nv])
+        scale = max(1.0, float(np.max(np.abs(s)))) if nv else 1.0
+        assert np.max(np.abs(g_s[q, :nv] - s), initial=0.0) <= 1e-5 * scale
+        assert np.all(np.isneginf(g_s[q, nv:]))
+        check_topk(g_idx[q], s, nv, k)
+
+
 def test_topk_ties_go_to_lower_index():
     """Many exactly equal scores: the selection must be the lowest indices."""
     v = v4()
