@@ -570,6 +570,49 @@ class Workload:
         return ins, outs
 
 
+def dominant_roofline(wl, flush, steps, stream, dist, peaks, abytes):
+    """The workload's dominant kernel timed alone as a graph replay (CUDA events
+    on its stream, L2 flushed between launches) against the HBM copy peak:
+    the CSA indexer (scores only) when the workload has a CSA layer, else the
+    HCA layer's dense MQA (query image + MQA).  Returns (roofline dict, ms)."""
+    import torch
+    import long_context_compressed_kv_b200 as v
+    csa = [lay for lay in wl.layers if lay.csa]
+    if csa:
+        lay = csa[0]
+        scores = torch.empty(lay.B, lay.max_vis, dtype=torch.float32, device="cuda")
+
+        def run():
+            v.index_topk(lay.desc, qI=lay.qI, qI_sf=lay.qI_sf, w=lay.w, q_pos=lay.pos,
+                         keys=lay.keys, keys_sf=lay.keys_sf, key_rows=lay.kv_rows,
+                         max_vis=lay.max_vis, idx_out=None, scores_out=scores, ws=lay.ws)
+        name, nbytes = "index_scores (CSA indexer, MXFP4 keys)", abytes["csa"]["index"]
+    else:
+        lay = wl.layers[0]
+
+        def run():
+            v.dense_mqa(lay.desc, Q=lay.Q, q_pos=lay.pos, kv=lay.kv, kv_scale=lay.kv_scale,
+                        kv_rows=lay.kv_rows, swa=lay.swa, swa_scale=lay.swa_scale,
+                        swa_rows=lay.swa_rows, max_vis=lay.max_vis, out=lay.out, ws=lay.ws,
+                        sink=lay.sink, lse=lay.lse)
+        name, nbytes = "dense_mqa (HCA shared-KV MQA, E4M3 entries)", abytes["hca"]["mqa"]
+    for _ in range(3):
+        flush()
+        run()
+    # timed as a graph replay: a direct call would also time the host-side enqueue
+    g = capture_graph(run)
+    t = float(np.mean(timed_device(g.replay, flush, steps, stream)))
+    t = max_over_ranks(t, dist)
+    achieved = nbytes / (t / 1e3) / 1e9
+    roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": _index_traffic() if csa and wl.w.name == HEADLINE else None,
+            "peak_source": peaks["source"], "launch_us": round(t * 1e3, 2),
+            "algorithmic_bytes": int(nbytes)}
+    del g
+    return roof, t
+
+
 def run_gpu(args, dist, rank, world):
     import torch
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
@@ -603,34 +646,11 @@ def run_gpu(args, dist, rank, world):
     q_step = wl.queries_per_step()
     value = job_value(ms, q_step, world)
 
-    # ---- dominant kernel: the indexer score kernel of the CSA layer, timed alone
-    import long_context_compressed_kv_b200 as v
-    csa = [lay for lay in wl.layers if lay.csa]
-    roof = None
-    abytes = algorithmic_bytes(wl.w)
+    # ---- dominant kernel, timed alone
     peaks = _peaks()
-    if csa:
-        lay = csa[0]
-        scores = torch.empty(lay.B, lay.max_vis, dtype=torch.float32, device="cuda")
-
-        def idx_only():
-            v.index_topk(lay.desc, qI=lay.qI, qI_sf=lay.qI_sf, w=lay.w, q_pos=lay.pos,
-                         keys=lay.keys, keys_sf=lay.keys_sf, key_rows=lay.kv_rows,
-                         max_vis=lay.max_vis, idx_out=None, scores_out=scores, ws=lay.ws)
-        for _ in range(3):
-            flush()
-            idx_only()
-        # timed as a graph replay: a direct call would also time the host-side enqueue
-        g_idx = capture_graph(idx_only)
-        t_idx = float(np.mean(timed_device(g_idx.replay, flush, max(args.steps, 10), stream)))
-        t_idx = max_over_ranks(t_idx, dist)
-        bytes_idx = abytes["csa"]["index"]
-        achieved = bytes_idx / (t_idx / 1e3) / 1e9
-        roof = {"kernel": "index_scores (CSA indexer, MXFP4 keys)", "bound": "hbm",
-                "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": _index_traffic(),
-                "peak_source": peaks["source"], "launch_us": round(t_idx * 1e3, 2),
-                "algorithmic_bytes": int(bytes_idx)}
+    abytes = algorithmic_bytes(wl.w)
+    roof, t_idx = dominant_roofline(wl, flush, max(args.steps, 10), stream, dist, peaks, abytes)
+    csa = [lay for lay in wl.layers if lay.csa]
     step_bytes = sum(sum(vv for kk, vv in d.items() if kk in ("index", "mqa"))
                      for d in abytes.values())
     step_roof = {"bytes": int(step_bytes), "us": round(ms * 1e3, 2),
@@ -665,7 +685,7 @@ def run_gpu(args, dist, rank, world):
     e2e_val = world * q_step / (e2e_ms / 1e3)
     e2e_eager = world * q_step / (e2e["eager"] / 1e3)
     peaks_tc = measure_tc_peaks(stream)
-    if roof is not None:
+    if roof is not None and csa:
         fp4 = abytes["csa"]["keys"] * 2 * csa[0].desc.H_I * csa[0].desc.d_I
         ach_t = fp4 / (t_idx / 1e3) / 1e12
         roof["tensor"] = {"format": "mxfp4", "flops_per_launch": int(fp4),
@@ -687,9 +707,11 @@ def run_gpu(args, dist, rank, world):
             t2 = float(np.mean(timed_device(w2.replay, flush, args.steps, stream)))
             b2 = algorithmic_bytes(w2.w)
             sb = sum(sum(vv for kk, vv in d.items() if kk in ("index", "mqa")) for d in b2.values())
+            r2, _ = dominant_roofline(w2, flush, max(args.steps, 10), stream, None, peaks, b2)
             also[name] = {"queries_per_s": round(w2.queries_per_step() / (t2 / 1e3), 1),
                           "us_per_step": round(t2 * 1e3, 2),
-                          "frac_hbm": round(sb / (t2 / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+                          "frac_hbm": round(sb / (t2 / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                          "roofline": r2}
             del w2
             torch.cuda.empty_cache()
     return dict(value=value, ms=ms, roof=roof, step_roof=step_roof, clocks=clk.summary(),
