@@ -694,6 +694,37 @@ def run_gpu(args, dist, rank, world):
                           "frac": round(ach_t / peaks_tc["fp4_mxf4_tflops"], 4),
                           "peak_source": "measured in this run (tcgen05 probe)"}
 
+    # ---- the BF16-score selector variant on the same CSA layer: index + top-k
+    # with fp32 scores against bf16 scores, and the recall of the bf16
+    # selection against the fp32 one
+    bf16_sel = None
+    if csa and world == 1:
+        import long_context_compressed_kv_b200 as v
+        lay = csa[0]
+        idx32 = torch.empty_like(lay.idx)
+        idx16 = torch.empty_like(lay.idx)
+        times = {}
+        for name, out_idx, sd in (("fp32", idx32, v.F32), ("bf16", idx16, v.BF16)):
+            def sel(out_idx=out_idx, sd=sd):
+                v.index_topk(lay.desc, qI=lay.qI, qI_sf=lay.qI_sf, w=lay.w, q_pos=lay.pos,
+                             keys=lay.keys, keys_sf=lay.keys_sf, key_rows=lay.kv_rows,
+                             max_vis=lay.max_vis, idx_out=out_idx, ws=lay.ws, score_dtype=sd)
+            for _ in range(3):
+                flush()
+                sel()
+            g_sel = capture_graph(sel)
+            times[name] = float(np.mean(timed_device(g_sel.replay, flush, max(args.steps, 10),
+                                                     stream)))
+            del g_sel
+        a32, a16 = idx32.cpu().numpy(), idx16.cpu().numpy()
+        rec = [len(np.intersect1d(a32[b][a32[b] >= 0], a16[b][a16[b] >= 0])) /
+               max(1, int((a32[b] >= 0).sum())) for b in range(a32.shape[0])]
+        bf16_sel = {"index_topk_us_fp32_scores": round(times["fp32"] * 1e3, 2),
+                    "index_topk_us_bf16_scores": round(times["bf16"] * 1e3, 2),
+                    "speedup": round(times["fp32"] / times["bf16"], 3),
+                    "recall_of_fp32_selection": round(float(np.mean(rec)), 4),
+                    "note": "synthetic N(0,1) keys and queries, not trained weights"}
+
     also = {}
     if not args.no_also and world == 1:
         del wl
@@ -717,6 +748,7 @@ def run_gpu(args, dist, rank, world):
     return dict(value=value, ms=ms, roof=roof, step_roof=step_roof, clocks=clk.summary(),
                 e2e=dict(value=e2e_val, h2d=h2d, d2h=d2h, ms=e2e_ms, eager_value=e2e_eager,
                          eager_ms=e2e["eager"]), also=also, tc_peaks=peaks_tc,
+                bf16_selector=bf16_sel,
                 launches=launches, q_step=q_step,
                 per_step=per_step)
 
@@ -1092,6 +1124,7 @@ def main():
             "cpu_baseline": cpu,
             "clocks": res["clocks"],
             "also": res["also"],
+            "bf16_score_selector": res.get("bf16_selector"),
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -141,7 +141,11 @@ typedef struct {
  * V4A_MXFP4 runs on the tcgen05 block-scaled tensor-core kernel only and needs
  * d_I = 128, H_I in {32, 64, 128} and key_rows % 4 == 0 (else
  * V4A_ERR_UNSUPPORTED), with qI, qI_sf, w, keys, keys_sf 16-byte aligned
- * (else V4A_ERR_INVALID_ARG).  */
+ * (else V4A_ERR_INVALID_ARG).
+ * score_dtype V4A_BF16 ([deep-read] "FP4 QAT、可恢复 rollout 与百万 Token RL":
+ * the selector on BF16 scores) rounds every score to bf16 (nearest even)
+ * before the top-k, which then selects exactly among those bf16 values (ties
+ * to the lower index); scores_out, if given, receives them as bf16.  */
 typedef struct {
   int32_t n_q;                /* queries, 1 .. 2^20 */
   int32_t B;                  /* sequences */
@@ -155,7 +159,9 @@ typedef struct {
   int64_t key_rows;           /* rows per sequence; n_vis(p) must not exceed it */
   int64_t max_vis;            /* upper bound of n_vis over the queries (<= key_rows) */
   int32_t* idx_out;           /* device [n_q][top_k]; NULL = scores only (scores_out required) */
-  float* scores_out;          /* device [n_q][max_vis] or NULL; entries >= n_vis are -inf */
+  void* scores_out;           /* device [n_q][max_vis] float (bf16 with score_dtype V4A_BF16)
+                                 or NULL; entries >= n_vis are -inf */
+  int32_t score_dtype;        /* V4A_F32 (0) or V4A_BF16 */
 } v4attn_index_args;
 
 /* ---------------------------------------------------------------- MQA

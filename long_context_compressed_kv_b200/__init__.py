@@ -110,11 +110,11 @@ def compress(desc: LayerDesc, *, m: int, overlap: bool, c: int, Ca, Za, Cb=None,
 
 def index_topk(desc: LayerDesc, *, qI, w, q_pos, keys, key_rows: int, max_vis: int, idx_out, ws,
                qI_sf=None, keys_sf=None, q_seq=None, B: Optional[int] = None, scores_out=None,
-               stream=None):
+               score_dtype: int = F32, stream=None):
     n_q = int(q_pos.numel())
     a = IndexArgs(n_q, B if B is not None else n_q, _p(qI), _p(qI_sf), _p(w), _p(q_seq),
                   _p(q_pos), _p(keys), _p(keys_sf), key_rows, max_vis, _p(idx_out),
-                  _p(scores_out))
+                  _p(scores_out), score_dtype)
     _check("v4attn_index_topk", _lib.v4attn_index_topk(ctypes.byref(desc), ctypes.byref(a),
                                                        _p(ws), ws.numel(), _stream(stream)))
 
@@ -127,7 +127,7 @@ def index_topk_noalloc(desc: LayerDesc, *, qI, w, q_pos, keys, key_rows: int, ma
     n_q = int(q_pos.numel())
     a = IndexArgs(n_q, B if B is not None else n_q, _p(qI), _p(qI_sf), _p(w), _p(q_seq),
                   _p(q_pos), _p(keys), _p(keys_sf), key_rows, max_vis, _p(idx_out),
-                  _p(scores_out))
+                  _p(scores_out), F32)
     _check("v4attn_index_topk_noalloc",
            _lib.v4attn_index_topk_noalloc(ctypes.byref(desc), ctypes.byref(a), _stream(stream)))
 
@@ -149,7 +149,7 @@ def debug_index_stall(desc: LayerDesc, *, qI, w, q_pos, keys, key_rows: int, max
     n_q = int(q_pos.numel())
     a = IndexArgs(n_q, B if B is not None else n_q, _p(qI), _p(qI_sf), _p(w), _p(q_seq),
                   _p(q_pos), _p(keys), _p(keys_sf), key_rows, max_vis, _p(idx_out),
-                  _p(scores_out))
+                  _p(scores_out), F32)
     _check("v4attn_debug_index_stall",
            _lib.v4attn_debug_index_stall(ctypes.byref(desc), ctypes.byref(a), _p(ws), ws.numel(),
                                          int(wait_ns), _stream(stream)))

@@ -41,7 +41,7 @@ class IndexArgs(ctypes.Structure):
     _fields_ = [("n_q", c_i32), ("B", c_i32), ("qI", c_ptr), ("qI_sf", c_ptr), ("w", c_ptr),
                 ("q_seq", c_ptr), ("q_pos", c_ptr), ("keys", c_ptr), ("keys_sf", c_ptr),
                 ("key_rows", c_i64), ("max_vis", c_i64), ("idx_out", c_ptr),
-                ("scores_out", c_ptr)]
+                ("scores_out", c_ptr), ("score_dtype", c_i32)]
 
 
 class MqaArgs(ctypes.Structure):

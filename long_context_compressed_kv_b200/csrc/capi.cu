@@ -176,6 +176,9 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
   if (!a->qI || !a->w || !a->q_pos || !a->keys || (!a->idx_out && !a->scores_out))
     return V4A_ERR_INVALID_ARG;
   if (d->idx_dtype == V4A_MXFP4 && (!a->qI_sf || !a->keys_sf)) return V4A_ERR_INVALID_ARG;
+  if (a->score_dtype != V4A_F32 && a->score_dtype != V4A_BF16) return V4A_ERR_INVALID_ARG;
+  const int sbf = a->score_dtype == V4A_BF16 ? 1 : 0;
+  const size_t s_esz = sbf ? 2 : 4;
   if (a->key_rows < 1 || a->max_vis < 0 || a->max_vis > a->key_rows) return V4A_ERR_INVALID_ARG;
   if (!ws) return V4A_ERR_WORKSPACE;
   if (ws_bytes < body_off + index_need(a->n_q, a->max_vis)) return V4A_ERR_WORKSPACE;
@@ -207,8 +210,10 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
   if (dry) return V4A_OK;
   for (int32_t q0 = 0; q0 < a->n_q; q0 += kQChunk) {
     const int32_t cn = std::min(kQChunk, a->n_q - q0);
-    float* scores = a->scores_out ? a->scores_out + (int64_t)q0 * ld
-                                  : reinterpret_cast<float*>(w8 + body_off);
+    float* scores = a->scores_out
+                        ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a->scores_out) +
+                                                   (size_t)q0 * ld * s_esz)
+                        : reinterpret_cast<float*>(w8 + body_off);
     if (a->max_vis > 0) {
       IndexParams P;
       P.n_q = cn;
@@ -229,6 +234,7 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
       P.max_vis = a->max_vis;
       P.scores = scores;
       P.scores_ld = ld;
+      P.score_bf16 = sbf;
       P.status = status;
       P.wait_ns = wait_ns;
       P.stall = stall;
@@ -241,6 +247,7 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
     T.k = d->top_k;
     T.scores = scores;
     T.scores_ld = ld;
+    T.score_bf16 = sbf;
     T.max_vis = a->max_vis;
     T.q_pos = a->q_pos + q0;
     T.idx_out = a->idx_out + (int64_t)q0 * d->top_k;

@@ -62,6 +62,16 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
   __nv_bfloat16 h = __float2bfloat16_rn(x);
   return *reinterpret_cast<uint16_t*>(&h);
 }
+// element i of a score row held as fp32, or as bf16 (round to nearest even)
+__device__ __forceinline__ void put_score(float* row, int64_t i, float v, int bf16) {
+  if (bf16)
+    reinterpret_cast<uint16_t*>(row)[i] = f32_to_bf16_bits(v);
+  else
+    row[i] = v;
+}
+__device__ __forceinline__ float get_score(const float* row, int64_t i, int bf16) {
+  return bf16 ? __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(row)[i] << 16) : row[i];
+}
 __device__ __forceinline__ float exp2i(int e) {   // 2^e for e in the normal range
   return __int_as_float((e + 127) << 23);
 }

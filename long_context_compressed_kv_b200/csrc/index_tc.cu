@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int64_t from = (int64_t)(s.tile_prefix[q + 1] - s.tile_prefix[q]) * KT;
         for (int u = 0; u < QPG; ++u)
           for (int64_t i = from + et; i < P.max_vis; i += EPI_GROUPS * 128)
-            P.scores[(int64_t)(q * QPG + u) * P.scores_ld + i] = -INFINITY;
+            put_score(P.scores, (int64_t)(q * QPG + u) * P.scores_ld + i, -INFINITY, P.score_bf16);
       }
     }
     TileIter t;
@@ -422,9 +422,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         const int64_t i = (int64_t)(t.lt + k) * KT + r;
         if (i < P.max_vis) {
-          P.scores[(int64_t)(t.q * QPG) * P.scores_ld + i] = (i < nv) ? s0 + s1 : -INFINITY;
+          put_score(P.scores, (int64_t)(t.q * QPG) * P.scores_ld + i, (i < nv) ? s0 + s1 : -INFINITY,
+                    P.score_bf16);
           if (PAIR)
-            P.scores[(int64_t)(t.q * QPG + 1) * P.scores_ld + i] = (i < nv2) ? u0 + u1 : -INFINITY;
+            put_score(P.scores, (int64_t)(t.q * QPG + 1) * P.scores_ld + i,
+                      (i < nv2) ? u0 + u1 : -INFINITY, P.score_bf16);
         }
       }
       if (seg_end) {

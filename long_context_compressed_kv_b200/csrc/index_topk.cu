@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(128) index_scores_simt(IndexParams P) {
       score = fmaf(ws[h], fmaxf(acc, 0.f), score);
     }
   }
-  P.scores[(int64_t)q * P.scores_ld + i] = score;
+  put_score(P.scores, (int64_t)q * P.scores_ld + i, score, P.score_bf16);
 }
 
 cudaError_t launch_index_scores(const IndexParams& P, cudaStream_t st) {
@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select(TopkParams P) {
     __syncthreads();
     const uint32_t prefix = sh_prefix, mask = sh_mask;
     for (int i = threadIdx.x; i < nv; i += blockDim.x) {
-      const uint32_t key = float_key(s[i]);
+      const uint32_t key = float_key(get_score(s, i, P.score_bf16));
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select(TopkParams P) {
   int base_sel = 0, base_eq = 0;
   for (int c0 = 0; c0 < nv; c0 += blockDim.x) {
     const int i = c0 + threadIdx.x;
-    const uint32_t key = (i < nv) ? float_key(s[i]) : 0u;
+    const uint32_t key = (i < nv) ? float_key(get_score(s, i, P.score_bf16)) : 0u;
     const int gt = (i < nv) && key > T;
     const int eq = (i < nv) && key == T;
     int tot_eq, tot_sel;

@@ -69,8 +69,9 @@ struct IndexParams {
   const void* keys;
   const uint8_t* keys_sf;
   int64_t key_rows, max_vis;
-  float* scores;        // [n_q][max_vis]
+  float* scores;        // [n_q][max_vis] fp32, or bf16 when score_bf16
   int64_t scores_ld;
+  int score_bf16 = 0;
   uint32_t* status;
   uint32_t wait_ns = 0; // bound of the tensor-core kernel's waits (0: the default, 1 s)
   int stall = 0;        // debug: the tensor-core kernel's MMA warp waits on a barrier
@@ -79,8 +80,9 @@ struct IndexParams {
 
 struct TopkParams {
   int n_q, m, k;
-  const float* scores;
+  const float* scores;  // fp32, or bf16 when score_bf16
   int64_t scores_ld, max_vis;
+  int score_bf16 = 0;
   const int64_t* q_pos;
   int32_t* idx_out;
 };
@@ -121,6 +123,8 @@ struct MqaParams {
   uint32_t* grid_bar = nullptr;   // tensor-core path: [count, generation] in the workspace header
   uint8_t* qbuf;        // tensor-core path: [n_q] coded query images (kMqaQImageStride bytes)
   int q_ready = 0;      // the images in qbuf are already coded (decode: by the append kernel)
+  int pair = 0;         // tensor-core path: two consecutive queries of one sequence per CTA
+                        // (H <= 64: head rows 0..63 the first, 64..127 the second)
   void* out;
   int out_dtype;
   float* lse;

@@ -43,15 +43,18 @@ __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w &
 // RoPE chunks each), and issue all of their loads before the RoPE angles are
 // computed; every thread of the block must call this (one __syncthreads).
 // cs / sn: 32 floats of shared memory each.
+// Image row h holds head h - row0 of Qrow0 (rows outside [row0, row0 + H) are
+// zero): row0 = 64 puts a second query's heads in rows 64.. of a shared image.
 __device__ __forceinline__ void qimage_code_rows(const __nv_bfloat16* Qrow0, int H, int64_t p,
                                                  float theta, uint8_t* img, int hblk,
                                                  float* cs, float* sn, bool rmsnorm = false,
-                                                 float eps = 0.f) {
+                                                 float eps = 0.f, int row0 = 0) {
   const int tid = threadIdx.x;
   const bool worker = tid < 64;
   const int h = hblk * 16 + ((tid & 63) >> 2), part = tid & 3;
-  const bool live = worker && h < H;
-  const uint4* src = reinterpret_cast<const uint4*>(Qrow0 + (int64_t)(live ? h : 0) * 512);
+  const int hs = h - row0;
+  const bool live = worker && hs >= 0 && hs < H;
+  const uint4* src = reinterpret_cast<const uint4*>(Qrow0 + (int64_t)(live ? hs : 0) * 512);
   uint4 nope[14], rope[2];
 #pragma unroll
   for (int i = 0; i < 14; ++i) nope[i] = live ? src[part * 14 + i] : make_uint4(0u, 0u, 0u, 0u);

@@ -88,7 +88,7 @@ struct Smem {
       float fself[128], invl[128];            // merge factor of this split, 1 / denominator
     } mg;
   };
-  float rcs[32], rsn[32];                     // RoPE angles of the query position (dh = 1)
+  float rcs[2][32], rsn[2][32];               // RoPE angles of the query positions (dh = 1)
   int verdict;                                // the grid barrier's outcome, for the whole CTA
   float xl[KG - 1][128];                      // the other groups' row sums, for the epilogue
   uint64_t full[KST], empty[KST], sfull[2], pfull[2], pdone[2], xbar[4][2];
@@ -245,30 +245,59 @@ struct Geo {
   int b;
   int64_t p, n_vis;
   int n_main, n_swa, nmp, total, s0, T;
+  // pairs: the two queries' positions and visible entries (rows 0..63 / 64..127)
+  int64_t pq[2], nq[2];
 };
 
+// Position and visible entries of query q, checked against the call's bounds.
+__device__ __forceinline__ void query_span(const MqaParams& P, int q, int& b, int64_t& p,
+                                           int64_t& nv) {
+  b = P.q_seq ? P.q_seq[q] : P.q_base + q;
+  p = P.q_pos[q];
+  nv = (p + 1) / P.m;
+  if (b < 0 || b >= P.B) {
+    if (threadIdx.x == 0) flag(P.status, ST_BAD_SEQ);
+    b = 0;
+    nv = 0;
+    p = -1;
+  }
+  if (nv > P.kv_rows) {
+    if (threadIdx.x == 0) flag(P.status, ST_BAD_POSITION);
+    nv = P.kv_rows;
+  }
+  if (!P.idx && nv > P.max_vis) {
+    if (threadIdx.x == 0) flag(P.status, ST_BAD_POSITION);
+    nv = P.max_vis;
+  }
+}
+
+// q: the query, or with P.pair the pair (queries 2q, 2q + 1 of one sequence:
+// the union of their visible entries and of their windows, each row masked to
+// its own query's in the softmax)
+template <bool PAIR>
 __device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
   Geo g;
-  g.b = P.q_seq ? P.q_seq[q] : P.q_base + q;
-  g.p = P.q_pos[q];
-  g.n_vis = (g.p + 1) / P.m;
-  if (g.b < 0 || g.b >= P.B) {
-    if (threadIdx.x == 0) flag(P.status, ST_BAD_SEQ);
-    g.b = 0;
-    g.n_vis = 0;
-    g.p = -1;
+  if (PAIR) {
+    int b1;
+    query_span(P, 2 * q, g.b, g.pq[0], g.nq[0]);
+    query_span(P, 2 * q + 1, b1, g.pq[1], g.nq[1]);
+    if (b1 != g.b) {
+      if (threadIdx.x == 0) flag(P.status, ST_BAD_SEQ);
+      g.nq[1] = 0;
+      g.pq[1] = -1;
+    }
+    g.p = max(g.pq[0], g.pq[1]);
+    g.n_vis = max(g.nq[0], g.nq[1]);
+    const int64_t lo = max((int64_t)0, min(g.pq[0], g.pq[1]) - P.n_win + 1);
+    g.n_main = (int)g.n_vis;
+    g.n_swa = g.p >= 0 ? (int)(g.p - lo + 1) : 0;
+  } else {
+    query_span(P, q, g.b, g.p, g.n_vis);
+    g.pq[0] = g.pq[1] = g.p;
+    g.nq[0] = g.nq[1] = g.n_vis;
+    g.n_main = P.idx ? P.n_sel : (int)g.n_vis;
+    g.n_swa = (int)min((int64_t)P.n_win, g.p + 1);
   }
-  if (g.n_vis > P.kv_rows) {
-    if (threadIdx.x == 0) flag(P.status, ST_BAD_POSITION);
-    g.n_vis = P.kv_rows;
-  }
-  int64_t nm = P.idx ? (int64_t)P.n_sel : g.n_vis;
-  if (!P.idx && nm > P.max_vis) {
-    if (threadIdx.x == 0) flag(P.status, ST_BAD_POSITION);
-    nm = P.max_vis;
-  }
-  g.n_main = (int)nm;
-  g.n_swa = (int)min((int64_t)P.n_win, g.p + 1);
   if (g.n_swa < 0) g.n_swa = 0;
   g.nmp = (g.n_main + NK - 1) / NK * NK;
   g.total = g.nmp + (g.n_swa + NK - 1) / NK * NK;
@@ -295,14 +324,18 @@ __device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
 // is read by eight SMs): the query image of the main kernel.
 __global__ void __launch_bounds__(64) mqa_tc_qprep_kernel(MqaParams P) {
   __shared__ float cs[32], sn[32];
-  const int q = blockIdx.x;
+  // pairs: image blockIdx.x holds query 2x in rows 0..63, 2x + 1 in rows 64..127
+  const int second = (P.pair && blockIdx.y >= 4) ? 1 : 0;
+  const int q = P.pair ? 2 * blockIdx.x + second : blockIdx.x;
   qimage_code_rows(reinterpret_cast<const __nv_bfloat16*>(P.Q) + (int64_t)q * P.H * 512, P.H,
-                   P.q_pos[q], P.theta, P.qbuf + (int64_t)q * kMqaQImageStride, blockIdx.y, cs, sn,
-                   P.q_rmsnorm != 0, P.eps);
+                   P.q_pos[q], P.theta, P.qbuf + (int64_t)blockIdx.x * kMqaQImageStride, blockIdx.y, cs, sn,
+                   P.q_rmsnorm != 0, P.eps, second ? 64 : 0);
 }
 
 // 576 threads = 18 warps: on the SM sub-partition that holds five of them at
 // most 16384 / 5 registers a warp, hence 96 registers a thread
+// PAIR: two consecutive queries of one sequence per CTA (see MqaParams::pair)
+template <bool PAIR>
 __global__ void __launch_bounds__(NTHR, 1)
     mqa_tc_kernel(MqaParams P, const __grid_constant__ Maps maps) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -314,7 +347,7 @@ __global__ void __launch_bounds__(NTHR, 1)
   const int split = (int)(blockIdx.x % (unsigned)C);
   const int unit = (int)(blockIdx.x / (unsigned)C);
   const int dh = unit & 1, q = unit >> 1;
-  const Geo g = geometry(P, q, split);
+  const Geo g = geometry<PAIR>(P, q, split);
   // the grid barrier's generation before this CTA arrives (merging launches)
   const uint32_t bar_gen0 = (C > 1 && threadIdx.x == 0) ? ld_acquire_gpu(P.grid_bar + 1) : 0u;
   // every CTA, also one with no tiles (T = 0), takes part in the merge below
@@ -441,10 +474,12 @@ __global__ void __launch_bounds__(NTHR, 1)
     // the angles of the output's inverse RoPE (dims 448..511, one pair a
     // lane), computed here while the other warps still work through the tiles
     if (dh == 1) {
-      float c = 1.f, sv = 0.f;
-      if (g.p >= 0) rope_cs(g.p, lane, 64, P.theta, c, sv);
-      s.rcs[lane] = c;
-      s.rsn[lane] = sv;
+      for (int u = 0; u < (PAIR ? 2 : 1); ++u) {
+        float c = 1.f, sv = 0.f;
+        if (g.pq[u] >= 0) rope_cs(g.pq[u], lane, 64, P.theta, c, sv);
+        s.rcs[u][lane] = c;
+        s.rsn[u][lane] = sv;
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
@@ -523,6 +558,11 @@ __global__ void __launch_bounds__(NTHR, 1)
     bool live = mbar_wait_warp(&s.qready, 0, P.status, 1);
     const float qs = s.qsc[h];
     const int ctid = (warp - 2) * 32 + lane;             // 0 .. 511: share of the V conversion
+    // pairs: this row's query (rows 64..127 the second): its visible entries
+    // and its window [p - n_win + 1, p] among the pair's union
+    const int rq = (PAIR && h >= 64) ? 1 : 0;
+    const int64_t lim_e = g.nq[rq], w_lo = g.pq[rq] - P.n_win + 1, w_hi = g.pq[rq];
+    const int64_t tok0 = g.p - g.n_swa + 1 - g.nmp;      // window token of key vk + g.nmp .. is tok0 + vk
     for (int t = 0; t < g.T && live; ++t) {
       const int a = t & 1, st = t % KST, xb = t & 1;
       if (!mbar_wait_warp(&s.sfull[a], (t >> 1) & 1, P.status, 6) ||
@@ -548,8 +588,18 @@ __global__ void __launch_bounds__(NTHR, 1)
         const float kj = ksc[j];
         const float v = (qs * kj * __uint_as_float(sn_[j]) + __uint_as_float(sr_[j])) * sl2;
         s2[j] = (kj != 0.f) ? v : -INFINITY;             // a zero scale marks an empty slot
-        ms = fmaxf(ms, s2[j]);
       }
+      if (PAIR) {                                      // uniform: the row's own query only
+        const int vk = g.s0 + t * NK + grp * KPG;
+#pragma unroll
+        for (int j = 0; j < KPG; ++j) {
+          const bool ok = vk + j < g.nmp ? (vk + j < lim_e)
+                                         : (tok0 + vk + j >= w_lo && tok0 + vk + j <= w_hi);
+          if (!ok) s2[j] = -INFINITY;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < KPG; ++j) ms = fmaxf(ms, s2[j]);
       // the tile's row maximum: exchanged with the other key groups of the
       // same TMEM lane quarter (the same head rows); past this exchange every
       // group has read its S columns, so P may overwrite them
@@ -651,6 +701,9 @@ __global__ void __launch_bounds__(NTHR, 1)
   tc_fence_before();
   __syncthreads();
   const float log2e = 1.4426950408889634f;
+  // the output (query, head) of TMEM lane / image row hh
+  auto row_q = [&](int hh) -> int64_t { return PAIR ? 2 * (int64_t)q + (hh >> 6) : q; };
+  auto row_h = [&](int hh) -> int { return PAIR ? (hh & 63) : hh; };
   uint8_t* stage = &s.q[0];                             // q .. kv3: free, every MMA / copy is done
   float* fac = reinterpret_cast<float*>(stage);         // [C][128] row factors (after the copy-out)
   float* lsp = fac + C * 128;                           // [C][128] row sums
@@ -710,7 +763,7 @@ __global__ void __launch_bounds__(NTHR, 1)
   const bool fast = C > 1 && C <= kFastSplits && 128 * ng <= NTHR;
   const uint2* po0 = reinterpret_cast<const uint2*>(P.part_o) + (int64_t)(blockIdx.x - split) * (128 * 64);
   const int f_hh = fast ? tid / max(ng, 1) : 0, f_col = fast ? 4 * (g0 + tid % max(ng, 1)) : 0;
-  const bool f_item = fast && tid < 128 * ng && f_hh < P.H;
+  const bool f_item = fast && tid < 128 * ng && row_h(f_hh) < P.H;
   uint2 pre[kFastSplits];
   if (C > 1) {
     // (4) the C splits' row maxima and sums of this (query, half): every
@@ -765,8 +818,8 @@ __global__ void __launch_bounds__(NTHR, 1)
     // the merged row maximum (with the sink, log2 units) and denominator; the
     // factor of each split: exp2(max_r - M) for O (C = 1), times l_r for the
     // normalised partials O_r / l_r (C > 1)
-    const int hh = tid;
-    const float z = (P.sink && hh < P.H) ? P.sink[hh] * log2e : -INFINITY;
+    const int hh = tid, head = row_h(hh);
+    const float z = (P.sink && head < P.H) ? P.sink[head] * log2e : -INFINITY;
     float M = z;
     if (C == 1) {
       M = fmaxf(M, s.mg.rms[hh]);
@@ -788,27 +841,27 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     if (M != -INFINITY && z != -INFINITY) den += ex2f(z - M);
     s.mg.invl[hh] = den > 0.f ? 1.f / den : 0.f;
-    if (P.lse && dh == 0 && split == 0 && hh < P.H && merge_ok)
-      P.lse[(int64_t)q * P.H + hh] = den > 0.f ? M * 0.6931471805599453f + logf(den) : -INFINITY;
+    if (P.lse && dh == 0 && split == 0 && head < P.H && merge_ok)
+      P.lse[row_q(hh) * P.H + head] = den > 0.f ? M * 0.6931471805599453f + logf(den) : -INFINITY;
   }
   __syncthreads();
-  const int64_t obase = (int64_t)q * P.H * 512 + dh * 256;
   // the final value of output column `col` (this half) of row hh from its
   // merged (summed, scaled) value: / denominator, R(-p) on RoPE pairs, stored
   auto emit4 = [&](int hh, int col, float4 a) {
     const float il = s.mg.invl[hh];
     float o[4] = {a.x * il, a.y * il, a.z * il, a.w * il};
     if (dh == 1 && col >= 192) {
+      const int u = (PAIR && hh >= 64) ? 1 : 0;
 #pragma unroll
       for (int e = 0; e < 4; e += 2) {
         const int k = (col + e - 192) >> 1;
-        const float cs = s.rcs[k], sn = s.rsn[k];
+        const float cs = s.rcs[u][k], sn = s.rsn[u][k];
         const float r0 = o[e] * cs + o[e + 1] * sn, r1 = -o[e] * sn + o[e + 1] * cs;
         o[e] = r0;
         o[e + 1] = r1;
       }
     }
-    const int64_t off = obase + (int64_t)hh * 512 + col;
+    const int64_t off = (row_q(hh) * P.H + row_h(hh)) * 512 + dh * 256 + col;
     if (P.out_dtype == V4A_F32) {
       *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) + off) = make_float4(o[0], o[1], o[2], o[3]);
     } else {
@@ -830,7 +883,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         uint32_t r[32];
         tmem_ld32_nowait(ob + c, r);
         tmem_ld_wait();
-        if (hh < P.H)
+        if (row_h(hh) < P.H)
 #pragma unroll
           for (int k = 0; k < 32; k += 4)
             emit4(hh, c + k, make_float4(__uint_as_float(r[k]) * f, __uint_as_float(r[k + 1]) * f,
@@ -858,7 +911,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     } else
     for (int it = tid; it < 128 * ng; it += NTHR) {
       const int hh = it / ng, col = 4 * (g0 + it % ng);
-      if (hh >= P.H) continue;
+      if (row_h(hh) >= P.H) continue;
       float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int r0 = 0; r0 < C; r0 += 8) {              // eight loads in flight
         uint2 b[8];
@@ -924,11 +977,14 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   // per device: CTAs that can be resident at once (one per SM)
   static int resident[64] = {0};
   if (resident[dev] == 0) {
-    cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel,
+    cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(mqa_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0, n_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mqa_tc_kernel, NTHR, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mqa_tc_kernel<false>, NTHR, smem);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     resident[dev] = std::max(1, per_sm * n_sm);
@@ -941,9 +997,13 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   // sparse call spreads them over as many SMs as it can); one when fewer
   // than two fit, which needs no partials and no grid barrier
   MqaParams Q = P;
+  // Two consecutive queries per CTA (their 2 x H <= 128 head rows side by
+  // side, sharing every key tile) when a dense call's queries all belong to
+  // one sequence and are many: the prefill form of the HCA MQA
+  Q.pair = (!P.idx && P.H <= 64 && P.B == 1 && P.n_q >= 256 && P.n_q % 2 == 0 && !P.q_ready) ? 1 : 0;
   const int64_t n_main = P.idx ? (int64_t)P.n_sel : P.max_vis;
-  const int64_t tiles = (n_main + NK - 1) / NK + (P.n_win + NK - 1) / NK;
-  const int64_t units = 2 * (int64_t)P.n_q;
+  const int64_t tiles = (n_main + NK - 1) / NK + (P.n_win + NK - 1 + (Q.pair ? NK : 0)) / NK;
+  const int64_t units = 2 * (int64_t)(Q.pair ? P.n_q / 2 : P.n_q);
   const int64_t cap = std::min<int64_t>(resident[dev], kMqaTcMaxCtas);
   int64_t C = 1;
   if (units * 2 <= cap)
@@ -954,7 +1014,9 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
     return cudaErrorInvalidValue;
   const int64_t grid = units * C;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  if (!P.q_ready) mqa_tc_qprep_kernel<<<dim3((unsigned)P.n_q, 8), 64, 0, st>>>(P);
+  if (C > 1) Q.pair = 0;                            // (never with n_q >= 256)
+  if (!P.q_ready)
+    mqa_tc_qprep_kernel<<<dim3((unsigned)(Q.pair ? P.n_q / 2 : P.n_q), 8), 64, 0, st>>>(Q);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
   cfg.blockDim = dim3(NTHR, 1, 1);
@@ -965,7 +1027,8 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = C > 1 ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, mqa_tc_kernel, Q, m);
+  return Q.pair ? cudaLaunchKernelEx(&cfg, mqa_tc_kernel<true>, Q, m)
+                : cudaLaunchKernelEx(&cfg, mqa_tc_kernel<false>, Q, m);
 }
 
 }  // namespace v4a

@@ -121,21 +121,58 @@ __global__ void __launch_bounds__(TPB, 1) topk_cluster_kernel(TopkParams P) {
     return;                                     // uniform: no cluster barrier follows
   }
   const bool cached = len <= CACHE;
-  const float* src = P.scores + (int64_t)q * P.scores_ld + lo;
+  // this CTA's slice of the row (fp32, or bf16 halves of 32-bit words)
+  const int sbf = P.score_bf16;
+  const float* src = sbf ? reinterpret_cast<const float*>(
+                               reinterpret_cast<const uint16_t*>(P.scores) + (int64_t)q * P.scores_ld + lo)
+                         : P.scores + (int64_t)q * P.scores_ld + lo;
   if (rank == 0)
     for (int t = threadIdx.x; t < MAXPASS * NB; t += TPB) tot[t] = 0;
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  // bf16 rows: 16-bit order-preserving keys, so that at most two radix
+  // passes resolve them
   auto take_key = [&](int i, float x) {
-    const uint32_t k = float_key(x);
+    const uint32_t k = sbf ? float_key(x) >> 16 : float_key(x);
     if (cached) keys[padi(i)] = k;
     kmin = min(kmin, k);
     kmax = max(kmax, k);
   };
-  // scalar head up to a 16-byte boundary, then 16-byte loads, 8 in flight per thread
-  const int head = min(len, (int)((16 - (reinterpret_cast<uintptr_t>(src) & 15)) & 15) / 4);
-  if ((int)threadIdx.x < head) take_key(threadIdx.x, src[threadIdx.x]);
-  const float4* src4 = reinterpret_cast<const float4*>(src + head);
-  const int n4 = (len - head) / 4;
+  // scalar head up to a 16-byte boundary, then 16-byte loads, 8 in flight per
+  // thread (bf16 rows: 8 loads of one score in flight, coalesced across the warp)
+  const int head = sbf ? len : min(len, (int)((16 - (reinterpret_cast<uintptr_t>(src) & 15)) & 15) / 4);
+  if (sbf) {
+    // scalar head up to an 8-byte boundary, then 8-byte loads (4 scores), 8 in flight
+    const uint16_t* s16 = reinterpret_cast<const uint16_t*>(src);
+    auto bf = [](uint32_t b) { return __uint_as_float(b << 16); };
+    const int hb = min(len, (int)((8 - (reinterpret_cast<uintptr_t>(s16) & 7)) & 7) / 2);
+    if ((int)threadIdx.x < hb) take_key(threadIdx.x, bf(s16[threadIdx.x]));
+    const uint2* s8 = reinterpret_cast<const uint2*>(s16 + hb);
+    const int n8 = (len - hb) / 4;
+    for (int j0 = 0; j0 < n8; j0 += 8 * TPB) {
+      uint2 v8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * TPB + threadIdx.x;
+        v8[u] = (j < n8) ? s8[j] : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * TPB + threadIdx.x;
+        if (j < n8) {
+          const int i = hb + 4 * j;
+          take_key(i, bf(v8[u].x & 0xFFFFu));
+          take_key(i + 1, bf(v8[u].x >> 16));
+          take_key(i + 2, bf(v8[u].y & 0xFFFFu));
+          take_key(i + 3, bf(v8[u].y >> 16));
+        }
+      }
+    }
+    for (int i = hb + 4 * n8 + threadIdx.x; i < len; i += TPB) take_key(i, bf(s16[i]));
+  } else if ((int)threadIdx.x < head) {
+    take_key(threadIdx.x, src[threadIdx.x]);
+  }
+  const float4* src4 = reinterpret_cast<const float4*>(src + (sbf ? 0 : head));
+  const int n4 = sbf ? 0 : (len - head) / 4;
   for (int j0 = 0; j0 < n4; j0 += 8 * TPB) {
     float4 v[8];
 #pragma unroll
@@ -155,8 +192,12 @@ __global__ void __launch_bounds__(TPB, 1) topk_cluster_kernel(TopkParams P) {
       }
     }
   }
-  for (int i = head + 4 * n4 + threadIdx.x; i < len; i += TPB) take_key(i, src[i]);
-  auto key_at = [&](int i) -> uint32_t { return cached ? keys[padi(i)] : float_key(src[i]); };
+  if (!sbf)
+    for (int i = head + 4 * n4 + threadIdx.x; i < len; i += TPB) take_key(i, src[i]);
+  auto key_at = [&](int i) -> uint32_t {
+    return cached ? keys[padi(i)]
+                  : (sbf ? float_key(get_score(src, i, 1)) >> 16 : float_key(src[i]));
+  };
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));

@@ -208,6 +208,55 @@ def test_index_topk_one_sequence_pairs(H_I, nq):
         check_topk(g_idx[q], s, nv, k)
 
 
+@pytest.mark.parametrize("one_seq", [False, True])
+def test_index_topk_bf16_scores(one_seq):
+    """score_dtype BF16: every score rounded to bf16 (checked against the
+    oracle's scores of the GPU's stored keys within bf16 rounding), the
+    selection exact among those bf16 values (ties to the lower index), and
+    its recall of the fp32 selection reported (the bf16 grid makes near-ties
+    of the fp32 scores exact ties)."""
+    v = v4()
+    rng = np.random.default_rng(11 + one_seq)
+    H_I, d_I, k = 64, 128, 256
+    B, N = (1, 16384) if one_seq else (3, 20000)
+    keys = rng.standard_normal((B, N, d_I)).astype(np.float32)
+    positions = (np.array([4 * N - 1, 4 * N - 5, 4 * 700 + 3, 4 * 700 + 4, 9, 4 * 129])
+                 if one_seq else np.array([4 * N - 1, 4 * 7000 + 2, 4 * 100, 4 * N - 9]))
+    nq = len(positions)
+    q_seq = np.zeros(nq, np.int32) if one_seq else np.array([0, 1, 2, 1], np.int32)
+    qI = rng.standard_normal((nq, H_I, d_I)).astype(np.float32)
+    w = rng.uniform(0, 1, (nq, H_I)).astype(np.float32)
+    ly = synth.Layer("csa", 4, 16, 512, 64, 128, H_I, d_I, k, idx_fp4=True)
+    desc = desc_for(ly)
+    krows, ksf = code_rows(desc, dev(keys), v.MXFP4)
+    qrows, qsf = code_rows(desc, dev(qI.reshape(1, nq * H_I, d_I)), v.MXFP4)
+    qrows, qsf = qrows.reshape(nq, H_I, -1), qsf.reshape(nq, H_I, -1)
+    idx = torch.full((nq, k), -9, dtype=torch.int32, device="cuda")
+    scores = torch.zeros(nq, N, dtype=torch.bfloat16, device="cuda")
+    ws = v.workspace(desc, nq, N)
+    v.index_topk(desc, qI=qrows, qI_sf=qsf, w=dev(w), q_pos=dev(positions, torch.int64),
+                 q_seq=dev(q_seq, torch.int32), B=B, keys=krows, keys_sf=ksf, key_rows=N,
+                 max_vis=N, idx_out=idx, scores_out=scores, ws=ws, score_dtype=v.BF16)
+    torch.cuda.synchronize()
+    assert v.device_status(ws) == 0
+    kd = read_keys(krows, ksf, v.MXFP4)
+    qd = read_keys(qrows, qsf, v.MXFP4)
+    g_idx, g_s = idx.cpu().numpy(), scores.float().cpu().numpy()
+    recall = []
+    for q in range(nq):
+        nv = int(ocomp.n_visible(positions[q], 4))
+        s = oidx.scores(qd[q], w[q], kd[q_seq[q], :nv])
+        scale = max(1.0, float(np.max(np.abs(s)))) if nv else 1.0
+        # bf16 round to nearest of an fp32 sum within 1e-5 of the oracle's
+        assert np.all(np.abs(g_s[q, :nv] - s) <= 2.0 ** -8 * np.abs(s) + 1e-5 * scale)
+        assert np.all(np.isneginf(g_s[q, nv:]))
+        assert np.array_equal(g_idx[q], oidx.topk(g_s[q], nv, k))       # exact among bf16 values
+        ref = oidx.topk(s, nv, k)
+        kk = min(k, nv)
+        recall.append(len(np.intersect1d(g_idx[q][:kk], ref[:kk])) / kk)
+    assert np.mean(recall) >= 0.9, recall
+
+
 def test_topk_ties_go_to_lower_index():
     """Many exactly equal scores: the selection must be the lowest indices."""
     v = v4()
@@ -325,6 +374,51 @@ def test_mqa_parity(sparse, fp8, H, d, d_rope, q_rmsnorm):
         keys = np.concatenate([e_val[b, rows], s_val[b, toks % swa_rows]], 0)
         o, l = oracle_attention(Q[q], p, keys, sink, ly, fp8, q_rmsnorm=q_rmsnorm)
         check_output(g_out[q], o, g_lse[q], l, not fp8, ("query", q))
+
+
+@pytest.mark.parametrize("H", [64, 48])
+def test_dense_mqa_one_sequence_pairs(H):
+    """Dense MQA over many queries of one sequence (the prefill form): the
+    tensor-core kernel runs two consecutive queries per CTA (rows 0..63 /
+    64..127), each row masked to its own query's entries and window.
+    Positions: consecutive runs crossing block boundaries, gaps inside a pair,
+    a pair of equal positions, position 0."""
+    v = v4()
+    rng = np.random.default_rng(H)
+    m, N, n_win, d, d_rope = 128, 40, 128, 512, 64
+    ly = synth.Layer("hca", m, H, d, d_rope, n_win)
+    desc = desc_for(ly)
+    fmt = v.E4M3_BF16ROPE
+    L = m * N
+    ents = rng.standard_normal((1, N, d)).astype(np.float32)
+    swa_vals = rng.standard_normal((1, L, d)).astype(np.float32)
+    kv, kv_sc = code_rows(desc, dev(ents), fmt, d_rope=d_rope)
+    swa, swa_sc = code_rows(desc, dev(swa_vals), fmt, d_rope=d_rope)
+    pos = list(range(2 * m - 100, 2 * m + 100)) + [0, 1, 3000, 3000, 4000, 4900, 127, 128]
+    pos += sorted(rng.integers(0, L, 256 - len(pos)).tolist())
+    positions = np.array(pos[:256])
+    nq = len(positions)
+    Q = synth.bf16_values(rng.standard_normal((nq, H, d)).astype(np.float32))
+    sink = rng.standard_normal(H).astype(np.float32)
+    out = torch.zeros(nq, H, d, dtype=torch.float32, device="cuda")
+    lse = torch.zeros(nq, H, dtype=torch.float32, device="cuda")
+    ws = v.workspace(desc, nq, N)
+    v.dense_mqa(desc, Q=dev(Q, torch.bfloat16), q_pos=dev(positions, torch.int64),
+                q_seq=dev(np.zeros(nq), torch.int32), B=1, kv=kv, kv_scale=kv_sc, kv_rows=N,
+                swa=swa, swa_scale=swa_sc, swa_rows=L, max_vis=N, out=out, ws=ws,
+                sink=dev(sink), lse=lse)
+    torch.cuda.synchronize()
+    assert v.device_status(ws) == 0
+    g_out, g_lse = out.cpu().numpy(), lse.cpu().numpy()
+    e_val = read_kv(kv, kv_sc, fmt, d, d_rope)
+    s_val = read_kv(swa, swa_sc, fmt, d, d_rope)
+    for q in range(nq):
+        p = int(positions[q])
+        nv = int(ocomp.n_visible(p, m))
+        toks = omqa.window_tokens(p, n_win)
+        keys = np.concatenate([e_val[0, :nv], s_val[0, toks]], 0)
+        o, l = oracle_attention(Q[q], p, keys, sink, ly, True)
+        check_output(g_out[q], o, g_lse[q], l, False, ("query", q))
 
 
 def test_mqa_no_sink_and_empty_selection():
