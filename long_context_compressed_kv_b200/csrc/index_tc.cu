@@ -43,22 +43,31 @@ namespace {
 
 constexpr int KT = 128;                 // keys per tile (MMA M)
 constexpr int KROW = 64;                // bytes per key row (128 E2M1)
-constexpr int TPS = 4;                  // tiles per ring stage (32 KB of key codes)
-constexpr int STAGES = 5;
 constexpr int KTILE_BYTES = KT * KROW;  // 8 KB
 constexpr int SF_BYTES = 512;           // 128 rows x 4 scale bytes
 constexpr int MAXQ = 1024;              // queries per launch on this path
 constexpr int EPI_GROUPS = 2;           // epilogue warp groups, alternating tiles
 constexpr int NTHREADS = 64 + EPI_GROUPS * 128;
 constexpr int MAX_ACC = 8;              // accumulator stages in TMEM
-constexpr uint32_t TM_COLS = 512;
 
-// accumulator stages that fit in 512 TMEM columns next to their key scales (4
-// columns each) and the two query-scale slots (4 columns each)
-__host__ __device__ constexpr int n_acc(int N) {
-  return (512 - 8) / (N + 4) < MAX_ACC ? (512 - 8) / (N + 4) : MAX_ACC;
-}
+// Per MMA width N: N <= 64 runs two CTAs per SM (each its own MMA-issuing
+// thread, whose tcgen05 issue rate bounds the kernel; half of TMEM each; a
+// ring of 3 stages of up to 3 tiles), N = 128 one CTA per SM (all of TMEM, 5
+// stages of up to 4 tiles: 32 KB, the size from which one stage per barrier
+// round trip streams at HBM speed).  Accumulators: as many as fit the CTA's
+// TMEM columns next to their key scales (4 columns each) and the two
+// query-scale slots (4 columns each).
+template <int N>
+struct Cfg {
+  static constexpr int CPS = N <= 64 ? 2 : 1;
+  static constexpr int STAGES = CPS == 2 ? 3 : 5;
+  static constexpr int TPS = CPS == 2 ? 3 : 4;
+  static constexpr uint32_t TM_COLS = CPS == 2 ? 256 : 512;
+  static constexpr int NACC = ((int)TM_COLS - 8) / (N + 4) < MAX_ACC ? ((int)TM_COLS - 8) / (N + 4)
+                                                                      : MAX_ACC;
+};
 
+template <int STAGES, int TPS>
 struct Smem {
   alignas(1024) uint8_t keys[STAGES][TPS][KTILE_BYTES];
   alignas(1024) uint8_t q[2][128 * KROW];
@@ -80,13 +89,15 @@ struct TileIter {
 
 }  // namespace
 
-__device__ __forceinline__ void fail(Smem& s, uint32_t* status) {
+template <class S>
+__device__ __forceinline__ void fail(S& s, uint32_t* status) {
   s.abort = 1;
   flag(status, ST_TIMEOUT);
 }
 
 // Decode tile g into (query, local tile); `it` tracks segments (query changes).
-__device__ __forceinline__ void locate(const Smem& s, int n_q, int g, TileIter& t) {
+template <class S>
+__device__ __forceinline__ void locate(const S& s, int n_q, int g, TileIter& t) {
   while (t.qcur + 1 <= n_q && s.tile_prefix[t.qcur + 1] <= g) ++t.qcur;
   if (t.qcur != t.q) {
     t.q = t.qcur;
@@ -95,12 +106,13 @@ __device__ __forceinline__ void locate(const Smem& s, int n_q, int g, TileIter& 
   t.lt = g - s.tile_prefix[t.q];
 }
 
-// Tiles in the stage that starts at tile g: up to `tps` (at most TPS and at
+// Tiles in the stage that starts at tile g: up to `tps` (at most the stage's and at
 // most the accumulator count, so that the tiles of one stage never wait for
 // each other's accumulator: the epilogue frees a stage's accumulators only
 // after that stage's single commit), all of one query group, all inside this
 // CTA's range.  Every role walks the stages with this same rule.
-__device__ __forceinline__ int stage_tiles(const Smem& s, const TileIter& t, int g, int g1, int tps) {
+template <class S>
+__device__ __forceinline__ int stage_tiles(const S& s, const TileIter& t, int g, int g1, int tps) {
   const int to_seg = s.tile_prefix[t.q + 1] - g, to_end = g1 - g;
   const int n = to_seg < to_end ? to_seg : to_end;
   return n < tps ? n : tps;
@@ -110,17 +122,22 @@ __device__ __forceinline__ int stage_tiles(const Smem& s, const TileIter& t, int
 // sequence side by side (2 x H_I columns), so that every key tile serves both:
 // half the MMAs per score where many queries share their keys (prefill)
 template <int N, bool PAIR>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(NTHREADS, Cfg<N>::CPS)
     index_tc_kernel(IndexParams P, const __grid_constant__ CUtensorMap tm_keys,
                     const __grid_constant__ CUtensorMap tm_q) {
+  constexpr int STAGES = Cfg<N>::STAGES, TPS = Cfg<N>::TPS;
+  constexpr uint32_t TM_COLS = Cfg<N>::TM_COLS;
+  using Smem = v4a::Smem<STAGES, TPS>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int NACC = n_acc(N);
+  constexpr int NACC = Cfg<N>::NACC;
   static_assert(NACC >= 2 && NACC * (N + 4) + 8 <= (int)TM_COLS, "TMEM budget");
   constexpr int TPS_N = NACC < TPS ? NACC : TPS;        // tiles per stage for this N
-  constexpr bool W_IN_REGS = N <= 64;
+  // head weights in registers (one CTA per SM: registers to spare) or read
+  // from shared memory (two CTAs per SM: at most 102 registers a thread)
+  constexpr bool W_IN_REGS = N <= 64 && Cfg<N>::CPS == 1;
   constexpr int QPG = PAIR ? 2 : 1;                     // queries per MMA group
   constexpr int HG = N / QPG;                           // heads of one query
   const int n_g = P.n_q / QPG;                          // query groups (n_q even with PAIR)
@@ -395,7 +412,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int a = it % NACC;
         const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + a * N;
         float s0 = 0.f, s1 = 0.f, u0 = 0.f, u1 = 0.f;   // even / odd heads; u: the second query
-        constexpr int CH = N <= 64 ? N : 64;      // columns per TMEM round trip
+        constexpr int CH = Cfg<N>::CPS == 2 ? 32 : (N <= 64 ? N : 64);   // columns per TMEM round trip
 #pragma unroll
         for (int c0 = 0; c0 < N; c0 += CH) {
           uint32_t v[CH];
@@ -537,31 +554,30 @@ cudaError_t launch_index_tc(const IndexParams& P, cudaStream_t st) {
   const bool pair = P.B == 1 && P.n_q >= 2 && P.n_q % 2 == 0 && P.H_I <= 64;
   const int nmma = pair ? 2 * P.H_I : P.H_I;
   if (!make_rows_map(&tq, P.qI, (int64_t)P.n_q * P.H_I, KROW, nmma)) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(Smem) + 1024;
-  static unsigned long long configured = 0;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !(configured & (1ull << dev))) {
-    cudaError_t e = cudaSuccess;
-    for (const void* f : {(const void*)index_tc_kernel<32, false>, (const void*)index_tc_kernel<64, false>,
-                          (const void*)index_tc_kernel<128, false>, (const void*)index_tc_kernel<64, true>,
-                          (const void*)index_tc_kernel<128, true>})
-      if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured |= 1ull << dev;
-  }
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = sms;   // persistent: one CTA per SM, contiguous tile ranges
+  // persistent: Cfg<N>::CPS CTAs per SM, each over a contiguous range of tiles
+  auto launch = [&](auto kernel, auto cfg_tag) -> cudaError_t {
+    using C = decltype(cfg_tag);
+    const size_t smem = sizeof(Smem<C::STAGES, C::TPS>) + 1024;
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kernel<<<C::CPS * sms, NTHREADS, smem, st>>>(P, tk, tq);
+    return cudaSuccess;
+  };
+  cudaError_t e = cudaSuccess;
   switch (nmma * (pair ? -1 : 1)) {
-    case 32: index_tc_kernel<32, false><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
-    case 64: index_tc_kernel<64, false><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
-    case 128: index_tc_kernel<128, false><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
-    case -64: index_tc_kernel<64, true><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
-    case -128: index_tc_kernel<128, true><<<grid, NTHREADS, smem, st>>>(P, tk, tq); break;
+    case 32: e = launch(index_tc_kernel<32, false>, Cfg<32>{}); break;
+    case 64: e = launch(index_tc_kernel<64, false>, Cfg<64>{}); break;
+    case 128: e = launch(index_tc_kernel<128, false>, Cfg<128>{}); break;
+    case -64: e = launch(index_tc_kernel<64, true>, Cfg<64>{}); break;
+    case -128: e = launch(index_tc_kernel<128, true>, Cfg<128>{}); break;
     default: return cudaErrorInvalidValue;
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
