@@ -78,6 +78,7 @@ struct Smem {
   uint64_t full[STAGES], empty[STAGES], accstage[STAGES], qfull[2], qempty[2],
       accempty[MAX_ACC], done, never;
   int tile_prefix[MAXQ + 1];
+  int seq[MAXQ];                                    // sequence of each query group
   uint32_t tmem_base;
   int abort;
 };
@@ -157,20 +158,9 @@ __global__ void __launch_bounds__(NTHREADS, Cfg<N>::CPS)
     }
     return nv;
   };
-  // tiles per query group, loaded in parallel, then a serial prefix over shared memory
-  for (int q = threadIdx.x; q < n_g; q += NTHREADS) {
-    int64_t nv = visible(q * QPG);
-    if (PAIR) nv = max(nv, visible(q * QPG + 1));
-    s.tile_prefix[q + 1] = (int)((nv + KT - 1) / KT);
-  }
-  __syncthreads();
+  // set-up that needs no global memory first (barriers, TMEM), so that it
+  // overlaps the position loads below
   if (threadIdx.x == 0) {
-    int acc = 0;
-    s.tile_prefix[0] = 0;
-    for (int q = 0; q < n_g; ++q) {
-      acc += s.tile_prefix[q + 1];
-      s.tile_prefix[q + 1] = acc;
-    }
     s.abort = 0;
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&s.full[i], 1);    // the producer lane's arrive + TMA / bulk bytes
@@ -187,6 +177,23 @@ __global__ void __launch_bounds__(NTHREADS, Cfg<N>::CPS)
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(&s.tmem_base, TM_COLS);
+  // tiles and sequence of each query group (positions loaded in parallel,
+  // one round trip), then a serial prefix over shared memory
+  for (int q = threadIdx.x; q < n_g; q += NTHREADS) {
+    int64_t nv = visible(q * QPG);
+    if (PAIR) nv = max(nv, visible(q * QPG + 1));
+    s.tile_prefix[q + 1] = (int)((nv + KT - 1) / KT);
+    s.seq[q] = P.q_seq ? P.q_seq[q * QPG] : P.q_base + q * QPG;   // used only with tiles
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    s.tile_prefix[0] = 0;
+    for (int q = 0; q < n_g; ++q) {
+      acc += s.tile_prefix[q + 1];
+      s.tile_prefix[q + 1] = acc;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -218,8 +225,7 @@ __global__ void __launch_bounds__(NTHREADS, Cfg<N>::CPS)
       locate(s, n_g, g, t);
       const int n = stage_tiles(s, t, g, g1, TPS_N);
       if (t.seg != seg_before) {
-        // read once per query: a global load per stage would sit on the issue path
-        b = P.q_seq ? P.q_seq[t.q * QPG] : P.q_base + t.q * QPG;
+        b = s.seq[t.q];
         const int j = t.seg & 1, uq = t.seg >> 1;
         if (uq >= 1 && !mbar_wait_warp(&s.qempty[j], (uq - 1) & 1, P.status, -1, lim)) {
           fail(s, P.status);

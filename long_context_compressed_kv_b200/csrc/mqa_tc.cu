@@ -368,6 +368,11 @@ __global__ void __launch_bounds__(NTHR, 1)
     mbar_init(&s.done, 1);
     mbar_init(&s.lbar, NSM - 4);
     fence_mbar_init();
+    // the query image by four bulk copies on qready, issued before the CTA's
+    // first barrier so that it overlaps the TMEM allocation and the set-up
+    const uint8_t* qimg = P.qbuf + (int64_t)q * kMqaQImageStride;
+    mbar_arrive_expect_tx(&s.qready, QIMG);
+    for (int k = 0; k < 4; ++k) bulk_load(s.q + k * QCHUNK, qimg + k * QCHUNK, QCHUNK, &s.qready);
   }
   if (warp == 1) tmem_alloc(&s.tmem_base, 512);
   tc_fence_before();
@@ -377,17 +382,12 @@ __global__ void __launch_bounds__(NTHR, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ loads
-    // The query image by four bulk copies on qready.  Entry / window rows by
-    // TMA (complete_tx bytes on full[st]); the 64 entry scales by cp.async,
+    // (The query image is already on its way: thread 0 issued it with the
+    // barriers.)  Entry / window rows by TMA (complete_tx bytes on full[st]);
+    // the 64 entry scales by cp.async,
     // zero-filled for empty slots (a stored scale is a nonzero power of two,
     // so a zero scale marks an empty slot); every lane arrives on full[st]
     // through cp.async.mbarrier.arrive.noinc once its scale copies land.
-    if (lane == 0) {
-      const uint8_t* qimg = P.qbuf + (int64_t)q * kMqaQImageStride;
-      mbar_arrive_expect_tx(&s.qready, QIMG);
-      for (int k = 0; k < 4; ++k)
-        bulk_load(s.q + k * QCHUNK, qimg + k * QCHUNK, QCHUNK, &s.qready);
-    }
     const int64_t kv_base = (int64_t)g.b * P.kv_rows, sw_base = (int64_t)g.b * P.swa_rows;
     // global row of key r of tile vk, or -1 when the slot is empty
     auto row_of = [&](int vk, int r, bool main_tile) -> int64_t {
