@@ -340,9 +340,19 @@ __global__ void __launch_bounds__(TPB, 1) topk_cluster_kernel(TopkParams P) {
       eq += key == T;
     }
   }
-  int tot_gt, tot_eq;
-  const int gt_before_t = block_scan(gt, wsum, tot_gt);
-  const int eq_before_t = block_scan(eq, wsum, tot_eq);
+  int tot_gt, tot_eq, gt_before_t, eq_before_t;
+  if (len < 65536) {
+    // both counts in one scan: 16 bits each, no carry while the slice is shorter
+    int tot;
+    const int pre = block_scan(gt | (eq << 16), wsum, tot);
+    gt_before_t = pre & 0xFFFF;
+    eq_before_t = pre >> 16;
+    tot_gt = tot & 0xFFFF;
+    tot_eq = tot >> 16;
+  } else {
+    gt_before_t = block_scan(gt, wsum, tot_gt);
+    eq_before_t = block_scan(eq, wsum, tot_eq);
+  }
   if (threadIdx.x == 0) {
     cnt[0] = tot_gt;
     cnt[1] = tot_eq;
