@@ -52,7 +52,7 @@ def build_decode_layer(w, li, inp, in_dtype=None, out_dtype=None):
     """A DecodeLayer holding the coded synthetic history of ``synth.decode_layer_inputs``
     and the new token's inputs, ready for ``step``."""
     import torch
-    from long_context_compressed_kv_b200.decode import DecodeLayer
+    from long_context_compressed_kv_b200.decode_layer import DecodeLayer
     ly = w.layers[li]
     p, ring = inp["p"], inp["ring"]
     lay = DecodeLayer(desc_for(ly), w.B, kv_rows=inp["n_hist"] + 1, swa_rows=ly.n_win,
@@ -150,7 +150,7 @@ class PrefillPair:
             vals = torch.from_numpy(q0["qI"]).to(dev).reshape(1, -1, csa.d_I)
             qrows = self.qI[sl].reshape(1, -1, csa.d_I // 2)
             qsf = self.qI_sf[sl].reshape(1, -1, csa.d_I // 32)
-            from long_context_compressed_kv_b200.decode import code_rows as _code_rows
+            from long_context_compressed_kv_b200.decode_layer import code_rows as _code_rows
             _code_rows(self.dc, vals, v.MXFP4, qrows, qsf, 0)
             self.qI[sl] = qrows.reshape(len(rows), csa.H_I, -1)
             self.qI_sf[sl] = qsf.reshape(len(rows), csa.H_I, -1)
@@ -780,6 +780,13 @@ def run_gpu(args, dist, rank, world):
                     "recall_of_fp32_selection": round(float(np.mean(rec)), 4),
                     "note": "synthetic N(0,1) keys and queries, not trained weights"}
 
+    # ---- the same step on paged caches: every layer's compressed cache (and
+    # the CSA indexer keys) scattered over a shuffled pool of 128-token blocks
+    # behind a block table, the window and tails per sequence as before
+    paged = None
+    if world == 1:
+        paged = paged_decode_measure(wl, flush, args.steps, stream)
+
     also = {}
     if not args.no_also and world == 1:
         del wl
@@ -801,11 +808,92 @@ def run_gpu(args, dist, rank, world):
             del w2
             torch.cuda.empty_cache()
     return dict(value=value, ms=ms, roof=roof, step_roof=step_roof, clocks=clk.summary(),
+                paged=paged,
                 e2e=dict(value=e2e_val, h2d=h2d, d2h=d2h, ms=e2e_ms, eager_value=e2e_eager,
                          eager_ms=e2e["eager"]), also=also, tc_peaks=peaks_tc,
                 bf16_selector=bf16_sel,
                 launches=launches, q_step=q_step,
                 per_step=per_step)
+
+
+def paged_decode_measure(wl, flush, steps, stream, spare_blocks=16, seed=1):
+    """The workload's decode step with paged compressed caches: per layer a
+    pool of B * blocks_per_seq + spare_blocks blocks (epb = 128 / m entries a
+    block) holding each sequence's entries (and, for CSA, indexer keys) in a
+    shuffled order, a block table, and one captured graph of every layer's
+    v4attn_decode on them; timed like the step itself.  Also checks that the
+    outputs equal the contiguous step's (CSA: bit for bit; HCA, whose paged
+    entries are gathered rather than tiled and so split over other CTAs,
+    within 5e-3 of the output's RMS, the f16 rounding of the split partials,
+    plus one bf16 step of the element)."""
+    import torch
+    import long_context_compressed_kv_b200 as v
+    rng = np.random.default_rng(seed)
+    calls, outs = [], []
+    for lay in wl.layers:
+        epb = 128 // lay.m
+        bps = lay.kv_rows // epb
+        n = lay.B * bps + spare_blocks
+        table = rng.permutation(n)[: lay.B * bps].astype(np.int64)
+        sel = torch.from_numpy(table).cuda()
+        bt = sel.to(torch.int32).view(lay.B, bps).contiguous()
+
+        def scatter(rows, n=n, epb=epb, bps=bps, sel=sel, B=lay.B):
+            pool = torch.zeros((n * epb,) + tuple(rows.shape[2:]), dtype=rows.dtype,
+                               device=rows.device)
+            pool.view((n, epb) + tuple(rows.shape[2:]))[sel] = \
+                rows.reshape((B * bps, epb) + tuple(rows.shape[2:]))
+            return pool
+        pkv, psc = scatter(lay.kv), scatter(lay.kv_scale)
+        out, lse = torch.zeros_like(lay.out), torch.zeros_like(lay.lse)
+        kw = {}
+        if lay.csa:
+            pk, psf = scatter(lay.keys), scatter(lay.keys_sf)
+            idx = torch.full_like(lay.idx, -1)
+            kw = dict(x_idx=lay.x_idx, itail=lay.itail, ibias=lay.ibias, keys=pk, keys_sf=psf,
+                      key_rows=n * epb, qI=lay.qI, qI_sf=lay.qI_sf, w=lay.w, idx_out=idx)
+
+        def call(lay=lay, pkv=pkv, psc=psc, n=n, epb=epb, bt=bt, out=out, lse=lse, kw=kw):
+            v.decode(lay.desc, pos=lay.pos, x_main=lay.x_main, tail=lay.tail, bias=lay.bias,
+                     kv=pkv, kv_scale=psc, kv_rows=n * epb, swa=lay.swa,
+                     swa_scale=lay.swa_scale, swa_rows=lay.swa_rows, Q=lay.Q, out=out,
+                     ws=lay.ws, max_vis=lay.max_vis, sink=lay.sink, lse=lse, block_table=bt,
+                     **kw)
+        calls.append(call)
+        outs.append((lay, out, lse))
+
+    def step():
+        for c in calls:
+            c()
+    step()
+    torch.cuda.synchronize()
+    wl.replay()                       # the contiguous step's outputs, to compare
+    torch.cuda.synchronize()
+    same = {}
+    for lay, out, lse in outs:
+        name = "csa" if lay.csa else "hca"
+        if lay.csa:
+            same[name] = bool(torch.equal(out, lay.out) and torch.equal(lse, lay.lse))
+        else:
+            # within 5e-3 of the RMS (the split partials' f16 rounding) plus one
+            # bf16 step of the element (the output's own rounding may flip)
+            ref = lay.out.float()
+            rms = float(ref.pow(2).mean().sqrt())
+            same[name] = bool(((out.float() - ref).abs() <= 5e-3 * rms + ref.abs() / 128).all())
+    g = capture_graph(step)
+    for _ in range(3):
+        flush()
+        g.replay()
+    t = float(np.mean(timed_device(g.replay, flush, steps, stream)))
+    for lay, _, _ in outs:
+        v.device_status(lay.ws)       # raises on a device-side check (a bad table entry)
+    del g
+    return {"queries_per_s": round(wl.queries_per_step() / (t / 1e3), 1),
+            "us_per_step": round(t * 1e3, 2),
+            "outputs_match_contiguous": same,
+            "how": "pools of 128-token blocks (32 CSA entries + 32 indexer keys, or 1 HCA "
+                   "entry, a block) in shuffled order behind a block table; one graph of "
+                   "both layers' decode calls; L2 flushed between steps"}
 
 
 def measure_tc_peaks(stream, reps=5, n_iter=16384):
@@ -1182,6 +1270,7 @@ def main():
             "clocks": res["clocks"],
             "also": res["also"],
             "bf16_score_selector": res.get("bf16_selector"),
+            "paged_kv": res.get("paged"),
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -44,6 +44,21 @@
  *       V4A_MXFP4          c/2 bytes of E2M1 pairs (element 2j in the low
  *                          nibble) plus c/32 E8M0 scale bytes in a separate
  *                          array (OCP MX v1.0: X = floor(log2 amax) - 2).
+ *   - Paged caches ([deep-read] "异构 KV cache 与磁盘前缀复用": a classical
+ *     block cache over blocks of lcm(4, 128) = 128 raw tokens, next to the
+ *     per-sequence state cache of window and uncompressed tail).  With
+ *     block_table == NULL the compressed caches are per sequence: entry e of
+ *     sequence b at row b * rows + e.  With a block table (device int32
+ *     [B][blocks_per_seq]) they are pools shared by all sequences, `rows`
+ *     rows in all: one block holds epb = 128 / m consecutive entries (32 CSA
+ *     entries and 32 indexer keys, or 1 HCA entry), and entry e of sequence
+ *     b is at row block_table[b * blocks_per_seq + e / epb] * epb + e % epb.
+ *     rows must be a multiple of epb, a sequence sees at most
+ *     blocks_per_seq * epb entries, and a table entry outside
+ *     [0, rows / epb) is caught by the kernels (status bit, the access
+ *     skipped).  The window and tail rings stay per sequence.  Paged caches
+ *     need the tensor-core formats (E4M3 entries, MXFP4 keys; else
+ *     V4A_ERR_UNSUPPORTED).
  */
 #ifndef V4ATTN_H
 #define V4ATTN_H
@@ -162,6 +177,9 @@ typedef struct {
   void* scores_out;           /* device [n_q][max_vis] float (bf16 with score_dtype V4A_BF16)
                                  or NULL; entries >= n_vis are -inf */
   int32_t score_dtype;        /* V4A_F32 (0) or V4A_BF16 */
+  const int32_t* block_table; /* device [B][blocks_per_seq], or NULL: keys / keys_sf per
+                                 sequence (see "Paged caches"; key_rows = pool rows) */
+  int32_t blocks_per_seq;
 } v4attn_index_args;
 
 /* ---------------------------------------------------------------- MQA
@@ -204,6 +222,9 @@ typedef struct {
   void* out;                  /* device [n_q][H][d] */
   int32_t out_dtype;          /* V4A_F32 or V4A_BF16 */
   float* lse;                 /* device [n_q][H] or NULL */
+  const int32_t* block_table; /* device [B][blocks_per_seq], or NULL: kv / kv_scale per
+                                 sequence (see "Paged caches"; kv_rows = pool rows) */
+  int32_t blocks_per_seq;
 } v4attn_mqa_args;
 
 /* ---------------------------------------------------------------- decode
@@ -241,6 +262,10 @@ typedef struct {
   void* out; int32_t out_dtype; float* lse;            /* [B][H][d], [B][H] or NULL */
   int32_t* idx_out;                                    /* CSA: [B][top_k] selected entries (required) */
   int64_t max_vis;                                     /* upper bound of n_vis after the step */
+  const int32_t* block_table;  /* device [B][blocks_per_seq] or NULL: the main cache and the
+                                  indexer keys as pools (see "Paged caches"); the new entry
+                                  goes to its block's row, the window and tails stay per sequence */
+  int32_t blocks_per_seq;
 } v4attn_decode_args;
 
 /* ---------------------------------------------------------------- projection

@@ -108,13 +108,24 @@ def compress(desc: LayerDesc, *, m: int, overlap: bool, c: int, Ca, Za, Cb=None,
                                                    _stream(stream)))
 
 
+def _bt(block_table):
+    """(pointer, blocks per sequence) of an int32 [B][blocks_per_seq] block table, or (None, 0)."""
+    if block_table is None:
+        return None, 0
+    assert block_table.dim() == 2 and block_table.is_contiguous()
+    return _p(block_table), int(block_table.shape[1])
+
+
 def index_topk(desc: LayerDesc, *, qI, w, q_pos, keys, key_rows: int, max_vis: int, idx_out, ws,
                qI_sf=None, keys_sf=None, q_seq=None, B: Optional[int] = None, scores_out=None,
-               score_dtype: int = F32, stream=None):
+               score_dtype: int = F32, block_table=None, stream=None):
+    """Indexer scores + top-k (see include/v4attn.h); with ``block_table``
+    (int32 [B][blocks_per_seq]) the keys are a paged pool of ``key_rows`` rows."""
     n_q = int(q_pos.numel())
+    bt, bps = _bt(block_table)
     a = IndexArgs(n_q, B if B is not None else n_q, _p(qI), _p(qI_sf), _p(w), _p(q_seq),
                   _p(q_pos), _p(keys), _p(keys_sf), key_rows, max_vis, _p(idx_out),
-                  _p(scores_out), score_dtype)
+                  _p(scores_out), score_dtype, bt, bps)
     _check("v4attn_index_topk", _lib.v4attn_index_topk(ctypes.byref(desc), ctypes.byref(a),
                                                        _p(ws), ws.numel(), _stream(stream)))
 
@@ -179,38 +190,41 @@ def workspace_init(ws, stream=None):
 
 
 def _mqa(fn, desc, Q, q_pos, kv, kv_rows, swa, swa_rows, out, ws, kv_scale, swa_scale, q_seq, B,
-         idx, n_sel, max_vis, sink, lse, q_rmsnorm, stream):
+         idx, n_sel, max_vis, sink, lse, q_rmsnorm, stream, block_table=None):
     n_q = int(q_pos.numel())
+    bt, bps = _bt(block_table)
     a = MqaArgs(n_q, B if B is not None else n_q, _p(Q), _dt(Q), int(q_rmsnorm), _p(q_seq),
                 _p(q_pos), _p(kv), _p(kv_scale), kv_rows, _p(swa), _p(swa_scale), swa_rows,
-                _p(idx), n_sel, max_vis, _p(sink), _p(out), _dt(out), _p(lse))
+                _p(idx), n_sel, max_vis, _p(sink), _p(out), _dt(out), _p(lse), bt, bps)
     _check(fn, getattr(_lib, fn)(ctypes.byref(desc), ctypes.byref(a), _p(ws), ws.numel(),
                                  _stream(stream)))
 
 
 def sparse_mqa(desc: LayerDesc, *, Q, q_pos, kv, kv_rows: int, swa, swa_rows: int, idx, out, ws,
                kv_scale=None, swa_scale=None, q_seq=None, B=None, sink=None, lse=None,
-               q_rmsnorm=False, stream=None):
+               q_rmsnorm=False, block_table=None, stream=None):
     _mqa("v4attn_sparse_mqa", desc, Q, q_pos, kv, kv_rows, swa, swa_rows, out, ws, kv_scale,
-         swa_scale, q_seq, B, idx, int(idx.shape[-1]), 0, sink, lse, q_rmsnorm, stream)
+         swa_scale, q_seq, B, idx, int(idx.shape[-1]), 0, sink, lse, q_rmsnorm, stream,
+         block_table)
 
 
 def dense_mqa(desc: LayerDesc, *, Q, q_pos, kv, kv_rows: int, swa, swa_rows: int, max_vis: int,
               out, ws, kv_scale=None, swa_scale=None, q_seq=None, B=None, sink=None, lse=None,
-              q_rmsnorm=False, stream=None):
+              q_rmsnorm=False, block_table=None, stream=None):
     _mqa("v4attn_dense_mqa", desc, Q, q_pos, kv, kv_rows, swa, swa_rows, out, ws, kv_scale,
-         swa_scale, q_seq, B, None, 0, max_vis, sink, lse, q_rmsnorm, stream)
+         swa_scale, q_seq, B, None, 0, max_vis, sink, lse, q_rmsnorm, stream, block_table)
 
 
 def decode(desc: LayerDesc, *, pos, x_main, tail, bias, kv, kv_rows: int, swa, swa_rows: int,
            Q, out, ws, max_vis: int, kv_scale=None, swa_scale=None, x_idx=None, itail=None,
            ibias=None, keys=None, keys_sf=None, key_rows: int = 0, qI=None, qI_sf=None, w=None,
-           sink=None, lse=None, idx_out=None, stream=None):
+           sink=None, lse=None, idx_out=None, block_table=None, stream=None):
+    bt, bps = _bt(block_table)
     a = DecodeArgs(int(pos.numel()), _p(pos), _dt(x_main), _p(x_main), _p(tail), _p(bias),
                    _p(x_idx), _p(itail), _p(ibias), _p(kv), _p(kv_scale), kv_rows, _p(keys),
                    _p(keys_sf), key_rows, _p(swa), _p(swa_scale), swa_rows, _p(Q), _dt(Q),
                    _p(qI), _p(qI_sf), _p(w), _p(sink), _p(out), _dt(out), _p(lse), _p(idx_out),
-                   max_vis)
+                   max_vis, bt, bps)
     _check("v4attn_decode", _lib.v4attn_decode(ctypes.byref(desc), ctypes.byref(a), _p(ws),
                                                ws.numel(), _stream(stream)))
 

@@ -41,7 +41,8 @@ class IndexArgs(ctypes.Structure):
     _fields_ = [("n_q", c_i32), ("B", c_i32), ("qI", c_ptr), ("qI_sf", c_ptr), ("w", c_ptr),
                 ("q_seq", c_ptr), ("q_pos", c_ptr), ("keys", c_ptr), ("keys_sf", c_ptr),
                 ("key_rows", c_i64), ("max_vis", c_i64), ("idx_out", c_ptr),
-                ("scores_out", c_ptr), ("score_dtype", c_i32)]
+                ("scores_out", c_ptr), ("score_dtype", c_i32), ("block_table", c_ptr),
+                ("blocks_per_seq", c_i32)]
 
 
 class MqaArgs(ctypes.Structure):
@@ -49,7 +50,8 @@ class MqaArgs(ctypes.Structure):
                 ("q_rmsnorm", c_i32), ("q_seq", c_ptr), ("q_pos", c_ptr), ("kv", c_ptr),
                 ("kv_scale", c_ptr), ("kv_rows", c_i64), ("swa", c_ptr), ("swa_scale", c_ptr),
                 ("swa_rows", c_i64), ("idx", c_ptr), ("n_sel", c_i32), ("max_vis", c_i64),
-                ("sink", c_ptr), ("out", c_ptr), ("out_dtype", c_i32), ("lse", c_ptr)]
+                ("sink", c_ptr), ("out", c_ptr), ("out_dtype", c_i32), ("lse", c_ptr),
+                ("block_table", c_ptr), ("blocks_per_seq", c_i32)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -59,7 +61,8 @@ class DecodeArgs(ctypes.Structure):
                 ("keys", c_ptr), ("keys_sf", c_ptr), ("key_rows", c_i64), ("swa", c_ptr),
                 ("swa_scale", c_ptr), ("swa_rows", c_i64), ("Q", c_ptr), ("q_dtype", c_i32),
                 ("qI", c_ptr), ("qI_sf", c_ptr), ("w", c_ptr), ("sink", c_ptr), ("out", c_ptr),
-                ("out_dtype", c_i32), ("lse", c_ptr), ("idx_out", c_ptr), ("max_vis", c_i64)]
+                ("out_dtype", c_i32), ("lse", c_ptr), ("idx_out", c_ptr), ("max_vis", c_i64),
+                ("block_table", c_ptr), ("blocks_per_seq", c_i32)]
 
 
 class ProjectArgs(ctypes.Structure):

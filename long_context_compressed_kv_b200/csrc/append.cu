@@ -286,6 +286,10 @@ __device__ __forceinline__ void copy_share(uint8_t* dst, const uint8_t* src, int
 }
 }  // namespace
 
+// PAGED: the entry and the indexer key go to their block's slot in the pools
+// (A.kv_pages / A.key_pages); a compile-time switch, so that the per-sequence
+// kernel carries none of it
+template <bool PAGED>
 __global__ void __launch_bounds__(kThr, 2) decode_append_kernel(AppendParams A) {
   __shared__ float red[72];
   __shared__ float xch[2 * kCl];
@@ -364,7 +368,13 @@ __global__ void __launch_bounds__(kThr, 2) decode_append_kernel(AppendParams A) 
     float rc, rs;
     pool_channels(a, c_lo, CW, ebuf, part, bsm, rq, rc, rs);
     const int64_t rb = row_bytes(A.kv_dtype, A.d, A.d_rope);
-    const int64_t row = (int64_t)b * A.kv_rows + i % A.kv_rows;
+    // the entry's row: its block's slot in the pool, or this sequence's row
+    // (the same for every CTA of the cluster, so all of them return together)
+    const int64_t row = PAGED ? page_row(A.kv_pages, b, i) : (int64_t)b * A.kv_rows + i % A.kv_rows;
+    if (PAGED && row < 0) {
+      if (rank == 0 && threadIdx.x == 0) flag(A.status, ST_BAD_INDEX);
+      return;
+    }
     uint8_t* orow = reinterpret_cast<uint8_t*>(A.kv) + row * rb;
     // this CTA's channels, offset so that finish_main writes them in place
     finish_main(ebuf, c_lo, CW, A.d, A.d_rope, true, true, rc, rs, A.eps, A.kv_dtype, orow,
@@ -382,7 +392,12 @@ __global__ void __launch_bounds__(kThr, 2) decode_append_kernel(AppendParams A) 
   RopeReq none{false, 0, 0, 0, 0.f};
   float rc, rs;
   pool_channels(a, c_lo, CW, ebuf, part, bsm, none, rc, rs);
-  const int64_t row = (int64_t)b * A.key_rows + i % A.key_rows;
+  const int64_t row =
+      PAGED ? page_row(A.key_pages, b, i) : (int64_t)b * A.key_rows + i % A.key_rows;
+  if (PAGED && row < 0) {                            // after the pooling: no barrier follows
+    if (rank == 0 && threadIdx.x == 0) flag(A.status, ST_BAD_INDEX);
+    return;
+  }
   if (A.idx_dtype == V4A_MXFP4) {
     finish_mxfp4(ebuf, c_lo, reinterpret_cast<uint8_t*>(A.keys) + row * (A.dI / 2),
                  reinterpret_cast<uint8_t*>(A.keys_sf) + row * (A.dI / 32));
@@ -406,7 +421,8 @@ cudaError_t launch_decode_append(const AppendParams& A, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_append_kernel, A);
+  return A.kv_pages.bt ? cudaLaunchKernelEx(&cfg, decode_append_kernel<true>, A)
+                       : cudaLaunchKernelEx(&cfg, decode_append_kernel<false>, A);
 }
 
 }  // namespace v4a

@@ -166,6 +166,31 @@ v4attn_status tc_status(int code) {
   return code == 0 ? V4A_OK : (code == 1 ? V4A_ERR_INVALID_ARG : V4A_ERR_UNSUPPORTED);
 }
 
+// Paged caches (see "Paged caches" in v4attn.h): a block table needs at least
+// one block per sequence, 128 % m == 0 (blocks of 128 raw tokens), the
+// tensor-core formats and a pool of whole blocks.
+static v4attn_status check_pages(const v4attn_layer_desc* d, const int32_t* bt, int32_t bps,
+                                 int64_t rows, bool tc_format) {
+  if (!bt) return V4A_OK;
+  if (bps < 1 || rows < 1 || (reinterpret_cast<uintptr_t>(bt) & 3)) return V4A_ERR_INVALID_ARG;
+  if (128 % d->m != 0 || !tc_format) return V4A_ERR_UNSUPPORTED;
+  if (rows % (128 / d->m) != 0) return V4A_ERR_INVALID_ARG;
+  return V4A_OK;
+}
+static PageMap page_map(const v4attn_layer_desc* d, const int32_t* bt, int32_t bps, int64_t rows) {
+  PageMap pm;
+  if (!bt) return pm;
+  pm.bt = bt;
+  pm.bps = bps;
+  pm.epb = 128 / d->m;
+  pm.n_blocks = rows / pm.epb;
+  return pm;
+}
+// Entries a sequence can hold: its part of the cache, or its blocks of the pool.
+static int64_t seq_cap(const v4attn_layer_desc* d, const int32_t* bt, int32_t bps, int64_t rows) {
+  return bt ? (int64_t)bps * (128 / d->m) : rows;
+}
+
 // `dry`: validate and return without launching.  `wait_ns` / `stall`: the
 // failure-detection test hook (see v4attn_debug_index_stall).
 v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args* a, void* ws,
@@ -179,7 +204,13 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
   if (a->score_dtype != V4A_F32 && a->score_dtype != V4A_BF16) return V4A_ERR_INVALID_ARG;
   const int sbf = a->score_dtype == V4A_BF16 ? 1 : 0;
   const size_t s_esz = sbf ? 2 : 4;
-  if (a->key_rows < 1 || a->max_vis < 0 || a->max_vis > a->key_rows) return V4A_ERR_INVALID_ARG;
+  if (const v4attn_status sp = check_pages(d, a->block_table, a->blocks_per_seq, a->key_rows,
+                                           d->idx_dtype == V4A_MXFP4))
+    return sp;
+  const PageMap pages = page_map(d, a->block_table, a->blocks_per_seq, a->key_rows);
+  if (a->key_rows < 1 || a->max_vis < 0 ||
+      a->max_vis > seq_cap(d, a->block_table, a->blocks_per_seq, a->key_rows))
+    return V4A_ERR_INVALID_ARG;
   if (!ws) return V4A_ERR_WORKSPACE;
   if (ws_bytes < body_off + index_need(a->n_q, a->max_vis)) return V4A_ERR_WORKSPACE;
   uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
@@ -204,6 +235,7 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
     P.keys_sf = a->keys_sf;
     P.key_rows = a->key_rows;
     P.max_vis = a->max_vis;
+    P.pages = pages;
     const v4attn_status s = tc_status(index_tc_check(P));
     if (s != V4A_OK) return s;
   }
@@ -236,6 +268,7 @@ v4attn_status run_index_topk(const v4attn_layer_desc* d, const v4attn_index_args
       P.scores_ld = ld;
       P.score_bf16 = sbf;
       P.status = status;
+      P.pages = pages;
       P.wait_ns = wait_ns;
       P.stall = stall;
       if (const cudaError_t e = index_scores_dispatch(P, st)) return cuda_status(e);
@@ -268,7 +301,12 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
   if (a->out_dtype != V4A_F32 && a->out_dtype != V4A_BF16) return V4A_ERR_UNSUPPORTED;
   if (a->kv_rows < 1) return V4A_ERR_INVALID_ARG;
   if (sparse && (!a->idx || a->n_sel < 1 || a->n_sel > 4096)) return V4A_ERR_INVALID_ARG;
-  if (!sparse && (a->max_vis < 0 || a->max_vis > a->kv_rows)) return V4A_ERR_INVALID_ARG;
+  if (const v4attn_status sp = check_pages(d, a->block_table, a->blocks_per_seq, a->kv_rows,
+                                           d->kv_dtype == V4A_E4M3_BF16ROPE))
+    return sp;
+  if (!sparse && (a->max_vis < 0 ||
+                  a->max_vis > seq_cap(d, a->block_table, a->blocks_per_seq, a->kv_rows)))
+    return V4A_ERR_INVALID_ARG;
   if (!aligned16(a->kv) || (a->swa && !aligned16(a->swa)) || !aligned16(a->out))
     return V4A_ERR_INVALID_ARG;
   if (!ws) return V4A_ERR_WORKSPACE;
@@ -322,6 +360,7 @@ v4attn_status run_mqa(const v4attn_layer_desc* d, const v4attn_mqa_args* a, void
     P.out_dtype = a->out_dtype;
     P.lse = a->lse ? a->lse + (int64_t)q0 * d->H : nullptr;
     P.status = reinterpret_cast<uint32_t*>(ws);
+    P.pages = page_map(d, a->block_table, a->blocks_per_seq, a->kv_rows);
     if (q0 == 0 && d->kv_dtype == V4A_E4M3_BF16ROPE) {
       const v4attn_status s = tc_status(mqa_tc_check(P));
       if (s != V4A_OK) return s;
@@ -390,7 +429,13 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
   if (csa && (!a->x_idx || !a->itail || !a->keys || !a->qI || !a->w || !a->idx_out))
     return V4A_ERR_INVALID_ARG;
   if (a->in_dtype != V4A_F32 && a->in_dtype != V4A_BF16) return V4A_ERR_UNSUPPORTED;
-  if (a->max_vis < 0 || a->max_vis > a->kv_rows || (csa && a->max_vis > a->key_rows))
+  if (const v4attn_status sp = check_pages(desc, a->block_table, a->blocks_per_seq, a->kv_rows,
+                                           desc->kv_dtype == V4A_E4M3_BF16ROPE &&
+                                               (!csa || desc->idx_dtype == V4A_MXFP4)))
+    return sp;
+  if (csa && a->block_table && a->key_rows % (128 / desc->m) != 0) return V4A_ERR_INVALID_ARG;
+  if (a->max_vis < 0 || a->max_vis > seq_cap(desc, a->block_table, a->blocks_per_seq, a->kv_rows) ||
+      (csa && a->max_vis > seq_cap(desc, a->block_table, a->blocks_per_seq, a->key_rows)))
     return V4A_ERR_INVALID_ARG;
   if (!ws) return V4A_ERR_WORKSPACE;
   if (ws_bytes < total_need(desc, a->B, a->max_vis)) return V4A_ERR_WORKSPACE;
@@ -445,6 +490,9 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
   A.keys = csa ? a->keys : nullptr;
   A.keys_sf = csa ? a->keys_sf : nullptr;
   A.key_rows = csa ? a->key_rows : 0;
+  A.kv_pages = page_map(desc, a->block_table, a->blocks_per_seq, a->kv_rows);
+  if (csa) A.key_pages = page_map(desc, a->block_table, a->blocks_per_seq, a->key_rows);
+  A.status = reinterpret_cast<uint32_t*>(ws);
   // the tensor-core MQA's query images, coded in the same launch when its
   // format applies and the step's queries fit one query chunk
   const bool fuse_q = desc->kv_dtype == V4A_E4M3_BF16ROPE && a->q_dtype == V4A_BF16 &&
@@ -472,6 +520,8 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
     ix.key_rows = a->key_rows;
     ix.max_vis = a->max_vis;
     ix.idx_out = a->idx_out;
+    ix.block_table = a->block_table;
+    ix.blocks_per_seq = a->blocks_per_seq;
     s = run_index_topk(desc, &ix, ws, ws_bytes, stream, body_mqa(desc, a->B), true);
     if (s != V4A_OK) return s;
   }
@@ -495,6 +545,8 @@ v4attn_status v4attn_decode(const v4attn_layer_desc* desc, const v4attn_decode_a
   q.out = a->out;
   q.out_dtype = a->out_dtype;
   q.lse = a->lse;
+  q.block_table = a->block_table;
+  q.blocks_per_seq = a->blocks_per_seq;
   s = run_mqa(desc, &q, ws, ws_bytes, stream, csa, fuse_q, true);
   if (s != V4A_OK) return s;
   if (const cudaError_t e = launch_decode_append(A, stream)) return cuda_status(e);

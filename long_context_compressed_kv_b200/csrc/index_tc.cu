@@ -121,8 +121,14 @@ __device__ __forceinline__ int stage_tiles(const S& s, const TileIter& t, int g,
 
 // N = MMA N: the indexer heads, or with PAIR two consecutive queries of one
 // sequence side by side (2 x H_I columns), so that every key tile serves both:
-// half the MMAs per score where many queries share their keys (prefill)
-template <int N, bool PAIR>
+// half the MMAs per score where many queries share their keys (prefill).
+// PAGED: the keys are a pool of 32-key blocks (a classical block of 128 raw
+// tokens holds 32 indexer keys) reached through P.pages; a 128-key tile is
+// four blocks, each loaded by its own TMA box of 32 rows (tm_keys then has a
+// box of {64 B, 8, 4}), so MMA row 32 kb + 8 c + l holds key 32 kb + 4 l + c
+// of the tile's block kb, and the producer's lanes copy the key scales into
+// the matching scale-factor order (lane 8 c + l, column kb) one 4-byte word each.
+template <int N, bool PAIR, bool PAGED>
 __global__ void __launch_bounds__(NTHREADS, Cfg<N>::CPS)
     index_tc_kernel(IndexParams P, const __grid_constant__ CUtensorMap tm_keys,
                     const __grid_constant__ CUtensorMap tm_q) {
@@ -144,6 +150,8 @@ __global__ void __launch_bounds__(NTHREADS, Cfg<N>::CPS)
   const int n_g = P.n_q / QPG;                          // query groups (n_q even with PAIR)
   const uint32_t lim = P.wait_ns ? P.wait_ns : (uint32_t)kWaitNs;   // bound of every wait
 
+  // keys a sequence can hold: its part of the cache, or its blocks of the pool
+  const int64_t cap = PAGED ? (int64_t)P.pages.bps * P.pages.epb : P.key_rows;
   // visible keys of query q (checked); a group's tiles cover its largest
   auto visible = [&](int q) -> int64_t {
     int64_t nv = (P.q_pos[q] + 1) / P.m;
@@ -152,9 +160,9 @@ __global__ void __launch_bounds__(NTHREADS, Cfg<N>::CPS)
       flag(P.status, ST_BAD_SEQ);
       nv = 0;
     }
-    if (nv > P.key_rows || nv > P.max_vis) {
+    if (nv > cap || nv > P.max_vis) {
       flag(P.status, ST_BAD_POSITION);
-      nv = min(P.key_rows, P.max_vis);
+      nv = min(cap, P.max_vis);
     }
     return nv;
   };
@@ -163,7 +171,9 @@ __global__ void __launch_bounds__(NTHREADS, Cfg<N>::CPS)
   if (threadIdx.x == 0) {
     s.abort = 0;
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&s.full[i], 1);    // the producer lane's arrive + TMA / bulk bytes
+      // the producer lane's arrive + TMA / bulk bytes (paged: every producer
+      // lane's arrive, once its scale copies have landed, + TMA bytes)
+      mbar_init(&s.full[i], PAGED ? 32 : 1);
       mbar_init(&s.empty[i], 1);   // the epilogue's releaser, once the stage's MMAs are done
       mbar_init(&s.accstage[i], 1);   // one commit after all MMAs of a stage
     }
@@ -220,12 +230,17 @@ __global__ void __launch_bounds__(NTHREADS, Cfg<N>::CPS)
     int stg = 0;
     int qissued = 0;                            // query-buffer loads issued
     int b = 0;                                  // sequence of the current query
+    int64_t nvg = 0;                            // paged: visible keys of the current group
     for (int g = g0; g < g1 && !aborted(); ++stg) {
       const int seg_before = t.seg;
       locate(s, n_g, g, t);
       const int n = stage_tiles(s, t, g, g1, TPS_N);
       if (t.seg != seg_before) {
         b = s.seq[t.q];
+        if constexpr (PAGED) {
+          nvg = min((int64_t)(P.q_pos[t.q * QPG] + 1) / P.m, min(cap, P.max_vis));
+          if (PAIR) nvg = max(nvg, min((int64_t)(P.q_pos[t.q * QPG + 1] + 1) / P.m, min(cap, P.max_vis)));
+        }
         const int j = t.seg & 1, uq = t.seg >> 1;
         if (uq >= 1 && !mbar_wait_warp(&s.qempty[j], (uq - 1) & 1, P.status, -1, lim)) {
           fail(s, P.status);
@@ -245,6 +260,44 @@ __global__ void __launch_bounds__(NTHREADS, Cfg<N>::CPS)
       if (u >= 1 && !mbar_wait_warp(&s.empty[st], (u - 1) & 1, P.status, -1, lim)) {
         fail(s, P.status);
         break;
+      }
+      if constexpr (PAGED) {
+        // block kb of tile k: keys (lt + k) * 128 + 32 kb .. +31 of the sequence,
+        // pool rows pr .. pr + 31; blocks at or past the group's visible keys
+        // are not loaded (their rows are masked in the epilogue)
+        int64_t pr[TPS * 4];
+        uint32_t bytes = 0;
+#pragma unroll
+        for (int i = 0; i < TPS * 4; ++i) {
+          pr[i] = -1;
+          if (i < 4 * n) {
+            const int64_t e = (int64_t)(t.lt + i / 4) * KT + 32 * (i % 4);
+            if (e < nvg) {
+              pr[i] = page_row(P.pages, b, e);
+              if (pr[i] < 0 && lane == 0) flag(P.status, ST_BAD_INDEX);
+            }
+            if (pr[i] >= 0) bytes += 32 * KROW;
+          }
+        }
+        if (lane == 0) mbar_expect_tx(&s.full[st], bytes);
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int i = 0; i < TPS * 4; ++i)
+            if (pr[i] >= 0)
+              tma_load_3d(s.keys[st][i / 4] + (i % 4) * 32 * KROW, &tm_keys, &s.full[st], 0,
+                          (int)(pr[i] >> 2), 0);
+        }
+        // lane 8 c + l, column kb: the scale word of key 32 kb + 4 l + c
+        const int kin = 4 * (lane & 7) + (lane >> 3);
+#pragma unroll
+        for (int i = 0; i < TPS * 4; ++i)
+          if (i < 4 * n)
+            cp_async4(&s.sfa_raw[st][(i / 4) * KT + 4 * lane + (i % 4)],
+                      ksf32 + (pr[i] >= 0 ? pr[i] + kin : 0), pr[i] >= 0);
+        cp_async_arrive_noinc(&s.full[st]);
+        g += n;
+        continue;
       }
       const int64_t row0 = (int64_t)b * P.key_rows + (int64_t)t.lt * KT;
       if (lane == 0) {
@@ -362,7 +415,8 @@ __global__ void __launch_bounds__(NTHREADS, Cfg<N>::CPS)
     // TMEM lanes 32*(w%4) .. +31 (one key per thread)
     const int grp = (warp - 2) >> 2;
     const int quad = warp & 3;
-    const int r = 4 * lane + quad;              // key of TMEM lane 32 * quad + lane
+    // key of TMEM lane 32 * quad + lane (its MMA row) within the tile
+    const int r = PAGED ? 32 * quad + 4 * (lane & 7) + (lane >> 3) : 4 * lane + quad;
     {
       // keys beyond the last tile of each query (group): -inf
       const int et = threadIdx.x - 64;
@@ -525,13 +579,14 @@ bool make_rows_map_sw(CUtensorMap* map, const void* base, int64_t rows, int row_
 // 3-D uint8 view of the MXFP4 key codes (64-byte rows, row count divisible by
 // 4): dims {64 B, rows / 4, 4} with strides {256 B, 64 B}.  A box {64, 32, 4}
 // at (0, row0 / 4, 0) lands rows row0 + 4l + c at shared-memory row 32c + l,
-// 64-byte swizzled; rows past the end of the array read as zero.
-static bool make_keys_map(CUtensorMap* map, const void* base, int64_t rows) {
+// 64-byte swizzled; rows past the end of the array read as zero.  With
+// box_l = 8 (paged keys: one 32-key block) row0 + 4l + c lands at row 8c + l.
+static bool make_keys_map(CUtensorMap* map, const void* base, int64_t rows, int box_l = 32) {
   EncodeTiledFn enc = encode_fn();
   if (!enc || rows < 4 || (rows & 3) || rows > (1ll << 31)) return false;
   cuuint64_t dims[3] = {(cuuint64_t)KROW, (cuuint64_t)(rows / 4), 4};
   cuuint64_t strides[2] = {(cuuint64_t)(4 * KROW), (cuuint64_t)KROW};
-  cuuint32_t box[3] = {(cuuint32_t)KROW, 32, 4};
+  cuuint32_t box[3] = {(cuuint32_t)KROW, (cuuint32_t)box_l, 4};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
@@ -545,7 +600,11 @@ int index_tc_check(const IndexParams& P) {
   // the scale and weight rows are moved by 1-D bulk copies: 16-byte aligned
   // sources, i.e. 16-byte aligned bases and a key row count divisible by 4
   // (the 3-D key view needs the latter too)
-  if (P.key_rows % 4 != 0 || (int64_t)P.B * P.key_rows > (1ll << 31)) return 2;
+  if (P.key_rows % 4 != 0 ||
+      (P.pages.bt ? P.key_rows : (int64_t)P.B * P.key_rows) > (1ll << 31))
+    return 2;
+  // paged keys: a pool of whole 32-key blocks (m = 4: 128 raw tokens a block)
+  if (P.pages.bt && (P.pages.epb != 32 || P.key_rows % 32 != 0)) return 2;
   if (((uintptr_t)P.keys & 15) || ((uintptr_t)P.qI & 15) || ((uintptr_t)P.keys_sf & 15) ||
       ((uintptr_t)P.qI_sf & 15) || ((uintptr_t)P.w & 15))
     return 1;
@@ -554,7 +613,10 @@ int index_tc_check(const IndexParams& P) {
 
 cudaError_t launch_index_tc(const IndexParams& P, cudaStream_t st) {
   CUtensorMap tk, tq;
-  if (!make_keys_map(&tk, P.keys, (int64_t)P.B * P.key_rows)) return cudaErrorInvalidValue;
+  const bool paged = P.pages.bt != nullptr;
+  if (!(paged ? make_keys_map(&tk, P.keys, P.key_rows, 8)
+              : make_keys_map(&tk, P.keys, (int64_t)P.B * P.key_rows)))
+    return cudaErrorInvalidValue;
   // two consecutive queries per MMA (N = 2 H_I) when every query belongs to
   // the one sequence of the call and they pair up evenly
   const bool pair = P.B == 1 && P.n_q >= 2 && P.n_q % 2 == 0 && P.H_I <= 64;
@@ -575,13 +637,24 @@ cudaError_t launch_index_tc(const IndexParams& P, cudaStream_t st) {
     return cudaSuccess;
   };
   cudaError_t e = cudaSuccess;
-  switch (nmma * (pair ? -1 : 1)) {
-    case 32: e = launch(index_tc_kernel<32, false>, Cfg<32>{}); break;
-    case 64: e = launch(index_tc_kernel<64, false>, Cfg<64>{}); break;
-    case 128: e = launch(index_tc_kernel<128, false>, Cfg<128>{}); break;
-    case -64: e = launch(index_tc_kernel<64, true>, Cfg<64>{}); break;
-    case -128: e = launch(index_tc_kernel<128, true>, Cfg<128>{}); break;
-    default: return cudaErrorInvalidValue;
+  if (paged) {
+    switch (nmma * (pair ? -1 : 1)) {
+      case 32: e = launch(index_tc_kernel<32, false, true>, Cfg<32>{}); break;
+      case 64: e = launch(index_tc_kernel<64, false, true>, Cfg<64>{}); break;
+      case 128: e = launch(index_tc_kernel<128, false, true>, Cfg<128>{}); break;
+      case -64: e = launch(index_tc_kernel<64, true, true>, Cfg<64>{}); break;
+      case -128: e = launch(index_tc_kernel<128, true, true>, Cfg<128>{}); break;
+      default: return cudaErrorInvalidValue;
+    }
+  } else {
+    switch (nmma * (pair ? -1 : 1)) {
+      case 32: e = launch(index_tc_kernel<32, false, false>, Cfg<32>{}); break;
+      case 64: e = launch(index_tc_kernel<64, false, false>, Cfg<64>{}); break;
+      case 128: e = launch(index_tc_kernel<128, false, false>, Cfg<128>{}); break;
+      case -64: e = launch(index_tc_kernel<64, true, false>, Cfg<64>{}); break;
+      case -128: e = launch(index_tc_kernel<128, true, false>, Cfg<128>{}); break;
+      default: return cudaErrorInvalidValue;
+    }
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

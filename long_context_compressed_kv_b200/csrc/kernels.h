@@ -6,6 +6,28 @@
 
 namespace v4a {
 
+// Paged compressed caches (see "Paged caches" in v4attn.h): entry e of
+// sequence b at row bt[b * bps + e / epb] * epb + e % epb of a pool of
+// n_blocks * epb rows; bt == nullptr: per-sequence caches.
+struct PageMap {
+  const int32_t* bt = nullptr;
+  int32_t bps = 0;        // blocks per sequence (columns of the table)
+  int32_t epb = 1;        // entries per block: 128 / m
+  int64_t n_blocks = 0;   // blocks in the pool
+};
+
+#if defined(__CUDACC__)
+// Pool row of entry e of sequence b, or -1 when the table holds no valid
+// block for it (a table entry outside [0, n_blocks) or e past the table).
+__device__ __forceinline__ int64_t page_row(const PageMap& pm, int b, int64_t e) {
+  const int64_t lb = e / pm.epb;
+  if (e < 0 || lb >= pm.bps) return -1;
+  const int32_t pb = __ldg(pm.bt + (int64_t)b * pm.bps + lb);
+  if (pb < 0 || (int64_t)pb >= pm.n_blocks) return -1;
+  return (int64_t)pb * pm.epb + (e - lb * pm.epb);
+}
+#endif
+
 struct CompressParams {
   int m, overlap, c;
   const void *Ca, *Za, *Cb, *Zb;
@@ -56,6 +78,10 @@ struct AppendParams {
   const void* Q = nullptr;
   int H = 0;
   uint8_t* qimg = nullptr;
+  // paged caches: the entry's and the indexer key's rows come from the block
+  // table (a bad table entry sets ST_BAD_INDEX in *status and skips the write)
+  PageMap kv_pages, key_pages;
+  uint32_t* status = nullptr;
 };
 
 struct IndexParams {
@@ -76,6 +102,7 @@ struct IndexParams {
   uint32_t wait_ns = 0; // bound of the tensor-core kernel's waits (0: the default, 1 s)
   int stall = 0;        // debug: the tensor-core kernel's MMA warp waits on a barrier
                         // nothing completes, so that its bounded wait runs out
+  PageMap pages;        // paged keys (tensor-core kernel): key_rows = pool rows
 };
 
 struct TopkParams {
@@ -129,6 +156,7 @@ struct MqaParams {
   int out_dtype;
   float* lse;
   uint32_t* status;
+  PageMap pages;        // paged entries (tensor-core kernel): kv_rows = pool rows
 };
 
 struct ProjectParams {

@@ -249,7 +249,9 @@ struct Geo {
   int64_t pq[2], nq[2];
 };
 
-// Position and visible entries of query q, checked against the call's bounds.
+// Position and visible entries of query q, checked against the call's bounds
+// (PAGED: a sequence holds at most its table's blocks of entries).
+template <bool PAGED>
 __device__ __forceinline__ void query_span(const MqaParams& P, int q, int& b, int64_t& p,
                                            int64_t& nv) {
   b = P.q_seq ? P.q_seq[q] : P.q_base + q;
@@ -261,9 +263,10 @@ __device__ __forceinline__ void query_span(const MqaParams& P, int q, int& b, in
     nv = 0;
     p = -1;
   }
-  if (nv > P.kv_rows) {
+  const int64_t cap = PAGED ? (int64_t)P.pages.bps * P.pages.epb : P.kv_rows;
+  if (nv > cap) {
     if (threadIdx.x == 0) flag(P.status, ST_BAD_POSITION);
-    nv = P.kv_rows;
+    nv = cap;
   }
   if (!P.idx && nv > P.max_vis) {
     if (threadIdx.x == 0) flag(P.status, ST_BAD_POSITION);
@@ -274,13 +277,13 @@ __device__ __forceinline__ void query_span(const MqaParams& P, int q, int& b, in
 // q: the query, or with P.pair the pair (queries 2q, 2q + 1 of one sequence:
 // the union of their visible entries and of their windows, each row masked to
 // its own query's in the softmax)
-template <bool PAIR>
+template <bool PAIR, bool PAGED>
 __device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
   Geo g;
   if (PAIR) {
     int b1;
-    query_span(P, 2 * q, g.b, g.pq[0], g.nq[0]);
-    query_span(P, 2 * q + 1, b1, g.pq[1], g.nq[1]);
+    query_span<PAGED>(P, 2 * q, g.b, g.pq[0], g.nq[0]);
+    query_span<PAGED>(P, 2 * q + 1, b1, g.pq[1], g.nq[1]);
     if (b1 != g.b) {
       if (threadIdx.x == 0) flag(P.status, ST_BAD_SEQ);
       g.nq[1] = 0;
@@ -292,7 +295,7 @@ __device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
     g.n_main = (int)g.n_vis;
     g.n_swa = g.p >= 0 ? (int)(g.p - lo + 1) : 0;
   } else {
-    query_span(P, q, g.b, g.p, g.n_vis);
+    query_span<PAGED>(P, q, g.b, g.p, g.n_vis);
     g.pq[0] = g.pq[1] = g.p;
     g.nq[0] = g.nq[1] = g.n_vis;
     g.n_main = P.idx ? P.n_sel : (int)g.n_vis;
@@ -307,7 +310,7 @@ __device__ __forceinline__ Geo geometry(const MqaParams& P, int q, int split) {
   // call every tile is gathered and counts one.  Split `split` of C takes
   // the tiles whose cost prefix starts in [W split / C, W (split + 1) / C).
   const int mt = g.nmp / NK, wt = (g.total - g.nmp) / NK, C = P.n_split;
-  const int wc = P.idx ? 1 : kWinCost;
+  const int wc = (PAGED || P.idx) ? 1 : kWinCost;   // paged entries are gathered too
   const int64_t W = mt + (int64_t)wc * wt;
   auto tile_at = [&](int64_t x) -> int {        // first tile whose cost prefix is >= x
     return (int)(x <= mt ? x : mt + (x - mt + wc - 1) / wc);
@@ -334,8 +337,11 @@ __global__ void __launch_bounds__(64) mqa_tc_qprep_kernel(MqaParams P) {
 
 // 576 threads = 18 warps: on the SM sub-partition that holds five of them at
 // most 16384 / 5 registers a warp, hence 96 registers a thread
-// PAIR: two consecutive queries of one sequence per CTA (see MqaParams::pair)
-template <bool PAIR>
+// PAIR: two consecutive queries of one sequence per CTA (see MqaParams::pair).
+// PAGED: entry rows through the block table (P.pages), every main tile
+// gathered; a compile-time switch, so that the per-sequence kernel carries
+// none of it
+template <bool PAIR, bool PAGED>
 __global__ void __launch_bounds__(NTHR, 1)
     mqa_tc_kernel(MqaParams P, const __grid_constant__ Maps maps) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -347,7 +353,7 @@ __global__ void __launch_bounds__(NTHR, 1)
   const int split = (int)(blockIdx.x % (unsigned)C);
   const int unit = (int)(blockIdx.x / (unsigned)C);
   const int dh = unit & 1, q = unit >> 1;
-  const Geo g = geometry<PAIR>(P, q, split);
+  const Geo g = geometry<PAIR, PAGED>(P, q, split);
   // the grid barrier's generation before this CTA arrives (merging launches)
   const uint32_t bar_gen0 = (C > 1 && threadIdx.x == 0) ? ld_acquire_gpu(P.grid_bar + 1) : 0u;
   // every CTA, also one with no tiles (T = 0), takes part in the merge below
@@ -388,7 +394,10 @@ __global__ void __launch_bounds__(NTHR, 1)
     // zero-filled for empty slots (a stored scale is a nonzero power of two,
     // so a zero scale marks an empty slot); every lane arrives on full[st]
     // through cp.async.mbarrier.arrive.noinc once its scale copies land.
-    const int64_t kv_base = (int64_t)g.b * P.kv_rows, sw_base = (int64_t)g.b * P.swa_rows;
+    // paged entries: rows of the pool (through the block table), else of
+    // this sequence's part of the cache
+    const int64_t kv_base = PAGED ? 0 : (int64_t)g.b * P.kv_rows;
+    const int64_t sw_base = (int64_t)g.b * P.swa_rows;
     // global row of key r of tile vk, or -1 when the slot is empty
     auto row_of = [&](int vk, int r, bool main_tile) -> int64_t {
       if (main_tile) {
@@ -399,6 +408,11 @@ __global__ void __launch_bounds__(NTHR, 1)
         if (e >= g.n_vis) {
           flag(P.status, ST_BAD_INDEX);
           return -1;
+        }
+        if constexpr (PAGED) {
+          const int64_t row = page_row(P.pages, g.b, e);
+          if (row < 0) flag(P.status, ST_BAD_INDEX);
+          return row;
         }
         return kv_base + e;
       }
@@ -418,7 +432,7 @@ __global__ void __launch_bounds__(NTHR, 1)
       issued = t + 1;
       const int vk = g.s0 + t * NK;
       const bool main_tile = vk < g.nmp;
-      const bool contiguous = main_tile && !P.idx && vk + NK <= g.n_main;
+      const bool contiguous = !PAGED && main_tile && !P.idx && vk + NK <= g.n_main;
       if (lane == 0) mbar_expect_tx(&s.full[st], TILE_BYTES);
       __syncwarp();
       if (contiguous) {
@@ -949,7 +963,8 @@ bool make_rows_map_sw(CUtensorMap* map, const void* base, int64_t rows, int row_
 int mqa_tc_check(const MqaParams& P) {
   if (P.kv_dtype != V4A_E4M3_BF16ROPE || P.d != 512 || P.d_rope != 64 || P.H > 128 ||
       P.q_dtype != V4A_BF16 || P.n_win > 1024 || P.qbuf == nullptr ||
-      (int64_t)P.B * P.kv_rows >= (1ll << 31) || (int64_t)P.B * P.swa_rows >= (1ll << 31))
+      (P.pages.bt ? P.kv_rows : (int64_t)P.B * P.kv_rows) >= (1ll << 31) ||
+      (int64_t)P.B * P.swa_rows >= (1ll << 31))
     return 2;
   if (((uintptr_t)P.qbuf & 15) || ((uintptr_t)P.kv & 15) ||
       (P.n_win > 0 && ((uintptr_t)P.swa & 15)) || ((uintptr_t)P.Q & 15))
@@ -959,7 +974,7 @@ int mqa_tc_check(const MqaParams& P) {
 
 cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   Maps m;
-  const int64_t kv_rows = (int64_t)P.B * P.kv_rows;
+  const int64_t kv_rows = P.pages.bt ? P.kv_rows : (int64_t)P.B * P.kv_rows;   // rows the maps cover
   const int64_t sw_rows = (int64_t)P.B * P.swa_rows;
   const void* swa = P.swa ? (const void*)P.swa : (const void*)P.kv;
   const int64_t swr = P.swa ? sw_rows : kv_rows;
@@ -977,14 +992,15 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   // per device: CTAs that can be resident at once (one per SM)
   static int resident[64] = {0};
   if (resident[dev] == 0) {
-    cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(mqa_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
+    cudaError_t e = cudaSuccess;
+    for (auto k : {mqa_tc_kernel<false, false>, mqa_tc_kernel<true, false>,
+                   mqa_tc_kernel<false, true>, mqa_tc_kernel<true, true>})
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0, n_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mqa_tc_kernel<false>, NTHR, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mqa_tc_kernel<false, false>, NTHR,
+                                                      smem);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     resident[dev] = std::max(1, per_sm * n_sm);
@@ -994,8 +1010,8 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   // least kMinSplitTiles key tiles in a dense call (a split's fixed cost, its
   // start and its share of the merge, is worth about that many contiguous
   // tiles; gathered tiles are bound by the copy engine of their SM, so a
-  // sparse call spreads them over as many SMs as it can); one when fewer
-  // than two fit, which needs no partials and no grid barrier
+  // sparse call, or a paged one, spreads them over as many SMs as it can);
+  // one when fewer than two fit, which needs no partials and no grid barrier
   MqaParams Q = P;
   // Two consecutive queries per CTA (their 2 x H <= 128 head rows side by
   // side, sharing every key tile) when a dense call's queries all belong to
@@ -1007,7 +1023,8 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   const int64_t cap = std::min<int64_t>(resident[dev], kMqaTcMaxCtas);
   int64_t C = 1;
   if (units * 2 <= cap)
-    C = std::max<int64_t>(1, std::min<int64_t>({cap / units, P.idx ? tiles : tiles / kMinSplitTiles,
+    C = std::max<int64_t>(1, std::min<int64_t>({cap / units,
+                                               (P.idx || P.pages.bt) ? tiles : tiles / kMinSplitTiles,
                                                (int64_t)kMaxSplit}));
   Q.n_split = (int)C;
   if (C > 1 && (Q.part_o == nullptr || Q.part_ml == nullptr || Q.grid_bar == nullptr))
@@ -1027,8 +1044,11 @@ cudaError_t launch_mqa_tc(const MqaParams& P, cudaStream_t st) {
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = C > 1 ? 1 : 0;
-  return Q.pair ? cudaLaunchKernelEx(&cfg, mqa_tc_kernel<true>, Q, m)
-                : cudaLaunchKernelEx(&cfg, mqa_tc_kernel<false>, Q, m);
+  if (P.pages.bt)
+    return Q.pair ? cudaLaunchKernelEx(&cfg, mqa_tc_kernel<true, true>, Q, m)
+                  : cudaLaunchKernelEx(&cfg, mqa_tc_kernel<false, true>, Q, m);
+  return Q.pair ? cudaLaunchKernelEx(&cfg, mqa_tc_kernel<true, false>, Q, m)
+                : cudaLaunchKernelEx(&cfg, mqa_tc_kernel<false, false>, Q, m);
 }
 
 }  // namespace v4a

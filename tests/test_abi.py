@@ -212,3 +212,52 @@ def test_tensor_core_formats_are_refused_not_downgraded():
     a.max_vis = 4096
     assert lib.v4attn_decode(ctypes.byref(dc), ctypes.byref(a), ws, big, None) == \
         _abi.ERR_UNSUPPORTED
+
+
+@pytest.mark.skipif(not _no_gpu(), reason="host-only check with fake device pointers")
+def test_block_table_arguments_are_checked():
+    """Paged caches (include/v4attn.h, "Paged caches"): a block table needs at
+    least one block per sequence, a 4-byte aligned table, a pool of whole blocks
+    (32 CSA entries / indexer keys or 1 HCA entry a block), a visible bound
+    within the table, and the tensor-core formats; each violation is refused
+    before any launch (fake pointers, never dereferenced)."""
+    from long_context_compressed_kv_b200 import _abi
+    lib = _abi.load()
+    fake = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(1 << 21)
+    big = 1 << 40
+
+    def mqa(kind, m, kv_fmt, kv_rows, bps, max_vis, bt=fake):
+        d = _abi.LayerDesc(kind, m, 128, 64, 512, 64, 160000.0, 0.0, 64, 128, 64, kv_fmt,
+                           _abi.MXFP4, 1e-6)
+        q = _abi.MqaArgs()
+        q.n_q, q.B = 2, 2
+        for f in ("Q", "q_pos", "kv", "kv_scale", "swa", "swa_scale", "sink", "out"):
+            setattr(q, f, fake)
+        q.q_dtype, q.out_dtype = _abi.BF16, _abi.BF16
+        q.kv_rows, q.swa_rows, q.max_vis = kv_rows, 128, max_vis
+        q.block_table, q.blocks_per_seq = bt, bps
+        if kind == _abi.CSA:
+            q.idx, q.n_sel = fake, 64
+            return lib.v4attn_sparse_mqa(ctypes.byref(d), ctypes.byref(q), ws, big, None)
+        return lib.v4attn_dense_mqa(ctypes.byref(d), ctypes.byref(q), ws, big, None)
+    assert mqa(_abi.HCA, 128, _abi.E4M3_BF16ROPE, 1024, 0, 16) == _abi.ERR_INVALID_ARG
+    assert mqa(_abi.HCA, 128, _abi.E4M3_BF16ROPE, 1024, 8, 16,
+               ctypes.c_void_p((1 << 20) + 2)) == _abi.ERR_INVALID_ARG
+    assert mqa(_abi.HCA, 128, _abi.F32, 1024, 8, 8) == _abi.ERR_UNSUPPORTED
+    assert mqa(_abi.HCA, 128, _abi.E4M3_BF16ROPE, 1024, 8, 9) == _abi.ERR_INVALID_ARG
+    assert mqa(_abi.CSA, 4, _abi.E4M3_BF16ROPE, 1000, 8, 256) == _abi.ERR_INVALID_ARG
+
+    def index(idx_fmt, key_rows, bps, max_vis):
+        d = _abi.LayerDesc(_abi.CSA, 4, 128, 64, 512, 64, 160000.0, 0.0, 64, 128, 512,
+                           _abi.E4M3_BF16ROPE, idx_fmt, 1e-6)
+        ix = _abi.IndexArgs()
+        ix.n_q = ix.B = 2
+        for f in ("qI", "qI_sf", "w", "q_pos", "keys", "keys_sf", "idx_out"):
+            setattr(ix, f, fake)
+        ix.key_rows, ix.max_vis = key_rows, max_vis
+        ix.block_table, ix.blocks_per_seq = fake, bps
+        return lib.v4attn_index_topk(ctypes.byref(d), ctypes.byref(ix), ws, big, None)
+    assert index(_abi.F32, 4096, 16, 512) == _abi.ERR_UNSUPPORTED
+    assert index(_abi.MXFP4, 4096 + 16, 16, 512) == _abi.ERR_INVALID_ARG
+    assert index(_abi.MXFP4, 4096, 16, 513) == _abi.ERR_INVALID_ARG
