@@ -89,7 +89,7 @@ struct Smem {
     } mg;
   };
   float rcs[2][32], rsn[2][32];               // RoPE angles of the query positions (dh = 1)
-  int verdict;                                // the grid barrier's outcome, for the whole CTA
+  int bar_ok;                                 // the grid barrier's outcome, for the whole CTA
   float xl[KG - 1][128];                      // the other groups' row sums, for the epilogue
   uint64_t full[KST], empty[KST], sfull[2], pfull[2], pdone[2], xbar[4][2];
   uint64_t qready, ofinal, done, lbar;
@@ -764,10 +764,10 @@ __global__ void __launch_bounds__(NTHR, 1)
     if (tid == 0) {
       const bool ok = grid_barrier(P.grid_bar, P.grid_bar + 1, bar_gen0, gridDim.x, P.status);
       if (!ok) flag(P.status, ST_TIMEOUT | (1u << (16 + 13)));
-      s.verdict = ok ? 1 : 0;
+      s.bar_ok = ok ? 1 : 0;
     }
     __syncthreads();
-    merge_ok = s.verdict != 0;
+    merge_ok = s.bar_ok != 0;
   }
   // this CTA's column groups [g0, g1) of every row (four columns each); with
   // few splits and at most one (row, group) item a thread, every partial the
