@@ -19,19 +19,21 @@
 // layout, and go from the bulk-copied stage straight to TMEM with no rewrite
 // through registers (which would add generic-proxy stores and a proxy fence
 // per stage to the MMA warp).  The epilogue maps TMEM lane 32c + l back to key
-// 4l + c.  A ring stage holds up
-// to four consecutive 128-key tiles of one query (32 KB): on this part a
-// streaming read over one stage per barrier round trip reaches HBM speed only
-// from about 32 KB per stage on, while the work is still split between CTAs
-// tile by tile.  The accumulator has several TMEM stages so the epilogue of
-// tile i overlaps the MMAs of the tiles after it.  The MMA warp commits once
-// per stage (commits were its costliest instruction to issue); the first
-// epilogue warp, once it has seen that commit, hands the ring stage (and at a
-// query's end its query buffer) back to the producer.  Roles: warp 0 TMA producer,
-// warp 1 MMA issuer (one lane), warps 2..5 and 6..9 two epilogue groups on
-// alternate tiles (one thread per key row).  By its arithmetic intensity the
-// indexer is HBM-bound (68 bytes per key against 16384 FP4 FLOP); as built,
-// the MMA warp's tcgen05 instruction issue, not HBM, sets its time.
+// 4l + c.  A ring stage holds
+// up to three (two CTAs per SM, N <= 64) or four (one CTA per SM, N = 128)
+// consecutive 128-key tiles of one query: on this part a streaming read over
+// one stage per barrier round trip reaches HBM speed only from about 32 KB per
+// SM and stage on, while the work is still split between CTAs tile by tile.
+// The accumulator has several TMEM stages so the epilogue of tile i overlaps
+// the MMAs of the tiles after it.  The MMA warp commits once per stage
+// (commits were its costliest instruction to issue); the first epilogue warp,
+// once it has seen that commit, hands the ring stage (and at a query's end its
+// query buffer) back to the producer.  Roles: warp 0 TMA producer, warp 1 MMA
+// issuer (one lane), warps 2..5 and 6..9 two epilogue groups on alternate
+// tiles (one thread per key row).  By its arithmetic intensity the indexer is
+// HBM-bound (68 bytes per key against 16384 FP4 FLOP); as built, the
+// streaming itself (the per-stage barrier round trips from a landed load to
+// the stage's release) sets its time, the MMA issue next.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
