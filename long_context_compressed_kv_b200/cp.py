@@ -29,6 +29,19 @@ over NCCL on GPU tensors and over gloo on CPU ones):
 Between the two stages each rank compresses its owned entries
 (``v4attn_compress``) over its predecessor's tail rows followed by its own
 rows, reading absolute token t at row t - (start - n_tail).
+
+For decode over a history sharded by entries (each rank holding a contiguous
+slice of a sequence's compressed entries and indexer keys) two merges close
+the step:
+
+* ``merge_topk`` - every rank's k best (score, global index) pairs of its
+  slice merged into the sequence's k best (higher score first, ties to the
+  lower index, ascending output, -1 padding): each global winner is among
+  its own slice's k best, so the union of the local selections holds them;
+* ``merge_attention`` - the attention of the same queries over the ranks'
+  disjoint key sets (each normalised over its own keys, with its log
+  denominator; the sink counted on one rank only) merged into the attention
+  over their union: LSE = log sum_r exp(lse_r), o = sum_r exp(lse_r - LSE) o_r.
 """
 from __future__ import annotations
 
@@ -120,3 +133,50 @@ def gather_entries(local: torch.Tensor, n_valid: int, max_n: int, dist,
     parts = [torch.empty_like(pad) for _ in range(world)]
     dist.all_gather(parts, pad, group=group)
     return torch.cat([p[: int(c.item())] for p, c in zip(parts, all_counts)], 0)
+
+
+def merge_topk(scores: torch.Tensor, idx: torch.Tensor, k: int, dist, group=None) -> torch.Tensor:
+    """Global top-k from every rank's local selection.  scores [nq, kl] and
+    idx [nq, kl] (int64 global entry indices, -1 for no entry) hold a rank's
+    kl >= min(k, slice) best entries per query; returns int64 [nq, k]: the k
+    best over all ranks, higher score first with ties to the lower index,
+    in ascending index order, -1 padded (every rank gets it)."""
+    world = dist.get_world_size(group)
+    s_all = [torch.empty_like(scores) for _ in range(world)]
+    i_all = [torch.empty_like(idx) for _ in range(world)]
+    dist.all_gather(s_all, scores.contiguous(), group=group)
+    dist.all_gather(i_all, idx.contiguous(), group=group)
+    s = torch.cat(s_all, 1).to(torch.float64)
+    i = torch.cat(i_all, 1)
+    s = torch.where(i >= 0, s, torch.full_like(s, float("-inf")))
+    out = torch.full((s.shape[0], k), -1, dtype=torch.int64, device=s.device)
+    for q in range(s.shape[0]):
+        valid = i[q] >= 0
+        sq, iq = s[q][valid], i[q][valid]
+        # by score descending, then by index ascending (a stable two-key sort)
+        o1 = torch.argsort(iq, stable=True)
+        o2 = torch.argsort(-sq[o1], stable=True)
+        chosen = torch.sort(iq[o1][o2][:k]).values
+        out[q, : chosen.numel()] = chosen
+    return out
+
+
+def merge_attention(o: torch.Tensor, lse: torch.Tensor, dist, group=None):
+    """Attention over the union of the ranks' disjoint key sets from each
+    rank's part: o [..., H, d] normalised over the rank's keys (zero for a
+    rank with none), lse [..., H] the log of its denominator (-inf for none).
+    Returns (o, lse) of the union (every rank gets them)."""
+    world = dist.get_world_size(group)
+    o_all = [torch.empty_like(o) for _ in range(world)]
+    l_all = [torch.empty_like(lse) for _ in range(world)]
+    dist.all_gather(o_all, o.contiguous(), group=group)
+    dist.all_gather(l_all, lse.contiguous(), group=group)
+    L = torch.stack(l_all, 0)                                  # [R, ..., H]
+    top = torch.amax(L, 0)
+    top = torch.where(torch.isfinite(top), top, torch.zeros_like(top))
+    w = torch.exp(L - top)                                     # exp(-inf) = 0
+    den = w.sum(0)
+    lse_all = torch.log(den) + top
+    frac = torch.where(den > 0, w / den, torch.zeros_like(w))
+    out = sum(frac[r].unsqueeze(-1) * o_all[r] for r in range(world))
+    return out, lse_all

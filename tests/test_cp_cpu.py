@@ -104,3 +104,59 @@ def test_three_gloo_ranks_compress_like_one_process():
             assert np.array_equal(res[r][key], ref)
         checked += 1
     assert checked >= 2
+
+
+def _merge_main(rank, world, port, out):
+    from oracle import indexer as oidx, mqa as omqa
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        rng = np.random.default_rng(11)           # the same draws on every rank
+        nq, H, d, N, scale, k = 2, 3, 8, 20, 0.4, 8
+        q = rng.standard_normal((nq, H, d))
+        keys = rng.standard_normal((N, d))
+        sink = rng.standard_normal(H)
+        scores = np.round(rng.standard_normal((3, 50)) * 2) / 2   # many exact ties
+        # this rank's contiguous slices of the keys and of the score rows
+        a, b = cp.chunk_bounds(N, world)[rank]
+        parts = [omqa.attend(q[i], keys[a:b], scale, sink if rank == 0 else None)
+                 for i in range(nq)]
+        o = torch.from_numpy(np.stack([p[0] for p in parts]))
+        lse = torch.from_numpy(np.stack([p[1] for p in parts]))
+        mo, ml = cp.merge_attention(o, lse, dist)
+        sa, sb = cp.chunk_bounds(50, world)[rank]
+        loc = [oidx.topk(scores[r, sa:sb], sb - sa, k) for r in range(3)]
+        gidx = np.stack([np.where(l >= 0, l + sa, -1) for l in loc])
+        gsc = np.stack([np.where(g >= 0, scores[r, np.maximum(g, 0)], -np.inf)
+                        for r, g in enumerate(gidx)])
+        sel = cp.merge_topk(torch.from_numpy(gsc), torch.from_numpy(gidx), k, dist)
+        out[rank] = dict(o=mo.numpy(), lse=ml.numpy(), sel=sel.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_entry_sharded_decode_merges_match_one_process():
+    """A history sharded by entries over 3 gloo ranks: the attention parts
+    (sink on one rank) merge into the attention over all keys, and the local
+    top-k selections (scores with many exact ties) into the global top-k
+    (oracle attend / topk on each rank's slice stand in for the GPU calls)."""
+    from oracle import indexer as oidx, mqa as omqa
+    world = 3
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_merge_main, args=(world, port, out), nprocs=world, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    rng = np.random.default_rng(11)
+    nq, H, d, N, scale, k = 2, 3, 8, 20, 0.4, 8
+    q = rng.standard_normal((nq, H, d))
+    keys = rng.standard_normal((N, d))
+    sink = rng.standard_normal(H)
+    scores = np.round(rng.standard_normal((3, 50)) * 2) / 2
+    ref = [omqa.attend(q[i], keys, scale, sink) for i in range(nq)]
+    ref_sel = np.stack([oidx.topk(scores[r], 50, k) for r in range(3)])
+    for r in range(world):
+        assert np.allclose(res[r]["o"], np.stack([x[0] for x in ref]), rtol=1e-12, atol=1e-12)
+        assert np.allclose(res[r]["lse"], np.stack([x[1] for x in ref]), rtol=1e-12, atol=1e-12)
+        assert np.array_equal(res[r]["sel"], ref_sel)
